@@ -1,0 +1,411 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE expert layer: fwd+bwd tokens/s and grouped-GEMM
+TFLOP/s on B200, one process per GPU.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun as independent replicas (the layer keeps all
+experts on one GPU and has no exchange step): every rank runs the same
+workload on its own tokens, the timing is the max over ranks and `value`
+is the tokens of all ranks over that time (weak scaling).
+
+Timed region: W untimed warm-up steps, then exactly K steps, each bracketed
+by CUDA events on the stream the library launches on; between steps (and
+outside the events) a 512 MiB buffer is written to flush the 126 MB L2.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer fwd+bwd tokens/s and grouped-GEMM TFLOP/s (% of B200 peak), 1 GPU"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "e8"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-ratio", action="store_true", help="skip the E=128 vs E=8 measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.dev), "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        loaded = [r for r in rows if r[2] > 250.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3])
+                          if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in loaded), "reasons": reasons,
+                "samples": len(loaded), "power_w_max": max(r[2] for r in loaded)}
+
+
+# ------------------------------------------------------------------ oracle timing
+def _oracle_step(x, w_r, w_gu, w_d, dy, k, bias, route):
+    from oracle import moe_ref as R
+    fwd = R.layer_fwd(x, w_r, w_gu, w_d, k, bias=bias, route=route)
+    R.layer_bwd(fwd, dy, x, w_r, w_gu, w_d)
+
+
+def _oracle_inputs(cfg, T_s):
+    import torch
+    from mixture_experts_layer_39_b200.inputs import make_inputs
+    inp = make_inputs(cfg, seed=0, device="cuda" if torch.cuda.is_available() else "cpu")
+    f64 = lambda t: t.detach().to("cpu").double().numpy()
+    return (f64(inp["x"][:T_s]), f64(inp["w_r"]), f64(inp["w_gu"]), f64(inp["w_d"]),
+            f64(inp["dy"][:T_s]), None if inp["bias"] is None else f64(inp["bias"]),
+            None if inp["route"] is None else inp["route"][:T_s].cpu().numpy())
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def size_oracle_sample(cfg, seconds):
+    """Tokens per oracle step so that one step costs about `seconds`."""
+    T_s = min(128, cfg.T)
+    args = _oracle_inputs(cfg, T_s)
+    t0 = time.perf_counter()
+    _oracle_step(*args[:4], args[4], cfg.k, args[5], args[6])
+    dt = max(time.perf_counter() - t0, 1e-3)
+    T_fit = int(T_s * seconds / dt)
+    return max(min(128, cfg.T), min(cfg.T, T_fit // 64 * 64 if T_fit >= 64 else T_fit))
+
+
+def cpu_baseline(cfg, seconds):
+    T_s = size_oracle_sample(cfg, seconds)
+    args = _oracle_inputs(cfg, T_s)
+    t0 = time.perf_counter()
+    _oracle_step(*args[:4], args[4], cfg.k, args[5], args[6])
+    dt = time.perf_counter() - t0
+    return {"value": T_s / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"oracle fwd+bwd (NumPy float64, bf16 storage rounding) on the first "
+                       f"{T_s} of {cfg.T} tokens of workload {cfg.name} with all {cfg.E} experts' "
+                       f"full weights; one pass, {dt:.1f} s"),
+            "seconds": dt, "tokens": T_s}
+
+
+# ------------------------------------------------------------------ our arm
+def gemm_traffic(cfg_name):
+    """DRAM bytes per step of the grouped-GEMM launches from the committed ncu
+    summary, only while the kernel sources are the ones it was taken on."""
+    p = os.path.join(ROOT, "profiles", "grouped_gemm_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        d = json.load(fh)
+    h = hashlib.sha256()
+    for rel in ("mixture_experts_layer_39_b200/csrc/tc_gemm.cuh",
+                "mixture_experts_layer_39_b200/csrc/gemm.cu"):
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    if d.get("source_sha256") != h.hexdigest() or d.get("workload") != cfg_name:
+        return None
+    return d.get("dram_bytes_per_step")
+
+
+def measure(L, g, steps, warmup, flush, dev, with_gemm_events=True):
+    import torch
+    stream = torch.cuda.current_stream()
+
+    def one_step(ev=None):
+        L.router(g["x"], g["w_r"], g["bias"], g["route"])
+        L.permute(g["x"])
+        if ev: ev[0].record(stream)
+        L.experts_fwd(g["w_gu"], g["w_d"])
+        if ev: ev[1].record(stream)
+        L.combine()
+        L.combine_bwd(g["dy"])
+        L.router_bwd(g["x"], g["w_r"])
+        if ev: ev[2].record(stream)
+        L.experts_bwd(g["w_gu"], g["w_d"])
+        if ev: ev[3].record(stream)
+        L.permute_bwd()
+
+    for _ in range(warmup):
+        flush.fill_(1)
+        one_step()
+    torch.cuda.synchronize(dev)
+    n0 = L.handle.launch_count()
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    step_ev = [(mk(), mk()) for _ in range(steps)]
+    gemm_ev = [[mk() for _ in range(4)] for _ in range(steps)] if with_gemm_events else None
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        step_ev[i][0].record(stream)
+        one_step(gemm_ev[i] if gemm_ev else None)
+        step_ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    launches = L.handle.launch_count() - n0
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    gemm_ms = [e[0].elapsed_time(e[1]) + e[2].elapsed_time(e[3]) for e in gemm_ev] if gemm_ev else None
+    return step_ms, gemm_ms, launches
+
+
+def measure_e2e(L, g, steps, warmup, flush, dev):
+    """Same step through the public API with the per-step inputs (x, dY and
+    the random-routing ids when used) copied from pinned host memory and the
+    step's results (y, dX) read back, all inside the timed region."""
+    import torch
+    stream = torch.cuda.current_stream()
+    host_in = {n: g[n].cpu().pin_memory() for n in ("x", "dy") }
+    if g["route"] is not None:
+        host_in["route"] = g["route"].cpu().pin_memory()
+    dev_in = {n: torch.empty_like(g[n]) for n in host_in}
+    y_h = torch.empty(L.y.shape, dtype=L.y.dtype, pin_memory=True)
+    dx_h = torch.empty(L.dx.shape, dtype=L.dx.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = y_h.numel() * y_h.element_size() + dx_h.numel() * dx_h.element_size()
+
+    def one():
+        for n, t in host_in.items():
+            dev_in[n].copy_(t, non_blocking=True)
+        L.step(dev_in["x"], g["w_r"], g["w_gu"], g["w_d"], dev_in["dy"], g["bias"],
+               dev_in.get("route"))
+        y_h.copy_(L.y, non_blocking=True)
+        dx_h.copy_(L.dx, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize(dev)
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    evs = [(mk(), mk()) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        evs[i][0].record(stream)
+        one()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    return [a.elapsed_time(b) for a, b in evs], h2d, d2h
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from mixture_experts_layer_39_b200.inputs import CONFIGS, make_inputs
+    from mixture_experts_layer_39_b200.layer import MoELayer
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def max_over_ranks(v):
+        if ws == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    cfg = CONFIGS[args.workload]
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    sampler = ClockSampler(local)
+
+    def bench_cfg(c, steps, warmup, with_e2e):
+        g = make_inputs(c, seed=rank, device=dev)
+        L = MoELayer(c.T, c.d, c.f, c.E, c.k, device=dev)
+        barrier()
+        step_ms, gemm_ms, launches = measure(L, g, steps, warmup, flush, dev)
+        barrier()
+        out = {"total_ms": max_over_ranks(sum(step_ms)), "step_ms": step_ms,
+               "gemm_ms": gemm_ms, "launches": launches, "counts": L.counts.cpu().numpy()}
+        if with_e2e:
+            e2e_ms, h2d, d2h = measure_e2e(L, g, steps, min(warmup, 3), flush, dev)
+            barrier()
+            out.update({"e2e_total_ms": max_over_ranks(sum(e2e_ms)), "h2d": h2d, "d2h": d2h})
+        st = L.handle.get_status()
+        if st != 0:
+            raise RuntimeError(f"device status {st} after the benchmark")
+        del L, g
+        torch.cuda.empty_cache()
+        return out
+
+    sampler.start()
+    main = bench_cfg(cfg, args.steps, args.warmup, True)
+    ratio = None
+    if not args.no_ratio and cfg.name == "e8":
+        other = bench_cfg(CONFIGS["e128"], args.steps, args.warmup, False)
+        ratio = other
+    clocks = sampler.stop()
+
+    K = args.steps
+    tokens = cfg.T * K * ws
+    value = tokens / (main["total_ms"] / 1e3)
+    e2e_value = tokens / (main["e2e_total_ms"] / 1e3)
+    peaks, peak_kind = load_peaks()
+    gemm_flops = cfg.gemm_flops_fwd_bwd()
+    gemm_ms = statistics.mean(main["gemm_ms"])
+    achieved = gemm_flops / (gemm_ms / 1e3) / 1e12
+    traffic = gemm_traffic(cfg.name)
+    counts = main["counts"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": K,
+        "warmup": args.warmup, "ms_per_step": main["total_ms"] / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations, N(0,1/d) weights, learned-style routing)",
+        "config": {"workload": f"{cfg.name}: T={cfg.T} d_model={cfg.d} d_ff={cfg.f} E={cfg.E} "
+                               f"top_k={cfg.k} (4x4096 tokens)",
+                   "global_batch": cfg.T * ws, "parallelism": f"replicas{ws}" if ws > 1 else "1 GPU",
+                   "l2": "flushed between timed steps (512 MiB write outside the step events)"},
+        "roofline": {"bound": "tensor", "kernel": "grouped_gemm_kernel (6 launches per step)",
+                     "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                     "peak_source": f"{peak_kind} bf16 burst"},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": main["h2d"],
+                "d2h_bytes_per_step": main["d2h"]},
+        "gpu_launches": main["launches"],
+        "grouped_gemm": {"tflops": achieved, "ms_per_step": gemm_ms,
+                         "share_of_step": gemm_ms / (main["total_ms"] / K)},
+        "routing": {"max_over_mean_load": float(counts.max() / counts.mean()),
+                    "zero_experts": int((counts == 0).sum())},
+        "clocks": clocks,
+    }
+    if ratio is not None:
+        r_value = CONFIGS["e128"].T * K * ws / (ratio["total_ms"] / 1e3)
+        line["e128"] = {"value": r_value, "unit": UNIT, "vs_e8": r_value / value,
+                        "grouped_gemm_tflops": CONFIGS["e128"].gemm_flops_fwd_bwd()
+                        / (statistics.mean(ratio["gemm_ms"]) / 1e3) / 1e12}
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = {k: v for k, v in cpu_baseline(cfg, args.cpu_seconds).items()
+                                if k in ("value", "unit", "cores", "kind", "sample")}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    """The oracle, as it stands, on the host cores: each step is the layer's
+    fwd+bwd on a bounded sample of the workload's tokens."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    from mixture_experts_layer_39_b200.inputs import CONFIGS
+    cfg = CONFIGS[args.workload]
+    per_step = max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    T_s = size_oracle_sample(cfg, min(per_step, 5.0))
+    inp = _oracle_inputs(cfg, T_s)
+    for _ in range(args.warmup):
+        _oracle_step(*inp[:4], inp[4], cfg.k, inp[5], inp[6])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(*inp[:4], inp[4], cfg.k, inp[5], inp[6])
+    dt = time.perf_counter() - t0
+    value = T_s * args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": f"{cfg.name}: T={cfg.T} d_model={cfg.d} "
+                                                    f"d_ff={cfg.f} E={cfg.E} top_k={cfg.k}"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"each step: oracle fwd+bwd on the first {T_s} of {cfg.T} tokens"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,249 @@
+/*
+ * moe.h -- C ABI of libmoe.so, the dropless mixture-of-experts expert layer
+ * (one training step, one GPU, NVIDIA B200 / sm_100a).
+ *
+ * The layer, as the Olmo-core 3 pages describe it in words:
+ *   - a router computes a score distribution over the experts for every
+ *     token and keeps the k best (discosf.com article on Olmo-core 3,
+ *     section 1.1 "sparse computation" and section 2.1 "how a token is sent
+ *     to the experts in one forward pass");
+ *   - the routing metadata stays on the GPU so the host never waits for a
+ *     copy back; routed tokens are written straight into each expert's
+ *     contiguous input buffer; all experts' small GEMMs run as one grouped
+ *     GEMM whose schedule is read on the device (Olmo-core 3 introduction
+ *     page, section 2 "three parallelisms plus three routing
+ *     optimisations");
+ *   - no token is dropped when an expert is over-subscribed (vibecoding.ru
+ *     news item on Olmo-core 3, paragraph on grouped_gemm and dropless MoE);
+ *   - expert outputs are put back in the original token order (discosf.com
+ *     article, section 2.1);
+ *   - MXFP8 is offered for selected operations (Olmo-core 3 introduction
+ *     page, section 3 "MXFP8").
+ * The pages give no formulas; the readings used are stated per call.
+ *
+ * Conventions for every call below
+ *   - Pointers named as device pointers must point to device memory of the
+ *     handle's device; all of them are owned by the caller.  No call
+ *     allocates, frees or copies to the host; all scratch comes from `ws`
+ *     (size from moe_workspace_size).  The one exception is moe_create,
+ *     which allocates a 256-byte control block freed by moe_destroy.
+ *   - Every call only enqueues work on `stream` (a cudaStream_t, may be 0)
+ *     and returns; nothing synchronises the host except moe_get_status.
+ *   - Host-side checks run before any launch: a NULL required pointer, a
+ *     bad size or a misaligned pointer returns MOE_ERR_INVALID_ARG, a shape
+ *     outside the supported set returns MOE_ERR_UNSUPPORTED, and nothing is
+ *     launched.  A failed launch returns MOE_ERR_CUDA.
+ *   - Problems only the device can see (an expert id outside [0, E) in a
+ *     caller-written topk_idx, a bounded wait that ran out) never trap: the
+ *     kernel records a code in the handle's status word, skips the bad
+ *     entry, and moe_get_status reports it later.
+ *   - Layouts are row-major.  bf16 = bfloat16 (round to nearest even).
+ *   - Supported shapes: 1 <= k <= min(E, 8), 1 <= E <= 1024, T >= 1,
+ *     d_model and d_ff multiples of 256.
+ *
+ * Routed-row space.  Every expert e owns a segment of rows
+ * [offsets[e], offsets[e+1]) in the permuted buffers; segments start at
+ * multiples of 32 rows, hold counts[e] real rows in ascending (token, slot)
+ * order followed by zero pad rows.  Buffers in this space have
+ * M_cap = T*k + 31*E rows (moe_max_rows); rows at and past offsets[E] are
+ * never read or written.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,
+  MOE_ERR_UNSUPPORTED = 2,
+  MOE_ERR_CUDA = 3,
+  MOE_ERR_WORKSPACE = 4,
+  MOE_ERR_DEVICE_CHECK = 5, /* device saw a bad index / offset */
+  MOE_ERR_TIMEOUT = 6       /* a bounded device-side wait gave up */
+} moe_status_t;
+
+enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_MXFP8 = 1 };
+enum { MOE_FLAG_RENORM = 1 }; /* gate weights divided by their sum over k */
+
+typedef struct moe_shape {
+  int T;         /* tokens */
+  int d_model;   /* d */
+  int d_ff;      /* f, per-expert hidden width */
+  int n_experts; /* E */
+  int top_k;     /* k */
+  int dtype;     /* MOE_DTYPE_BF16 or MOE_DTYPE_MXFP8 (expert GEMM operands) */
+  int flags;     /* MOE_FLAG_* */
+} moe_shape_t;
+
+typedef struct moe_context* moe_handle_t;
+
+typedef void* moe_stream_t; /* a cudaStream_t */
+
+/* Creates a handle bound to CUDA device `device`: caches the SM count and
+ * allocates the device status word.  *h receives the handle. */
+MOE_API moe_status_t moe_create(moe_handle_t* h, int device);
+
+/* Frees the handle's control block.  Pending work must have finished. */
+MOE_API moe_status_t moe_destroy(moe_handle_t h);
+
+/* Bytes of scratch every step call of this shape may use, in one buffer
+ * shared by all calls (calls on one stream run in order, so they can share
+ * it).  Must be 256-byte aligned. */
+MOE_API moe_status_t moe_workspace_size(moe_handle_t h, const moe_shape_t* s, size_t* bytes);
+
+/* M_cap = T*k + 31*E: rows of every buffer in the routed-row space. */
+MOE_API moe_status_t moe_max_rows(const moe_shape_t* s, int64_t* rows);
+
+/* Router forward (top-k softmax).
+ *   L[t,e] = sum_i x[t,i] * w_router[e,i] (+ bias[e]), fp32 accumulate;
+ *   probs  = softmax over all E experts, fp32;
+ *   topk_idx[t, 0..k-1] = the k largest L[t,:], ties to the lower expert
+ *     index, ordered by descending logit;  when route_in != NULL its ids
+ *     are used instead (random-routing benchmark mode of the pages);
+ *   topk_w[t,j] = probs[t, topk_idx[t,j]] (divided by their sum when
+ *     MOE_FLAG_RENORM).
+ * In : x [T,d] bf16, w_router [E,d] bf16, bias [E] fp32 or NULL,
+ *      route_in [T,k] int32 or NULL (must hold k distinct ids in [0,E)).
+ * Out: topk_idx [T,k] int32, topk_w [T,k] fp32, probs [T,E] fp32 (kept for
+ *      the backward), logits [T,E] fp32 or NULL (optional copy of L).
+ * One warp per token does the softmax and the top-k in registers. */
+MOE_API moe_status_t moe_router_topk(moe_handle_t h, const moe_shape_t* s,
+                             const void* x, const void* w_router, const float* bias,
+                             const int32_t* route_in, int32_t* topk_idx, float* topk_w,
+                             float* probs, float* logits, void* ws, size_t ws_bytes,
+                             moe_stream_t stream);
+
+/* Routing metadata + rowwise permute, all on the device.
+ *   counts[e]   = number of (t,j) with topk_idx[t,j] == e;
+ *   offsets[e]  = sum_{e'<e} roundup(counts[e'], 32); offsets[E] = M_pad;
+ *   row_map[t,j]= offsets[e] + #{(t',j') before (t,j) in t*k+j order with
+ *                 the same expert e};
+ *   x_perm[row_map[t,j]] = x[t]; pad rows of every segment are zero.
+ * In : x [T,d] bf16, topk_idx [T,k] int32.
+ * Out: counts [E] int32, offsets [E+1] int32, row_map [T,k] int32,
+ *      x_perm [M_cap,d] bf16.
+ * An id outside [0,E) sets MOE_ERR_DEVICE_CHECK and that entry is skipped
+ * (its row_map entry is -1). */
+MOE_API moe_status_t moe_permute(moe_handle_t h, const moe_shape_t* s, const void* x,
+                         const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                         int32_t* row_map, void* x_perm, void* ws, size_t ws_bytes,
+                         moe_stream_t stream);
+
+/* Grouped SwiGLU expert FFN, forward.  For the rows of expert e:
+ *   A = X W_gu[e][0:f]^T, U = X W_gu[e][f:2f]^T   (fp32 accumulate)
+ *   au[:, 0:f] = bf16(A), au[:, f:2f] = bf16(U)   (saved for the backward)
+ *   h = bf16(silu(A) * U), silu(z) = z / (1 + exp(-z))
+ *   o_perm = bf16(h W_down[e]^T)
+ * In : x_perm [M_cap,d] bf16, offsets [E+1] int32 (from moe_permute),
+ *      w_gu [E,2f,d] bf16, w_down [E,d,f] bf16.
+ * Out: au [M_cap,2f] bf16, h [M_cap,f] bf16, o_perm [M_cap,d] bf16.
+ * Persistent tcgen05/TMEM kernels fed by TMA; the tile schedule is decoded
+ * from `offsets` on the device. */
+MOE_API moe_status_t moe_grouped_swiglu_fwd(moe_handle_t h, const moe_shape_t* s, const void* x_perm,
+                                    const int32_t* offsets, const void* w_gu,
+                                    const void* w_down, void* au, void* hbuf, void* o_perm,
+                                    void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Weighted unpermute-combine ("restore"):
+ *   y[t] = bf16( sum_j topk_w[t,j] * o_perm[row_map[t,j]] ), fp32 sum in
+ *   slot order.
+ * In : o_perm [M_cap,d] bf16, row_map [T,k] int32, topk_w [T,k] fp32.
+ * Out: y [T,d] bf16. */
+MOE_API moe_status_t moe_unpermute_combine(moe_handle_t h, const moe_shape_t* s, const void* o_perm,
+                                   const int32_t* row_map, const float* topk_w, void* y,
+                                   moe_stream_t stream);
+
+/* Backward of the combine:
+ *   do_perm[row_map[t,j]] = bf16(topk_w[t,j] * dy[t]); pad rows = 0;
+ *   d_topk_w[t,j] = sum_i dy[t,i] * o_perm[row_map[t,j], i]  (fp32).
+ * In : dy [T,d] bf16, o_perm, row_map, topk_w, offsets [E+1], counts [E].
+ * Out: do_perm [M_cap,d] bf16, d_topk_w [T,k] fp32. */
+MOE_API moe_status_t moe_unpermute_combine_bwd(moe_handle_t h, const moe_shape_t* s, const void* dy,
+                                       const void* o_perm, const int32_t* row_map,
+                                       const float* topk_w, const int32_t* offsets,
+                                       const int32_t* counts, void* do_perm, float* d_topk_w,
+                                       moe_stream_t stream);
+
+/* Grouped SwiGLU expert FFN, backward (dgrad and wgrad).  Per expert e:
+ *   dH = do_perm W_down[e]                       (fp32 accumulate)
+ *   s = sigmoid(A), A and U read from au
+ *   dau[:,0:f] = bf16(dH U s (1 + A (1 - s))),  dau[:,f:2f] = bf16(dH silu(A))
+ *   dw_down[e] = bf16(do_perm_e^T h_e)           (sum over e's rows)
+ *   dx_perm    = bf16(dau W_gu[e])
+ *   dw_gu[e]   = bf16(dau_e^T x_perm_e)
+ * Experts with no rows get zero weight gradients.
+ * In : do_perm, x_perm, au, hbuf [M_cap,*] bf16, offsets [E+1], w_gu, w_down.
+ * Out: dau [M_cap,2f] bf16, dx_perm [M_cap,d] bf16, dw_gu [E,2f,d] bf16,
+ *      dw_down [E,d,f] bf16. */
+MOE_API moe_status_t moe_grouped_swiglu_bwd(moe_handle_t h, const moe_shape_t* s, const void* do_perm,
+                                    const void* x_perm, const void* au, const void* hbuf,
+                                    const int32_t* offsets, const void* w_gu,
+                                    const void* w_down, void* dau, void* dx_perm, void* dw_gu,
+                                    void* dw_down, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream);
+
+/* Backward of the permute:
+ *   dx[t] = bf16( sum_j dx_perm[row_map[t,j]] + dx_router[t] ), fp32 sum,
+ *   rounded once.  dx_router may be NULL.
+ * In : dx_perm [M_cap,d] bf16, row_map [T,k], dx_router [T,d] fp32 or NULL.
+ * Out: dx [T,d] bf16. */
+MOE_API moe_status_t moe_permute_bwd(moe_handle_t h, const moe_shape_t* s, const void* dx_perm,
+                             const int32_t* row_map, const float* dx_router, void* dx,
+                             moe_stream_t stream);
+
+/* Router backward (through the selected probabilities; top-k itself has no
+ * gradient):
+ *   g = d_topk_w, or with MOE_FLAG_RENORM g_j = (dw_j - sum_i dw_i w_i) / S
+ *   dp[t, topk_idx[t,j]] = g[t,j], 0 elsewhere
+ *   dL = probs * (dp - sum_e probs dp)
+ *   dx_router = dL w_router            [T,d] fp32 (fed to moe_permute_bwd)
+ *   dw_router = bf16(dL^T x)           [E,d]
+ *   dbias     = sum_t dL               [E] fp32, written when non-NULL
+ * In : d_topk_w [T,k] fp32, probs [T,E] fp32, topk_idx [T,k], x [T,d] bf16,
+ *      w_router [E,d] bf16. */
+MOE_API moe_status_t moe_router_topk_bwd(moe_handle_t h, const moe_shape_t* s, const float* d_topk_w,
+                                 const float* probs, const int32_t* topk_idx, const void* x,
+                                 const void* w_router, float* dx_router, void* dw_router,
+                                 float* dbias, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* MXFP8 quantisation of a bf16 matrix [rows, cols] (OCP MX v1.0 reading of
+ * the pages' "MXFP8"): blocks of 32 consecutive elements, along each row
+ * (axis = 1) or down each column (axis = 0); per block the E8M0 scale code
+ * is clamp(floor(log2(amax)) - 8, -127, 127) + 127 (code 0 for an all-zero
+ * block) and each element is the E4M3 code of round-to-nearest-even
+ * (v / 2^(code-127)), saturated to +-448.
+ * In : in [rows, cols] bf16; rows (axis 0) or cols (axis 1) multiple of 32.
+ * Out: q [rows, cols] uint8 (E4M3 codes), scales uint8 (E8M0 codes),
+ *      [rows, cols/32] for axis 1, [rows/32, cols] for axis 0. */
+MOE_API moe_status_t moe_mxfp8_quantize(moe_handle_t h, const void* in, int64_t rows, int64_t cols,
+                                int axis, uint8_t* q, uint8_t* scales, moe_stream_t stream);
+
+/* Waits for the device, then returns the status word recorded by kernels
+ * (MOE_OK if none) in *device_status and clears it.  The only call that
+ * synchronises; not meant for use inside a step. */
+MOE_API moe_status_t moe_get_status(moe_handle_t h, int* device_status);
+
+/* Number of kernels this handle has launched since it was created (a host
+ * counter: it costs nothing on the device and does not synchronise). */
+MOE_API moe_status_t moe_get_launch_count(moe_handle_t h, uint64_t* launches);
+
+/* Static description of a status code. */
+MOE_API const char* moe_status_string(moe_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,425 @@
+// extern "C" entry points of libmoe.so (declared and documented in
+// include/moe.h): argument checks, workspace carving, launch order.
+#include <cstdio>
+#include <cstdlib>
+#include <new>
+
+#include "gemm.cuh"
+#include "kernels.cuh"
+
+struct moe_context {
+  int device;
+  int num_sms;
+  moe::DeviceCtl* ctl;      // device status word
+  uint64_t launches = 0;    // kernels launched through this handle
+};
+
+namespace {
+
+using moe::ceil_div64;
+
+// Makes the handle's device current for the duration of a call.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) { ok = false; return; }
+    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) {
+      int cur = -1;
+      if (cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+  }
+};
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+moe_status_t check_shape(const moe_shape_t* s) {
+  if (s == nullptr) return MOE_ERR_INVALID_ARG;
+  if (s->T < 1 || s->d_model < 1 || s->d_ff < 1 || s->n_experts < 1 || s->top_k < 1)
+    return MOE_ERR_INVALID_ARG;
+  if (s->top_k > s->n_experts) return MOE_ERR_INVALID_ARG;
+  if (s->top_k > 8 || s->n_experts > 1024) return MOE_ERR_UNSUPPORTED;
+  if (s->d_model % 256 != 0 || s->d_ff % 256 != 0) return MOE_ERR_UNSUPPORTED;
+  if (s->dtype != MOE_DTYPE_BF16 && s->dtype != MOE_DTYPE_MXFP8) return MOE_ERR_INVALID_ARG;
+  const int64_t m_cap = static_cast<int64_t>(s->T) * s->top_k + 31ll * s->n_experts;
+  if (m_cap >= (1ll << 31) - 256) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+int64_t max_rows(const moe_shape_t* s) {
+  return static_cast<int64_t>(s->T) * s->top_k + 31ll * s->n_experts;
+}
+
+bool router_on_tensor_cores(int E) { return E > 64; }
+
+moe_status_t check_router_shape(const moe_shape_t* s) {
+  const int E = s->n_experts;
+  if (E <= 64) return MOE_OK;
+  if (E % 128 == 0) return MOE_OK;
+  return MOE_ERR_UNSUPPORTED;
+}
+
+size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+// Router backward workspace layout.
+struct RouterBwdWs {
+  size_t dl, db_part, part, total;
+  int nblocks, n_part, group_len;
+};
+
+RouterBwdWs router_bwd_layout(const moe_context* h, const moe_shape_t* s) {
+  RouterBwdWs w{};
+  const int T = s->T, d = s->d_model, E = s->n_experts;
+  w.nblocks = moe::router_bwd_blocks(h->num_sms);
+  size_t off = 0;
+  w.dl = off;
+  off += align256(static_cast<size_t>(T) * E * (router_on_tensor_cores(E) ? 2 : 4));
+  w.db_part = off;
+  off += align256(static_cast<size_t>(w.nblocks) * E * 4);
+  w.part = off;
+  if (router_on_tensor_cores(E)) {
+    w.n_part = moe::router_dw_groups(h->num_sms, T, d, E, &w.group_len);
+  } else {
+    w.n_part = static_cast<int>(ceil_div64(T, moe::router_dw_small_chunk()));
+    w.group_len = moe::router_dw_small_chunk();
+  }
+  off += align256(static_cast<size_t>(w.n_part) * E * d * 4);
+  w.total = off;
+  return w;
+}
+
+size_t workspace_bytes(const moe_context* h, const moe_shape_t* s) {
+  const int64_t T = s->T, E = s->n_experts;
+  size_t need = 0;
+  auto upd = [&](size_t v) { need = v > need ? v : need; };
+  upd(align256(static_cast<size_t>(T) * E * 4));                                   // router logits
+  upd(align256(static_cast<size_t>(moe::n_subchunks(s->T, s->top_k)) * E * 4));    // permute
+  upd(router_bwd_layout(h, s).total);                                              // router bwd
+  return need;
+}
+
+moe_status_t check_ws(const moe_context* h, const moe_shape_t* s, void* ws, size_t ws_bytes) {
+  if (ws == nullptr || !aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < workspace_bytes(h, s)) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                          \
+  do {                                         \
+    const moe_status_t _st = (expr);           \
+    if (_st != MOE_OK) return _st;             \
+  } while (0)
+
+#define MOE_CHECK_HANDLE(h, s)                                  \
+  do {                                                          \
+    if ((h) == nullptr) return MOE_ERR_INVALID_ARG;             \
+    MOE_TRY(check_shape(s));                                    \
+  } while (0)
+
+#define MOE_GUARD(h)                         \
+  DeviceGuard _guard((h)->device);           \
+  if (!_guard.ok) return MOE_ERR_CUDA
+
+template <typename... P>
+bool all_nonnull(P... p) { return ((p != nullptr) && ...); }
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_create(moe_handle_t* out, int device) {
+  if (out == nullptr) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  int n = 0;
+  if (cudaGetDeviceCount(&n) != cudaSuccess || device < 0 || device >= n) return MOE_ERR_INVALID_ARG;
+  DeviceGuard g(device);
+  if (!g.ok) return MOE_ERR_CUDA;
+  auto* h = new (std::nothrow) moe_context();
+  if (h == nullptr) return MOE_ERR_CUDA;
+  h->device = device;
+  if (cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) {
+    delete h;
+    return MOE_ERR_CUDA;
+  }
+  if (cudaMalloc(&h->ctl, 256) != cudaSuccess) {
+    delete h;
+    return MOE_ERR_CUDA;
+  }
+  if (cudaMemset(h->ctl, 0, 256) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    cudaFree(h->ctl);
+    delete h;
+    return MOE_ERR_CUDA;
+  }
+  *out = h;
+  return MOE_OK;
+}
+
+moe_status_t moe_destroy(moe_handle_t h) {
+  if (h == nullptr) return MOE_ERR_INVALID_ARG;
+  {
+    DeviceGuard g(h->device);
+    cudaFree(h->ctl);
+  }
+  delete h;
+  return MOE_OK;
+}
+
+moe_status_t moe_workspace_size(moe_handle_t h, const moe_shape_t* s, size_t* bytes) {
+  MOE_CHECK_HANDLE(h, s);
+  if (bytes == nullptr) return MOE_ERR_INVALID_ARG;
+  *bytes = workspace_bytes(h, s);
+  return MOE_OK;
+}
+
+moe_status_t moe_max_rows(const moe_shape_t* s, int64_t* rows) {
+  MOE_TRY(check_shape(s));
+  if (rows == nullptr) return MOE_ERR_INVALID_ARG;
+  *rows = max_rows(s);
+  return MOE_OK;
+}
+
+moe_status_t moe_router_topk(moe_handle_t h, const moe_shape_t* s, const void* x,
+                             const void* w_router, const float* bias, const int32_t* route_in,
+                             int32_t* topk_idx, float* topk_w, float* probs, float* logits,
+                             void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  MOE_TRY(check_router_shape(s));
+  if (!all_nonnull(x, w_router, topk_idx, topk_w, probs)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(w_router, 16)) return MOE_ERR_INVALID_ARG;
+  const int T = s->T, d = s->d_model, E = s->n_experts, k = s->top_k;
+  const bool renorm = (s->flags & MOE_FLAG_RENORM) != 0;
+  auto st = static_cast<cudaStream_t>(stream);
+  MOE_GUARD(h);
+  if (!router_on_tensor_cores(E)) {
+    h->launches += 1;
+    return cuda_status(moe::launch_router_fused(
+        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_router), bias,
+        route_in, T, d, E, k, renorm, topk_idx, topk_w, probs, logits, h->ctl, st));
+  }
+  float* lg = logits;
+  if (lg == nullptr) {
+    MOE_TRY(check_ws(h, s, ws, ws_bytes));
+    lg = static_cast<float*>(ws);
+  } else if (!aligned(lg, 16)) {
+    return MOE_ERR_INVALID_ARG;
+  }
+  moe::GemmCtx c{h->num_sms, h->ctl};
+  h->launches += 2;
+  MOE_TRY(moe::gemm_router_logits(c, x, w_router, lg, T, d, E, st));
+  return cuda_status(moe::launch_softmax_topk(lg, bias, route_in, T, E, k, renorm, topk_idx, topk_w,
+                                              probs, logits, h->ctl, st));
+}
+
+moe_status_t moe_permute(moe_handle_t h, const moe_shape_t* s, const void* x,
+                         const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                         int32_t* row_map, void* x_perm, void* ws, size_t ws_bytes,
+                         moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  if (!all_nonnull(x, topk_idx, counts, offsets, row_map, x_perm)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(x_perm, 16)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(h, s, ws, ws_bytes));
+  const int T = s->T, d = s->d_model, E = s->n_experts, k = s->top_k;
+  auto st = static_cast<cudaStream_t>(stream);
+  MOE_GUARD(h);
+  auto* sub = static_cast<int32_t*>(ws);
+  h->launches += 4;
+  MOE_TRY(cuda_status(moe::launch_route_hist(topk_idx, T, k, E, sub, h->ctl, st)));
+  MOE_TRY(cuda_status(moe::launch_route_scan(sub, moe::n_subchunks(T, k), E, counts, offsets, st)));
+  MOE_TRY(cuda_status(moe::launch_route_rank(topk_idx, T, k, E, sub, offsets, row_map, st)));
+  return cuda_status(moe::launch_permute_scatter(static_cast<const __nv_bfloat16*>(x), row_map,
+                                                 offsets, counts, T, d, k, E,
+                                                 static_cast<__nv_bfloat16*>(x_perm), st));
+}
+
+moe_status_t moe_grouped_swiglu_fwd(moe_handle_t h, const moe_shape_t* s, const void* x_perm,
+                                    const int32_t* offsets, const void* w_gu, const void* w_down,
+                                    void* au, void* hbuf, void* o_perm, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  (void)ws;
+  (void)ws_bytes;
+  if (s->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (!all_nonnull(x_perm, offsets, w_gu, w_down, au, hbuf, o_perm)) return MOE_ERR_INVALID_ARG;
+  for (const void* p : {x_perm, w_gu, w_down, static_cast<const void*>(au),
+                        static_cast<const void*>(hbuf), static_cast<const void*>(o_perm)})
+    if (!aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  const int d = s->d_model, f = s->d_ff, E = s->n_experts;
+  const int64_t m_cap = max_rows(s);
+  auto st = static_cast<cudaStream_t>(stream);
+  MOE_GUARD(h);
+  moe::GemmCtx c{h->num_sms, h->ctl};
+  h->launches += 2;
+  MOE_TRY(moe::gemm_fwd_gate_up(c, x_perm, offsets, w_gu, au, hbuf, E, d, f, m_cap, st));
+  return moe::gemm_fwd_down(c, hbuf, offsets, w_down, o_perm, E, d, f, m_cap, st);
+}
+
+moe_status_t moe_unpermute_combine(moe_handle_t h, const moe_shape_t* s, const void* o_perm,
+                                   const int32_t* row_map, const float* topk_w, void* y,
+                                   moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  if (!all_nonnull(o_perm, row_map, topk_w, y)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(o_perm, 16) || !aligned(y, 16)) return MOE_ERR_INVALID_ARG;
+  MOE_GUARD(h);
+  h->launches += 1;
+  return cuda_status(moe::launch_combine(static_cast<const __nv_bfloat16*>(o_perm), row_map, topk_w,
+                                         s->T, s->d_model, s->top_k,
+                                         static_cast<__nv_bfloat16*>(y),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_unpermute_combine_bwd(moe_handle_t h, const moe_shape_t* s, const void* dy,
+                                       const void* o_perm, const int32_t* row_map,
+                                       const float* topk_w, const int32_t* offsets,
+                                       const int32_t* counts, void* do_perm, float* d_topk_w,
+                                       moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  if (!all_nonnull(dy, o_perm, row_map, topk_w, offsets, counts, do_perm, d_topk_w))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(dy, 16) || !aligned(o_perm, 16) || !aligned(do_perm, 16)) return MOE_ERR_INVALID_ARG;
+  MOE_GUARD(h);
+  h->launches += 1;
+  return cuda_status(moe::launch_combine_bwd(
+      static_cast<const __nv_bfloat16*>(dy), static_cast<const __nv_bfloat16*>(o_perm), row_map,
+      topk_w, offsets, counts, s->T, s->d_model, s->top_k, s->n_experts,
+      static_cast<__nv_bfloat16*>(do_perm), d_topk_w, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_grouped_swiglu_bwd(moe_handle_t h, const moe_shape_t* s, const void* do_perm,
+                                    const void* x_perm, const void* au, const void* hbuf,
+                                    const int32_t* offsets, const void* w_gu, const void* w_down,
+                                    void* dau, void* dx_perm, void* dw_gu, void* dw_down, void* ws,
+                                    size_t ws_bytes, moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  (void)ws;
+  (void)ws_bytes;
+  if (s->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (!all_nonnull(do_perm, x_perm, au, hbuf, offsets, w_gu, w_down, dau, dx_perm, dw_gu, dw_down))
+    return MOE_ERR_INVALID_ARG;
+  for (const void* p : {do_perm, x_perm, au, hbuf, w_gu, w_down, static_cast<const void*>(dau),
+                        static_cast<const void*>(dx_perm), static_cast<const void*>(dw_gu),
+                        static_cast<const void*>(dw_down)})
+    if (!aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  const int d = s->d_model, f = s->d_ff, E = s->n_experts;
+  const int64_t m_cap = max_rows(s);
+  auto st = static_cast<cudaStream_t>(stream);
+  MOE_GUARD(h);
+  moe::GemmCtx c{h->num_sms, h->ctl};
+  h->launches += 4;
+  MOE_TRY(moe::gemm_dgrad_down_swiglu(c, do_perm, offsets, w_down, au, dau, E, d, f, m_cap, st));
+  MOE_TRY(moe::gemm_wgrad_down(c, do_perm, hbuf, offsets, dw_down, E, d, f, m_cap, st));
+  MOE_TRY(moe::gemm_dgrad_gate_up(c, dau, offsets, w_gu, dx_perm, E, d, f, m_cap, st));
+  return moe::gemm_wgrad_gate_up(c, dau, x_perm, offsets, dw_gu, E, d, f, m_cap, st);
+}
+
+moe_status_t moe_permute_bwd(moe_handle_t h, const moe_shape_t* s, const void* dx_perm,
+                             const int32_t* row_map, const float* dx_router, void* dx,
+                             moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  if (!all_nonnull(dx_perm, row_map, dx)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(dx_perm, 16) || !aligned(dx, 16) || !aligned(dx_router, 16))
+    return MOE_ERR_INVALID_ARG;
+  MOE_GUARD(h);
+  h->launches += 1;
+  return cuda_status(moe::launch_permute_bwd(static_cast<const __nv_bfloat16*>(dx_perm), row_map,
+                                             dx_router, s->T, s->d_model, s->top_k,
+                                             static_cast<__nv_bfloat16*>(dx),
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_router_topk_bwd(moe_handle_t h, const moe_shape_t* s, const float* d_topk_w,
+                                 const float* probs, const int32_t* topk_idx, const void* x,
+                                 const void* w_router, float* dx_router, void* dw_router,
+                                 float* dbias, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  MOE_TRY(check_router_shape(s));
+  if (!all_nonnull(d_topk_w, probs, topk_idx, x, w_router, dx_router, dw_router))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(dx_router, 16))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(h, s, ws, ws_bytes));
+  const int T = s->T, d = s->d_model, E = s->n_experts, k = s->top_k;
+  const bool renorm = (s->flags & MOE_FLAG_RENORM) != 0;
+  auto st = static_cast<cudaStream_t>(stream);
+  MOE_GUARD(h);
+  const RouterBwdWs L = router_bwd_layout(h, s);
+  auto* base = static_cast<uint8_t*>(ws);
+  auto* db_part = reinterpret_cast<float*>(base + L.db_part);
+  auto* part = reinterpret_cast<float*>(base + L.part);
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  const auto* wb = static_cast<const __nv_bfloat16*>(w_router);
+  h->launches += router_on_tensor_cores(E) ? 4 : 3;
+  if (dbias != nullptr) h->launches += 1;
+  if (!router_on_tensor_cores(E)) {
+    auto* dl = reinterpret_cast<float*>(base + L.dl);
+    MOE_TRY(cuda_status(moe::launch_router_bwd_dl(d_topk_w, probs, topk_idx, wb, T, d, E, k, renorm,
+                                                  true, dl, nullptr, dx_router, db_part, L.nblocks,
+                                                  h->ctl, st)));
+    MOE_TRY(cuda_status(moe::launch_router_dw_small(dl, xb, T, d, E, part, st)));
+  } else {
+    auto* dl = reinterpret_cast<__nv_bfloat16*>(base + L.dl);
+    MOE_TRY(cuda_status(moe::launch_router_bwd_dl(d_topk_w, probs, topk_idx, wb, T, d, E, k, renorm,
+                                                  false, nullptr, dl, nullptr, db_part, L.nblocks,
+                                                  h->ctl, st)));
+    moe::GemmCtx c{h->num_sms, h->ctl};
+    MOE_TRY(moe::gemm_router_dx(c, dl, w_router, dx_router, T, d, E, st));
+    MOE_TRY(moe::gemm_router_dw_partial(c, dl, x, part, T, d, E, L.n_part, L.group_len, st));
+  }
+  MOE_TRY(cuda_status(moe::launch_reduce_partials_bf16(part, L.n_part, static_cast<int64_t>(E) * d,
+                                                       static_cast<__nv_bfloat16*>(dw_router), st)));
+  if (dbias != nullptr)
+    MOE_TRY(cuda_status(moe::launch_reduce_rows_f32(db_part, L.nblocks, E, dbias, st)));
+  return MOE_OK;
+}
+
+moe_status_t moe_mxfp8_quantize(moe_handle_t h, const void* in, int64_t rows, int64_t cols,
+                                int axis, uint8_t* q, uint8_t* scales, moe_stream_t stream) {
+  if (h == nullptr || !all_nonnull(in, q, scales)) return MOE_ERR_INVALID_ARG;
+  if (rows < 1 || cols < 1 || (axis != 0 && axis != 1)) return MOE_ERR_INVALID_ARG;
+  if (axis == 1 && (cols % 32 != 0 || !aligned(in, 16) || !aligned(q, 16)))
+    return MOE_ERR_INVALID_ARG;
+  if (axis == 0 && (rows % 32 != 0 || cols % 2 != 0 || !aligned(in, 4) || !aligned(q, 2) ||
+                    !aligned(scales, 2)))
+    return MOE_ERR_INVALID_ARG;
+  MOE_GUARD(h);
+  h->launches += 1;
+  return cuda_status(moe::launch_mxfp8_quantize(static_cast<const __nv_bfloat16*>(in), rows, cols,
+                                                axis, q, scales, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_get_status(moe_handle_t h, int* device_status) {
+  if (h == nullptr || device_status == nullptr) return MOE_ERR_INVALID_ARG;
+  MOE_GUARD(h);
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  moe::DeviceCtl c{};
+  if (cudaMemcpy(&c, h->ctl, sizeof(c), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemset(h->ctl, 0, sizeof(c)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  *device_status = c.status;
+  return MOE_OK;
+}
+
+moe_status_t moe_get_launch_count(moe_handle_t h, uint64_t* launches) {
+  if (h == nullptr || launches == nullptr) return MOE_ERR_INVALID_ARG;
+  *launches = h->launches;
+  return MOE_OK;
+}
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MOE_ERR_DEVICE_CHECK: return "device-side index check failed";
+    case MOE_ERR_TIMEOUT: return "device-side bounded wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

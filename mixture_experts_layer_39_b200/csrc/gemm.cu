@@ -1,0 +1,282 @@
+// Host side of the tcgen05 grouped GEMMs: TMA descriptors and launches for
+// every contraction of the layer.
+//
+//   forward   gate/up : [M, d] x W_gu[e]^T  -> SwiGLU epilogue -> AU, H
+//             down    : [M, f] x W_d[e]^T   -> O
+//   backward  dgrad-down : dO x W_d[e]      -> SwiGLU-backward epilogue -> dAU
+//             dgrad-gu   : dAU x W_gu[e]    -> dX_perm
+//             wgrad-down : dO_e^T H_e       -> dW_d[e]   (contraction over e's rows)
+//             wgrad-gu   : dAU_e^T X_e      -> dW_gu[e]
+//   router    logits  : x W_r^T (E multiple of 128), dX_router = dL W_r,
+//             dW_r partials = dL^T x over token chunks
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "gemm.cuh"
+#include "tc_gemm.cuh"
+
+namespace moe {
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 map over a row-major [outer, inner] matrix.
+bool tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+             uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D bf16 map over [groups, outer, inner].
+bool tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t groups,
+             uint64_t row_bytes, uint64_t group_bytes, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {inner, outer, groups};
+  cuuint64_t strides[2] = {row_bytes, group_bytes};
+  cuuint32_t box[3] = {box_inner, box_outer, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP>
+moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const tc::GemmArgs& args, int grid,
+                    cudaStream_t st) {
+  constexpr int STAGES = BN == 256 ? 4 : 6;
+  auto kern = tc::grouped_gemm_kernel<BN, A_MN, B_MN, EPI, KGROUP, STAGES>;
+  const size_t smem = tc::SmemPlan<BN, STAGES>::bytes(args.n_groups);
+  static size_t configured = 0;  // largest size this instantiation was opened for
+  if (smem > configured) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    configured = smem;
+  }
+  if (grid <= 0) return MOE_OK;
+  kern<<<grid, tc::kThreads, smem, st>>>(a, b, args);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+tc::GemmArgs base_args(const GemmCtx& c) {
+  tc::GemmArgs a{};
+  a.ctl = c.ctl;
+  return a;
+}
+
+}  // namespace
+
+moe_status_t gemm_fwd_gate_up(const GemmCtx& c, const void* x_perm, const int32_t* offsets,
+                              const void* w_gu, void* au, void* h, int E, int d, int f,
+                              int64_t m_cap, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, x_perm, d, m_cap, 2ull * d, 64, 128)) return MOE_ERR_CUDA;
+  if (!tmap_3d(&tb, w_gu, d, 2ull * f, E, 2ull * d, 4ull * f * d, 64, 128)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  a.n_tiles_n = f / 128;
+  a.k_blocks = d / tc::BK;
+  a.n_groups = E;
+  a.offsets = offsets;
+  a.total_len = static_cast<int>(m_cap);
+  a.m_cap = m_cap;
+  a.out = au;
+  a.ldo = 2ll * f;
+  a.out2 = h;
+  a.ldo2 = f;
+  a.f = f;
+  return launch<256, false, false, tc::EPI_SWIGLU_FWD, false>(ta, tb, a, c.num_sms, st);
+}
+
+moe_status_t gemm_fwd_down(const GemmCtx& c, const void* h, const int32_t* offsets,
+                           const void* w_d, void* o_perm, int E, int d, int f, int64_t m_cap,
+                           cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, h, f, m_cap, 2ull * f, 64, 128)) return MOE_ERR_CUDA;
+  if (!tmap_3d(&tb, w_d, f, d, E, 2ull * f, 2ull * d * f, 64, 256)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  a.n_tiles_n = d / 256;
+  a.k_blocks = f / tc::BK;
+  a.n_groups = E;
+  a.offsets = offsets;
+  a.total_len = static_cast<int>(m_cap);
+  a.m_cap = m_cap;
+  a.out = o_perm;
+  a.ldo = d;
+  return launch<256, false, false, tc::EPI_BF16, false>(ta, tb, a, c.num_sms, st);
+}
+
+moe_status_t gemm_dgrad_down_swiglu(const GemmCtx& c, const void* do_perm, const int32_t* offsets,
+                                    const void* w_d, const void* au, void* dau, int E, int d,
+                                    int f, int64_t m_cap, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, do_perm, d, m_cap, 2ull * d, 64, 128)) return MOE_ERR_CUDA;
+  // W_d[e] is [d (contraction), f (output)]: N-major operand
+  if (!tmap_3d(&tb, w_d, f, d, E, 2ull * f, 2ull * d * f, 64, 64)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  a.n_tiles_n = f / 256;
+  a.k_blocks = d / tc::BK;
+  a.n_groups = E;
+  a.offsets = offsets;
+  a.total_len = static_cast<int>(m_cap);
+  a.m_cap = m_cap;
+  a.out = dau;
+  a.ldo = 2ll * f;
+  a.aux = static_cast<const __nv_bfloat16*>(au);
+  a.ld_aux = 2ll * f;
+  a.f = f;
+  return launch<256, false, true, tc::EPI_SWIGLU_BWD, false>(ta, tb, a, c.num_sms, st);
+}
+
+moe_status_t gemm_dgrad_gate_up(const GemmCtx& c, const void* dau, const int32_t* offsets,
+                                const void* w_gu, void* dx_perm, int E, int d, int f,
+                                int64_t m_cap, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, dau, 2ull * f, m_cap, 4ull * f, 64, 128)) return MOE_ERR_CUDA;
+  // W_gu[e] is [2f (contraction), d (output)]: N-major operand
+  if (!tmap_3d(&tb, w_gu, d, 2ull * f, E, 2ull * d, 4ull * f * d, 64, 64)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  a.n_tiles_n = d / 256;
+  a.k_blocks = 2 * f / tc::BK;
+  a.n_groups = E;
+  a.offsets = offsets;
+  a.total_len = static_cast<int>(m_cap);
+  a.m_cap = m_cap;
+  a.out = dx_perm;
+  a.ldo = d;
+  return launch<256, false, true, tc::EPI_BF16, false>(ta, tb, a, c.num_sms, st);
+}
+
+moe_status_t gemm_wgrad_down(const GemmCtx& c, const void* do_perm, const void* h,
+                             const int32_t* offsets, void* dw_d, int E, int d, int f,
+                             int64_t m_cap, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  // A = dO^T (M = d along the rows' contiguous axis), B = H (N = f)
+  if (!tmap_2d(&ta, do_perm, d, m_cap, 2ull * d, 64, 64)) return MOE_ERR_CUDA;
+  if (!tmap_3d(&tb, h, f, m_cap, 1, 2ull * f, 2ull * f * m_cap, 64, 64)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  a.n_tiles_n = f / 256;
+  a.m_tiles_fixed = d / tc::BM;
+  a.n_groups = E;
+  a.offsets = offsets;
+  a.total_len = static_cast<int>(m_cap);
+  a.out = dw_d;
+  a.ldo = f;
+  a.out_gstride = static_cast<int64_t>(d) * f;
+  const int64_t tiles = static_cast<int64_t>(E) * a.m_tiles_fixed * a.n_tiles_n;
+  const int grid = static_cast<int>(tiles < c.num_sms ? tiles : c.num_sms);
+  return launch<256, true, true, tc::EPI_BF16, true>(ta, tb, a, grid, st);
+}
+
+moe_status_t gemm_wgrad_gate_up(const GemmCtx& c, const void* dau, const void* x_perm,
+                                const int32_t* offsets, void* dw_gu, int E, int d, int f,
+                                int64_t m_cap, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, dau, 2ull * f, m_cap, 4ull * f, 64, 64)) return MOE_ERR_CUDA;
+  if (!tmap_3d(&tb, x_perm, d, m_cap, 1, 2ull * d, 2ull * d * m_cap, 64, 64)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  a.n_tiles_n = d / 256;
+  a.m_tiles_fixed = 2 * f / tc::BM;
+  a.n_groups = E;
+  a.offsets = offsets;
+  a.total_len = static_cast<int>(m_cap);
+  a.out = dw_gu;
+  a.ldo = d;
+  a.out_gstride = 2ll * f * d;
+  const int64_t tiles = static_cast<int64_t>(E) * a.m_tiles_fixed * a.n_tiles_n;
+  const int grid = static_cast<int>(tiles < c.num_sms ? tiles : c.num_sms);
+  return launch<256, true, true, tc::EPI_BF16, true>(ta, tb, a, grid, st);
+}
+
+moe_status_t gemm_router_logits(const GemmCtx& c, const void* x, const void* w_r, float* logits,
+                                int T, int d, int E, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, x, d, T, 2ull * d, 64, 128)) return MOE_ERR_CUDA;
+  if (!tmap_3d(&tb, w_r, d, E, 1, 2ull * d, 2ull * d * E, 64, 128)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  a.n_tiles_n = E / 128;
+  a.k_blocks = d / tc::BK;
+  a.n_groups = 1;
+  a.offsets = nullptr;
+  a.uniform_len = T;
+  a.total_len = T;
+  a.m_cap = T;
+  a.out = logits;
+  a.ldo = E;
+  const int64_t tiles = ceil_div64(T, tc::BM) * a.n_tiles_n;
+  const int grid = static_cast<int>(tiles < c.num_sms ? tiles : c.num_sms);
+  return launch<128, false, false, tc::EPI_F32, false>(ta, tb, a, grid, st);
+}
+
+moe_status_t gemm_router_dx(const GemmCtx& c, const void* dl_bf16, const void* w_r,
+                            float* dx_router, int T, int d, int E, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, dl_bf16, E, T, 2ull * E, 64, 128)) return MOE_ERR_CUDA;
+  if (!tmap_3d(&tb, w_r, d, E, 1, 2ull * d, 2ull * d * E, 64, 64)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  a.n_tiles_n = d / 256;
+  a.k_blocks = E / tc::BK;
+  a.n_groups = 1;
+  a.offsets = nullptr;
+  a.uniform_len = T;
+  a.total_len = T;
+  a.m_cap = T;
+  a.out = dx_router;
+  a.ldo = d;
+  const int64_t tiles = ceil_div64(T, tc::BM) * a.n_tiles_n;
+  const int grid = static_cast<int>(tiles < c.num_sms ? tiles : c.num_sms);
+  return launch<256, false, true, tc::EPI_F32, false>(ta, tb, a, grid, st);
+}
+
+int router_dw_groups(int num_sms, int T, int d, int E, int* group_len) {
+  const int tiles_per_group = (E / tc::BM) * (d / 256);
+  int g = num_sms / (tiles_per_group > 0 ? tiles_per_group : 1);
+  if (g < 1) g = 1;
+  int64_t len = ceil_div64(ceil_div64(T, g), 64) * 64;
+  g = static_cast<int>(ceil_div64(T, len));
+  *group_len = static_cast<int>(len);
+  return g;
+}
+
+moe_status_t gemm_router_dw_partial(const GemmCtx& c, const void* dl_bf16, const void* x,
+                                    float* partial, int T, int d, int E, int n_groups,
+                                    int group_len, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, dl_bf16, E, T, 2ull * E, 64, 64)) return MOE_ERR_CUDA;
+  if (!tmap_3d(&tb, x, d, T, 1, 2ull * d, 2ull * d * T, 64, 64)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  a.n_tiles_n = d / 256;
+  a.m_tiles_fixed = E / tc::BM;
+  a.n_groups = n_groups;
+  a.offsets = nullptr;
+  a.uniform_len = group_len;
+  a.total_len = T;
+  a.out = partial;
+  a.ldo = d;
+  a.out_gstride = static_cast<int64_t>(E) * d;
+  const int64_t tiles = static_cast<int64_t>(n_groups) * a.m_tiles_fixed * a.n_tiles_n;
+  const int grid = static_cast<int>(tiles < c.num_sms ? tiles : c.num_sms);
+  return launch<256, true, true, tc::EPI_F32, true>(ta, tb, a, grid, st);
+}
+
+}  // namespace moe

@@ -1,0 +1,40 @@
+// Host launchers of the tcgen05 grouped GEMMs (implemented in gemm.cu).
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+struct GemmCtx {
+  int num_sms;
+  DeviceCtl* ctl;
+};
+
+moe_status_t gemm_fwd_gate_up(const GemmCtx& c, const void* x_perm, const int32_t* offsets,
+                              const void* w_gu, void* au, void* h, int E, int d, int f,
+                              int64_t m_cap, cudaStream_t st);
+moe_status_t gemm_fwd_down(const GemmCtx& c, const void* h, const int32_t* offsets,
+                           const void* w_d, void* o_perm, int E, int d, int f, int64_t m_cap,
+                           cudaStream_t st);
+moe_status_t gemm_dgrad_down_swiglu(const GemmCtx& c, const void* do_perm, const int32_t* offsets,
+                                    const void* w_d, const void* au, void* dau, int E, int d,
+                                    int f, int64_t m_cap, cudaStream_t st);
+moe_status_t gemm_dgrad_gate_up(const GemmCtx& c, const void* dau, const int32_t* offsets,
+                                const void* w_gu, void* dx_perm, int E, int d, int f,
+                                int64_t m_cap, cudaStream_t st);
+moe_status_t gemm_wgrad_down(const GemmCtx& c, const void* do_perm, const void* h,
+                             const int32_t* offsets, void* dw_d, int E, int d, int f,
+                             int64_t m_cap, cudaStream_t st);
+moe_status_t gemm_wgrad_gate_up(const GemmCtx& c, const void* dau, const void* x_perm,
+                                const int32_t* offsets, void* dw_gu, int E, int d, int f,
+                                int64_t m_cap, cudaStream_t st);
+moe_status_t gemm_router_logits(const GemmCtx& c, const void* x, const void* w_r, float* logits,
+                                int T, int d, int E, cudaStream_t st);
+moe_status_t gemm_router_dx(const GemmCtx& c, const void* dl_bf16, const void* w_r,
+                            float* dx_router, int T, int d, int E, cudaStream_t st);
+int router_dw_groups(int num_sms, int T, int d, int E, int* group_len);
+moe_status_t gemm_router_dw_partial(const GemmCtx& c, const void* dl_bf16, const void* x,
+                                    float* partial, int T, int d, int E, int n_groups,
+                                    int group_len, cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,65 @@
+// Declarations of the memory-bound kernels' host launchers (router,
+// routing metadata, permute, combine and their backwards, MXFP8 quantise).
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// Sub-chunk of flat (token, slot) entries handled by one warp in the
+// routing histogram / rank kernels.
+constexpr int kSubChunk = 256;
+
+inline int64_t n_subchunks(int T, int k) { return ceil_div64(static_cast<int64_t>(T) * k, kSubChunk); }
+
+// ---- router forward
+cudaError_t launch_router_fused(const __nv_bfloat16* x, const __nv_bfloat16* w_r, const float* bias,
+                                const int32_t* route_in, int T, int d, int E, int k, bool renorm,
+                                int32_t* idx, float* w, float* probs, float* logits,
+                                DeviceCtl* ctl, cudaStream_t st);
+cudaError_t launch_softmax_topk(const float* logits_in, const float* bias, const int32_t* route_in,
+                                int T, int E, int k, bool renorm, int32_t* idx, float* w,
+                                float* probs, float* logits_out, DeviceCtl* ctl, cudaStream_t st);
+
+// ---- routing metadata + permute
+cudaError_t launch_route_hist(const int32_t* idx, int T, int k, int E, int32_t* sub_counts,
+                              DeviceCtl* ctl, cudaStream_t st);
+cudaError_t launch_route_scan(int32_t* sub_counts, int64_t n_sub, int E, int32_t* counts,
+                              int32_t* offsets, cudaStream_t st);
+cudaError_t launch_route_rank(const int32_t* idx, int T, int k, int E, const int32_t* sub_base,
+                              const int32_t* offsets, int32_t* row_map, cudaStream_t st);
+cudaError_t launch_permute_scatter(const __nv_bfloat16* x, const int32_t* row_map,
+                                   const int32_t* offsets, const int32_t* counts, int T, int d,
+                                   int k, int E, __nv_bfloat16* x_perm, cudaStream_t st);
+
+// ---- combine and backwards
+cudaError_t launch_combine(const __nv_bfloat16* o_perm, const int32_t* row_map, const float* w,
+                           int T, int d, int k, __nv_bfloat16* y, cudaStream_t st);
+cudaError_t launch_combine_bwd(const __nv_bfloat16* dy, const __nv_bfloat16* o_perm,
+                               const int32_t* row_map, const float* w, const int32_t* offsets,
+                               const int32_t* counts, int T, int d, int k, int E,
+                               __nv_bfloat16* do_perm, float* dw, cudaStream_t st);
+cudaError_t launch_permute_bwd(const __nv_bfloat16* dx_perm, const int32_t* row_map,
+                               const float* dx_router, int T, int d, int k, __nv_bfloat16* dx,
+                               cudaStream_t st);
+
+// ---- router backward
+int router_bwd_blocks(int num_sms);
+cudaError_t launch_router_bwd_dl(const float* dw, const float* probs, const int32_t* idx,
+                                 const __nv_bfloat16* w_r, int T, int d, int E, int k, bool renorm,
+                                 bool fuse_dx, float* dl_f32, __nv_bfloat16* dl_bf16,
+                                 float* dx_router, float* db_partial, int nblocks,
+                                 DeviceCtl* ctl, cudaStream_t st);
+int router_dw_small_chunk();
+cudaError_t launch_router_dw_small(const float* dl, const __nv_bfloat16* x, int T, int d, int E,
+                                   float* partial, cudaStream_t st);
+cudaError_t launch_reduce_partials_bf16(const float* partial, int n_part, int64_t n,
+                                        __nv_bfloat16* out, cudaStream_t st);
+cudaError_t launch_reduce_rows_f32(const float* partial, int n_part, int E, float* out,
+                                   cudaStream_t st);
+
+// ---- MXFP8
+cudaError_t launch_mxfp8_quantize(const __nv_bfloat16* in, int64_t rows, int64_t cols, int axis,
+                                  uint8_t* q, uint8_t* scales, cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,381 @@
+// Routing metadata, rowwise permute, combine and their backwards.
+//
+// "Routing metadata stays on the GPU, so the host never waits for a copy
+// back" and "routed data is written straight into the expert's input
+// buffer" -- Olmo-core 3 introduction page, section 2 (GPU-resident routing,
+// rowwise expert parallelism).  "The routing result becomes a permutation
+// index; tokens are regrouped per expert, processed, then restored to their
+// original order" -- discosf.com article, section 2.1.
+//
+// Metadata is computed in three deterministic steps so that the row of every
+// (token, slot) entry is exactly the stable expert-major order:
+//   hist : each warp counts the experts of one 256-entry sub-chunk;
+//   scan : per expert, an exclusive scan over sub-chunks (the base of each
+//          sub-chunk) and the padded segment offsets;
+//   rank : each warp walks its sub-chunk in order, 32 entries at a time; the
+//          rank of an entry among equal experts in a batch comes from
+//          __match_any_sync, and the per-expert running base advances by the
+//          batch's count.
+#include "kernels.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kWarps = 8;
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+__global__ void __launch_bounds__(kWarps * 32)
+    route_hist_kernel(const int32_t* __restrict__ idx, int64_t n_entries, int E, int64_t n_sub,
+                      int32_t* __restrict__ sub_counts, DeviceCtl* ctl) {
+  extern __shared__ int s_cnt[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* cnt = s_cnt + warp * E;
+  for (int e = lane; e < E; e += 32) cnt[e] = 0;
+  __syncwarp();
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+  if (c >= n_sub) return;
+  const int64_t beg = c * kSubChunk;
+  const int64_t end = beg + kSubChunk < n_entries ? beg + kSubChunk : n_entries;
+  for (int64_t i = beg + lane; i < end; i += 32) {
+    const int e = __ldg(idx + i);
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+    else report(ctl, MOE_ERR_DEVICE_CHECK, 200);
+  }
+  __syncwarp();
+  for (int e = lane; e < E; e += 32) sub_counts[c * E + e] = cnt[e];
+}
+
+// One block; thread e scans expert e over the sub-chunks, then the block
+// scans the padded counts into segment offsets.
+__global__ void __launch_bounds__(1024)
+    route_scan_kernel(int32_t* __restrict__ sub, int64_t n_sub, int E, int32_t* __restrict__ counts,
+                      int32_t* __restrict__ offsets) {
+  __shared__ int s_warp[32];
+  const int e = threadIdx.x;
+  int run = 0;
+  if (e < E) {
+    int64_t c = 0;
+    for (; c + 4 <= n_sub; c += 4) {
+      const int v0 = sub[(c + 0) * E + e], v1 = sub[(c + 1) * E + e];
+      const int v2 = sub[(c + 2) * E + e], v3 = sub[(c + 3) * E + e];
+      sub[(c + 0) * E + e] = run;
+      sub[(c + 1) * E + e] = run + v0;
+      sub[(c + 2) * E + e] = run + v0 + v1;
+      sub[(c + 3) * E + e] = run + v0 + v1 + v2;
+      run += v0 + v1 + v2 + v3;
+    }
+    for (; c < n_sub; ++c) {
+      const int v = sub[c * E + e];
+      sub[c * E + e] = run;
+      run += v;
+    }
+    counts[e] = run;
+  }
+  const int padded = e < E ? (run + kSegAlign - 1) / kSegAlign * kSegAlign : 0;
+  // block exclusive scan of `padded`
+  const int lane = e & 31, warp = e >> 5;
+  int v = padded;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  if (lane == 31) s_warp[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int w = s_warp[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += u;
+    }
+    s_warp[lane] = w;
+  }
+  __syncthreads();
+  const int incl = v + (warp > 0 ? s_warp[warp - 1] : 0);
+  if (e < E) offsets[e] = incl - padded;
+  if (e == E - 1) offsets[E] = incl;
+}
+
+__global__ void __launch_bounds__(kWarps * 32)
+    route_rank_kernel(const int32_t* __restrict__ idx, int64_t n_entries, int E, int64_t n_sub,
+                      const int32_t* __restrict__ sub_base, const int32_t* __restrict__ offsets,
+                      int32_t* __restrict__ row_map) {
+  extern __shared__ int s_base_all[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* base = s_base_all + warp * E;
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+  if (c >= n_sub) return;
+  for (int e = lane; e < E; e += 32) base[e] = __ldg(offsets + e) + sub_base[c * E + e];
+  __syncwarp();
+  const int64_t beg = c * kSubChunk;
+  const int64_t end = beg + kSubChunk < n_entries ? beg + kSubChunk : n_entries;
+  for (int64_t i0 = beg; i0 < end; i0 += 32) {
+    const int64_t i = i0 + lane;
+    const bool valid = i < end;
+    const int e = valid ? __ldg(idx + i) : -1;
+    const bool good = valid && e >= 0 && e < E;
+    const int key = good ? e : -1 - lane;  // lanes without an expert match only themselves
+    const uint32_t peers = __match_any_sync(0xffffffffu, key);
+    int row = -1;
+    if (good) row = base[e] + __popc(peers & lanemask_lt());
+    __syncwarp();
+    if (good && (peers & lanemask_lt()) == 0) base[e] += __popc(peers);
+    __syncwarp();
+    if (valid) row_map[i] = row;
+  }
+}
+
+// Warps [0, T): token t, reads x[t] once and writes its k rows.
+// Warps [T, T+E): expert e, zero-fills the pad rows of its segment.
+__global__ void __launch_bounds__(kWarps * 32)
+    permute_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ row_map,
+                           const int32_t* __restrict__ offsets, const int32_t* __restrict__ counts,
+                           int T, int nvec, int k, int E, uint4* __restrict__ x_perm) {
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+  if (gw < T) {
+    int rows[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) rows[j] = j < k ? __ldg(row_map + gw * k + j) : -1;
+    const uint4* src = x + gw * nvec;
+    for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
+      uint4 val[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (v0 + 32 * u < nvec) val[u] = __ldg(src + v0 + 32 * u);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (rows[j] < 0) continue;
+        uint4* dst = x_perm + static_cast<int64_t>(rows[j]) * nvec;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = val[u];
+      }
+    }
+  } else if (gw < static_cast<int64_t>(T) + E) {
+    const int e = static_cast<int>(gw - T);
+    const int64_t r0 = static_cast<int64_t>(__ldg(offsets + e)) + __ldg(counts + e);
+    const int64_t r1 = __ldg(offsets + e + 1);
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (int64_t r = r0; r < r1; ++r)
+      for (int v = lane; v < nvec; v += 32) x_perm[r * nvec + v] = z;
+  }
+}
+
+__device__ __forceinline__ void unpack8(const uint4& q, float* f) {
+  f[0] = bf16_lo(q.x); f[1] = bf16_hi(q.x);
+  f[2] = bf16_lo(q.y); f[3] = bf16_hi(q.y);
+  f[4] = bf16_lo(q.z); f[5] = bf16_hi(q.z);
+  f[6] = bf16_lo(q.w); f[7] = bf16_hi(q.w);
+}
+
+__device__ __forceinline__ uint4 pack8(const float* f) {
+  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                    pack_bf16x2(f[6], f[7]));
+}
+
+// y[t] = bf16(sum_j w[t,j] * O[row_map[t,j]]), fp32 in slot order.
+__global__ void __launch_bounds__(kWarps * 32)
+    combine_kernel(const uint4* __restrict__ o, const int32_t* __restrict__ row_map,
+                   const float* __restrict__ w, int T, int nvec, int k, uint4* __restrict__ y) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+  if (t >= T) return;
+  int rows[8];
+  float wt[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    rows[j] = j < k ? __ldg(row_map + t * k + j) : -1;
+    wt[j] = j < k ? __ldg(w + t * k + j) : 0.f;
+  }
+  for (int v0 = lane; v0 < nvec; v0 += 64) {
+    float acc[2][8];
+    uint4 q[2][8];
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (rows[j] >= 0 && v0 + 32 * u < nvec)
+          q[u][j] = __ldg(o + static_cast<int64_t>(rows[j]) * nvec + v0 + 32 * u);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[u][c] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (rows[j] < 0) continue;
+        float f[8];
+        unpack8(q[u][j], f);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[u][c] = fmaf(wt[j], f[c], acc[u][c]);
+      }
+      if (v0 + 32 * u < nvec) y[t * nvec + v0 + 32 * u] = pack8(acc[u]);
+    }
+  }
+}
+
+// dO[row_map[t,j]] = bf16(w * dY[t]); dw[t,j] = <dY[t], O[row_map[t,j]]>;
+// warps past T zero the pad rows of dO.
+__global__ void __launch_bounds__(kWarps * 32)
+    combine_bwd_kernel(const uint4* __restrict__ dy, const uint4* __restrict__ o,
+                       const int32_t* __restrict__ row_map, const float* __restrict__ w,
+                       const int32_t* __restrict__ offsets, const int32_t* __restrict__ counts,
+                       int T, int nvec, int k, int E, uint4* __restrict__ dO,
+                       float* __restrict__ dw) {
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+  if (gw < T) {
+    const int64_t t = gw;
+    int rows[8];
+    float wt[8], part[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      rows[j] = j < k ? __ldg(row_map + t * k + j) : -1;
+      wt[j] = j < k ? __ldg(w + t * k + j) : 0.f;
+      part[j] = 0.f;
+    }
+    for (int v = lane; v < nvec; v += 32) {
+      float g[8];
+      unpack8(__ldg(dy + t * nvec + v), g);
+      uint4 q[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (rows[j] >= 0) q[j] = __ldg(o + static_cast<int64_t>(rows[j]) * nvec + v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (rows[j] < 0) continue;
+        float f[8], s[8];
+        unpack8(q[j], f);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          part[j] = fmaf(g[c], f[c], part[j]);
+          s[c] = wt[j] * g[c];
+        }
+        dO[static_cast<int64_t>(rows[j]) * nvec + v] = pack8(s);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j >= k) break;
+      const float r = warp_sum(part[j]);
+      if (lane == 0) dw[t * k + j] = r;
+    }
+  } else if (gw < static_cast<int64_t>(T) + E) {
+    const int e = static_cast<int>(gw - T);
+    const int64_t r0 = static_cast<int64_t>(__ldg(offsets + e)) + __ldg(counts + e);
+    const int64_t r1 = __ldg(offsets + e + 1);
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (int64_t r = r0; r < r1; ++r)
+      for (int v = lane; v < nvec; v += 32) dO[r * nvec + v] = z;
+  }
+}
+
+// dX[t] = bf16(sum_j dX_perm[row_map[t,j]] + dX_router[t]), fp32, rounded once.
+__global__ void __launch_bounds__(kWarps * 32)
+    permute_bwd_kernel(const uint4* __restrict__ dxp, const int32_t* __restrict__ row_map,
+                       const float4* __restrict__ dxr, int T, int nvec, int k,
+                       uint4* __restrict__ dx) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+  if (t >= T) return;
+  int rows[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) rows[j] = j < k ? __ldg(row_map + t * k + j) : -1;
+  for (int v = lane; v < nvec; v += 32) {
+    uint4 q[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (rows[j] >= 0) q[j] = __ldg(dxp + static_cast<int64_t>(rows[j]) * nvec + v);
+    float acc[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (rows[j] < 0) continue;
+      float f[8];
+      unpack8(q[j], f);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] += f[c];
+    }
+    if (dxr != nullptr) {
+      const float4 a = __ldg(dxr + (t * nvec + v) * 2);
+      const float4 b = __ldg(dxr + (t * nvec + v) * 2 + 1);
+      acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+      acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    }
+    dx[t * nvec + v] = pack8(acc);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_route_hist(const int32_t* idx, int T, int k, int E, int32_t* sub_counts,
+                              DeviceCtl* ctl, cudaStream_t st) {
+  const int64_t n_sub = n_subchunks(T, k);
+  const unsigned grid = static_cast<unsigned>(ceil_div64(n_sub, kWarps));
+  route_hist_kernel<<<grid, kWarps * 32, kWarps * E * sizeof(int), st>>>(
+      idx, static_cast<int64_t>(T) * k, E, n_sub, sub_counts, ctl);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_scan(int32_t* sub_counts, int64_t n_sub, int E, int32_t* counts,
+                              int32_t* offsets, cudaStream_t st) {
+  route_scan_kernel<<<1, 1024, 0, st>>>(sub_counts, n_sub, E, counts, offsets);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_rank(const int32_t* idx, int T, int k, int E, const int32_t* sub_base,
+                              const int32_t* offsets, int32_t* row_map, cudaStream_t st) {
+  const int64_t n_sub = n_subchunks(T, k);
+  const unsigned grid = static_cast<unsigned>(ceil_div64(n_sub, kWarps));
+  route_rank_kernel<<<grid, kWarps * 32, kWarps * E * sizeof(int), st>>>(
+      idx, static_cast<int64_t>(T) * k, E, n_sub, sub_base, offsets, row_map);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_scatter(const __nv_bfloat16* x, const int32_t* row_map,
+                                   const int32_t* offsets, const int32_t* counts, int T, int d,
+                                   int k, int E, __nv_bfloat16* x_perm, cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>(ceil_div64(static_cast<int64_t>(T) + E, kWarps));
+  permute_scatter_kernel<<<grid, kWarps * 32, 0, st>>>(
+      reinterpret_cast<const uint4*>(x), row_map, offsets, counts, T, d / 8, k, E,
+      reinterpret_cast<uint4*>(x_perm));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const __nv_bfloat16* o_perm, const int32_t* row_map, const float* w,
+                           int T, int d, int k, __nv_bfloat16* y, cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>(ceil_div64(T, kWarps));
+  combine_kernel<<<grid, kWarps * 32, 0, st>>>(reinterpret_cast<const uint4*>(o_perm), row_map, w,
+                                               T, d / 8, k, reinterpret_cast<uint4*>(y));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_bwd(const __nv_bfloat16* dy, const __nv_bfloat16* o_perm,
+                               const int32_t* row_map, const float* w, const int32_t* offsets,
+                               const int32_t* counts, int T, int d, int k, int E,
+                               __nv_bfloat16* do_perm, float* dw, cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>(ceil_div64(static_cast<int64_t>(T) + E, kWarps));
+  combine_bwd_kernel<<<grid, kWarps * 32, 0, st>>>(
+      reinterpret_cast<const uint4*>(dy), reinterpret_cast<const uint4*>(o_perm), row_map, w,
+      offsets, counts, T, d / 8, k, E, reinterpret_cast<uint4*>(do_perm), dw);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_bwd(const __nv_bfloat16* dx_perm, const int32_t* row_map,
+                               const float* dx_router, int T, int d, int k, __nv_bfloat16* dx,
+                               cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>(ceil_div64(T, kWarps));
+  permute_bwd_kernel<<<grid, kWarps * 32, 0, st>>>(
+      reinterpret_cast<const uint4*>(dx_perm), row_map, reinterpret_cast<const float4*>(dx_router),
+      T, d / 8, k, reinterpret_cast<uint4*>(dx));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

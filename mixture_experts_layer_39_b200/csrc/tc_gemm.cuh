@@ -1,0 +1,599 @@
+// Persistent grouped GEMM on the 5th-generation tensor cores (tcgen05 + TMEM),
+// fed by TMA, for sm_100a.
+//
+// "Grouped GEMM: merge the many small expert GEMMs into one launch so the
+// GPU stays busy" and "device-scheduled grouped GEMM" -- Olmo-core 3
+// introduction page, section 2 (three routing optimisations).  Here the
+// schedule is decoded on the device from the expert offsets, so routing
+// never forces a device-to-host copy.
+//
+// One CTA per SM, 6 warps:
+//   warp 0      TMA producer (one lane): A/B tiles into a STAGES-deep ring
+//   warp 1      MMA issuer (one lane): tcgen05.mma 128 x BN x 16, fp32 in TMEM;
+//               also owns the TMEM allocation
+//   warps 2..5  epilogue: tcgen05.ld from TMEM -> registers -> global
+// Two TMEM accumulators (2 x BN columns) let the epilogue of tile i overlap
+// the main loop of tile i+1.
+//
+// Two grouping modes:
+//   M-grouped (KGROUP=false): rows of A are split in groups (experts); group
+//     g owns rows [off(g), off(g+1)) and multiplies B[g].  Tiles are 128-row
+//     slices of a group; rows past off(g+1) are masked at the store.
+//   K-grouped (KGROUP=true, weight gradients): group g owns the contraction
+//     range [off(g), off(g+1)) and writes its own output matrix g.  A group
+//     with an empty range writes zeros.
+//
+// Operand layouts in shared memory are the canonical 128-byte-swizzled
+// UMMA layouts: K-major = rows of 64 bf16 along K (TMA box {64, rows});
+// MN-major = 64-element chunks along M/N, one 128-byte row per K index (TMA
+// box {64, 64}), chunks 8 KB apart.
+//
+// Every mbarrier wait is bounded (kWaitLimitNs, globaltimer); on expiry the
+// CTA records MOE_ERR_TIMEOUT, drains its own TMA copies and MMAs, frees
+// TMEM and returns.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace moe {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BK = 64;  // bf16 elements per smem row: 128 bytes = one swizzle row
+constexpr int kThreads = 192;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+enum Epi : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_SWIGLU_FWD = 2, EPI_SWIGLU_BWD = 3 };
+
+struct GemmArgs {
+  int n_tiles_n;     // tiles along N per (group, m-tile)
+  int k_blocks;      // M-grouped: contraction length / BK
+  int n_groups;
+  const int* offsets;  // [n_groups + 1] on the device, or nullptr: uniform groups
+  int uniform_len;     // group length when offsets == nullptr
+  int total_len;       // clamp of all group boundaries (rows of the grouped operand)
+  int m_tiles_fixed;   // K-grouped: M / BM
+  int64_t m_cap;       // M-grouped: rows of the output buffer (store bound)
+  void* out;
+  int64_t ldo;
+  int64_t out_gstride;  // K-grouped: elements between group outputs
+  void* out2;           // SwiGLU forward: H
+  int64_t ldo2;
+  const __nv_bfloat16* aux;  // SwiGLU backward: saved [A | U]
+  int64_t ld_aux;
+  int f;  // SwiGLU: width of one half ([A | U] column offset of U)
+  DeviceCtl* ctl;
+};
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: true when the phase completed; false when another role
+// aborted or the time limit passed (then the abort flag is raised).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          bool honour_abort = true) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (honour_abort && *abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (layout code 2),
+// descriptor version 1 at bits 46-47; addresses and offsets in 16-byte units.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
+                                                    uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+// Instruction descriptor of kind::f16 with bf16 inputs and fp32 accumulate.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4)                       // D format fp32
+         | (1u << 7)                     // A format bf16
+         | (1u << 10)                    // B format bf16
+         | ((a_mn ? 1u : 0u) << 15)      // A major
+         | ((b_mn ? 1u : 0u) << 16)      // B major
+         | ((uint32_t)(N >> 3) << 17)    // N / 8
+         | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+// 32 lanes x 32 consecutive fp32 columns of TMEM.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- scheduling
+struct Tile {
+  int group;
+  int row0;     // M-grouped: first row of the tile; K-grouped: first row of M
+  int row_end;  // M-grouped: end of the group's rows (store mask)
+  int n_tile;
+  int k_lo;     // K-grouped: first contraction row
+  int k_blocks;
+  int last_k16;  // MMAs of K=16 in the last k-block (1..4)
+};
+
+__device__ __forceinline__ int group_off(const GemmArgs& a, int g) {
+  int v;
+  if (a.offsets != nullptr) {
+    v = __ldg(a.offsets + g);
+  } else {
+    long long u = static_cast<long long>(g) * a.uniform_len;
+    v = static_cast<int>(u < a.total_len ? u : a.total_len);
+  }
+  v = v < 0 ? 0 : v;
+  return v > a.total_len ? a.total_len : v;
+}
+
+template <bool KGROUP>
+__device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* s_tile_start, int t) {
+  Tile tl;
+  if constexpr (!KGROUP) {
+    const int mt = t / a.n_tiles_n;
+    tl.n_tile = t - mt * a.n_tiles_n;
+    int lo = 0, hi = a.n_groups - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_tile_start[mid] <= mt) lo = mid; else hi = mid - 1;
+    }
+    tl.group = lo;
+    const int g0 = group_off(a, lo), g1 = group_off(a, lo + 1);
+    tl.row0 = g0 + (mt - s_tile_start[lo]) * BM;
+    tl.row_end = g1 > g0 ? g1 : g0;
+    tl.k_lo = 0;
+    tl.k_blocks = a.k_blocks;
+    tl.last_k16 = 4;
+  } else {
+    const int per = a.m_tiles_fixed * a.n_tiles_n;
+    tl.group = t / per;
+    const int r = t - tl.group * per;
+    const int mt = r / a.n_tiles_n;
+    tl.n_tile = r - mt * a.n_tiles_n;
+    tl.row0 = mt * BM;
+    tl.row_end = 0;
+    const int g0 = group_off(a, tl.group), g1 = group_off(a, tl.group + 1);
+    const int len = g1 > g0 ? g1 - g0 : 0;
+    tl.k_lo = g0;
+    tl.k_blocks = (len + BK - 1) / BK;
+    const int rem = len - (tl.k_blocks - 1) * BK;
+    tl.last_k16 = tl.k_blocks > 0 ? (rem + 15) / 16 : 0;
+  }
+  return tl;
+}
+
+// ---------------------------------------------------------------- epilogue helpers
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d4[q] = w;
+  }
+}
+
+__device__ __forceinline__ void store_f32x32(float* dst, const float* v) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float* v) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 w = __ldg(s4 + q);
+    v[8 * q + 0] = bf16_lo(w.x); v[8 * q + 1] = bf16_hi(w.x);
+    v[8 * q + 2] = bf16_lo(w.y); v[8 * q + 3] = bf16_hi(w.y);
+    v[8 * q + 4] = bf16_lo(w.z); v[8 * q + 5] = bf16_hi(w.z);
+    v[8 * q + 6] = bf16_lo(w.w); v[8 * q + 7] = bf16_hi(w.w);
+  }
+}
+
+// ---------------------------------------------------------------- the kernel
+template <int BN, int STAGES>
+struct SmemPlan {
+  static constexpr int kABytes = BM * BK * 2;
+  static constexpr int kBBytes = BN * BK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kBarOff = STAGES * kStageBytes;                 // 1024-aligned stages
+  static constexpr int kBarBytes = (2 * STAGES + 5) * 8;               // full, empty, tfull x2, tempty x2, drain
+  static constexpr int kMiscOff = kBarOff + kBarBytes;                 // tmem base, abort flag
+  static constexpr int kTileOff = kMiscOff + 16;                       // group tile starts
+  static constexpr int bytes(int n_groups) { return 1024 + kTileOff + 4 * (n_groups + 1); }
+};
+
+template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+  static_assert(BN == 128 || BN == 256, "BN");
+  static_assert(!(EPI == EPI_SWIGLU_FWD && B_MN), "SwiGLU forward takes K-major weights");
+  using Plan = SmemPlan<BN, STAGES>;
+  constexpr uint32_t kTmemCols = 2 * BN;
+  constexpr uint32_t kIdesc = idesc_bf16(BM, BN, A_MN, B_MN);
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Plan::kBarOff);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + Plan::kMiscOff);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + Plan::kMiscOff + 4);
+  int* s_tile_start = reinterpret_cast<int*>(smem + Plan::kTileOff);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t smem_base = smem_u32(smem);
+  auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
+  auto empty_bar = [&](int s) { return smem_u32(&bars[STAGES + s]); };
+  auto tfull_bar = [&](int b) { return smem_u32(&bars[2 * STAGES + b]); };
+  auto tempty_bar = [&](int b) { return smem_u32(&bars[2 * STAGES + 2 + b]); };
+  const uint32_t drain_bar = smem_u32(&bars[2 * STAGES + 4]);
+
+  // ---- set-up: barriers, TMEM, group tile starts
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(s_tmem)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  int total_tiles;
+  if constexpr (!KGROUP) {
+    // tiles per group, then an exclusive scan by warp 2
+    for (int g = threadIdx.x; g < args.n_groups; g += kThreads) {
+      const int len = group_off(args, g + 1) - group_off(args, g);
+      s_tile_start[g + 1] = len > 0 ? (len + BM - 1) / BM : 0;
+    }
+    __syncthreads();
+    if (warp == 2) {
+      int carry = 0;
+      for (int base = 0; base < args.n_groups; base += 32) {
+        const int g = base + lane;
+        int v = g < args.n_groups ? s_tile_start[g + 1] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v += u;
+        }
+        if (g < args.n_groups) s_tile_start[g + 1] = carry + v;
+        carry += __shfl_sync(0xffffffffu, v, 31);
+      }
+      if (lane == 0) s_tile_start[0] = 0;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  if constexpr (!KGROUP) {
+    total_tiles = s_tile_start[args.n_groups] * args.n_tiles_n;
+  } else {
+    total_tiles = args.n_groups * args.m_tiles_fixed * args.n_tiles_n;
+  }
+
+  if (warp == 0) {
+    // ================================================================ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_parity = 0;  // per-stage: a load is in flight / its phase
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        const Tile tl = decode_tile<KGROUP>(args, s_tile_start, t);
+        for (int kb = 0; kb < tl.k_blocks; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, s_abort)) { ok = false; break; }
+          const uint32_t sa = smem_base + stage * Plan::kStageBytes;
+          const uint32_t sb = sa + Plan::kABytes;
+          const uint32_t fb = full_bar(stage);
+          mbar_arrive_expect_tx(fb, Plan::kStageBytes);
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          if constexpr (!KGROUP) {
+            const int k0 = kb * BK;
+            // A: K-major rows of the group's slice
+            tma_load_2d(sa, &tmA, fb, k0, tl.row0);
+            if constexpr (EPI == EPI_SWIGLU_FWD) {
+              const int nh = tl.n_tile * (BN / 2);
+              tma_load_3d(sb, &tmB, fb, k0, nh, tl.group);
+              tma_load_3d(sb + (BN / 2) * BK * 2, &tmB, fb, k0, args.f + nh, tl.group);
+            } else if constexpr (!B_MN) {
+              tma_load_3d(sb, &tmB, fb, k0, tl.n_tile * BN, tl.group);
+            } else {
+#pragma unroll
+              for (int j = 0; j < BN / 64; ++j)
+                tma_load_3d(sb + j * (64 * BK * 2), &tmB, fb, tl.n_tile * BN + 64 * j, k0,
+                            tl.group);
+            }
+          } else {
+            const int kr = tl.k_lo + kb * BK;
+#pragma unroll
+            for (int j = 0; j < BM / 64; ++j)
+              tma_load_2d(sa + j * (64 * BK * 2), &tmA, fb, tl.row0 + 64 * j, kr);
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_3d(sb + j * (64 * BK * 2), &tmB, fb, tl.n_tile * BN + 64 * j, kr, 0);
+          }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        report(args.ctl, MOE_ERR_TIMEOUT, 1);
+        // let every copy this thread started land before the CTA exits
+        for (int s = 0; s < STAGES; ++s)
+          if (armed & (1u << s)) mbar_wait(full_bar(s), (armed_parity >> s) & 1u, s_abort, false);
+      }
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        const Tile tl = decode_tile<KGROUP>(args, s_tile_start, t);
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, s_abort)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < tl.k_blocks; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, s_abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_base + stage * Plan::kStageBytes;
+          const uint32_t sb = sa + Plan::kABytes;
+          const int n16 = (kb == tl.k_blocks - 1) ? tl.last_k16 : 4;
+          for (int kk = 0; kk < n16; ++kk) {
+            const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * 2048, 64 * BK * 2, 1024)
+                                     : smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 64 * BK * 2, 1024)
+                                     : smem_desc_sw128(sb + kk * 32, 16, 1024);
+            mma_bf16(d_tmem, ad, bd, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(empty_bar(stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(tfull_bar(acc));
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok) report(args.ctl, MOE_ERR_TIMEOUT, 2);
+      // all MMAs issued by this thread have finished once the drain barrier flips
+      mma_commit(drain_bar);
+      mbar_wait(drain_bar, 0, s_abort, false);
+    }
+  } else {
+    // ================================================================ epilogue
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int r_local = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+      const Tile tl = decode_tile<KGROUP>(args, s_tile_start, t);
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull_bar(acc), acc_phase, s_abort));
+      if (!ok) {
+        if (lane == 0) report(args.ctl, MOE_ERR_TIMEOUT, 3);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const bool zero_acc = KGROUP && tl.k_blocks == 0;
+      int64_t row;
+      bool row_ok;
+      if constexpr (!KGROUP) {
+        row = static_cast<int64_t>(tl.row0) + r_local;
+        row_ok = row < tl.row_end && row < args.m_cap;
+      } else {
+        row = static_cast<int64_t>(tl.row0) + r_local;
+        row_ok = true;
+      }
+      float v[32];
+      if constexpr (EPI == EPI_BF16 || EPI == EPI_F32) {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tbase + c, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = zero_acc ? 0.f : __uint_as_float(r[i]);
+          if (row_ok) {
+            const int64_t col = static_cast<int64_t>(tl.n_tile) * BN + c;
+            const int64_t gofs = KGROUP ? static_cast<int64_t>(tl.group) * args.out_gstride : 0;
+            if constexpr (EPI == EPI_BF16) {
+              store_bf16x32(static_cast<__nv_bfloat16*>(args.out) + gofs + row * args.ldo + col, v);
+            } else {
+              store_f32x32(static_cast<float*>(args.out) + gofs + row * args.ldo + col, v);
+            }
+          }
+        }
+      } else if constexpr (EPI == EPI_SWIGLU_FWD) {
+        constexpr int BNH = BN / 2;
+#pragma unroll 1
+        for (int c = 0; c < BNH; c += 32) {
+          uint32_t ra[32], ru[32];
+          tmem_ld32(tbase + c, ra);
+          tmem_ld32(tbase + BNH + c, ru);
+          tmem_ld_wait();
+          if (row_ok) {
+            const int64_t col = static_cast<int64_t>(tl.n_tile) * BNH + c;
+            __nv_bfloat16* au = static_cast<__nv_bfloat16*>(args.out) + row * args.ldo;
+            float a[32], u[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              a[i] = __uint_as_float(ra[i]);
+              u[i] = __uint_as_float(ru[i]);
+              v[i] = a[i] / (1.0f + __expf(-a[i])) * u[i];
+            }
+            store_bf16x32(au + col, a);
+            store_bf16x32(au + args.f + col, u);
+            store_bf16x32(static_cast<__nv_bfloat16*>(args.out2) + row * args.ldo2 + col, v);
+          }
+        }
+      } else {  // EPI_SWIGLU_BWD
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tbase + c, r);
+          const int64_t col = static_cast<int64_t>(tl.n_tile) * BN + c;
+          float a[32], u[32];
+          if (row_ok) {
+            load_bf16x32(args.aux + row * args.ld_aux + col, a);
+            load_bf16x32(args.aux + row * args.ld_aux + args.f + col, u);
+          }
+          tmem_ld_wait();
+          if (row_ok) {
+            float du[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float dh = __uint_as_float(r[i]);
+              const float s = 1.0f / (1.0f + __expf(-a[i]));
+              v[i] = dh * u[i] * s * (1.0f + a[i] * (1.0f - s));
+              du[i] = dh * a[i] * s;
+            }
+            __nv_bfloat16* dau = static_cast<__nv_bfloat16*>(args.out) + row * args.ldo;
+            store_bf16x32(dau + col, v);
+            store_bf16x32(dau + args.f + col, du);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+}  // namespace tc
+}  // namespace moe

@@ -1,0 +1,106 @@
+"""One training step of the dropless MoE expert layer through the C ABI.
+
+MoELayer owns the device buffers of one shape (PyTorch allocates them; the
+library never does) and issues the calls of a forward and a backward pass
+in order on the current stream:
+
+  forward : moe_router_topk -> moe_permute -> moe_grouped_swiglu_fwd
+            -> moe_unpermute_combine
+  backward: moe_unpermute_combine_bwd -> moe_router_topk_bwd
+            -> moe_grouped_swiglu_bwd -> moe_permute_bwd
+
+Nothing in a step copies to the host or synchronises.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import ops
+from ._lib import MOE_DTYPE_BF16
+
+BF16 = torch.bfloat16
+I32 = torch.int32
+F32 = torch.float32
+
+
+class MoELayer:
+    def __init__(self, T, d, f, E, k, device="cuda", renorm=False, keep_logits=False,
+                 handle: ops.Handle | None = None):
+        self.T, self.d, self.f, self.E, self.k = T, d, f, E, k
+        dev = torch.device(device)
+        self.device = dev
+        self.handle = handle if handle is not None else ops.Handle(dev.index or 0)
+        self.shape = ops.make_shape(T, d, f, E, k, MOE_DTYPE_BF16, renorm)
+        M = ops.max_rows(self.shape)
+        self.M_cap = M
+        z = lambda *s, dt=BF16: torch.empty(*s, dtype=dt, device=dev)
+        self.ws = torch.empty(self.handle.workspace_size(self.shape), dtype=torch.uint8, device=dev)
+        # forward state
+        self.idx, self.w = z(T, k, dt=I32), z(T, k, dt=F32)
+        self.probs = z(T, E, dt=F32)
+        self.logits = z(T, E, dt=F32) if keep_logits else None
+        self.counts, self.offsets = z(E, dt=I32), z(E + 1, dt=I32)
+        self.row_map = z(T, k, dt=I32)
+        self.x_perm, self.au, self.h = z(M, d), z(M, 2 * f), z(M, f)
+        self.o_perm, self.y = z(M, d), z(T, d)
+        # backward state
+        self.do_perm, self.dw = z(M, d), z(T, k, dt=F32)
+        self.dau, self.dx_perm = z(M, 2 * f), z(M, d)
+        self.dw_gu, self.dw_d = z(E, 2 * f, d), z(E, d, f)
+        self.dx_router, self.dw_r = z(T, d, dt=F32), z(E, d)
+        self.db = z(E, dt=F32)
+        self.dx = z(T, d)
+
+    # ------------------------------------------------------------- forward
+    def router(self, x, w_r, bias=None, route=None, stream=None):
+        ops.moe_router_topk(self.handle, self.shape, x, w_r, bias, route, self.idx, self.w,
+                            self.probs, self.logits, self.ws, stream)
+
+    def permute(self, x, stream=None):
+        ops.moe_permute(self.handle, self.shape, x, self.idx, self.counts, self.offsets,
+                        self.row_map, self.x_perm, self.ws, stream)
+
+    def experts_fwd(self, w_gu, w_d, stream=None):
+        ops.moe_grouped_swiglu_fwd(self.handle, self.shape, self.x_perm, self.offsets, w_gu, w_d,
+                                   self.au, self.h, self.o_perm, self.ws, stream)
+
+    def combine(self, stream=None):
+        ops.moe_unpermute_combine(self.handle, self.shape, self.o_perm, self.row_map, self.w,
+                                  self.y, stream)
+
+    def forward(self, x, w_r, w_gu, w_d, bias=None, route=None, stream=None):
+        self.router(x, w_r, bias, route, stream)
+        self.permute(x, stream)
+        self.experts_fwd(w_gu, w_d, stream)
+        self.combine(stream)
+        return self.y
+
+    # ------------------------------------------------------------- backward
+    def combine_bwd(self, dy, stream=None):
+        ops.moe_unpermute_combine_bwd(self.handle, self.shape, dy, self.o_perm, self.row_map,
+                                      self.w, self.offsets, self.counts, self.do_perm, self.dw,
+                                      stream)
+
+    def router_bwd(self, x, w_r, stream=None):
+        ops.moe_router_topk_bwd(self.handle, self.shape, self.dw, self.probs, self.idx, x, w_r,
+                                self.dx_router, self.dw_r, self.db, self.ws, stream)
+
+    def experts_bwd(self, w_gu, w_d, stream=None):
+        ops.moe_grouped_swiglu_bwd(self.handle, self.shape, self.do_perm, self.x_perm, self.au,
+                                   self.h, self.offsets, w_gu, w_d, self.dau, self.dx_perm,
+                                   self.dw_gu, self.dw_d, self.ws, stream)
+
+    def permute_bwd(self, stream=None):
+        ops.moe_permute_bwd(self.handle, self.shape, self.dx_perm, self.row_map, self.dx_router,
+                            self.dx, stream)
+
+    def backward(self, dy, x, w_r, w_gu, w_d, stream=None):
+        self.combine_bwd(dy, stream)
+        self.router_bwd(x, w_r, stream)
+        self.experts_bwd(w_gu, w_d, stream)
+        self.permute_bwd(stream)
+        return self.dx
+
+    def step(self, x, w_r, w_gu, w_d, dy, bias=None, route=None, stream=None):
+        self.forward(x, w_r, w_gu, w_d, bias, route, stream)
+        self.backward(dy, x, w_r, w_gu, w_d, stream)

@@ -1,0 +1,143 @@
+"""Python binding of the C ABI with the same names (moe_router_topk, ...).
+
+Each function takes torch tensors that already live on the handle's device
+and forwards their data pointers, sizes and the current CUDA stream to
+libmoe.so.  No arithmetic of the layer happens here.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import MoeShape
+
+
+class MoeError(RuntimeError):
+    def __init__(self, name, status):
+        self.status = status
+        super().__init__(f"{name} returned {_lib.STATUS_NAMES.get(status, status)}")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _call(name, *args):
+    st = getattr(_lib.load(), name)(*args)
+    if st != _lib.MOE_OK:
+        raise MoeError(name, st)
+
+
+def make_shape(T, d, f, E, k, dtype=_lib.MOE_DTYPE_BF16, renorm=False) -> MoeShape:
+    return MoeShape(T, d, f, E, k, dtype, _lib.MOE_FLAG_RENORM if renorm else 0)
+
+
+class Handle:
+    """Owns a moe_handle_t bound to one CUDA device."""
+
+    def __init__(self, device: int = 0):
+        self.device = device
+        self._h = ctypes.c_void_p()
+        _call("moe_create", ctypes.byref(self._h), device)
+
+    @property
+    def ptr(self):
+        return self._h
+
+    def close(self):
+        if self._h:
+            _lib.load().moe_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def workspace_size(self, shape: MoeShape) -> int:
+        n = ctypes.c_size_t()
+        _call("moe_workspace_size", self._h, ctypes.byref(shape), ctypes.byref(n))
+        return n.value
+
+    def launch_count(self) -> int:
+        v = ctypes.c_uint64()
+        _call("moe_get_launch_count", self._h, ctypes.byref(v))
+        return v.value
+
+    def get_status(self) -> int:
+        v = ctypes.c_int()
+        _call("moe_get_status", self._h, ctypes.byref(v))
+        return v.value
+
+
+def max_rows(shape: MoeShape) -> int:
+    n = ctypes.c_int64()
+    _call("moe_max_rows", ctypes.byref(shape), ctypes.byref(n))
+    return n.value
+
+
+def moe_router_topk(h, shape, x, w_router, bias, route_in, topk_idx, topk_w, probs, logits, ws,
+                    stream=None):
+    _call("moe_router_topk", h.ptr, ctypes.byref(shape), _ptr(x), _ptr(w_router), _ptr(bias),
+          _ptr(route_in), _ptr(topk_idx), _ptr(topk_w), _ptr(probs), _ptr(logits), _ptr(ws),
+          ws.numel() if ws is not None else 0, _stream(stream))
+
+
+def moe_permute(h, shape, x, topk_idx, counts, offsets, row_map, x_perm, ws, stream=None):
+    _call("moe_permute", h.ptr, ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(counts),
+          _ptr(offsets), _ptr(row_map), _ptr(x_perm), _ptr(ws), ws.numel(), _stream(stream))
+
+
+def moe_grouped_swiglu_fwd(h, shape, x_perm, offsets, w_gu, w_down, au, hbuf, o_perm, ws,
+                           stream=None):
+    _call("moe_grouped_swiglu_fwd", h.ptr, ctypes.byref(shape), _ptr(x_perm), _ptr(offsets),
+          _ptr(w_gu), _ptr(w_down), _ptr(au), _ptr(hbuf), _ptr(o_perm), _ptr(ws),
+          ws.numel() if ws is not None else 0, _stream(stream))
+
+
+def moe_unpermute_combine(h, shape, o_perm, row_map, topk_w, y, stream=None):
+    _call("moe_unpermute_combine", h.ptr, ctypes.byref(shape), _ptr(o_perm), _ptr(row_map),
+          _ptr(topk_w), _ptr(y), _stream(stream))
+
+
+def moe_unpermute_combine_bwd(h, shape, dy, o_perm, row_map, topk_w, offsets, counts, do_perm,
+                              d_topk_w, stream=None):
+    _call("moe_unpermute_combine_bwd", h.ptr, ctypes.byref(shape), _ptr(dy), _ptr(o_perm),
+          _ptr(row_map), _ptr(topk_w), _ptr(offsets), _ptr(counts), _ptr(do_perm),
+          _ptr(d_topk_w), _stream(stream))
+
+
+def moe_grouped_swiglu_bwd(h, shape, do_perm, x_perm, au, hbuf, offsets, w_gu, w_down, dau,
+                           dx_perm, dw_gu, dw_down, ws, stream=None):
+    _call("moe_grouped_swiglu_bwd", h.ptr, ctypes.byref(shape), _ptr(do_perm), _ptr(x_perm),
+          _ptr(au), _ptr(hbuf), _ptr(offsets), _ptr(w_gu), _ptr(w_down), _ptr(dau),
+          _ptr(dx_perm), _ptr(dw_gu), _ptr(dw_down), _ptr(ws),
+          ws.numel() if ws is not None else 0, _stream(stream))
+
+
+def moe_permute_bwd(h, shape, dx_perm, row_map, dx_router, dx, stream=None):
+    _call("moe_permute_bwd", h.ptr, ctypes.byref(shape), _ptr(dx_perm), _ptr(row_map),
+          _ptr(dx_router), _ptr(dx), _stream(stream))
+
+
+def moe_router_topk_bwd(h, shape, d_topk_w, probs, topk_idx, x, w_router, dx_router, dw_router,
+                        dbias, ws, stream=None):
+    _call("moe_router_topk_bwd", h.ptr, ctypes.byref(shape), _ptr(d_topk_w), _ptr(probs),
+          _ptr(topk_idx), _ptr(x), _ptr(w_router), _ptr(dx_router), _ptr(dw_router), _ptr(dbias),
+          _ptr(ws), ws.numel(), _stream(stream))
+
+
+def moe_mxfp8_quantize(h, inp, axis, q, scales, stream=None):
+    rows, cols = inp.shape
+    _call("moe_mxfp8_quantize", h.ptr, _ptr(inp), rows, cols, axis, _ptr(q), _ptr(scales),
+          _stream(stream))

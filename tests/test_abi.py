@@ -1,0 +1,80 @@
+"""The C-ABI library loads and exports every entry point include/moe.h
+declares; host-only logic runs without a GPU (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixture_experts_layer_39_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_lib.LIB_PATH):
+        from mixture_experts_layer_39_b200 import build
+        build.build()
+    return _lib.load()
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("moe_router_topk", "moe_permute", "moe_grouped_swiglu_fwd", "moe_grouped_swiglu_bwd",
+              "moe_unpermute_combine", "moe_mxfp8_quantize"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _lib.SIGNATURES, n
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert lib.moe_status_string(code)
+    assert b"unknown" in lib.moe_status_string(99)
+
+
+def test_max_rows_and_shape_checks(lib):
+    s = _lib.MoeShape(16384, 2048, 1024, 128, 4, 0, 0)
+    n = ctypes.c_int64()
+    assert lib.moe_max_rows(ctypes.byref(s), ctypes.byref(n)) == 0
+    assert n.value == 16384 * 4 + 31 * 128
+    bad = [
+        _lib.MoeShape(16, 200, 256, 8, 2, 0, 0),     # d not a multiple of 256 -> unsupported
+        _lib.MoeShape(16, 256, 256, 8, 9, 0, 0),     # k > E -> invalid
+        _lib.MoeShape(16, 256, 256, 2048, 2, 0, 0),  # E > 1024 -> unsupported
+        _lib.MoeShape(0, 256, 256, 8, 2, 0, 0),      # T = 0 -> invalid
+        _lib.MoeShape(16, 256, 256, 8, 2, 7, 0),     # unknown dtype -> invalid
+    ]
+    want = [2, 1, 2, 1, 1]
+    for s_, w in zip(bad, want):
+        assert lib.moe_max_rows(ctypes.byref(s_), ctypes.byref(n)) == w
+
+
+def test_null_handle_rejected_before_any_launch(lib):
+    s = _lib.MoeShape(16, 256, 256, 8, 2, 0, 0)
+    assert lib.moe_router_topk(None, ctypes.byref(s), *([None] * 9), 0, None) == 1
+    assert lib.moe_permute(None, ctypes.byref(s), *([None] * 7), 0, None) == 1
+    assert lib.moe_destroy(None) == 1
+    h = ctypes.c_void_p()
+    assert lib.moe_create(None, 0) == 1
+
+
+def test_create_without_device_fails_cleanly(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    h = ctypes.c_void_p()
+    assert lib.moe_create(ctypes.byref(h), 0) != 0
+    assert not h.value
