@@ -141,6 +141,27 @@ MOE_API moe_status_t moe_permute(moe_handle_t h, const moe_shape_t* s, const voi
                          int32_t* row_map, void* x_perm, void* ws, size_t ws_bytes,
                          moe_stream_t stream);
 
+/* moe_permute without a workspace argument, for callers that cannot provide
+ * scratch memory at all (no workspace buffer and no permission to allocate,
+ * e.g. a plug-in inside a host program that owns every byte of device memory,
+ * or a latency-critical path that must never call cudaMalloc).  The pages
+ * describe no such call; it is an addition of this library.
+ * Same arguments, outputs and device-side checks as moe_permute.  Its scratch
+ * is a fixed 1 MiB array inside the library (one per GPU that loads it, held
+ * until the process exits), so the shape must satisfy
+ *   ceil(T*k / 256) * E <= MOE_NOALLOC_SCRATCH_INTS,
+ * otherwise MOE_ERR_WORKSPACE is returned before any launch.  The first call
+ * on a device looks up the array's device address (a host-side step, done
+ * once per device with that device current); make that first call before
+ * any stream capture.  All calls share the array: calls whose work can
+ * overlap on the GPU (unordered streams, several host threads) race on it.
+ * Nothing is allocated or freed by this call. */
+#define MOE_NOALLOC_SCRATCH_INTS (1 << 18)
+MOE_API moe_status_t moe_permute_noalloc(moe_handle_t h, const moe_shape_t* s, const void* x,
+                                         const int32_t* topk_idx, int32_t* counts,
+                                         int32_t* offsets, int32_t* row_map, void* x_perm,
+                                         moe_stream_t stream);
+
 /* Grouped SwiGLU expert FFN, forward.  For the rows of expert e:
  *   A = X W_gu[e][0:f]^T, U = X W_gu[e][f:2f]^T   (fp32 accumulate)
  *   au[:, 0:f] = bf16(A), au[:, f:2f] = bf16(U)   (saved for the backward)

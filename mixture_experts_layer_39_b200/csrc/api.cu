@@ -4,50 +4,17 @@
 #include <cstdlib>
 #include <new>
 
+#include "context.cuh"
 #include "gemm.cuh"
 #include "kernels.cuh"
-
-struct moe_context {
-  int device;
-  int num_sms;
-  moe::DeviceCtl* ctl;      // device status word
-  uint64_t launches = 0;    // kernels launched through this handle
-};
 
 namespace {
 
 using moe::ceil_div64;
 
-// Makes the handle's device current for the duration of a call.
-struct DeviceGuard {
-  int prev = -1;
-  bool ok = true;
-  explicit DeviceGuard(int dev) {
-    if (cudaGetDevice(&prev) != cudaSuccess) { ok = false; return; }
-    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
-  }
-  ~DeviceGuard() {
-    if (prev >= 0) {
-      int cur = -1;
-      if (cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
-    }
-  }
-};
-
-bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-
-moe_status_t check_shape(const moe_shape_t* s) {
-  if (s == nullptr) return MOE_ERR_INVALID_ARG;
-  if (s->T < 1 || s->d_model < 1 || s->d_ff < 1 || s->n_experts < 1 || s->top_k < 1)
-    return MOE_ERR_INVALID_ARG;
-  if (s->top_k > s->n_experts) return MOE_ERR_INVALID_ARG;
-  if (s->top_k > 8 || s->n_experts > 1024) return MOE_ERR_UNSUPPORTED;
-  if (s->d_model % 256 != 0 || s->d_ff % 256 != 0) return MOE_ERR_UNSUPPORTED;
-  if (s->dtype != MOE_DTYPE_BF16 && s->dtype != MOE_DTYPE_MXFP8) return MOE_ERR_INVALID_ARG;
-  const int64_t m_cap = static_cast<int64_t>(s->T) * s->top_k + 31ll * s->n_experts;
-  if (m_cap >= (1ll << 31) - 256) return MOE_ERR_UNSUPPORTED;
-  return MOE_OK;
-}
+using moe::aligned;
+using moe::check_shape;
+using moe::DeviceGuard;
 
 int64_t max_rows(const moe_shape_t* s) {
   return static_cast<int64_t>(s->T) * s->top_k + 31ll * s->n_experts;

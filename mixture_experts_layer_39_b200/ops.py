@@ -98,6 +98,13 @@ def moe_permute(h, shape, x, topk_idx, counts, offsets, row_map, x_perm, ws, str
           _ptr(offsets), _ptr(row_map), _ptr(x_perm), _ptr(ws), ws.numel(), _stream(stream))
 
 
+def moe_permute_noalloc(h, shape, x, topk_idx, counts, offsets, row_map, x_perm, stream=None):
+    """moe_permute for callers that cannot supply scratch memory: the library
+    uses a fixed 1 MiB array of its own instead of a workspace."""
+    _call("moe_permute_noalloc", h.ptr, ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(counts),
+          _ptr(offsets), _ptr(row_map), _ptr(x_perm), _stream(stream))
+
+
 def moe_grouped_swiglu_fwd(h, shape, x_perm, offsets, w_gu, w_down, au, hbuf, o_perm, ws,
                            stream=None):
     _call("moe_grouped_swiglu_fwd", h.ptr, ctypes.byref(shape), _ptr(x_perm), _ptr(offsets),
