@@ -64,9 +64,10 @@ bool tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, u
 template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP>
 moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const tc::GemmArgs& args, int grid,
                     cudaStream_t st) {
-  constexpr int STAGES = BN == 256 ? 4 : 6;
+  // the SwiGLU-backward epilogue's landing buffers take the fourth stage's room
+  constexpr int STAGES = BN == 256 ? (EPI == tc::EPI_SWIGLU_BWD ? 3 : 4) : 6;
   auto kern = tc::grouped_gemm_kernel<BN, A_MN, B_MN, EPI, KGROUP, STAGES>;
-  const size_t smem = tc::SmemPlan<BN, STAGES>::bytes(args.n_groups);
+  const size_t smem = tc::SmemPlan<BN, STAGES, EPI>::bytes(args.n_groups);
   static size_t configured = 0;  // largest size this instantiation was opened for
   if (smem > configured) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -47,38 +47,55 @@ __global__ void __launch_bounds__(kWarps * 32)
     else report(ctl, MOE_ERR_DEVICE_CHECK, 200);
   }
   __syncwarp();
-  for (int e = lane; e < E; e += 32) sub_counts[c * E + e] = cnt[e];
+  for (int e = lane; e < E; e += 32) sub_counts[static_cast<int64_t>(e) * n_sub + c] = cnt[e];
 }
 
-// One block; thread e scans expert e over the sub-chunks, then the block
-// scans the padded counts into segment offsets.
+// One block of 32 warps.  Warp w scans experts w, w+32, ... over their
+// sub-chunk counts (stored expert-major, so each scan reads contiguous
+// memory), leaving each sub-chunk's base; then the block scans the padded
+// counts into the segment offsets.
 __global__ void __launch_bounds__(1024)
     route_scan_kernel(int32_t* __restrict__ sub, int64_t n_sub, int E, int32_t* __restrict__ counts,
                       int32_t* __restrict__ offsets) {
+  __shared__ int s_tot[1024];
   __shared__ int s_warp[32];
-  const int e = threadIdx.x;
-  int run = 0;
-  if (e < E) {
-    int64_t c = 0;
-    for (; c + 4 <= n_sub; c += 4) {
-      const int v0 = sub[(c + 0) * E + e], v1 = sub[(c + 1) * E + e];
-      const int v2 = sub[(c + 2) * E + e], v3 = sub[(c + 3) * E + e];
-      sub[(c + 0) * E + e] = run;
-      sub[(c + 1) * E + e] = run + v0;
-      sub[(c + 2) * E + e] = run + v0 + v1;
-      sub[(c + 3) * E + e] = run + v0 + v1 + v2;
-      run += v0 + v1 + v2 + v3;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int e = warp; e < E; e += 32) {
+    int32_t* row = sub + static_cast<int64_t>(e) * n_sub;
+    int carry = 0;
+    for (int64_t base = 0; base < n_sub; base += 32 * 4) {
+      int v[4];
+      int local = 0;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t i = base + lane * 4 + u;
+        v[u] = i < n_sub ? row[i] : 0;
+        local += v[u];
+      }
+      int incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      int run = carry + incl - local;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t i = base + lane * 4 + u;
+        if (i < n_sub) row[i] = run;
+        run += v[u];
+      }
+      carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    for (; c < n_sub; ++c) {
-      const int v = sub[c * E + e];
-      sub[c * E + e] = run;
-      run += v;
+    if (lane == 0) {
+      counts[e] = carry;
+      s_tot[e] = carry;
     }
-    counts[e] = run;
   }
+  __syncthreads();
+  const int e = threadIdx.x;
+  const int run = e < E ? s_tot[e] : 0;
   const int padded = e < E ? (run + kSegAlign - 1) / kSegAlign * kSegAlign : 0;
-  // block exclusive scan of `padded`
-  const int lane = e & 31, warp = e >> 5;
   int v = padded;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -111,7 +128,8 @@ __global__ void __launch_bounds__(kWarps * 32)
   int* base = s_base_all + warp * E;
   const int64_t c = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
   if (c >= n_sub) return;
-  for (int e = lane; e < E; e += 32) base[e] = __ldg(offsets + e) + sub_base[c * E + e];
+  for (int e = lane; e < E; e += 32)
+    base[e] = __ldg(offsets + e) + sub_base[static_cast<int64_t>(e) * n_sub + c];
   __syncwarp();
   const int64_t beg = c * kSubChunk;
   const int64_t end = beg + kSubChunk < n_entries ? beg + kSubChunk : n_entries;
@@ -222,7 +240,7 @@ __global__ void __launch_bounds__(kWarps * 32)
 
 // dO[row_map[t,j]] = bf16(w * dY[t]); dw[t,j] = <dY[t], O[row_map[t,j]]>;
 // warps past T zero the pad rows of dO.
-__global__ void __launch_bounds__(kWarps * 32)
+__global__ void __launch_bounds__(kWarps * 32, 3)
     combine_bwd_kernel(const uint4* __restrict__ dy, const uint4* __restrict__ o,
                        const int32_t* __restrict__ row_map, const float* __restrict__ w,
                        const int32_t* __restrict__ offsets, const int32_t* __restrict__ counts,

@@ -38,115 +38,145 @@ __device__ __forceinline__ void topk_registers(const float (&l)[NE], int E, int 
   }
 }
 
-// Logits on CUDA cores for small E: each lane owns 8 consecutive features
-// per 256-feature slice; TPW tokens share every weight load.
-template <int NE, int TPW>
+// Logits on CUDA cores for small E.  W_r is converted to fp32 once per
+// block into shared memory (when it fits; else read as bf16 through L1);
+// a warp takes TPW tokens at a time so every weight read serves TPW tokens,
+// and each lane owns 8 consecutive features per 256.
+template <int NE, int TPW, bool W_SMEM>
 __global__ void __launch_bounds__(kWarps * 32)
     router_fused_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w_r,
                         const float* __restrict__ bias, const int32_t* __restrict__ route_in,
                         int T, int d, int E, int k, int renorm, int32_t* __restrict__ idx_out,
                         float* __restrict__ w_out, float* __restrict__ probs,
                         float* __restrict__ logits, DeviceCtl* ctl) {
+  extern __shared__ float4 s_wf[];  // [E][d] fp32 when W_SMEM
   const int lane = threadIdx.x & 31;
-  const int64_t t0 = (static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5)) * TPW;
-  if (t0 >= T) return;
   const int nvec = d >> 3;
   const uint4* xv = reinterpret_cast<const uint4*>(x);
   const uint4* wv = reinterpret_cast<const uint4*>(w_r);
-
-  float acc[TPW][NE];
+  if constexpr (W_SMEM) {
+    for (int i = threadIdx.x; i < E * nvec; i += blockDim.x) {
+      const uint4 q = __ldg(wv + i);
+      s_wf[2 * i] = make_float4(bf16_lo(q.x), bf16_hi(q.x), bf16_lo(q.y), bf16_hi(q.y));
+      s_wf[2 * i + 1] = make_float4(bf16_lo(q.z), bf16_hi(q.z), bf16_lo(q.w), bf16_hi(q.w));
+    }
+    __syncthreads();
+  }
+  const int64_t groups = ceil_div64(T, TPW);
+  for (int64_t grp = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5); grp < groups;
+       grp += static_cast<int64_t>(gridDim.x) * kWarps) {
+    const int64_t t0 = grp * TPW;
+    float acc[TPW][NE];
 #pragma unroll
-  for (int i = 0; i < TPW; ++i)
+    for (int i = 0; i < TPW; ++i)
 #pragma unroll
-    for (int e = 0; e < NE; ++e) acc[i][e] = 0.f;
+      for (int e = 0; e < NE; ++e) acc[i][e] = 0.f;
 
-  for (int v = lane; v < nvec; v += 32) {
-    float xf[TPW][8];
+    uint4 xq[TPW];
 #pragma unroll
     for (int i = 0; i < TPW; ++i) {
       const int64_t t = t0 + i < T ? t0 + i : T - 1;
-      const uint4 q = __ldg(xv + t * nvec + v);
-      xf[i][0] = bf16_lo(q.x); xf[i][1] = bf16_hi(q.x);
-      xf[i][2] = bf16_lo(q.y); xf[i][3] = bf16_hi(q.y);
-      xf[i][4] = bf16_lo(q.z); xf[i][5] = bf16_hi(q.z);
-      xf[i][6] = bf16_lo(q.w); xf[i][7] = bf16_hi(q.w);
+      xq[i] = lane < nvec ? __ldg(xv + t * nvec + lane) : make_uint4(0, 0, 0, 0);
     }
+    for (int v = lane; v < nvec; v += 32) {
+      float xf[TPW][8];
 #pragma unroll
-    for (int e = 0; e < NE; ++e) {
-      if (e < E) {
-        const uint4 q = __ldg(wv + static_cast<int64_t>(e) * nvec + v);
-        float wf[8];
-        wf[0] = bf16_lo(q.x); wf[1] = bf16_hi(q.x);
-        wf[2] = bf16_lo(q.y); wf[3] = bf16_hi(q.y);
-        wf[4] = bf16_lo(q.z); wf[5] = bf16_hi(q.z);
-        wf[6] = bf16_lo(q.w); wf[7] = bf16_hi(q.w);
-#pragma unroll
-        for (int i = 0; i < TPW; ++i)
-#pragma unroll
-          for (int c = 0; c < 8; ++c) acc[i][e] = fmaf(xf[i][c], wf[c], acc[i][e]);
+      for (int i = 0; i < TPW; ++i) {
+        xf[i][0] = bf16_lo(xq[i].x); xf[i][1] = bf16_hi(xq[i].x);
+        xf[i][2] = bf16_lo(xq[i].y); xf[i][3] = bf16_hi(xq[i].y);
+        xf[i][4] = bf16_lo(xq[i].z); xf[i][5] = bf16_hi(xq[i].z);
+        xf[i][6] = bf16_lo(xq[i].w); xf[i][7] = bf16_hi(xq[i].w);
       }
-    }
-  }
-
+      if (v + 32 < nvec) {  // next features in flight while this slice is multiplied
 #pragma unroll
-  for (int i = 0; i < TPW; ++i) {
-    const int64_t t = t0 + i;
-    if (t >= T) break;
-    float l[NE];
-#pragma unroll
-    for (int e = 0; e < NE; ++e) {
-      l[e] = warp_sum(acc[i][e]);
-      if (e < E && bias != nullptr) l[e] += __ldg(bias + e);
-    }
-    float m = -FLT_MAX;
-#pragma unroll
-    for (int e = 0; e < NE; ++e) if (e < E) m = fmaxf(m, l[e]);
-    float s = 0.f;
-    float p[NE];
-#pragma unroll
-    for (int e = 0; e < NE; ++e) {
-      p[e] = e < E ? expf(l[e] - m) : 0.f;
-      s += p[e];
-    }
-    const float inv = 1.0f / s;
-#pragma unroll
-    for (int e = 0; e < NE; ++e) p[e] *= inv;
-#pragma unroll
-    for (int e = 0; e < NE; ++e) {
-      if (e < E && (e & 31) == lane) {
-        probs[t * E + e] = p[e];
-        if (logits != nullptr) logits[t * E + e] = l[e];
-      }
-    }
-    int chosen[8];
-    if (route_in == nullptr) {
-      topk_registers<NE>(l, E, k, chosen);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) chosen[j] = j < k ? __ldg(route_in + t * k + j) : 0;
-    }
-    float wsel[8];
-    float wsum = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float pv = 0.f;
-      if (j < k) {
-        const int c = chosen[j];
-        if (c >= 0 && c < E) {
-#pragma unroll
-          for (int e = 0; e < NE; ++e) if (e == c) pv = p[e];
-        } else if (lane == 0) {
-          report(ctl, MOE_ERR_DEVICE_CHECK, 100);
+        for (int i = 0; i < TPW; ++i) {
+          const int64_t t = t0 + i < T ? t0 + i : T - 1;
+          xq[i] = __ldg(xv + t * nvec + v + 32);
         }
       }
-      wsel[j] = pv;
-      wsum += pv;
-    }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j < k && lane == j) {
-        idx_out[t * k + j] = chosen[j];
-        w_out[t * k + j] = renorm ? wsel[j] / wsum : wsel[j];
+      for (int e = 0; e < NE; ++e) {
+        if (e < E) {
+          float wf[8];
+          if constexpr (W_SMEM) {
+            const float4 a = s_wf[2 * (e * nvec + v)], b = s_wf[2 * (e * nvec + v) + 1];
+            wf[0] = a.x; wf[1] = a.y; wf[2] = a.z; wf[3] = a.w;
+            wf[4] = b.x; wf[5] = b.y; wf[6] = b.z; wf[7] = b.w;
+          } else {
+            const uint4 q = __ldg(wv + static_cast<int64_t>(e) * nvec + v);
+            wf[0] = bf16_lo(q.x); wf[1] = bf16_hi(q.x);
+            wf[2] = bf16_lo(q.y); wf[3] = bf16_hi(q.y);
+            wf[4] = bf16_lo(q.z); wf[5] = bf16_hi(q.z);
+            wf[6] = bf16_lo(q.w); wf[7] = bf16_hi(q.w);
+          }
+#pragma unroll
+          for (int i = 0; i < TPW; ++i)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) acc[i][e] = fmaf(xf[i][c], wf[c], acc[i][e]);
+        }
+      }
+    }
+
+#pragma unroll
+    for (int i = 0; i < TPW; ++i) {
+      const int64_t t = t0 + i;
+      if (t >= T) break;
+      float l[NE];
+#pragma unroll
+      for (int e = 0; e < NE; ++e) {
+        l[e] = warp_sum(acc[i][e]);
+        if (e < E && bias != nullptr) l[e] += __ldg(bias + e);
+      }
+      float m = -FLT_MAX;
+#pragma unroll
+      for (int e = 0; e < NE; ++e) if (e < E) m = fmaxf(m, l[e]);
+      float sum = 0.f;
+      float p[NE];
+#pragma unroll
+      for (int e = 0; e < NE; ++e) {
+        p[e] = e < E ? expf(l[e] - m) : 0.f;
+        sum += p[e];
+      }
+      const float inv = 1.0f / sum;
+#pragma unroll
+      for (int e = 0; e < NE; ++e) p[e] *= inv;
+#pragma unroll
+      for (int e = 0; e < NE; ++e) {
+        if (e < E && (e & 31) == lane) {
+          probs[t * E + e] = p[e];
+          if (logits != nullptr) logits[t * E + e] = l[e];
+        }
+      }
+      int chosen[8];
+      if (route_in == nullptr) {
+        topk_registers<NE>(l, E, k, chosen);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) chosen[j] = j < k ? __ldg(route_in + t * k + j) : 0;
+      }
+      float wsel[8];
+      float wsum = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float pv = 0.f;
+        if (j < k) {
+          const int c = chosen[j];
+          if (c >= 0 && c < E) {
+#pragma unroll
+            for (int e = 0; e < NE; ++e) if (e == c) pv = p[e];
+          } else if (lane == 0) {
+            report(ctl, MOE_ERR_DEVICE_CHECK, 100);
+          }
+        }
+        wsel[j] = pv;
+        wsum += pv;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < k && lane == j) {
+          idx_out[t * k + j] = chosen[j];
+          w_out[t * k + j] = renorm ? wsel[j] / wsum : wsel[j];
+        }
       }
     }
   }
@@ -252,17 +282,32 @@ cudaError_t launch_router_fused(const __nv_bfloat16* x, const __nv_bfloat16* w_r
                                 const int32_t* route_in, int T, int d, int E, int k, bool renorm,
                                 int32_t* idx, float* w, float* probs, float* logits,
                                 DeviceCtl* ctl, cudaStream_t st) {
-  auto go = [&](auto kern, int tpw) {
-    const int64_t warps = ceil_div64(T, tpw);
-    const unsigned grid = static_cast<unsigned>(ceil_div64(warps, kWarps));
-    kern<<<grid, kWarps * 32, 0, st>>>(x, w_r, bias, route_in, T, d, E, k, renorm ? 1 : 0, idx, w,
-                                       probs, logits, ctl);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const size_t w_smem = static_cast<size_t>(E) * d * 4;
+  auto go = [&](auto kern_smem, auto kern_l1, int tpw) {
+    const int64_t groups = ceil_div64(T, tpw);
+    const int64_t want = ceil_div64(groups, kWarps);
+    if (w_smem <= 96 * 1024) {
+      if (w_smem > 48 * 1024 &&
+          cudaFuncSetAttribute(kern_smem, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(w_smem)) != cudaSuccess)
+        return cudaErrorInvalidValue;
+      const unsigned grid = static_cast<unsigned>(want < 2 * sms ? want : 2 * sms);
+      kern_smem<<<grid, kWarps * 32, w_smem, st>>>(x, w_r, bias, route_in, T, d, E, k,
+                                                   renorm ? 1 : 0, idx, w, probs, logits, ctl);
+    } else {
+      const unsigned grid = static_cast<unsigned>(want < 8 * sms ? want : 8 * sms);
+      kern_l1<<<grid, kWarps * 32, 0, st>>>(x, w_r, bias, route_in, T, d, E, k, renorm ? 1 : 0,
+                                            idx, w, probs, logits, ctl);
+    }
     return cudaGetLastError();
   };
-  if (E <= 8) return go(router_fused_kernel<8, 4>, 4);
-  if (E <= 16) return go(router_fused_kernel<16, 2>, 2);
-  if (E <= 32) return go(router_fused_kernel<32, 1>, 1);
-  if (E <= 64) return go(router_fused_kernel<64, 1>, 1);
+  if (E <= 8) return go(router_fused_kernel<8, 4, true>, router_fused_kernel<8, 4, false>, 4);
+  if (E <= 16) return go(router_fused_kernel<16, 2, true>, router_fused_kernel<16, 2, false>, 2);
+  if (E <= 32) return go(router_fused_kernel<32, 1, true>, router_fused_kernel<32, 1, false>, 1);
+  if (E <= 64) return go(router_fused_kernel<64, 1, true>, router_fused_kernel<64, 1, false>, 1);
   return cudaErrorInvalidValue;
 }
 

@@ -15,15 +15,26 @@ namespace {
 
 constexpr int kWarps = 8;
 
-template <int NPL, bool FUSE_DX>
+// NE: compile-time bound on E for the fused dX_router loop (E <= NE <= 32*NPL).
+template <int NPL, bool FUSE_DX, int NE = 32 * NPL>
 __global__ void __launch_bounds__(kWarps * 32)
     router_bwd_dl_kernel(const float* __restrict__ dw, const float* __restrict__ probs,
                          const int32_t* __restrict__ idx, const __nv_bfloat16* __restrict__ w_r,
                          int T, int d, int E, int k, int renorm, float* __restrict__ dl_f32,
                          __nv_bfloat16* __restrict__ dl_bf16, float* __restrict__ dx_router,
-                         float* __restrict__ db_partial) {
+                         float* __restrict__ db_partial, int stage_w) {
   __shared__ float s_db[kWarps][32 * NPL];
+  extern __shared__ uint4 s_wdyn[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint4* s_w = nullptr;
+  if constexpr (FUSE_DX) {
+    if (stage_w) {  // W_r staged once per block
+      const uint4* src = reinterpret_cast<const uint4*>(w_r);
+      for (int i = threadIdx.x; i < E * (d >> 3); i += blockDim.x) s_wdyn[i] = __ldg(src + i);
+      __syncthreads();
+      s_w = s_wdyn;
+    }
+  }
   float db[NPL];
 #pragma unroll
   for (int i = 0; i < NPL; ++i) db[i] = 0.f;
@@ -77,24 +88,26 @@ __global__ void __launch_bounds__(kWarps * 32)
       }
     }
     if constexpr (FUSE_DX) {
-      // dX_router[t, :] = sum_e dL[e] W_r[e, :]; lane owns 8 columns per 256
-      const uint4* wv = reinterpret_cast<const uint4*>(w_r);
+      // dX_router[t, :] = sum_e dL[e] W_r[e, :]; every lane gets all of dL
+      // once, then owns 8 columns per 256 (W_r from shared memory)
+      float dle[NE];
+#pragma unroll
+      for (int e = 0; e < NE; ++e) dle[e] = __shfl_sync(0xffffffffu, dl[e >> 5], e & 31);
+      const uint4* wv = s_w != nullptr ? s_w : reinterpret_cast<const uint4*>(w_r);
       float4* out = reinterpret_cast<float4*>(dx_router + t * d);
       for (int v = lane; v < nvec; v += 32) {
         float acc[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[c] = 0.f;
 #pragma unroll
-        for (int i = 0; i < NPL; ++i) {
-          for (int src = 0; src < 32; ++src) {
-            const int e = 32 * i + src;
-            const float dle = __shfl_sync(0xffffffffu, dl[i], src);
-            if (e >= E) break;
-            const uint4 q = __ldg(wv + static_cast<int64_t>(e) * nvec + v);
-            acc[0] = fmaf(dle, bf16_lo(q.x), acc[0]); acc[1] = fmaf(dle, bf16_hi(q.x), acc[1]);
-            acc[2] = fmaf(dle, bf16_lo(q.y), acc[2]); acc[3] = fmaf(dle, bf16_hi(q.y), acc[3]);
-            acc[4] = fmaf(dle, bf16_lo(q.z), acc[4]); acc[5] = fmaf(dle, bf16_hi(q.z), acc[5]);
-            acc[6] = fmaf(dle, bf16_lo(q.w), acc[6]); acc[7] = fmaf(dle, bf16_hi(q.w), acc[7]);
+        for (int e = 0; e < NE; ++e) {
+          if (e < E) {
+            const uint4 q = wv[static_cast<int64_t>(e) * nvec + v];
+            const float g = dle[e];
+            acc[0] = fmaf(g, bf16_lo(q.x), acc[0]); acc[1] = fmaf(g, bf16_hi(q.x), acc[1]);
+            acc[2] = fmaf(g, bf16_lo(q.y), acc[2]); acc[3] = fmaf(g, bf16_hi(q.y), acc[3]);
+            acc[4] = fmaf(g, bf16_lo(q.z), acc[4]); acc[5] = fmaf(g, bf16_hi(q.z), acc[5]);
+            acc[6] = fmaf(g, bf16_lo(q.w), acc[6]); acc[7] = fmaf(g, bf16_hi(q.w), acc[7]);
           }
         }
         out[2 * v] = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -115,14 +128,16 @@ __global__ void __launch_bounds__(kWarps * 32)
 }
 
 // dW_r partial over a chunk of tokens, CUDA cores (E <= 64): each thread
-// owns CPT consecutive columns and all E experts of them.
-constexpr int kChunk = 128;
+// owns CPT consecutive columns and all E experts of them; blocks tile
+// (column slice, token chunk).
+constexpr int kChunk = 64;
+constexpr int kDwThreads = 128;
 
 template <int NE, int CPT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kDwThreads)
     router_dw_small_kernel(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ x, int T,
                            int d, int E, float* __restrict__ partial) {
-  __shared__ float s_dl[kChunk * NE];
+  __shared__ float s_dl[kChunk * NE];  // 16 KB at NE = 64
   const int64_t t0 = static_cast<int64_t>(blockIdx.y) * kChunk;
   const int nt = T - t0 < kChunk ? static_cast<int>(T - t0) : kChunk;
   for (int i = threadIdx.x; i < nt * E; i += blockDim.x) {
@@ -130,18 +145,27 @@ __global__ void __launch_bounds__(256)
     s_dl[tt * NE + e] = dl[(t0 + tt) * E + e];
   }
   __syncthreads();
-  const int64_t col = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) * CPT;
+  const int64_t col = (static_cast<int64_t>(blockIdx.x) * kDwThreads + threadIdx.x) * CPT;
   if (col >= d) return;
   float acc[NE][CPT];
 #pragma unroll
   for (int e = 0; e < NE; ++e)
 #pragma unroll
     for (int c = 0; c < CPT; ++c) acc[e][c] = 0.f;
+#pragma unroll 4
   for (int tt = 0; tt < nt; ++tt) {
     float xv[CPT];
     const __nv_bfloat16* xr = x + (t0 + tt) * d + col;
+    if constexpr (CPT == 4) {
+      const uint2 q = __ldg(reinterpret_cast<const uint2*>(xr));
+      xv[0] = bf16_lo(q.x); xv[1] = bf16_hi(q.x); xv[2] = bf16_lo(q.y); xv[3] = bf16_hi(q.y);
+    } else if constexpr (CPT == 2) {
+      const uint32_t q = __ldg(reinterpret_cast<const unsigned int*>(xr));
+      xv[0] = bf16_lo(q); xv[1] = bf16_hi(q);
+    } else {
 #pragma unroll
-    for (int c = 0; c < CPT; ++c) xv[c] = __bfloat162float(xr[c]);
+      for (int c = 0; c < CPT; ++c) xv[c] = __bfloat162float(xr[c]);
+    }
 #pragma unroll
     for (int e = 0; e < NE; ++e) {
       if (e < E) {
@@ -159,23 +183,47 @@ __global__ void __launch_bounds__(256)
       for (int c = 0; c < CPT; ++c) out[static_cast<int64_t>(e) * d + col + c] = acc[e][c];
 }
 
-__global__ void reduce_partials_bf16_kernel(const float* __restrict__ partial, int n_part,
-                                            int64_t n, __nv_bfloat16* __restrict__ out) {
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    float s = 0.f;
-    for (int p = 0; p < n_part; ++p) s += partial[static_cast<int64_t>(p) * n + i];
-    out[i] = __float2bfloat16_rn(s);
+// out[i] = bf16(sum_p partial[p][i]).  A block owns 32 float4 columns; its
+// 8 warps take the partials p = w, w+8, ... and are summed in a fixed order.
+__global__ void __launch_bounds__(256)
+    reduce_partials_bf16_kernel(const float4* __restrict__ partial, int n_part, int64_t n4,
+                                __nv_bfloat16* __restrict__ out) {
+  __shared__ float4 s_part[8][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * 32 + lane;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (i < n4) {
+#pragma unroll 4
+    for (int p = warp; p < n_part; p += 8) {
+      const float4 v = __ldg(partial + static_cast<int64_t>(p) * n4 + i);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+  }
+  s_part[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0 && i < n4) {
+    float4 r = s_part[0][lane];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) {
+      r.x += s_part[w][lane].x; r.y += s_part[w][lane].y;
+      r.z += s_part[w][lane].z; r.w += s_part[w][lane].w;
+    }
+    uint2 packed = make_uint2(pack_bf16x2(r.x, r.y), pack_bf16x2(r.z, r.w));
+    reinterpret_cast<uint2*>(out)[i] = packed;
   }
 }
 
+// out[e] = sum_p partial[p][e]: one warp per e, lanes stride over p, then a
+// fixed-order butterfly.
 __global__ void reduce_rows_f32_kernel(const float* __restrict__ partial, int n_part, int E,
                                        float* __restrict__ out) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (e >= E) return;
   float s = 0.f;
-  for (int p = 0; p < n_part; ++p) s += partial[static_cast<int64_t>(p) * E + e];
-  out[e] = s;
+  for (int p = lane; p < n_part; p += 32) s += partial[static_cast<int64_t>(p) * E + e];
+  s = warp_sum(s);
+  if (lane == 0) out[e] = s;
 }
 
 }  // namespace
@@ -189,14 +237,24 @@ cudaError_t launch_router_bwd_dl(const float* dw, const float* probs, const int3
                                  float* dx_router, float* db_partial, int nblocks,
                                  DeviceCtl* ctl, cudaStream_t st) {
   (void)ctl;
+  const size_t w_bytes = static_cast<size_t>(E) * d * 2;
+  const bool stage = fuse_dx && w_bytes <= 96 * 1024;
+  const size_t smem = stage ? w_bytes : 0;
   auto go = [&](auto kern) {
-    kern<<<nblocks, kWarps * 32, 0, st>>>(dw, probs, idx, w_r, T, d, E, k, renorm ? 1 : 0, dl_f32,
-                                          dl_bf16, dx_router, db_partial);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return cudaErrorInvalidValue;
+    kern<<<nblocks, kWarps * 32, smem, st>>>(dw, probs, idx, w_r, T, d, E, k, renorm ? 1 : 0,
+                                             dl_f32, dl_bf16, dx_router, db_partial,
+                                             stage ? 1 : 0);
     return cudaGetLastError();
   };
   if (fuse_dx) {
-    if (E <= 32) return go(router_bwd_dl_kernel<1, true>);
-    if (E <= 64) return go(router_bwd_dl_kernel<2, true>);
+    if (E <= 8) return go(router_bwd_dl_kernel<1, true, 8>);
+    if (E <= 16) return go(router_bwd_dl_kernel<1, true, 16>);
+    if (E <= 32) return go(router_bwd_dl_kernel<1, true, 32>);
+    if (E <= 64) return go(router_bwd_dl_kernel<2, true, 64>);
     return cudaErrorInvalidValue;
   }
   if (E <= 128) return go(router_bwd_dl_kernel<4, false>);
@@ -210,28 +268,29 @@ cudaError_t launch_router_dw_small(const float* dl, const __nv_bfloat16* x, int 
                                    float* partial, cudaStream_t st) {
   const unsigned gy = static_cast<unsigned>(ceil_div64(T, kChunk));
   auto go = [&](auto kern, int cpt) {
-    const unsigned gx = static_cast<unsigned>(ceil_div64(d, 256 * cpt));
-    kern<<<dim3(gx, gy), 256, 0, st>>>(dl, x, T, d, E, partial);
+    const unsigned gx = static_cast<unsigned>(ceil_div64(d, kDwThreads * cpt));
+    kern<<<dim3(gx, gy), kDwThreads, 0, st>>>(dl, x, T, d, E, partial);
     return cudaGetLastError();
   };
-  if (E <= 8) return go(router_dw_small_kernel<8, 8>, 8);
-  if (E <= 16) return go(router_dw_small_kernel<16, 4>, 4);
-  if (E <= 32) return go(router_dw_small_kernel<32, 2>, 2);
+  if (E <= 8) return go(router_dw_small_kernel<8, 4>, 4);
+  if (E <= 16) return go(router_dw_small_kernel<16, 2>, 2);
+  if (E <= 32) return go(router_dw_small_kernel<32, 1>, 1);
   if (E <= 64) return go(router_dw_small_kernel<64, 1>, 1);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_reduce_partials_bf16(const float* partial, int n_part, int64_t n,
                                         __nv_bfloat16* out, cudaStream_t st) {
-  const unsigned grid = static_cast<unsigned>(ceil_div64(n, 256) < 4096 ? ceil_div64(n, 256) : 4096);
-  reduce_partials_bf16_kernel<<<grid, 256, 0, st>>>(partial, n_part, n, out);
+  const int64_t n4 = n / 4;  // n = E * d, a multiple of 256
+  reduce_partials_bf16_kernel<<<static_cast<unsigned>(ceil_div64(n4, 32)), 256, 0, st>>>(
+      reinterpret_cast<const float4*>(partial), n_part, n4, out);
   return cudaGetLastError();
 }
 
 cudaError_t launch_reduce_rows_f32(const float* partial, int n_part, int E, float* out,
                                    cudaStream_t st) {
-  reduce_rows_f32_kernel<<<static_cast<unsigned>(ceil_div64(E, 256)), 256, 0, st>>>(partial, n_part,
-                                                                                    E, out);
+  reduce_rows_f32_kernel<<<static_cast<unsigned>(ceil_div64(E, 8)), 256, 0, st>>>(partial, n_part,
+                                                                                 E, out);
   return cudaGetLastError();
 }
 

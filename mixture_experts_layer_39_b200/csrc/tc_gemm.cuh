@@ -202,6 +202,16 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Logistic function for the SwiGLU epilogues: sigma(z) = 1/2 + tanh(z/2)/2,
+// with the hardware tanh approximation (PTX tanh.approx.f32, relative error
+// about 2^-11: below the bf16 rounding the outputs take anyway).  One MUFU
+// operation instead of an exponential plus an IEEE division.
+__device__ __forceinline__ float sigmoid_fast(float z) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
+  return fmaf(0.5f, t, 0.5f);
+}
+
 // ---------------------------------------------------------------- scheduling
 struct Tile {
   int group;
@@ -262,39 +272,89 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* s_tile
 }
 
 // ---------------------------------------------------------------- epilogue helpers
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
+// Each epilogue warp owns 32 consecutive tile rows (its TMEM lane quarter)
+// and a 4 KB staging buffer: 32 rows x 128 bytes, 16-byte slots swizzled by
+// row (slot q of row r at q ^ (r & 7)) so that both access patterns below
+// are free of bank conflicts.
+//   row side       : lane r reads/writes the 8 slots of row r;
+//   coalesced side : lane i touches row 4j + i/8, slot i%8, so one warp
+//                    instruction moves four full 128-byte row segments.
+constexpr int kStageRowBytes = 128;
+constexpr int kEpiBufBytes = 32 * kStageRowBytes;
+
+__device__ __forceinline__ uint4* stage_slot(uint8_t* buf, int row, int q) {
+  return reinterpret_cast<uint4*>(buf + row * kStageRowBytes + ((q ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ void stage_write_row(uint8_t* buf, int lane, const uint4 (&v)[8]) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint4 w;
-    w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-    w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-    w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-    w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-    d4[q] = w;
+  for (int q = 0; q < 8; ++q) *stage_slot(buf, lane, q) = v[q];
+}
+
+__device__ __forceinline__ void stage_read_row(uint8_t* buf, int lane, uint4 (&v)[8]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) v[q] = *stage_slot(buf, lane, q);
+}
+
+__device__ __forceinline__ void stage_to_global(uint8_t* buf, uint8_t* g, int64_t ld_bytes,
+                                                int valid_rows, int lane) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int row = 4 * j + (lane >> 3);
+    const uint4 v = *stage_slot(buf, row, lane & 7);
+    if (row < valid_rows)
+      *reinterpret_cast<uint4*>(g + row * ld_bytes + ((lane & 7) << 4)) = v;
   }
 }
 
-__device__ __forceinline__ void store_f32x32(float* dst, const float* v) {
-  float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-  for (int q = 0; q < 8; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+// Writes this lane's 128-byte row `v` through the staging buffer to global.
+__device__ __forceinline__ void store_rows(uint8_t* buf, int lane, const uint4 (&v)[8], uint8_t* g,
+                                           int64_t ld_bytes, int valid_rows) {
+  stage_write_row(buf, lane, v);
+  __syncwarp();
+  stage_to_global(buf, g, ld_bytes, valid_rows, lane);
+  __syncwarp();
 }
 
-__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float* v) {
-  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+// 64 fp32 -> 64 bf16 (128 bytes)
+__device__ __forceinline__ void pack64(const float* f, uint4 (&v)[8]) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint4 w = __ldg(s4 + q);
-    v[8 * q + 0] = bf16_lo(w.x); v[8 * q + 1] = bf16_hi(w.x);
-    v[8 * q + 2] = bf16_lo(w.y); v[8 * q + 3] = bf16_hi(w.y);
-    v[8 * q + 4] = bf16_lo(w.z); v[8 * q + 5] = bf16_hi(w.z);
-    v[8 * q + 6] = bf16_lo(w.w); v[8 * q + 7] = bf16_hi(w.w);
+  for (int q = 0; q < 8; ++q)
+    v[q] = make_uint4(pack_bf16x2(f[8 * q + 0], f[8 * q + 1]), pack_bf16x2(f[8 * q + 2], f[8 * q + 3]),
+                      pack_bf16x2(f[8 * q + 4], f[8 * q + 5]), pack_bf16x2(f[8 * q + 6], f[8 * q + 7]));
+}
+
+// Asynchronous copy of the warp's 32 rows x 128 bytes at `g` into `buf`
+// (staging layout), zero-filling rows past valid_rows; no registers held.
+// (`safe` is any valid global address, used as the source of zero-size copies.)
+__device__ __forceinline__ void cp_async_rows(uint8_t* buf, const uint8_t* g, int64_t ld_bytes,
+                                              int valid_rows, int lane, const void* safe) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int row = 4 * j + (lane >> 3);
+    const bool ok = row < valid_rows;
+    const uint8_t* src = ok ? g + row * ld_bytes + ((lane & 7) << 4) : static_cast<const uint8_t*>(safe);
+    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(stage_slot(buf, row, lane & 7)));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(ok ? 16 : 0)
+                 : "memory");
   }
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 // ---------------------------------------------------------------- the kernel
-template <int BN, int STAGES>
+template <int BN, int STAGES, int EPI>
 struct SmemPlan {
   static constexpr int kABytes = BM * BK * 2;
   static constexpr int kBBytes = BN * BK * 2;
@@ -302,7 +362,11 @@ struct SmemPlan {
   static constexpr int kBarOff = STAGES * kStageBytes;                 // 1024-aligned stages
   static constexpr int kBarBytes = (2 * STAGES + 5) * 8;               // full, empty, tfull x2, tempty x2, drain
   static constexpr int kMiscOff = kBarOff + kBarBytes;                 // tmem base, abort flag
-  static constexpr int kTileOff = kMiscOff + 16;                       // group tile starts
+  static constexpr int kEpiOff = (kMiscOff + 16 + 127) / 128 * 128;    // 4 epilogue warps' buffers
+  // per warp: the 4 KB staging buffer, plus (SwiGLU backward) an 8 KB landing
+  // buffer that cp.async fills with the next chunk's saved [A | U] rows
+  static constexpr int kWarpEpiBytes = kEpiBufBytes + (EPI == EPI_SWIGLU_BWD ? 2 * kEpiBufBytes : 0);
+  static constexpr int kTileOff = kEpiOff + 4 * kWarpEpiBytes;         // group tile starts
   static constexpr int bytes(int n_groups) { return 1024 + kTileOff + 4 * (n_groups + 1); }
 };
 
@@ -312,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
   static_assert(BN == 128 || BN == 256, "BN");
   static_assert(!(EPI == EPI_SWIGLU_FWD && B_MN), "SwiGLU forward takes K-major weights");
-  using Plan = SmemPlan<BN, STAGES>;
+  using Plan = SmemPlan<BN, STAGES, EPI>;
   constexpr uint32_t kTmemCols = 2 * BN;
   constexpr uint32_t kIdesc = idesc_bf16(BM, BN, A_MN, B_MN);
 
@@ -486,13 +550,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ================================================================ epilogue
     const int quarter = warp & 3;  // TMEM lanes this warp may access
-    const int r_local = quarter * 32 + lane;
+    uint8_t* ebuf = smem + Plan::kEpiOff + (warp - 2) * Plan::kWarpEpiBytes;
+    uint8_t* lbuf_a = ebuf + kEpiBufBytes;       // SwiGLU backward: landing buffer for A
+    uint8_t* lbuf_u = ebuf + 2 * kEpiBufBytes;   // ... and for U
     int acc = 0;
     uint32_t acc_phase = 0;
+    // rows of this warp's quarter in the tile, and the row prefetch of a tile's
+    // saved [A | U] slice (SwiGLU backward) into L2
+    auto quarter_rows = [&](const Tile& tl) -> int {
+      if constexpr (KGROUP) {
+        return 32;
+      } else {
+        const int64_t first = static_cast<int64_t>(tl.row0) + quarter * 32;
+        int64_t lim = tl.row_end < args.m_cap ? tl.row_end : args.m_cap;
+        const int64_t n = lim - first;
+        return n <= 0 ? 0 : (n >= 32 ? 32 : static_cast<int>(n));
+      }
+    };
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
       const Tile tl = decode_tile<KGROUP>(args, s_tile_start, t);
+      const int vrows = quarter_rows(tl);
+      const int64_t row_first = static_cast<int64_t>(tl.row0) + quarter * 32;  // warp's first row
+      // SwiGLU backward: the saved [A | U] rows of the first 64 columns are
+      // requested before waiting for the accumulator, so their latency
+      // overlaps the main loop; each later chunk is requested one chunk ahead.
+      const __nv_bfloat16* aux = nullptr;
+      if constexpr (EPI == EPI_SWIGLU_BWD) {
+        aux = args.aux + row_first * args.ld_aux + static_cast<int64_t>(tl.n_tile) * BN;
+        cp_async_rows(lbuf_a, reinterpret_cast<const uint8_t*>(aux), args.ld_aux * 2, vrows, lane,
+                      args.aux);
+        cp_async_rows(lbuf_u, reinterpret_cast<const uint8_t*>(aux + args.f), args.ld_aux * 2, vrows,
+                      lane, args.aux);
+        cp_async_commit();
+      }
       const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull_bar(acc), acc_phase, s_abort));
       if (!ok) {
+        if constexpr (EPI == EPI_SWIGLU_BWD) cp_async_wait_all();  // own copies land first
         if (lane == 0) report(args.ctl, MOE_ERR_TIMEOUT, 3);
         break;
       }
@@ -500,82 +593,126 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
       const bool zero_acc = KGROUP && tl.k_blocks == 0;
-      int64_t row;
-      bool row_ok;
-      if constexpr (!KGROUP) {
-        row = static_cast<int64_t>(tl.row0) + r_local;
-        row_ok = row < tl.row_end && row < args.m_cap;
-      } else {
-        row = static_cast<int64_t>(tl.row0) + r_local;
-        row_ok = true;
-      }
-      float v[32];
-      if constexpr (EPI == EPI_BF16 || EPI == EPI_F32) {
+      const int64_t gofs = KGROUP ? static_cast<int64_t>(tl.group) * args.out_gstride : 0;
+      if constexpr (EPI == EPI_BF16) {
+        auto* base = static_cast<__nv_bfloat16*>(args.out) + gofs + row_first * args.ldo +
+                     static_cast<int64_t>(tl.n_tile) * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 64) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tbase + c, r0);
+          tmem_ld32(tbase + c + 32, r1);
+          tmem_ld_wait();
+          float f[64];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            f[i] = zero_acc ? 0.f : __uint_as_float(r0[i]);
+            f[32 + i] = zero_acc ? 0.f : __uint_as_float(r1[i]);
+          }
+          uint4 v[8];
+          pack64(f, v);
+          store_rows(ebuf, lane, v, reinterpret_cast<uint8_t*>(base + c), args.ldo * 2, vrows);
+        }
+      } else if constexpr (EPI == EPI_F32) {
+        auto* base = static_cast<float*>(args.out) + gofs + row_first * args.ldo +
+                     static_cast<int64_t>(tl.n_tile) * BN;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t r[32];
           tmem_ld32(tbase + c, r);
           tmem_ld_wait();
+          uint4 v[8];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = zero_acc ? 0.f : __uint_as_float(r[i]);
-          if (row_ok) {
-            const int64_t col = static_cast<int64_t>(tl.n_tile) * BN + c;
-            const int64_t gofs = KGROUP ? static_cast<int64_t>(tl.group) * args.out_gstride : 0;
-            if constexpr (EPI == EPI_BF16) {
-              store_bf16x32(static_cast<__nv_bfloat16*>(args.out) + gofs + row * args.ldo + col, v);
-            } else {
-              store_f32x32(static_cast<float*>(args.out) + gofs + row * args.ldo + col, v);
-            }
-          }
+          for (int q = 0; q < 8; ++q)
+            v[q] = zero_acc ? make_uint4(0, 0, 0, 0)
+                            : make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+          store_rows(ebuf, lane, v, reinterpret_cast<uint8_t*>(base + c), args.ldo * 4, vrows);
         }
       } else if constexpr (EPI == EPI_SWIGLU_FWD) {
         constexpr int BNH = BN / 2;
+        const int64_t col0 = static_cast<int64_t>(tl.n_tile) * BNH;
+        auto* au = static_cast<__nv_bfloat16*>(args.out) + row_first * args.ldo + col0;
+        auto* hh = static_cast<__nv_bfloat16*>(args.out2) + row_first * args.ldo2 + col0;
 #pragma unroll 1
-        for (int c = 0; c < BNH; c += 32) {
-          uint32_t ra[32], ru[32];
-          tmem_ld32(tbase + c, ra);
-          tmem_ld32(tbase + BNH + c, ru);
-          tmem_ld_wait();
-          if (row_ok) {
-            const int64_t col = static_cast<int64_t>(tl.n_tile) * BNH + c;
-            __nv_bfloat16* au = static_cast<__nv_bfloat16*>(args.out) + row * args.ldo;
-            float a[32], u[32];
+        for (int c = 0; c < BNH; c += 64) {
+          uint4 vg[8], vu[8], vh[8];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              a[i] = __uint_as_float(ra[i]);
-              u[i] = __uint_as_float(ru[i]);
-              v[i] = a[i] / (1.0f + __expf(-a[i])) * u[i];
+          for (int half = 0; half < 2; ++half) {
+            uint32_t g[32], u[32];
+            tmem_ld32(tbase + c + 32 * half, g);
+            tmem_ld32(tbase + BNH + c + 32 * half, u);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float a[8], b[8], h[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                a[i] = __uint_as_float(g[8 * q + i]);
+                b[i] = __uint_as_float(u[8 * q + i]);
+                h[i] = a[i] * sigmoid_fast(a[i]) * b[i];
+              }
+              vg[4 * half + q] = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]),
+                                            pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
+              vu[4 * half + q] = make_uint4(pack_bf16x2(b[0], b[1]), pack_bf16x2(b[2], b[3]),
+                                            pack_bf16x2(b[4], b[5]), pack_bf16x2(b[6], b[7]));
+              vh[4 * half + q] = make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]),
+                                            pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
             }
-            store_bf16x32(au + col, a);
-            store_bf16x32(au + args.f + col, u);
-            store_bf16x32(static_cast<__nv_bfloat16*>(args.out2) + row * args.ldo2 + col, v);
           }
+          store_rows(ebuf, lane, vg, reinterpret_cast<uint8_t*>(au + c), args.ldo * 2, vrows);
+          store_rows(ebuf, lane, vu, reinterpret_cast<uint8_t*>(au + args.f + c), args.ldo * 2, vrows);
+          store_rows(ebuf, lane, vh, reinterpret_cast<uint8_t*>(hh + c), args.ldo2 * 2, vrows);
         }
       } else {  // EPI_SWIGLU_BWD
+        auto* dau = static_cast<__nv_bfloat16*>(args.out) + row_first * args.ldo +
+                    static_cast<int64_t>(tl.n_tile) * BN;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t r[32];
-          tmem_ld32(tbase + c, r);
-          const int64_t col = static_cast<int64_t>(tl.n_tile) * BN + c;
-          float a[32], u[32];
-          if (row_ok) {
-            load_bf16x32(args.aux + row * args.ld_aux + col, a);
-            load_bf16x32(args.aux + row * args.ld_aux + args.f + col, u);
+        for (int c = 0; c < BN; c += 64) {
+          uint4 va[8], vu[8];
+          cp_async_wait_all();
+          __syncwarp();
+          stage_read_row(lbuf_a, lane, va);
+          stage_read_row(lbuf_u, lane, vu);
+          __syncwarp();
+          if (c + 64 < BN) {  // next chunk lands while this one is computed and stored
+            cp_async_rows(lbuf_a, reinterpret_cast<const uint8_t*>(aux + c + 64), args.ld_aux * 2,
+                          vrows, lane, args.aux);
+            cp_async_rows(lbuf_u, reinterpret_cast<const uint8_t*>(aux + args.f + c + 64),
+                          args.ld_aux * 2, vrows, lane, args.aux);
+            cp_async_commit();
           }
-          tmem_ld_wait();
-          if (row_ok) {
-            float du[32];
+          uint4 ou[8];  // dU in registers; dA goes straight to the staging buffer
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float dh = __uint_as_float(r[i]);
-              const float s = 1.0f / (1.0f + __expf(-a[i]));
-              v[i] = dh * u[i] * s * (1.0f + a[i] * (1.0f - s));
-              du[i] = dh * a[i] * s;
+          for (int half = 0; half < 2; ++half) {
+            uint32_t r[32];
+            tmem_ld32(tbase + c + 32 * half, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 qa = va[4 * half + q], qu = vu[4 * half + q];
+              const float a[8] = {bf16_lo(qa.x), bf16_hi(qa.x), bf16_lo(qa.y), bf16_hi(qa.y),
+                                  bf16_lo(qa.z), bf16_hi(qa.z), bf16_lo(qa.w), bf16_hi(qa.w)};
+              const float u[8] = {bf16_lo(qu.x), bf16_hi(qu.x), bf16_lo(qu.y), bf16_hi(qu.y),
+                                  bf16_lo(qu.z), bf16_hi(qu.z), bf16_lo(qu.w), bf16_hi(qu.w)};
+              float da[8], du[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float dh = __uint_as_float(r[8 * q + i]);
+                const float sg = sigmoid_fast(a[i]);
+                da[i] = dh * u[i] * sg * (1.0f + a[i] * (1.0f - sg));
+                du[i] = dh * a[i] * sg;
+              }
+              *stage_slot(ebuf, lane, 4 * half + q) =
+                  make_uint4(pack_bf16x2(da[0], da[1]), pack_bf16x2(da[2], da[3]),
+                             pack_bf16x2(da[4], da[5]), pack_bf16x2(da[6], da[7]));
+              ou[4 * half + q] = make_uint4(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]),
+                                            pack_bf16x2(du[4], du[5]), pack_bf16x2(du[6], du[7]));
             }
-            __nv_bfloat16* dau = static_cast<__nv_bfloat16*>(args.out) + row * args.ldo;
-            store_bf16x32(dau + col, v);
-            store_bf16x32(dau + args.f + col, du);
           }
+          __syncwarp();
+          stage_to_global(ebuf, reinterpret_cast<uint8_t*>(dau + c), args.ldo * 2, vrows, lane);
+          __syncwarp();
+          store_rows(ebuf, lane, ou, reinterpret_cast<uint8_t*>(dau + args.f + c), args.ldo * 2, vrows);
         }
       }
       tc_fence_before();
