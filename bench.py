@@ -43,6 +43,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-ratio", action="store_true", help="skip the E=128 vs E=8 measurement")
+    ap.add_argument("--no-mxfp8", action="store_true", help="skip the MXFP8 workload measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle sample")
@@ -293,9 +294,9 @@ def run_ours(args):
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     sampler = ClockSampler(local)
 
-    def bench_cfg(c, steps, warmup, with_e2e):
+    def bench_cfg(c, steps, warmup, with_e2e, dtype="bf16"):
         g = make_inputs(c, seed=rank, device=dev)
-        L = MoELayer(c.T, c.d, c.f, c.E, c.k, device=dev)
+        L = MoELayer(c.T, c.d, c.f, c.E, c.k, device=dev, dtype=dtype)
         barrier()
         step_ms, gemm_ms, launches = measure(L, g, steps, warmup, flush, dev)
         barrier()
@@ -316,8 +317,10 @@ def run_ours(args):
     main = bench_cfg(cfg, args.steps, args.warmup, True)
     ratio = None
     if not args.no_ratio and cfg.name == "e8":
-        other = bench_cfg(CONFIGS["e128"], args.steps, args.warmup, False)
-        ratio = other
+        ratio = bench_cfg(CONFIGS["e128"], args.steps, args.warmup, False)
+    mx = None
+    if not args.no_mxfp8 and cfg.name == "e8":
+        mx = bench_cfg(CONFIGS["mxfp8"], args.steps, args.warmup, False, dtype="mxfp8")
     clocks = sampler.stop()
 
     K = args.steps
@@ -357,6 +360,16 @@ def run_ours(args):
         line["e128"] = {"value": r_value, "unit": UNIT, "vs_e8": r_value / value,
                         "grouped_gemm_tflops": CONFIGS["e128"].gemm_flops_fwd_bwd()
                         / (statistics.mean(ratio["gemm_ms"]) / 1e3) / 1e12}
+    if mx is not None:
+        mc = CONFIGS["mxfp8"]
+        line["mxfp8"] = {
+            "workload": f"mxfp8: T={mc.T} d_model={mc.d} d_ff={mc.f} E={mc.E} top_k={mc.k}, "
+                        "uniform random expert ids, E4M3 + E8M0/32 expert GEMM operands",
+            "value": mc.T * K * ws / (mx["total_ms"] / 1e3), "unit": UNIT,
+            "ms_per_step": mx["total_ms"] / K,
+            "expert_calls_tflops": mc.gemm_flops_fwd_bwd() / (statistics.mean(mx["gemm_ms"]) / 1e3) / 1e12,
+            "expert_calls_note": "18*d*f*T*k GEMM FLOPs over the two expert calls, MXFP8 "
+                                 "quantisation kernels included"}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = {k: v for k, v in cpu_baseline(cfg, args.cpu_seconds).items()
                                 if k in ("value", "unit", "cores", "kind", "sample")}

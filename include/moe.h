@@ -43,10 +43,17 @@
  *
  * Routed-row space.  Every expert e owns a segment of rows
  * [offsets[e], offsets[e+1]) in the permuted buffers; segments start at
- * multiples of 32 rows, hold counts[e] real rows in ascending (token, slot)
- * order followed by zero pad rows.  Buffers in this space have
- * M_cap = T*k + 31*E rows (moe_max_rows); rows at and past offsets[E] are
- * never read or written.
+ * multiples of A rows (A = 32, or 128 when dtype is MOE_DTYPE_MXFP8), hold
+ * counts[e] real rows in ascending (token, slot) order followed by zero pad
+ * rows.  Buffers in this space have M_cap rows (moe_max_rows): T*k + 31*E,
+ * or roundup(T*k + 127*E, 128) in MXFP8 mode; rows at and past offsets[E]
+ * are never written.
+ *
+ * MXFP8 mode (shape dtype MOE_DTYPE_MXFP8): the expert GEMMs of
+ * moe_grouped_swiglu_fwd/bwd quantise every operand along its contraction
+ * axis (E4M3 elements, one E8M0 scale per 32) into the workspace and run
+ * block-scaled tcgen05 MMAs with fp32 accumulation; their outputs stay
+ * bf16.  The router, permute and combine are unchanged.
  */
 #ifndef MOE_H_
 #define MOE_H_
@@ -103,7 +110,7 @@ MOE_API moe_status_t moe_destroy(moe_handle_t h);
  * it).  Must be 256-byte aligned. */
 MOE_API moe_status_t moe_workspace_size(moe_handle_t h, const moe_shape_t* s, size_t* bytes);
 
-/* M_cap = T*k + 31*E: rows of every buffer in the routed-row space. */
+/* M_cap: rows of every buffer in the routed-row space (see above). */
 MOE_API moe_status_t moe_max_rows(const moe_shape_t* s, int64_t* rows);
 
 /* Router forward (top-k softmax).
@@ -127,7 +134,8 @@ MOE_API moe_status_t moe_router_topk(moe_handle_t h, const moe_shape_t* s,
 
 /* Routing metadata + rowwise permute, all on the device.
  *   counts[e]   = number of (t,j) with topk_idx[t,j] == e;
- *   offsets[e]  = sum_{e'<e} roundup(counts[e'], 32); offsets[E] = M_pad;
+ *   offsets[e]  = sum_{e'<e} roundup(counts[e'], A); offsets[E] = M_pad
+ *                 (A = 32, or 128 in MXFP8 mode);
  *   row_map[t,j]= offsets[e] + #{(t',j') before (t,j) in t*k+j order with
  *                 the same expert e};
  *   x_perm[row_map[t,j]] = x[t]; pad rows of every segment are zero.

@@ -16,9 +16,7 @@ using moe::aligned;
 using moe::check_shape;
 using moe::DeviceGuard;
 
-int64_t max_rows(const moe_shape_t* s) {
-  return static_cast<int64_t>(s->T) * s->top_k + 31ll * s->n_experts;
-}
+using moe::max_rows;
 
 bool router_on_tensor_cores(int E) { return E > 64; }
 
@@ -58,10 +56,52 @@ RouterBwdWs router_bwd_layout(const moe_context* h, const moe_shape_t* s) {
   return w;
 }
 
+// MXFP8 expert GEMMs: quantised operand copies (E4M3 codes + E8M0 scales)
+// carved from the workspace; the forward and the backward call reuse the
+// same bytes.
+struct MxWs {
+  size_t xq, xs, wguq, wgus, hq, hs, wdq, wds, fwd_total;
+  size_t doq, dos, wdq_c, wds_c, dauq, daus, wguq_c, wgus_c, doq_c, dos_c, hq_c, hs_c, dauq_c,
+      daus_c, xq_c, xs_c, bwd_total;
+};
+
+MxWs mx_layout(const moe_shape_t* s) {
+  const size_t M = static_cast<size_t>(max_rows(s)), d = s->d_model, f = s->d_ff,
+               E = s->n_experts;
+  MxWs w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  w.xq = take(M * d);           w.xs = take(M * d / 32);
+  w.wguq = take(E * 2 * f * d); w.wgus = take(E * 2 * f * d / 32);
+  w.hq = take(M * f);           w.hs = take(M * f / 32);
+  w.wdq = take(E * d * f);      w.wds = take(E * d * f / 32);
+  w.fwd_total = off;
+  off = 0;
+  w.doq = take(M * d);              w.dos = take(M * d / 32);
+  w.wdq_c = take(E * d * f);        w.wds_c = take(E * f * d / 32);
+  w.dauq = take(M * 2 * f);         w.daus = take(M * 2 * f / 32);
+  w.wguq_c = take(E * 2 * f * d);   w.wgus_c = take(E * d * 2 * f / 32);
+  w.doq_c = take(M * d);            w.dos_c = take(d * M / 32);
+  w.hq_c = take(M * f);             w.hs_c = take(f * M / 32);
+  w.dauq_c = take(M * 2 * f);       w.daus_c = take(2 * f * M / 32);
+  w.xq_c = take(M * d);             w.xs_c = take(d * M / 32);
+  w.bwd_total = off;
+  return w;
+}
+
 size_t workspace_bytes(const moe_context* h, const moe_shape_t* s) {
   const int64_t T = s->T, E = s->n_experts;
   size_t need = 0;
   auto upd = [&](size_t v) { need = v > need ? v : need; };
+  if (s->dtype == MOE_DTYPE_MXFP8) {
+    const MxWs w = mx_layout(s);
+    upd(w.fwd_total);
+    upd(w.bwd_total);
+  }
   upd(align256(static_cast<size_t>(T) * E * 4));                                   // router logits
   upd(align256(static_cast<size_t>(moe::n_subchunks(s->T, s->top_k)) * E * 4));    // permute
   upd(router_bwd_layout(h, s).total);                                              // router bwd
@@ -196,7 +236,8 @@ moe_status_t moe_permute(moe_handle_t h, const moe_shape_t* s, const void* x,
   auto* sub = static_cast<int32_t*>(ws);
   h->launches += 4;
   MOE_TRY(cuda_status(moe::launch_route_hist(topk_idx, T, k, E, sub, h->ctl, st)));
-  MOE_TRY(cuda_status(moe::launch_route_scan(sub, moe::n_subchunks(T, k), E, counts, offsets, st)));
+  MOE_TRY(cuda_status(
+      moe::launch_route_scan(sub, moe::n_subchunks(T, k), E, moe::seg_align(s), counts, offsets, st)));
   MOE_TRY(cuda_status(moe::launch_route_rank(topk_idx, T, k, E, sub, offsets, row_map, st)));
   return cuda_status(moe::launch_permute_scatter(static_cast<const __nv_bfloat16*>(x), row_map,
                                                  offsets, counts, T, d, k, E,
@@ -208,9 +249,6 @@ moe_status_t moe_grouped_swiglu_fwd(moe_handle_t h, const moe_shape_t* s, const 
                                     void* au, void* hbuf, void* o_perm, void* ws, size_t ws_bytes,
                                     moe_stream_t stream) {
   MOE_CHECK_HANDLE(h, s);
-  (void)ws;
-  (void)ws_bytes;
-  if (s->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
   if (!all_nonnull(x_perm, offsets, w_gu, w_down, au, hbuf, o_perm)) return MOE_ERR_INVALID_ARG;
   for (const void* p : {x_perm, w_gu, w_down, static_cast<const void*>(au),
                         static_cast<const void*>(hbuf), static_cast<const void*>(o_perm)})
@@ -220,6 +258,24 @@ moe_status_t moe_grouped_swiglu_fwd(moe_handle_t h, const moe_shape_t* s, const 
   auto st = static_cast<cudaStream_t>(stream);
   MOE_GUARD(h);
   moe::GemmCtx c{h->num_sms, h->ctl};
+  if (s->dtype == MOE_DTYPE_MXFP8) {
+    MOE_TRY(check_ws(h, s, ws, ws_bytes));
+    const MxWs L = mx_layout(s);
+    auto* b = static_cast<uint8_t*>(ws);
+    auto bf = [](const void* p) { return static_cast<const __nv_bfloat16*>(p); };
+    auto rows = [&](const void* in, int64_t r, int64_t cols, size_t q, size_t sc) {
+      return cuda_status(moe::launch_mxfp8_quantize(bf(in), r, cols, 1, b + q, b + sc, st));
+    };
+    h->launches += 6;
+    MOE_TRY(rows(x_perm, m_cap, d, L.xq, L.xs));
+    MOE_TRY(rows(w_gu, 2ll * E * f, d, L.wguq, L.wgus));
+    MOE_TRY(moe::gemm_mx_fwd_gate_up(c, {b + L.xq, b + L.xs}, offsets, {b + L.wguq, b + L.wgus}, au,
+                                     hbuf, E, d, f, m_cap, st));
+    MOE_TRY(rows(hbuf, m_cap, f, L.hq, L.hs));
+    MOE_TRY(rows(w_down, static_cast<int64_t>(E) * d, f, L.wdq, L.wds));
+    return moe::gemm_mx_fwd_down(c, {b + L.hq, b + L.hs}, offsets, {b + L.wdq, b + L.wds}, o_perm,
+                                 E, d, f, m_cap, st);
+  }
   h->launches += 2;
   MOE_TRY(moe::gemm_fwd_gate_up(c, x_perm, offsets, w_gu, au, hbuf, E, d, f, m_cap, st));
   return moe::gemm_fwd_down(c, hbuf, offsets, w_down, o_perm, E, d, f, m_cap, st);
@@ -262,9 +318,6 @@ moe_status_t moe_grouped_swiglu_bwd(moe_handle_t h, const moe_shape_t* s, const 
                                     void* dau, void* dx_perm, void* dw_gu, void* dw_down, void* ws,
                                     size_t ws_bytes, moe_stream_t stream) {
   MOE_CHECK_HANDLE(h, s);
-  (void)ws;
-  (void)ws_bytes;
-  if (s->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
   if (!all_nonnull(do_perm, x_perm, au, hbuf, offsets, w_gu, w_down, dau, dx_perm, dw_gu, dw_down))
     return MOE_ERR_INVALID_ARG;
   for (const void* p : {do_perm, x_perm, au, hbuf, w_gu, w_down, static_cast<const void*>(dau),
@@ -276,6 +329,39 @@ moe_status_t moe_grouped_swiglu_bwd(moe_handle_t h, const moe_shape_t* s, const 
   auto st = static_cast<cudaStream_t>(stream);
   MOE_GUARD(h);
   moe::GemmCtx c{h->num_sms, h->ctl};
+  if (s->dtype == MOE_DTYPE_MXFP8) {
+    MOE_TRY(check_ws(h, s, ws, ws_bytes));
+    const MxWs L = mx_layout(s);
+    auto* b = static_cast<uint8_t*>(ws);
+    auto bf = [](const void* p) { return static_cast<const __nv_bfloat16*>(p); };
+    auto rows = [&](const void* in, int64_t r, int64_t cols, size_t q, size_t sc) {
+      return cuda_status(moe::launch_mxfp8_quantize(bf(in), r, cols, 1, b + q, b + sc, st));
+    };
+    auto cols_t = [&](const void* in, int64_t r, int64_t cols, int64_t group, size_t q, size_t sc) {
+      return cuda_status(moe::launch_mxfp8_quantize_cols_t(bf(in), r, cols, group, b + q, b + sc, st));
+    };
+    const int64_t Ed = static_cast<int64_t>(E) * d, E2f = 2ll * E * f;
+    h->launches += 12;
+    // dgrad of the down projection (+ SwiGLU backward): dO along d, W_d along d
+    MOE_TRY(rows(do_perm, m_cap, d, L.doq, L.dos));
+    MOE_TRY(cols_t(w_down, Ed, f, d, L.wdq_c, L.wds_c));
+    MOE_TRY(moe::gemm_mx_dgrad_down_swiglu(c, {b + L.doq, b + L.dos}, offsets,
+                                           {b + L.wdq_c, b + L.wds_c}, au, dau, E, d, f, m_cap, st));
+    // dgrad of gate/up: dAU along 2f, W_gu along 2f
+    MOE_TRY(rows(dau, m_cap, 2ll * f, L.dauq, L.daus));
+    MOE_TRY(cols_t(w_gu, E2f, d, 2ll * f, L.wguq_c, L.wgus_c));
+    MOE_TRY(moe::gemm_mx_dgrad_gate_up(c, {b + L.dauq, b + L.daus}, offsets,
+                                       {b + L.wguq_c, b + L.wgus_c}, dx_perm, E, d, f, m_cap, st));
+    // weight gradients: every operand along tokens
+    MOE_TRY(cols_t(do_perm, m_cap, d, m_cap, L.doq_c, L.dos_c));
+    MOE_TRY(cols_t(hbuf, m_cap, f, m_cap, L.hq_c, L.hs_c));
+    MOE_TRY(moe::gemm_mx_wgrad(c, {b + L.doq_c, b + L.dos_c}, d, {b + L.hq_c, b + L.hs_c}, f,
+                               offsets, dw_down, E, m_cap, st));
+    MOE_TRY(cols_t(dau, m_cap, 2ll * f, m_cap, L.dauq_c, L.daus_c));
+    MOE_TRY(cols_t(x_perm, m_cap, d, m_cap, L.xq_c, L.xs_c));
+    return moe::gemm_mx_wgrad(c, {b + L.dauq_c, b + L.daus_c}, 2 * f, {b + L.xq_c, b + L.xs_c}, d,
+                              offsets, dw_gu, E, m_cap, st);
+  }
   h->launches += 4;
   MOE_TRY(moe::gemm_dgrad_down_swiglu(c, do_perm, offsets, w_down, au, dau, E, d, f, m_cap, st));
   MOE_TRY(moe::gemm_wgrad_down(c, do_perm, hbuf, offsets, dw_down, E, d, f, m_cap, st));

@@ -9,8 +9,12 @@
 
 namespace moe {
 
-// Segments of the routed-row space start at multiples of this many rows.
+// Segments of the routed-row space start at multiples of this many rows
+// (bf16 operands), or of kSegAlignMx rows when the expert GEMMs run in MXFP8
+// (so every 32-token scale block and every 128-token K-block of the weight
+// gradients lies inside one expert).
 constexpr int kSegAlign = 32;
+constexpr int kSegAlignMx = 128;
 
 struct DeviceCtl {
   int status;  // first recorded moe_status_t code, 0 when clean

@@ -30,6 +30,17 @@ struct DeviceGuard {
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+inline int seg_align(const moe_shape_t* s) {
+  return s->dtype == MOE_DTYPE_MXFP8 ? kSegAlignMx : kSegAlign;
+}
+
+// Rows of every buffer in the routed-row space.
+inline int64_t max_rows(const moe_shape_t* s) {
+  const int64_t a = seg_align(s);
+  const int64_t r = static_cast<int64_t>(s->T) * s->top_k + (a - 1) * s->n_experts;
+  return s->dtype == MOE_DTYPE_MXFP8 ? (r + a - 1) / a * a : r;
+}
+
 // Shape checks shared by every entry point (see include/moe.h, "Supported shapes").
 inline moe_status_t check_shape(const moe_shape_t* s) {
   if (s == nullptr) return MOE_ERR_INVALID_ARG;
@@ -39,8 +50,7 @@ inline moe_status_t check_shape(const moe_shape_t* s) {
   if (s->top_k > 8 || s->n_experts > 1024) return MOE_ERR_UNSUPPORTED;
   if (s->d_model % 256 != 0 || s->d_ff % 256 != 0) return MOE_ERR_UNSUPPORTED;
   if (s->dtype != MOE_DTYPE_BF16 && s->dtype != MOE_DTYPE_MXFP8) return MOE_ERR_INVALID_ARG;
-  const int64_t m_cap = static_cast<int64_t>(s->T) * s->top_k + 31ll * s->n_experts;
-  if (m_cap >= (1ll << 31) - 256) return MOE_ERR_UNSUPPORTED;
+  if (max_rows(s) >= (1ll << 31) - 256) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 

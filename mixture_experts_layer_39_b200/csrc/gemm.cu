@@ -33,41 +33,46 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 map over a row-major [outer, inner] matrix.
+// 2-D map over a row-major [outer, inner] matrix (bf16, or E4M3 codes as uint8).
 bool tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-             uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+             uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool u8 = false) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D bf16 map over [groups, outer, inner].
+// 3-D map over [groups, outer, inner].
 bool tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t groups,
-             uint64_t row_bytes, uint64_t group_bytes, uint32_t box_inner, uint32_t box_outer) {
+             uint64_t row_bytes, uint64_t group_bytes, uint32_t box_inner, uint32_t box_outer,
+             bool u8 = false) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {inner, outer, groups};
   cuuint64_t strides[2] = {row_bytes, group_bytes};
   cuuint32_t box[3] = {box_inner, box_outer, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+            const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP>
+template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, bool FP8 = false>
 moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const tc::GemmArgs& args, int grid,
                     cudaStream_t st) {
-  // the SwiGLU-backward epilogue's landing buffers take the fourth stage's room
-  constexpr int STAGES = BN == 256 ? (EPI == tc::EPI_SWIGLU_BWD ? 3 : 4) : 6;
-  auto kern = tc::grouped_gemm_kernel<BN, A_MN, B_MN, EPI, KGROUP, STAGES>;
-  const size_t smem = tc::SmemPlan<BN, STAGES, EPI>::bytes(args.n_groups);
+  // the SwiGLU-backward epilogue's landing buffers take one stage's room;
+  // MXFP8 stages are 32 KB of operands plus 1 KB of scale atoms
+  constexpr int STAGES = FP8 ? (EPI == tc::EPI_SWIGLU_BWD ? 5 : 6)
+                             : (BN == 256 ? (EPI == tc::EPI_SWIGLU_BWD ? 3 : 4) : 6);
+  auto kern = tc::grouped_gemm_kernel<BN, A_MN, B_MN, EPI, KGROUP, STAGES, FP8>;
+  const size_t smem = tc::SmemPlan<BN, STAGES, EPI, FP8>::bytes(args.n_groups);
   static size_t configured = 0;  // largest size this instantiation was opened for
   if (smem > configured) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -278,6 +283,121 @@ moe_status_t gemm_router_dw_partial(const GemmCtx& c, const void* dl_bf16, const
   const int64_t tiles = static_cast<int64_t>(n_groups) * a.m_tiles_fixed * a.n_tiles_n;
   const int grid = static_cast<int>(tiles < c.num_sms ? tiles : c.num_sms);
   return launch<256, true, true, tc::EPI_F32, true>(ta, tb, a, grid, st);
+}
+
+// ------------------------------------------------------------------ MXFP8
+// Operands are E4M3 codes with E8M0 scales stored [MN index][K/32]; tiles are
+// 128 x 128 and each stage carries 128 contraction elements (128 bytes).
+
+moe_status_t gemm_mx_fwd_gate_up(const GemmCtx& c, const MxOperand& x, const int32_t* offsets,
+                                 const MxOperand& w_gu, void* au, void* h, int E, int d, int f,
+                                 int64_t m_cap, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, x.q, d, m_cap, d, 128, 128, true)) return MOE_ERR_CUDA;
+  if (!tmap_3d(&tb, w_gu.q, d, 2ull * f, E, d, 2ull * f * d, 128, 64, true)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  a.n_tiles_n = f / 64;
+  a.k_blocks = d / 128;
+  a.n_groups = E;
+  a.offsets = offsets;
+  a.total_len = static_cast<int>(m_cap);
+  a.m_cap = m_cap;
+  a.out = au;
+  a.ldo = 2ll * f;
+  a.out2 = h;
+  a.ldo2 = f;
+  a.f = f;
+  a.sfa = x.s; a.ld_sfa = d / 32; a.sfa_rows = m_cap;
+  a.sfb = w_gu.s; a.ld_sfb = d / 32; a.sfb_rows = 2ll * f; a.sfb_gstride = 2ll * f * (d / 32);
+  return launch<128, false, false, tc::EPI_SWIGLU_FWD, false, true>(ta, tb, a, c.num_sms, st);
+}
+
+moe_status_t gemm_mx_fwd_down(const GemmCtx& c, const MxOperand& h, const int32_t* offsets,
+                              const MxOperand& w_d, void* o_perm, int E, int d, int f,
+                              int64_t m_cap, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, h.q, f, m_cap, f, 128, 128, true)) return MOE_ERR_CUDA;
+  if (!tmap_3d(&tb, w_d.q, f, d, E, f, 1ull * d * f, 128, 128, true)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  a.n_tiles_n = d / 128;
+  a.k_blocks = f / 128;
+  a.n_groups = E;
+  a.offsets = offsets;
+  a.total_len = static_cast<int>(m_cap);
+  a.m_cap = m_cap;
+  a.out = o_perm;
+  a.ldo = d;
+  a.sfa = h.s; a.ld_sfa = f / 32; a.sfa_rows = m_cap;
+  a.sfb = w_d.s; a.ld_sfb = f / 32; a.sfb_rows = d; a.sfb_gstride = 1ll * d * (f / 32);
+  return launch<128, false, false, tc::EPI_BF16, false, true>(ta, tb, a, c.num_sms, st);
+}
+
+moe_status_t gemm_mx_dgrad_down_swiglu(const GemmCtx& c, const MxOperand& dO, const int32_t* offsets,
+                                       const MxOperand& w_d_col, const void* au, void* dau, int E,
+                                       int d, int f, int64_t m_cap, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, dO.q, d, m_cap, d, 128, 128, true)) return MOE_ERR_CUDA;
+  // W_d[e] is [d (contraction), f (output)]: N-major, quantised along d
+  if (!tmap_3d(&tb, w_d_col.q, f, d, E, f, 1ull * d * f, 128, 128, true)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  a.n_tiles_n = f / 128;
+  a.k_blocks = d / 128;
+  a.n_groups = E;
+  a.offsets = offsets;
+  a.total_len = static_cast<int>(m_cap);
+  a.m_cap = m_cap;
+  a.out = dau;
+  a.ldo = 2ll * f;
+  a.aux = static_cast<const __nv_bfloat16*>(au);
+  a.ld_aux = 2ll * f;
+  a.f = f;
+  a.sfa = dO.s; a.ld_sfa = d / 32; a.sfa_rows = m_cap;
+  a.sfb = w_d_col.s; a.ld_sfb = d / 32; a.sfb_rows = f; a.sfb_gstride = 1ll * f * (d / 32);
+  return launch<128, false, true, tc::EPI_SWIGLU_BWD, false, true>(ta, tb, a, c.num_sms, st);
+}
+
+moe_status_t gemm_mx_dgrad_gate_up(const GemmCtx& c, const MxOperand& dau, const int32_t* offsets,
+                                   const MxOperand& w_gu_col, void* dx_perm, int E, int d, int f,
+                                   int64_t m_cap, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, dau.q, 2ull * f, m_cap, 2ull * f, 128, 128, true)) return MOE_ERR_CUDA;
+  if (!tmap_3d(&tb, w_gu_col.q, d, 2ull * f, E, d, 2ull * f * d, 128, 128, true)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  a.n_tiles_n = d / 128;
+  a.k_blocks = 2 * f / 128;
+  a.n_groups = E;
+  a.offsets = offsets;
+  a.total_len = static_cast<int>(m_cap);
+  a.m_cap = m_cap;
+  a.out = dx_perm;
+  a.ldo = d;
+  a.sfa = dau.s; a.ld_sfa = 2 * f / 32; a.sfa_rows = m_cap;
+  a.sfb = w_gu_col.s; a.ld_sfb = 2 * f / 32; a.sfb_rows = d; a.sfb_gstride = 1ll * d * (2 * f / 32);
+  return launch<128, false, true, tc::EPI_BF16, false, true>(ta, tb, a, c.num_sms, st);
+}
+
+moe_status_t gemm_mx_wgrad(const GemmCtx& c, const MxOperand& a_col, int M, const MxOperand& b_col,
+                           int N, const int32_t* offsets, void* dw, int E, int64_t m_cap,
+                           cudaStream_t st) {
+  // dW[e] (M x N) = A_e^T B_e over e's token rows; both operands are token-major
+  // (MN-major) and quantised along tokens, scales [M or N][m_cap/32]
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, a_col.q, M, m_cap, M, 128, 128, true)) return MOE_ERR_CUDA;
+  if (!tmap_3d(&tb, b_col.q, N, m_cap, 1, N, 1ull * N * m_cap, 128, 128, true)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  a.n_tiles_n = N / 128;
+  a.m_tiles_fixed = M / tc::BM;
+  a.n_groups = E;
+  a.offsets = offsets;
+  a.total_len = static_cast<int>(m_cap);
+  a.out = dw;
+  a.ldo = N;
+  a.out_gstride = static_cast<int64_t>(M) * N;
+  a.sfa = a_col.s; a.ld_sfa = m_cap / 32; a.sfa_rows = M;
+  a.sfb = b_col.s; a.ld_sfb = m_cap / 32; a.sfb_rows = N; a.sfb_gstride = 0;
+  const int64_t tiles = static_cast<int64_t>(E) * a.m_tiles_fixed * a.n_tiles_n;
+  const int grid = static_cast<int>(tiles < c.num_sms ? tiles : c.num_sms);
+  return launch<128, true, true, tc::EPI_BF16, true, true>(ta, tb, a, grid, st);
 }
 
 }  // namespace moe

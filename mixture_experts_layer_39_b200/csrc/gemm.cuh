@@ -10,6 +10,12 @@ struct GemmCtx {
   DeviceCtl* ctl;
 };
 
+// An MXFP8 operand: E4M3 codes and E8M0 scales ([MN index][K/32] bytes).
+struct MxOperand {
+  const uint8_t* q;
+  const uint8_t* s;
+};
+
 moe_status_t gemm_fwd_gate_up(const GemmCtx& c, const void* x_perm, const int32_t* offsets,
                               const void* w_gu, void* au, void* h, int E, int d, int f,
                               int64_t m_cap, cudaStream_t st);
@@ -36,5 +42,21 @@ int router_dw_groups(int num_sms, int T, int d, int E, int* group_len);
 moe_status_t gemm_router_dw_partial(const GemmCtx& c, const void* dl_bf16, const void* x,
                                     float* partial, int T, int d, int E, int n_groups,
                                     int group_len, cudaStream_t st);
+
+moe_status_t gemm_mx_fwd_gate_up(const GemmCtx& c, const MxOperand& x, const int32_t* offsets,
+                                 const MxOperand& w_gu, void* au, void* h, int E, int d, int f,
+                                 int64_t m_cap, cudaStream_t st);
+moe_status_t gemm_mx_fwd_down(const GemmCtx& c, const MxOperand& h, const int32_t* offsets,
+                              const MxOperand& w_d, void* o_perm, int E, int d, int f,
+                              int64_t m_cap, cudaStream_t st);
+moe_status_t gemm_mx_dgrad_down_swiglu(const GemmCtx& c, const MxOperand& dO, const int32_t* offsets,
+                                       const MxOperand& w_d_col, const void* au, void* dau, int E,
+                                       int d, int f, int64_t m_cap, cudaStream_t st);
+moe_status_t gemm_mx_dgrad_gate_up(const GemmCtx& c, const MxOperand& dau, const int32_t* offsets,
+                                   const MxOperand& w_gu_col, void* dx_perm, int E, int d, int f,
+                                   int64_t m_cap, cudaStream_t st);
+moe_status_t gemm_mx_wgrad(const GemmCtx& c, const MxOperand& a_col, int M, const MxOperand& b_col,
+                           int N, const int32_t* offsets, void* dw, int E, int64_t m_cap,
+                           cudaStream_t st);
 
 }  // namespace moe

@@ -24,7 +24,7 @@ cudaError_t launch_softmax_topk(const float* logits_in, const float* bias, const
 // ---- routing metadata + permute
 cudaError_t launch_route_hist(const int32_t* idx, int T, int k, int E, int32_t* sub_counts,
                               DeviceCtl* ctl, cudaStream_t st);
-cudaError_t launch_route_scan(int32_t* sub_counts, int64_t n_sub, int E, int32_t* counts,
+cudaError_t launch_route_scan(int32_t* sub_counts, int64_t n_sub, int E, int align, int32_t* counts,
                               int32_t* offsets, cudaStream_t st);
 cudaError_t launch_route_rank(const int32_t* idx, int T, int k, int E, const int32_t* sub_base,
                               const int32_t* offsets, int32_t* row_map, cudaStream_t st);
@@ -61,5 +61,9 @@ cudaError_t launch_reduce_rows_f32(const float* partial, int n_part, int E, floa
 // ---- MXFP8
 cudaError_t launch_mxfp8_quantize(const __nv_bfloat16* in, int64_t rows, int64_t cols, int axis,
                                   uint8_t* q, uint8_t* scales, cudaStream_t st);
+// Column-wise (32-row blocks) with scales stored [groups][cols][rows_per_group/32].
+cudaError_t launch_mxfp8_quantize_cols_t(const __nv_bfloat16* in, int64_t rows, int64_t cols,
+                                         int64_t rows_per_group, uint8_t* q, uint8_t* scales,
+                                         cudaStream_t st);
 
 }  // namespace moe

@@ -68,9 +68,13 @@ __global__ void mx_rowwise_kernel(const uint4* __restrict__ in, int64_t rows, in
   }
 }
 
-// axis 0: one thread per (32-row block, pair of adjacent columns).
+// axis 0: one thread per (32-row block, pair of adjacent columns).  Scales go
+// to [rows/32, cols] (scale_mode 0) or, for the GEMM operand layout, to
+// [groups, cols, rows_per_group/32] (scale_mode 1: a column's scales along
+// the contraction axis are contiguous inside each group of rows).
 __global__ void mx_colwise_kernel(const uint32_t* __restrict__ in, int64_t rows, int64_t cols,
-                                  uint16_t* __restrict__ q, uint16_t* __restrict__ scales) {
+                                  uint16_t* __restrict__ q, uint8_t* __restrict__ scales,
+                                  int scale_mode, int64_t rows_per_group) {
   const int64_t cpairs = cols / 2;
   const int64_t total = (rows / 32) * cpairs;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
@@ -94,7 +98,15 @@ __global__ void mx_colwise_kernel(const uint32_t* __restrict__ in, int64_t rows,
       const uint16_t hi = e4m3x2(b[r] * i1, 0.f) & 0xFF;
       q[(rb * 32 + r) * cpairs + cp] = static_cast<uint16_t>(lo | (hi << 8));
     }
-    scales[rb * cpairs + cp] = static_cast<uint16_t>((e0 + 127) | ((e1 + 127) << 8));
+    if (scale_mode == 0) {
+      reinterpret_cast<uint16_t*>(scales)[rb * cpairs + cp] =
+          static_cast<uint16_t>((e0 + 127) | ((e1 + 127) << 8));
+    } else {
+      const int64_t bpg = rows_per_group / 32;  // scale blocks per group
+      const int64_t g = rb / bpg, rl = rb - g * bpg;
+      scales[(g * cols + 2 * cp) * bpg + rl] = static_cast<uint8_t>(e0 + 127);
+      scales[(g * cols + 2 * cp + 1) * bpg + rl] = static_cast<uint8_t>(e1 + 127);
+    }
   }
 }
 
@@ -111,9 +123,18 @@ cudaError_t launch_mxfp8_quantize(const __nv_bfloat16* in, int64_t rows, int64_t
     const int64_t total = (rows / 32) * (cols / 2);
     const unsigned grid = static_cast<unsigned>(ceil_div64(total, 256) < 65535 ? ceil_div64(total, 256) : 65535);
     mx_colwise_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(in), rows, cols,
-                                            reinterpret_cast<uint16_t*>(q),
-                                            reinterpret_cast<uint16_t*>(scales));
+                                            reinterpret_cast<uint16_t*>(q), scales, 0, rows);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mxfp8_quantize_cols_t(const __nv_bfloat16* in, int64_t rows, int64_t cols,
+                                         int64_t rows_per_group, uint8_t* q, uint8_t* scales,
+                                         cudaStream_t st) {
+  const int64_t total = (rows / 32) * (cols / 2);
+  const unsigned grid = static_cast<unsigned>(ceil_div64(total, 256) < 65535 ? ceil_div64(total, 256) : 65535);
+  mx_colwise_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(in), rows, cols,
+                                          reinterpret_cast<uint16_t*>(q), scales, 1, rows_per_group);
   return cudaGetLastError();
 }
 

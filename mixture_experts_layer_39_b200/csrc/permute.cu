@@ -55,8 +55,8 @@ __global__ void __launch_bounds__(kWarps * 32)
 // memory), leaving each sub-chunk's base; then the block scans the padded
 // counts into the segment offsets.
 __global__ void __launch_bounds__(1024)
-    route_scan_kernel(int32_t* __restrict__ sub, int64_t n_sub, int E, int32_t* __restrict__ counts,
-                      int32_t* __restrict__ offsets) {
+    route_scan_kernel(int32_t* __restrict__ sub, int64_t n_sub, int E, int align,
+                      int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
   __shared__ int s_tot[1024];
   __shared__ int s_warp[32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(1024)
   __syncthreads();
   const int e = threadIdx.x;
   const int run = e < E ? s_tot[e] : 0;
-  const int padded = e < E ? (run + kSegAlign - 1) / kSegAlign * kSegAlign : 0;
+  const int padded = e < E ? (run + align - 1) / align * align : 0;
   int v = padded;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -342,9 +342,9 @@ cudaError_t launch_route_hist(const int32_t* idx, int T, int k, int E, int32_t* 
   return cudaGetLastError();
 }
 
-cudaError_t launch_route_scan(int32_t* sub_counts, int64_t n_sub, int E, int32_t* counts,
+cudaError_t launch_route_scan(int32_t* sub_counts, int64_t n_sub, int E, int align, int32_t* counts,
                               int32_t* offsets, cudaStream_t st) {
-  route_scan_kernel<<<1, 1024, 0, st>>>(sub_counts, n_sub, E, counts, offsets);
+  route_scan_kernel<<<1, 1024, 0, st>>>(sub_counts, n_sub, E, align, counts, offsets);
   return cudaGetLastError();
 }
 

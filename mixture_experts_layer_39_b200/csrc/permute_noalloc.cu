@@ -78,7 +78,8 @@ extern "C" moe_status_t moe_permute_noalloc(moe_handle_t h, const moe_shape_t* s
   auto st = static_cast<cudaStream_t>(stream);
   h->launches += 4;
   if (moe::launch_route_hist(topk_idx, T, k, E, sub, h->ctl, st) != cudaSuccess) return MOE_ERR_CUDA;
-  if (moe::launch_route_scan(sub, n_sub, E, counts, offsets, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::launch_route_scan(sub, n_sub, E, moe::seg_align(s), counts, offsets, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
   if (moe::launch_route_rank(topk_idx, T, k, E, sub, offsets, row_map, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (moe::launch_permute_scatter(static_cast<const __nv_bfloat16*>(x), row_map, offsets, counts,

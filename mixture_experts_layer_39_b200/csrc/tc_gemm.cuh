@@ -65,6 +65,14 @@ struct GemmArgs {
   int64_t ld_aux;
   int f;  // SwiGLU: width of one half ([A | U] column offset of U)
   DeviceCtl* ctl;
+  // MXFP8 operands: E8M0 scales stored [MN index][K/32] (bytes), B's per group
+  const uint8_t* sfa;
+  int64_t ld_sfa;       // bytes per A row (M index) = K_total / 32
+  int64_t sfa_rows;     // rows of the A scale array (reads are clamped to it)
+  const uint8_t* sfb;
+  int64_t ld_sfb;
+  int64_t sfb_rows;     // rows per group of the B scale array
+  int64_t sfb_gstride;  // bytes between groups of B scales (M-grouped)
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -178,6 +186,50 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
+// Instruction descriptor of kind::mxf8f6f4 (block-scaled): E4M3 A and B, E8M0
+// scales (bit 23), K = 32 per MMA.  The scale-factor ids (bits 4-5 for B,
+// 29-30 for A) select the byte of each 32-bit scale word and are or-ed in
+// per MMA.
+__host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, bool a_mn, bool b_mn) {
+  return ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+         (1u << 23) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}\n"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem),
+      "r"(accumulate)
+      : "memory");
+}
+
+// One 512-byte scale atom (32 rows x 16 bytes, no swizzle: 8-row groups 128 B
+// apart) from shared memory into 4 TMEM columns, copied to all four lane
+// quarters.
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(512u >> 4) << 16;   // leading byte offset (unused at 16 B width)
+  d |= static_cast<uint64_t>(128u >> 4) << 32;   // stride byte offset: 8 rows x 16 B
+  d |= static_cast<uint64_t>(1) << 46;           // descriptor version
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
+}
+
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc) {
+  const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(gsrc) : "memory");
+}
+
+// Arrives on the mbarrier once all prior cp.async of this thread completed
+// (the arrival is counted in the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -235,7 +287,7 @@ __device__ __forceinline__ int group_off(const GemmArgs& a, int g) {
   return v > a.total_len ? a.total_len : v;
 }
 
-template <bool KGROUP>
+template <bool KGROUP, int BKE = BK, int KMMA = 16>
 __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* s_tile_start, int t) {
   Tile tl;
   if constexpr (!KGROUP) {
@@ -264,9 +316,9 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* s_tile
     const int g0 = group_off(a, tl.group), g1 = group_off(a, tl.group + 1);
     const int len = g1 > g0 ? g1 - g0 : 0;
     tl.k_lo = g0;
-    tl.k_blocks = (len + BK - 1) / BK;
-    const int rem = len - (tl.k_blocks - 1) * BK;
-    tl.last_k16 = tl.k_blocks > 0 ? (rem + 15) / 16 : 0;
+    tl.k_blocks = (len + BKE - 1) / BKE;
+    const int rem = len - (tl.k_blocks - 1) * BKE;
+    tl.last_k16 = tl.k_blocks > 0 ? (rem + KMMA - 1) / KMMA : 0;
   }
   return tl;
 }
@@ -354,12 +406,16 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
 }
 
 // ---------------------------------------------------------------- the kernel
-template <int BN, int STAGES, int EPI>
+template <int BN, int STAGES, int EPI, bool FP8 = false>
 struct SmemPlan {
-  static constexpr int kABytes = BM * BK * 2;
-  static constexpr int kBBytes = BN * BK * 2;
+  // one stage holds 128-byte rows: 64 bf16 or 128 fp8 contraction elements
+  static constexpr int kABytes = BM * 128;
+  static constexpr int kBBytes = BN * 128;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kBarOff = STAGES * kStageBytes;                 // 1024-aligned stages
+  // MXFP8: per stage one 512-byte scale atom per 128 rows of A and of B
+  static constexpr int kSfStageBytes = FP8 ? 512 * (1 + BN / 128) : 0;
+  static constexpr int kSfOff = STAGES * kStageBytes;
+  static constexpr int kBarOff = kSfOff + STAGES * kSfStageBytes;      // 1024-aligned stages
   static constexpr int kBarBytes = (2 * STAGES + 5) * 8;               // full, empty, tfull x2, tempty x2, drain
   static constexpr int kMiscOff = kBarOff + kBarBytes;                 // tmem base, abort flag
   static constexpr int kEpiOff = (kMiscOff + 16 + 127) / 128 * 128;    // 4 epilogue warps' buffers
@@ -370,15 +426,22 @@ struct SmemPlan {
   static constexpr int bytes(int n_groups) { return 1024 + kTileOff + 4 * (n_groups + 1); }
 };
 
-template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, int STAGES>
+template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, int STAGES, bool FP8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
   static_assert(BN == 128 || BN == 256, "BN");
   static_assert(!(EPI == EPI_SWIGLU_FWD && B_MN), "SwiGLU forward takes K-major weights");
-  using Plan = SmemPlan<BN, STAGES, EPI>;
-  constexpr uint32_t kTmemCols = 2 * BN;
-  constexpr uint32_t kIdesc = idesc_bf16(BM, BN, A_MN, B_MN);
+  static_assert(!FP8 || BN == 128, "MXFP8 tiles are 128 x 128 (TMEM holds the scales too)");
+  using Plan = SmemPlan<BN, STAGES, EPI, FP8>;
+  // contraction elements per stage, per MMA, per 128-byte MN chunk of an MN-major operand
+  constexpr int BKE = FP8 ? 128 : BK;
+  constexpr int KMMA = FP8 ? 32 : 16;
+  constexpr int CH = FP8 ? 128 : 64;
+  constexpr uint32_t kChunkBytes = BKE * 128;      // one MN chunk of an MN-major stage
+  constexpr uint32_t kSfCols = 4 + 4 * (BN / 128); // TMEM columns of one scale buffer
+  constexpr uint32_t kTmemCols = FP8 ? 512 : 2 * BN;
+  constexpr uint32_t kIdesc = FP8 ? idesc_mxf8(BM, BN, A_MN, B_MN) : idesc_bf16(BM, BN, A_MN, B_MN);
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -400,7 +463,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- set-up: barriers, TMEM, group tile starts
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
+      // MXFP8: the 32 producer lanes' scale copies arrive on the full barrier too
+      mbar_init(full_bar(s), FP8 ? 33 : 1);
       mbar_init(empty_bar(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -459,54 +523,93 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ================================================================ producer
-    if (lane == 0) {
+    // lane 0 issues the TMA tile loads; with MXFP8 all 32 lanes also copy the
+    // stage's scale atoms (cp.async, arriving on the full barrier)
+    if (FP8 || lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // per-stage: a load is in flight / its phase
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-        const Tile tl = decode_tile<KGROUP>(args, s_tile_start, t);
+        const Tile tl = decode_tile<KGROUP, BKE, KMMA>(args, s_tile_start, t);
         for (int kb = 0; kb < tl.k_blocks; ++kb) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, s_abort)) { ok = false; break; }
+          bool got = mbar_wait(empty_bar(stage), phase ^ 1u, s_abort);
+          if constexpr (FP8) got = __all_sync(0xffffffffu, got);
+          if (!got) { ok = false; break; }
           const uint32_t sa = smem_base + stage * Plan::kStageBytes;
           const uint32_t sb = sa + Plan::kABytes;
           const uint32_t fb = full_bar(stage);
-          mbar_arrive_expect_tx(fb, Plan::kStageBytes);
-          armed |= 1u << stage;
-          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-          if constexpr (!KGROUP) {
-            const int k0 = kb * BK;
-            // A: K-major rows of the group's slice
-            tma_load_2d(sa, &tmA, fb, k0, tl.row0);
-            if constexpr (EPI == EPI_SWIGLU_FWD) {
-              const int nh = tl.n_tile * (BN / 2);
-              tma_load_3d(sb, &tmB, fb, k0, nh, tl.group);
-              tma_load_3d(sb + (BN / 2) * BK * 2, &tmB, fb, k0, args.f + nh, tl.group);
-            } else if constexpr (!B_MN) {
-              tma_load_3d(sb, &tmB, fb, k0, tl.n_tile * BN, tl.group);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(fb, Plan::kStageBytes);
+            armed |= 1u << stage;
+            armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+            if constexpr (!KGROUP) {
+              const int k0 = kb * BKE;
+              // A: K-major rows of the group's slice
+              tma_load_2d(sa, &tmA, fb, k0, tl.row0);
+              if constexpr (EPI == EPI_SWIGLU_FWD) {
+                const int nh = tl.n_tile * (BN / 2);
+                tma_load_3d(sb, &tmB, fb, k0, nh, tl.group);
+                tma_load_3d(sb + (BN / 2) * 128, &tmB, fb, k0, args.f + nh, tl.group);
+              } else if constexpr (!B_MN) {
+                tma_load_3d(sb, &tmB, fb, k0, tl.n_tile * BN, tl.group);
+              } else {
+#pragma unroll
+                for (int j = 0; j < BN / CH; ++j)
+                  tma_load_3d(sb + j * kChunkBytes, &tmB, fb, tl.n_tile * BN + CH * j, k0, tl.group);
+              }
             } else {
+              const int kr = tl.k_lo + kb * BKE;
 #pragma unroll
-              for (int j = 0; j < BN / 64; ++j)
-                tma_load_3d(sb + j * (64 * BK * 2), &tmB, fb, tl.n_tile * BN + 64 * j, k0,
-                            tl.group);
+              for (int j = 0; j < BM / CH; ++j)
+                tma_load_2d(sa + j * kChunkBytes, &tmA, fb, tl.row0 + CH * j, kr);
+#pragma unroll
+              for (int j = 0; j < BN / CH; ++j)
+                tma_load_3d(sb + j * kChunkBytes, &tmB, fb, tl.n_tile * BN + CH * j, kr, 0);
             }
-          } else {
-            const int kr = tl.k_lo + kb * BK;
+          }
+          if constexpr (FP8) {
+            // scale atoms: byte (r0*16 + r1*4 + s) = scale of row 32*r1 + r0, K-slice s
+            uint8_t* sfa_s = smem + Plan::kSfOff + stage * Plan::kSfStageBytes;
+            uint8_t* sfb_s = sfa_s + 512;
+            const int64_t kbyte = KGROUP ? (static_cast<int64_t>(tl.k_lo) >> 5) + kb * 4
+                                         : static_cast<int64_t>(kb) * 4;
 #pragma unroll
-            for (int j = 0; j < BM / 64; ++j)
-              tma_load_2d(sa + j * (64 * BK * 2), &tmA, fb, tl.row0 + 64 * j, kr);
+            for (int r1 = 0; r1 < 4; ++r1) {
+              int64_t row = static_cast<int64_t>(tl.row0) + 32 * r1 + lane;
+              row = row < args.sfa_rows ? row : args.sfa_rows - 1;
+              cp_async4(sfa_s + lane * 16 + r1 * 4, args.sfa + row * args.ld_sfa + kbyte);
+            }
+            const int64_t gofs = KGROUP ? 0 : static_cast<int64_t>(tl.group) * args.sfb_gstride;
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              tma_load_3d(sb + j * (64 * BK * 2), &tmB, fb, tl.n_tile * BN + 64 * j, kr, 0);
+            for (int j = 0; j < BN / 128; ++j) {
+#pragma unroll
+              for (int r1 = 0; r1 < 4; ++r1) {
+                const int local = 128 * j + 32 * r1 + lane;  // row of the B tile
+                int64_t n;
+                if constexpr (EPI == EPI_SWIGLU_FWD) {
+                  const int nh = tl.n_tile * (BN / 2);
+                  n = local < BN / 2 ? nh + local : args.f + nh + (local - BN / 2);
+                } else {
+                  n = static_cast<int64_t>(tl.n_tile) * BN + local;
+                }
+                n = n < args.sfb_rows ? n : args.sfb_rows - 1;
+                cp_async4(sfb_s + j * 512 + lane * 16 + r1 * 4,
+                          args.sfb + gofs + n * args.ld_sfb + kbyte);
+              }
+            }
+            cp_async_arrive_noinc(fb);
           }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
       if (!ok) {
-        report(args.ctl, MOE_ERR_TIMEOUT, 1);
-        // let every copy this thread started land before the CTA exits
-        for (int s = 0; s < STAGES; ++s)
-          if (armed & (1u << s)) mbar_wait(full_bar(s), (armed_parity >> s) & 1u, s_abort, false);
+        if (lane == 0) report(args.ctl, MOE_ERR_TIMEOUT, 1);
+        if constexpr (FP8) cp_async_wait_all();
+        // let every copy this warp started land before the CTA exits
+        if (lane == 0)
+          for (int s = 0; s < STAGES; ++s)
+            if (armed & (1u << s)) mbar_wait(full_bar(s), (armed_parity >> s) & 1u, s_abort, false);
       }
     }
   } else if (warp == 1) {
@@ -516,9 +619,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
+      uint32_t sf_buf = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-        const Tile tl = decode_tile<KGROUP>(args, s_tile_start, t);
+        const Tile tl = decode_tile<KGROUP, BKE, KMMA>(args, s_tile_start, t);
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, s_abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -528,12 +632,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sa = smem_base + stage * Plan::kStageBytes;
           const uint32_t sb = sa + Plan::kABytes;
           const int n16 = (kb == tl.k_blocks - 1) ? tl.last_k16 : 4;
+          uint32_t sf_col = 0;
+          if constexpr (FP8) {
+            // the atoms were written by cp.async (generic proxy); order them before
+            // the tensor core's reads, then copy them to TMEM (alternating buffers
+            // after the accumulators)
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            sf_col = tmem_base + 2 * BN + sf_buf * kSfCols;
+            sf_buf ^= 1u;
+            const uint32_t sfa_s = smem_base + Plan::kSfOff + stage * Plan::kSfStageBytes;
+            tmem_cp_sf(sf_col, sfa_s);
+#pragma unroll
+            for (int j = 0; j < BN / 128; ++j) tmem_cp_sf(sf_col + 4 + 4 * j, sfa_s + 512 + 512 * j);
+          }
           for (int kk = 0; kk < n16; ++kk) {
-            const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * 2048, 64 * BK * 2, 1024)
+            // K-major: the next MMA starts 32 bytes further along each 128-byte row;
+            // MN-major: KMMA rows of 128 bytes further
+            const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * KMMA * 128, kChunkBytes, 1024)
                                      : smem_desc_sw128(sa + kk * 32, 16, 1024);
-            const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 64 * BK * 2, 1024)
+            const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * KMMA * 128, kChunkBytes, 1024)
                                      : smem_desc_sw128(sb + kk * 32, 16, 1024);
-            mma_bf16(d_tmem, ad, bd, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            if constexpr (FP8) {
+              const uint32_t sid = static_cast<uint32_t>(kk);
+              mma_mxf8(d_tmem, ad, bd, kIdesc | (sid << 4) | (sid << 29), sf_col | (sid << 30),
+                       (sf_col + 4) | (sid << 30), (kb > 0 || kk > 0) ? 1u : 0u);
+            } else {
+              mma_bf16(d_tmem, ad, bd, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           mma_commit(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -568,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-      const Tile tl = decode_tile<KGROUP>(args, s_tile_start, t);
+      const Tile tl = decode_tile<KGROUP, BKE, KMMA>(args, s_tile_start, t);
       const int vrows = quarter_rows(tl);
       const int64_t row_first = static_cast<int64_t>(tl.row0) + quarter * 32;  // warp's first row
       // SwiGLU backward: the saved [A | U] rows of the first 64 columns are

@@ -16,7 +16,7 @@ from __future__ import annotations
 import torch
 
 from . import ops
-from ._lib import MOE_DTYPE_BF16
+from ._lib import MOE_DTYPE_BF16, MOE_DTYPE_MXFP8
 
 BF16 = torch.bfloat16
 I32 = torch.int32
@@ -25,12 +25,16 @@ F32 = torch.float32
 
 class MoELayer:
     def __init__(self, T, d, f, E, k, device="cuda", renorm=False, keep_logits=False,
-                 handle: ops.Handle | None = None):
+                 handle: ops.Handle | None = None, dtype: str = "bf16"):
+        """dtype: "bf16", or "mxfp8" for E4M3/E8M0 expert GEMM operands (the
+        library then also aligns expert segments to 128 rows)."""
         self.T, self.d, self.f, self.E, self.k = T, d, f, E, k
         dev = torch.device(device)
         self.device = dev
         self.handle = handle if handle is not None else ops.Handle(dev.index or 0)
-        self.shape = ops.make_shape(T, d, f, E, k, MOE_DTYPE_BF16, renorm)
+        self.dtype = dtype
+        code = {"bf16": MOE_DTYPE_BF16, "mxfp8": MOE_DTYPE_MXFP8}[dtype]
+        self.shape = ops.make_shape(T, d, f, E, k, code, renorm)
         M = ops.max_rows(self.shape)
         self.M_cap = M
         z = lambda *s, dt=BF16: torch.empty(*s, dtype=dt, device=dev)
