@@ -44,6 +44,8 @@ def parse_args():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-ratio", action="store_true", help="skip the E=128 vs E=8 measurement")
     ap.add_argument("--no-mxfp8", action="store_true", help="skip the MXFP8 workload measurement")
+    ap.add_argument("--dtype", choices=["bf16", "mxfp8"], default="bf16",
+                    help="expert GEMM operands of the main workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle sample")
@@ -314,7 +316,7 @@ def run_ours(args):
         return out
 
     sampler.start()
-    main = bench_cfg(cfg, args.steps, args.warmup, True)
+    main = bench_cfg(cfg, args.steps, args.warmup, True, dtype=args.dtype)
     ratio = None
     if not args.no_ratio and cfg.name == "e8":
         ratio = bench_cfg(CONFIGS["e128"], args.steps, args.warmup, False)
@@ -336,7 +338,7 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": K,
         "warmup": args.warmup, "ms_per_step": main["total_ms"] / K, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if args.dtype == "bf16" else "mxfp8 (e4m3 + e8m0/32)",
         "data": "synthetic (seeded N(0,1) activations, N(0,1/d) weights, learned-style routing)",
         "config": {"workload": f"{cfg.name}: T={cfg.T} d_model={cfg.d} d_ff={cfg.f} E={cfg.E} "
                                f"top_k={cfg.k} (4x4096 tokens)",

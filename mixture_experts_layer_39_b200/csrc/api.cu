@@ -29,6 +29,13 @@ moe_status_t check_router_shape(const moe_shape_t* s) {
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
+// 256-row CTA-pair tiles for the M-grouped expert GEMMs when the average
+// expert segment spans at least six of them (tail rows then waste < 1/12 of
+// the tiles); shorter segments keep 128-row tiles.
+bool pair_tiles(const moe_shape_t* s) {
+  return static_cast<int64_t>(s->T) * s->top_k >= 1536ll * s->n_experts;
+}
+
 // Router backward workspace layout.
 struct RouterBwdWs {
   size_t dl, db_part, part, total;
@@ -257,7 +264,7 @@ moe_status_t moe_grouped_swiglu_fwd(moe_handle_t h, const moe_shape_t* s, const 
   const int64_t m_cap = max_rows(s);
   auto st = static_cast<cudaStream_t>(stream);
   MOE_GUARD(h);
-  moe::GemmCtx c{h->num_sms, h->ctl};
+  moe::GemmCtx c{h->num_sms, h->ctl, pair_tiles(s)};
   if (s->dtype == MOE_DTYPE_MXFP8) {
     MOE_TRY(check_ws(h, s, ws, ws_bytes));
     const MxWs L = mx_layout(s);
@@ -328,7 +335,7 @@ moe_status_t moe_grouped_swiglu_bwd(moe_handle_t h, const moe_shape_t* s, const 
   const int64_t m_cap = max_rows(s);
   auto st = static_cast<cudaStream_t>(stream);
   MOE_GUARD(h);
-  moe::GemmCtx c{h->num_sms, h->ctl};
+  moe::GemmCtx c{h->num_sms, h->ctl, pair_tiles(s)};
   if (s->dtype == MOE_DTYPE_MXFP8) {
     MOE_TRY(check_ws(h, s, ws, ws_bytes));
     const MxWs L = mx_layout(s);

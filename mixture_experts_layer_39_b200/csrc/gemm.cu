@@ -64,15 +64,17 @@ bool tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, bool FP8 = false>
+template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, bool FP8 = false, bool PAIR = false>
 moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const tc::GemmArgs& args, int grid,
                     cudaStream_t st) {
   // the SwiGLU-backward epilogue's landing buffers take one stage's room;
-  // MXFP8 stages are 32 KB of operands plus 1 KB of scale atoms
-  constexpr int STAGES = FP8 ? (EPI == tc::EPI_SWIGLU_BWD ? 5 : 6)
-                             : (BN == 256 ? (EPI == tc::EPI_SWIGLU_BWD ? 3 : 4) : 6);
-  auto kern = tc::grouped_gemm_kernel<BN, A_MN, B_MN, EPI, KGROUP, STAGES, FP8>;
-  const size_t smem = tc::SmemPlan<BN, STAGES, EPI, FP8>::bytes(args.n_groups);
+  // MXFP8 stages are 32 KB of operands plus 1 KB of scale atoms; a CTA of a
+  // pair holds 32 KB of operands per stage
+  constexpr int STAGES = FP8    ? (EPI == tc::EPI_SWIGLU_BWD ? 5 : 6)
+                         : PAIR ? (EPI == tc::EPI_SWIGLU_BWD ? 5 : 6)
+                                : (BN == 256 ? (EPI == tc::EPI_SWIGLU_BWD ? 3 : 4) : 6);
+  auto kern = tc::grouped_gemm_kernel<BN, A_MN, B_MN, EPI, KGROUP, STAGES, FP8, PAIR>;
+  const size_t smem = tc::SmemPlan<BN, STAGES, EPI, FP8, PAIR>::bytes(args.n_groups);
   static size_t configured = 0;  // largest size this instantiation was opened for
   if (smem > configured) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -81,8 +83,26 @@ moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const tc::GemmAr
     configured = smem;
   }
   if (grid <= 0) return MOE_OK;
-  kern<<<grid, tc::kThreads, smem, st>>>(a, b, args);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  if constexpr (PAIR) {
+    grid &= ~1;  // whole pairs
+    if (grid <= 0) return MOE_OK;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(tc::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a, b, args) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  } else {
+    kern<<<grid, tc::kThreads, smem, st>>>(a, b, args);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
 }
 
 tc::GemmArgs base_args(const GemmCtx& c) {
@@ -111,6 +131,7 @@ moe_status_t gemm_fwd_gate_up(const GemmCtx& c, const void* x_perm, const int32_
   a.out2 = h;
   a.ldo2 = f;
   a.f = f;
+  if (c.pair_m) return launch<256, false, false, tc::EPI_SWIGLU_FWD, false, false, true>(ta, tb, a, c.num_sms, st);
   return launch<256, false, false, tc::EPI_SWIGLU_FWD, false>(ta, tb, a, c.num_sms, st);
 }
 
@@ -119,7 +140,8 @@ moe_status_t gemm_fwd_down(const GemmCtx& c, const void* h, const int32_t* offse
                            cudaStream_t st) {
   CUtensorMap ta, tb;
   if (!tmap_2d(&ta, h, f, m_cap, 2ull * f, 64, 128)) return MOE_ERR_CUDA;
-  if (!tmap_3d(&tb, w_d, f, d, E, 2ull * f, 2ull * d * f, 64, 256)) return MOE_ERR_CUDA;
+  if (!tmap_3d(&tb, w_d, f, d, E, 2ull * f, 2ull * d * f, 64, c.pair_m ? 128 : 256))
+    return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
   a.n_tiles_n = d / 256;
   a.k_blocks = f / tc::BK;
@@ -129,6 +151,7 @@ moe_status_t gemm_fwd_down(const GemmCtx& c, const void* h, const int32_t* offse
   a.m_cap = m_cap;
   a.out = o_perm;
   a.ldo = d;
+  if (c.pair_m) return launch<256, false, false, tc::EPI_BF16, false, false, true>(ta, tb, a, c.num_sms, st);
   return launch<256, false, false, tc::EPI_BF16, false>(ta, tb, a, c.num_sms, st);
 }
 
@@ -151,6 +174,7 @@ moe_status_t gemm_dgrad_down_swiglu(const GemmCtx& c, const void* do_perm, const
   a.aux = static_cast<const __nv_bfloat16*>(au);
   a.ld_aux = 2ll * f;
   a.f = f;
+  if (c.pair_m) return launch<256, false, true, tc::EPI_SWIGLU_BWD, false, false, true>(ta, tb, a, c.num_sms, st);
   return launch<256, false, true, tc::EPI_SWIGLU_BWD, false>(ta, tb, a, c.num_sms, st);
 }
 
@@ -170,6 +194,7 @@ moe_status_t gemm_dgrad_gate_up(const GemmCtx& c, const void* dau, const int32_t
   a.m_cap = m_cap;
   a.out = dx_perm;
   a.ldo = d;
+  if (c.pair_m) return launch<256, false, true, tc::EPI_BF16, false, false, true>(ta, tb, a, c.num_sms, st);
   return launch<256, false, true, tc::EPI_BF16, false>(ta, tb, a, c.num_sms, st);
 }
 
@@ -189,9 +214,10 @@ moe_status_t gemm_wgrad_down(const GemmCtx& c, const void* do_perm, const void* 
   a.out = dw_d;
   a.ldo = f;
   a.out_gstride = static_cast<int64_t>(d) * f;
+  a.m_tiles_fixed = d / (2 * tc::BM);  // CTA pairs: 256-row tiles
   const int64_t tiles = static_cast<int64_t>(E) * a.m_tiles_fixed * a.n_tiles_n;
-  const int grid = static_cast<int>(tiles < c.num_sms ? tiles : c.num_sms);
-  return launch<256, true, true, tc::EPI_BF16, true>(ta, tb, a, grid, st);
+  const int grid = static_cast<int>(2 * tiles < c.num_sms ? 2 * tiles : c.num_sms);
+  return launch<256, true, true, tc::EPI_BF16, true, false, true>(ta, tb, a, grid, st);
 }
 
 moe_status_t gemm_wgrad_gate_up(const GemmCtx& c, const void* dau, const void* x_perm,
@@ -209,9 +235,10 @@ moe_status_t gemm_wgrad_gate_up(const GemmCtx& c, const void* dau, const void* x
   a.out = dw_gu;
   a.ldo = d;
   a.out_gstride = 2ll * f * d;
+  a.m_tiles_fixed = 2 * f / (2 * tc::BM);  // CTA pairs: 256-row tiles
   const int64_t tiles = static_cast<int64_t>(E) * a.m_tiles_fixed * a.n_tiles_n;
-  const int grid = static_cast<int>(tiles < c.num_sms ? tiles : c.num_sms);
-  return launch<256, true, true, tc::EPI_BF16, true>(ta, tb, a, grid, st);
+  const int grid = static_cast<int>(2 * tiles < c.num_sms ? 2 * tiles : c.num_sms);
+  return launch<256, true, true, tc::EPI_BF16, true, false, true>(ta, tb, a, grid, st);
 }
 
 moe_status_t gemm_router_logits(const GemmCtx& c, const void* x, const void* w_r, float* logits,

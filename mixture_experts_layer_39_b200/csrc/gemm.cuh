@@ -8,6 +8,9 @@ namespace moe {
 struct GemmCtx {
   int num_sms;
   DeviceCtl* ctl;
+  // M-grouped bf16 GEMMs run 256-row tiles on CTA pairs (worth it when the
+  // experts' row segments are long compared with a tile)
+  bool pair_m = false;
 };
 
 // An MXFP8 operand: E4M3 codes and E8M0 scales ([MN index][K/32] bytes).

@@ -107,14 +107,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Bounded wait: true when the phase completed; false when another role
 // aborted or the time limit passed (then the abort flag is raised).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity);
+
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          bool honour_abort = true) {
-  if (mbar_try_wait(bar, parity)) return true;
+                                          bool honour_abort = true, bool cluster_scope = false) {
+  auto poll = [&]() {
+    return cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+  };
+  if (poll()) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+      if (poll()) return true;
     if (honour_abort && *abort_flag) return false;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       *abort_flag = 1;
@@ -138,6 +143,83 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
+// ---- CTA-pair (cta_group::2) helpers
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared-memory location in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Arrival on an mbarrier of another CTA of the cluster (release at cluster scope).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+// Bounded wait with cluster-scope acquire (barriers that receive arrivals from the peer CTA).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Tile loads of a CTA pair: the completion bytes go to the mbarrier `bar`,
+// which may live in either CTA of the pair (plain loads, one destination).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrives (once the pair's prior MMAs completed) on the barrier at this
+// shared-memory offset in both CTAs of the pair.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar), "h"(static_cast<uint16_t>(3))
       : "memory");
 }
 
@@ -266,6 +348,7 @@ __device__ __forceinline__ float sigmoid_fast(float z) {
 
 // ---------------------------------------------------------------- scheduling
 struct Tile {
+  int m64;      // M-grouped tail tile with at most 64 rows: issued as M = 64 MMAs
   int group;
   int row0;     // M-grouped: first row of the tile; K-grouped: first row of M
   int row_end;  // M-grouped: end of the group's rows (store mask)
@@ -287,7 +370,7 @@ __device__ __forceinline__ int group_off(const GemmArgs& a, int g) {
   return v > a.total_len ? a.total_len : v;
 }
 
-template <bool KGROUP, int BKE = BK, int KMMA = 16>
+template <bool KGROUP, int BKE = BK, int KMMA = 16, int MT = BM>
 __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* s_tile_start, int t) {
   Tile tl;
   if constexpr (!KGROUP) {
@@ -300,8 +383,9 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* s_tile
     }
     tl.group = lo;
     const int g0 = group_off(a, lo), g1 = group_off(a, lo + 1);
-    tl.row0 = g0 + (mt - s_tile_start[lo]) * BM;
+    tl.row0 = g0 + (mt - s_tile_start[lo]) * MT;
     tl.row_end = g1 > g0 ? g1 : g0;
+    tl.m64 = (tl.row_end - tl.row0) <= 64 ? 1 : 0;
     tl.k_lo = 0;
     tl.k_blocks = a.k_blocks;
     tl.last_k16 = 4;
@@ -311,8 +395,9 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* s_tile
     const int r = t - tl.group * per;
     const int mt = r / a.n_tiles_n;
     tl.n_tile = r - mt * a.n_tiles_n;
-    tl.row0 = mt * BM;
+    tl.row0 = mt * MT;
     tl.row_end = 0;
+    tl.m64 = 0;
     const int g0 = group_off(a, tl.group), g1 = group_off(a, tl.group + 1);
     const int len = g1 > g0 ? g1 - g0 : 0;
     tl.k_lo = g0;
@@ -406,11 +491,12 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
 }
 
 // ---------------------------------------------------------------- the kernel
-template <int BN, int STAGES, int EPI, bool FP8 = false>
+template <int BN, int STAGES, int EPI, bool FP8 = false, bool PAIR = false>
 struct SmemPlan {
-  // one stage holds 128-byte rows: 64 bf16 or 128 fp8 contraction elements
+  // one stage holds 128-byte rows: 64 bf16 or 128 fp8 contraction elements;
+  // in a CTA pair each CTA holds half of B's BN rows
   static constexpr int kABytes = BM * 128;
-  static constexpr int kBBytes = BN * 128;
+  static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * 128;
   static constexpr int kStageBytes = kABytes + kBBytes;
   // MXFP8: per stage one 512-byte scale atom per 128 rows of A and of B
   static constexpr int kSfStageBytes = FP8 ? 512 * (1 + BN / 128) : 0;
@@ -426,14 +512,25 @@ struct SmemPlan {
   static constexpr int bytes(int n_groups) { return 1024 + kTileOff + 4 * (n_groups + 1); }
 };
 
-template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, int STAGES, bool FP8 = false>
+// PAIR: a cluster of two CTAs computes a 256 x BN tile with tcgen05.mma
+// cta_group::2 (M = 256).  Each CTA loads its own 128 rows of A and half of
+// B's BN rows; the even CTA (leader) waits for both CTAs' bytes on its full
+// barrier, issues the MMAs and commits to both CTAs' barriers; each CTA's
+// TMEM holds its own 128 accumulator rows, so the epilogue is unchanged, and
+// the odd CTA's epilogue warps release the accumulator on the leader's
+// barrier.
+template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, int STAGES, bool FP8 = false,
+          bool PAIR = false>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
   static_assert(BN == 128 || BN == 256, "BN");
   static_assert(!(EPI == EPI_SWIGLU_FWD && B_MN), "SwiGLU forward takes K-major weights");
   static_assert(!FP8 || BN == 128, "MXFP8 tiles are 128 x 128 (TMEM holds the scales too)");
-  using Plan = SmemPlan<BN, STAGES, EPI, FP8>;
+  static_assert(!PAIR || (BN == 256 && !FP8), "CTA pairs run bf16 256 x 256 tiles");
+  using Plan = SmemPlan<BN, STAGES, EPI, FP8, PAIR>;
+  constexpr int MT = PAIR ? 2 * BM : BM;  // tile rows (of the pair)
+  constexpr int BNC = PAIR ? BN / 2 : BN;  // B rows held by one CTA
   // contraction elements per stage, per MMA, per 128-byte MN chunk of an MN-major operand
   constexpr int BKE = FP8 ? 128 : BK;
   constexpr int KMMA = FP8 ? 32 : 16;
@@ -441,7 +538,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kChunkBytes = BKE * 128;      // one MN chunk of an MN-major stage
   constexpr uint32_t kSfCols = 4 + 4 * (BN / 128); // TMEM columns of one scale buffer
   constexpr uint32_t kTmemCols = FP8 ? 512 : 2 * BN;
-  constexpr uint32_t kIdesc = FP8 ? idesc_mxf8(BM, BN, A_MN, B_MN) : idesc_bf16(BM, BN, A_MN, B_MN);
+  constexpr uint32_t kIdesc = FP8 ? idesc_mxf8(BM, BN, A_MN, B_MN) : idesc_bf16(MT, BN, A_MN, B_MN);
+  // M-grouped bf16 tail tiles of <= 64 rows run M = 64 MMAs: rows 16q..16q+15
+  // of the accumulator then sit in TMEM lanes 32q..32q+15
+  constexpr bool kTail64 = !FP8 && !KGROUP && !A_MN && !PAIR;
+  constexpr uint32_t kIdesc64 = idesc_bf16(64, BN, A_MN, B_MN);
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -454,6 +555,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t smem_base = smem_u32(smem);
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // CTA within the pair
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int n_units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
   auto empty_bar = [&](int s) { return smem_u32(&bars[STAGES + s]); };
   auto tfull_bar = [&](int b) { return smem_u32(&bars[2 * STAGES + b]); };
@@ -469,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), 4);
+      mbar_init(tempty_bar(b), PAIR ? 8 : 4);  // epilogue warps of one or both CTAs
     }
     mbar_init(drain_bar, 1);
     *s_abort = 0;
@@ -481,18 +585,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmB);
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(s_tmem)),
-                 "r"(kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if constexpr (PAIR) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(s_tmem)),
+                   "r"(kTmemCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(s_tmem)),
+                   "r"(kTmemCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
   }
   int total_tiles;
   if constexpr (!KGROUP) {
     // tiles per group, then an exclusive scan by warp 2
     for (int g = threadIdx.x; g < args.n_groups; g += kThreads) {
       const int len = group_off(args, g + 1) - group_off(args, g);
-      s_tile_start[g + 1] = len > 0 ? (len + BM - 1) / BM : 0;
+      s_tile_start[g + 1] = len > 0 ? (len + MT - 1) / MT : 0;
     }
     __syncthreads();
     if (warp == 2) {
@@ -513,6 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // the peer's barriers are initialised before any use
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
   if constexpr (!KGROUP) {
@@ -530,16 +643,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // per-stage: a load is in flight / its phase
       bool ok = true;
-      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-        const Tile tl = decode_tile<KGROUP, BKE, KMMA>(args, s_tile_start, t);
+      for (int t = unit; t < total_tiles && ok; t += n_units) {
+        const Tile tl = decode_tile<KGROUP, BKE, KMMA, MT>(args, s_tile_start, t);
         for (int kb = 0; kb < tl.k_blocks; ++kb) {
-          bool got = mbar_wait(empty_bar(stage), phase ^ 1u, s_abort);
+          bool got = mbar_wait(empty_bar(stage), phase ^ 1u, s_abort, true, PAIR);
           if constexpr (FP8) got = __all_sync(0xffffffffu, got);
           if (!got) { ok = false; break; }
           const uint32_t sa = smem_base + stage * Plan::kStageBytes;
           const uint32_t sb = sa + Plan::kABytes;
           const uint32_t fb = full_bar(stage);
-          if (lane == 0) {
+          if constexpr (PAIR) {
+            // both CTAs' bytes complete on the leader's full barrier
+            const uint32_t fbl = mapa_shared(fb, 0);
+            if (rank == 0) {
+              mbar_arrive_expect_tx(fb, 2 * Plan::kStageBytes);
+              armed |= 1u << stage;
+              armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+            }
+            if constexpr (!KGROUP) {
+              const int k0 = kb * BKE;
+              tma_load_2d_pair(sa, &tmA, fbl, k0, tl.row0 + BM * static_cast<int>(rank));
+              if constexpr (EPI == EPI_SWIGLU_FWD) {
+                // the pair's B tile is [gate rows | up rows]: CTA 0 loads gate, CTA 1 up
+                const int nh = tl.n_tile * (BN / 2);
+                tma_load_3d_pair(sb, &tmB, fbl, k0, (rank ? args.f : 0) + nh, tl.group);
+              } else if constexpr (!B_MN) {
+                tma_load_3d_pair(sb, &tmB, fbl, k0, tl.n_tile * BN + BNC * static_cast<int>(rank),
+                                 tl.group);
+              } else {
+#pragma unroll
+                for (int j = 0; j < BNC / CH; ++j)
+                  tma_load_3d_pair(sb + j * kChunkBytes, &tmB, fbl,
+                                   tl.n_tile * BN + BNC * static_cast<int>(rank) + CH * j, k0, tl.group);
+              }
+            } else {
+              const int kr = tl.k_lo + kb * BKE;
+#pragma unroll
+              for (int j = 0; j < BM / CH; ++j)
+                tma_load_2d_pair(sa + j * kChunkBytes, &tmA, fbl,
+                                 tl.row0 + BM * static_cast<int>(rank) + CH * j, kr);
+#pragma unroll
+              for (int j = 0; j < BNC / CH; ++j)
+                tma_load_3d_pair(sb + j * kChunkBytes, &tmB, fbl,
+                                 tl.n_tile * BN + BNC * static_cast<int>(rank) + CH * j, kr, 0);
+            }
+          } else if (lane == 0) {
             mbar_arrive_expect_tx(fb, Plan::kStageBytes);
             armed |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -614,20 +762,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
-    if (lane == 0) {
+    if (PAIR && lane == 0 && rank != 0) {
+      // the leader issues the pair's MMAs; wait for them before TMEM is freed
+      mbar_wait(drain_bar, 0, s_abort, false, true);
+    } else if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       uint32_t sf_buf = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-        const Tile tl = decode_tile<KGROUP, BKE, KMMA>(args, s_tile_start, t);
-        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, s_abort)) { ok = false; break; }
+      for (int t = unit; t < total_tiles && ok; t += n_units) {
+        const Tile tl = decode_tile<KGROUP, BKE, KMMA, MT>(args, s_tile_start, t);
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, s_abort, true, PAIR)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < tl.k_blocks; ++kb) {
-          if (!mbar_wait(full_bar(stage), phase, s_abort)) { ok = false; break; }
+          if (!mbar_wait(full_bar(stage), phase, s_abort, true, PAIR)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_base + stage * Plan::kStageBytes;
           const uint32_t sb = sa + Plan::kABytes;
@@ -656,21 +807,24 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t sid = static_cast<uint32_t>(kk);
               mma_mxf8(d_tmem, ad, bd, kIdesc | (sid << 4) | (sid << 29), sf_col | (sid << 30),
                        (sf_col + 4) | (sid << 30), (kb > 0 || kk > 0) ? 1u : 0u);
+            } else if constexpr (PAIR) {
+              mma_bf16_pair(d_tmem, ad, bd, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
             } else {
-              mma_bf16(d_tmem, ad, bd, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+              const uint32_t idesc = (kTail64 && tl.m64) ? kIdesc64 : kIdesc;
+              mma_bf16(d_tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
             }
           }
-          mma_commit(empty_bar(stage));
+          if constexpr (PAIR) mma_commit_pair(empty_bar(stage)); else mma_commit(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        mma_commit(tfull_bar(acc));
+        if constexpr (PAIR) mma_commit_pair(tfull_bar(acc)); else mma_commit(tfull_bar(acc));
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
       if (!ok) report(args.ctl, MOE_ERR_TIMEOUT, 2);
       // all MMAs issued by this thread have finished once the drain barrier flips
-      mma_commit(drain_bar);
-      mbar_wait(drain_bar, 0, s_abort, false);
+      if constexpr (PAIR) mma_commit_pair(drain_bar); else mma_commit(drain_bar);
+      mbar_wait(drain_bar, 0, s_abort, false, PAIR);
     }
   } else {
     // ================================================================ epilogue
@@ -682,20 +836,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t acc_phase = 0;
     // rows of this warp's quarter in the tile, and the row prefetch of a tile's
     // saved [A | U] slice (SwiGLU backward) into L2
+    // tile rows owned by this warp: 32 (16 in an M = 64 tail tile) starting at
+    // quarter_first; quarter_rows = how many of them are real rows
+    auto rows_per_warp = [&](const Tile& tl) -> int { return (kTail64 && tl.m64) ? 16 : 32; };
+    auto quarter_first = [&](const Tile& tl) -> int64_t {
+      return static_cast<int64_t>(tl.row0) + BM * static_cast<int>(rank) + quarter * rows_per_warp(tl);
+    };
     auto quarter_rows = [&](const Tile& tl) -> int {
       if constexpr (KGROUP) {
         return 32;
       } else {
-        const int64_t first = static_cast<int64_t>(tl.row0) + quarter * 32;
+        const int rpw = rows_per_warp(tl);
         int64_t lim = tl.row_end < args.m_cap ? tl.row_end : args.m_cap;
-        const int64_t n = lim - first;
-        return n <= 0 ? 0 : (n >= 32 ? 32 : static_cast<int>(n));
+        const int64_t n = lim - quarter_first(tl);
+        return n <= 0 ? 0 : (n >= rpw ? rpw : static_cast<int>(n));
       }
     };
-    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-      const Tile tl = decode_tile<KGROUP, BKE, KMMA>(args, s_tile_start, t);
+    for (int t = unit; t < total_tiles; t += n_units) {
+      const Tile tl = decode_tile<KGROUP, BKE, KMMA, MT>(args, s_tile_start, t);
       const int vrows = quarter_rows(tl);
-      const int64_t row_first = static_cast<int64_t>(tl.row0) + quarter * 32;  // warp's first row
+      const int64_t row_first = quarter_first(tl);  // warp's first row
       // SwiGLU backward: the saved [A | U] rows of the first 64 columns are
       // requested before waiting for the accumulator, so their latency
       // overlaps the main loop; each later chunk is requested one chunk ahead.
@@ -708,7 +868,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       lane, args.aux);
         cp_async_commit();
       }
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull_bar(acc), acc_phase, s_abort));
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull_bar(acc), acc_phase, s_abort, true, PAIR));
       if (!ok) {
         if constexpr (EPI == EPI_SWIGLU_BWD) cp_async_wait_all();  // own copies land first
         if (lane == 0) report(args.ctl, MOE_ERR_TIMEOUT, 3);
@@ -842,18 +1002,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (lane == 0) {
+        if (PAIR && rank != 0) mbar_arrive_remote(mapa_shared(tempty_bar(acc), 0));
+        else mbar_arrive(tempty_bar(acc));
+      }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // the peer is done with this CTA's TMEM and barriers
   tc_fence_after();
   if (warp == 1) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"(kTmemCols)
-                 : "memory");
+    if constexpr (PAIR) {
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(kTmemCols)
+                   : "memory");
+    } else {
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(kTmemCols)
+                   : "memory");
+    }
   }
 }
 

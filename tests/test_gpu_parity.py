@@ -161,6 +161,8 @@ SMALL_CASES = [
     (333, 256, 256, 64, 8, "renorm"),      # k = 8, renormalised gate weights
     (400, 512, 256, 8, 2, "bias"),         # router bias
     (384, 256, 256, 12, 3, "random"),      # caller-given ids (random routing)
+    (3072, 256, 256, 8, 4, "learned"),     # long segments: 256-row CTA-pair tiles
+    (2080, 512, 256, 1, 1, "learned"),     # one expert, pair tiles with a ragged tail
 ]
 
 
