@@ -207,7 +207,7 @@ def measure(L, g, steps, warmup, flush, dev, with_gemm_events=True):
         if ev: ev[2].record(stream)
         L.experts_bwd(g["w_gu"], g["w_d"])
         if ev: ev[3].record(stream)
-        L.permute_bwd()
+        L.permute_bwd(g["w_r"])
 
     for _ in range(warmup):
         flush.fill_(1)

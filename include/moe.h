@@ -232,14 +232,38 @@ MOE_API moe_status_t moe_permute_bwd(moe_handle_t h, const moe_shape_t* s, const
                              const int32_t* row_map, const float* dx_router, void* dx,
                              moe_stream_t stream);
 
+/* Backward of the permute with the router's share of the input gradient
+ * added in the same pass (the two contributions of step a14/a15 of the
+ * layer: the pages name only the steps, the formulas are the plain
+ * backward of the router and of the permute):
+ *   dL[t]  = as in moe_router_topk_bwd, from d_topk_w, probs and topk_idx
+ *   dx[t]  = bf16( sum_j dx_perm[row_map[t,j]] + dL[t] w_router ), fp32,
+ *            rounded once; dL[t] w_router sums experts in increasing order.
+ * Gives the same bits as moe_router_topk_bwd (with dx_router) followed by
+ * moe_permute_bwd, but never stores dL w_router.  n_experts <= 64 only
+ * (MOE_ERR_UNSUPPORTED otherwise: for n_experts a multiple of 128 that
+ * product runs on the tensor cores inside moe_router_topk_bwd).
+ * In : dx_perm [M_cap,d] bf16, row_map [T,k], d_topk_w [T,k] fp32,
+ *      probs [T,E] fp32, topk_idx [T,k], w_router [E,d] bf16.
+ * Out: dx [T,d] bf16.  All pointers device, caller-owned; no workspace. */
+MOE_API moe_status_t moe_permute_router_bwd(moe_handle_t h, const moe_shape_t* s,
+                                            const void* dx_perm, const int32_t* row_map,
+                                            const float* d_topk_w, const float* probs,
+                                            const int32_t* topk_idx, const void* w_router,
+                                            void* dx, moe_stream_t stream);
+
 /* Router backward (through the selected probabilities; top-k itself has no
  * gradient):
  *   g = d_topk_w, or with MOE_FLAG_RENORM g_j = (dw_j - sum_i dw_i w_i) / S
  *   dp[t, topk_idx[t,j]] = g[t,j], 0 elsewhere
  *   dL = probs * (dp - sum_e probs dp)
- *   dx_router = dL w_router            [T,d] fp32 (fed to moe_permute_bwd)
+ *   dx_router = dL w_router            [T,d] fp32 (fed to moe_permute_bwd),
+ *                                      written when non-NULL
  *   dw_router = bf16(dL^T x)           [E,d]
  *   dbias     = sum_t dL               [E] fp32, written when non-NULL
+ * With dx_router NULL the call leaves the input gradient to
+ * moe_permute_router_bwd (n_experts <= 64), which forms dL w_router on the
+ * fly instead of passing [T,d] fp32 through device memory.
  * In : d_topk_w [T,k] fp32, probs [T,E] fp32, topk_idx [T,k], x [T,d] bf16,
  *      w_router [E,d] bf16. */
 MOE_API moe_status_t moe_router_topk_bwd(moe_handle_t h, const moe_shape_t* s, const float* d_topk_w,

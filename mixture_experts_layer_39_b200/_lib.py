@@ -43,6 +43,7 @@ SIGNATURES = {
     "moe_unpermute_combine_bwd": [P, SP, P, P, P, P, P, P, P, P, P],
     "moe_grouped_swiglu_bwd": [P, SP, P, P, P, P, P, P, P, P, P, P, P, P, c_size_t, P],
     "moe_permute_bwd": [P, SP, P, P, P, P, P],
+    "moe_permute_router_bwd": [P, SP, P, P, P, P, P, P, P, P],
     "moe_router_topk_bwd": [P, SP, P, P, P, P, P, P, P, P, P, c_size_t, P],
     "moe_mxfp8_quantize": [P, P, c_int64, c_int64, c_int, P, P, P],
     "moe_get_status": [P, ctypes.POINTER(c_int)],

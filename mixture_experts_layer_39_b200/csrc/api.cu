@@ -55,8 +55,7 @@ RouterBwdWs router_bwd_layout(const moe_context* h, const moe_shape_t* s) {
   if (router_on_tensor_cores(E)) {
     w.n_part = moe::router_dw_groups(h->num_sms, T, d, E, &w.group_len);
   } else {
-    w.n_part = static_cast<int>(ceil_div64(T, moe::router_dw_small_chunk()));
-    w.group_len = moe::router_dw_small_chunk();
+    w.n_part = moe::router_dw_chunks(h->num_sms, T, d, E, &w.group_len);
   }
   off += align256(static_cast<size_t>(w.n_part) * E * d * 4);
   w.total = off;
@@ -391,14 +390,33 @@ moe_status_t moe_permute_bwd(moe_handle_t h, const moe_shape_t* s, const void* d
                                              static_cast<cudaStream_t>(stream)));
 }
 
+moe_status_t moe_permute_router_bwd(moe_handle_t h, const moe_shape_t* s, const void* dx_perm,
+                                    const int32_t* row_map, const float* d_topk_w,
+                                    const float* probs, const int32_t* topk_idx,
+                                    const void* w_router, void* dx, moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  MOE_TRY(check_router_shape(s));
+  if (s->n_experts > 64) return MOE_ERR_UNSUPPORTED;
+  if (!all_nonnull(dx_perm, row_map, d_topk_w, probs, topk_idx, w_router, dx))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(dx_perm, 16) || !aligned(dx, 16) || !aligned(w_router, 16))
+    return MOE_ERR_INVALID_ARG;
+  MOE_GUARD(h);
+  h->launches += 1;
+  return cuda_status(moe::launch_permute_router_bwd(
+      static_cast<const __nv_bfloat16*>(dx_perm), row_map, d_topk_w, probs, topk_idx,
+      static_cast<const __nv_bfloat16*>(w_router), s->T, s->d_model, s->n_experts, s->top_k,
+      (s->flags & MOE_FLAG_RENORM) != 0, static_cast<__nv_bfloat16*>(dx),
+      static_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_router_topk_bwd(moe_handle_t h, const moe_shape_t* s, const float* d_topk_w,
                                  const float* probs, const int32_t* topk_idx, const void* x,
                                  const void* w_router, float* dx_router, void* dw_router,
                                  float* dbias, void* ws, size_t ws_bytes, moe_stream_t stream) {
   MOE_CHECK_HANDLE(h, s);
   MOE_TRY(check_router_shape(s));
-  if (!all_nonnull(d_topk_w, probs, topk_idx, x, w_router, dx_router, dw_router))
-    return MOE_ERR_INVALID_ARG;
+  if (!all_nonnull(d_topk_w, probs, topk_idx, x, w_router, dw_router)) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(dx_router, 16))
     return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_ws(h, s, ws, ws_bytes));
@@ -412,28 +430,32 @@ moe_status_t moe_router_topk_bwd(moe_handle_t h, const moe_shape_t* s, const flo
   auto* part = reinterpret_cast<float*>(base + L.part);
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
   const auto* wb = static_cast<const __nv_bfloat16*>(w_router);
-  h->launches += router_on_tensor_cores(E) ? 4 : 3;
-  if (dbias != nullptr) h->launches += 1;
+  const bool want_dx = dx_router != nullptr;
   if (!router_on_tensor_cores(E)) {
+    // dL and its per-block db sums (and dX_router when asked), then dW_r
+    // partial rows in one pass over x, then one reduction for dW_r and db
+    h->launches += 3;
     auto* dl = reinterpret_cast<float*>(base + L.dl);
     MOE_TRY(cuda_status(moe::launch_router_bwd_dl(d_topk_w, probs, topk_idx, wb, T, d, E, k, renorm,
-                                                  true, dl, nullptr, dx_router, db_part, L.nblocks,
-                                                  h->ctl, st)));
-    MOE_TRY(cuda_status(moe::launch_router_dw_small(dl, xb, T, d, E, part, st)));
-  } else {
-    auto* dl = reinterpret_cast<__nv_bfloat16*>(base + L.dl);
-    MOE_TRY(cuda_status(moe::launch_router_bwd_dl(d_topk_w, probs, topk_idx, wb, T, d, E, k, renorm,
-                                                  false, nullptr, dl, nullptr, db_part, L.nblocks,
-                                                  h->ctl, st)));
-    moe::GemmCtx c{h->num_sms, h->ctl};
-    MOE_TRY(moe::gemm_router_dx(c, dl, w_router, dx_router, T, d, E, st));
-    MOE_TRY(moe::gemm_router_dw_partial(c, dl, x, part, T, d, E, L.n_part, L.group_len, st));
+                                                  want_dx, dl, nullptr, dx_router, db_part,
+                                                  L.nblocks, h->ctl, st)));
+    MOE_TRY(cuda_status(moe::launch_router_dw(dl, xb, T, d, E, L.n_part, L.group_len, part, st)));
+    return cuda_status(moe::launch_reduce_dw(part, L.n_part, static_cast<int64_t>(E) * d, db_part,
+                                             L.nblocks, E, static_cast<__nv_bfloat16*>(dw_router),
+                                             dbias, st));
   }
-  MOE_TRY(cuda_status(moe::launch_reduce_partials_bf16(part, L.n_part, static_cast<int64_t>(E) * d,
-                                                       static_cast<__nv_bfloat16*>(dw_router), st)));
-  if (dbias != nullptr)
-    MOE_TRY(cuda_status(moe::launch_reduce_rows_f32(db_part, L.nblocks, E, dbias, st)));
-  return MOE_OK;
+  // E a multiple of 128: dL in bf16, both products on the tensor cores
+  h->launches += want_dx ? 4 : 3;
+  auto* dl = reinterpret_cast<__nv_bfloat16*>(base + L.dl);
+  MOE_TRY(cuda_status(moe::launch_router_bwd_dl(d_topk_w, probs, topk_idx, wb, T, d, E, k, renorm,
+                                                false, nullptr, dl, nullptr, db_part, L.nblocks,
+                                                h->ctl, st)));
+  moe::GemmCtx c{h->num_sms, h->ctl};
+  if (want_dx) MOE_TRY(moe::gemm_router_dx(c, dl, w_router, dx_router, T, d, E, st));
+  MOE_TRY(moe::gemm_router_dw_partial(c, dl, x, part, T, d, E, L.n_part, L.group_len, st));
+  return cuda_status(moe::launch_reduce_dw(part, L.n_part, static_cast<int64_t>(E) * d, db_part,
+                                           L.nblocks, E, static_cast<__nv_bfloat16*>(dw_router),
+                                           dbias, st));
 }
 
 moe_status_t moe_mxfp8_quantize(moe_handle_t h, const void* in, int64_t rows, int64_t cols,

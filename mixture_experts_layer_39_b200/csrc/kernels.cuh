@@ -44,19 +44,28 @@ cudaError_t launch_permute_bwd(const __nv_bfloat16* dx_perm, const int32_t* row_
                                cudaStream_t st);
 
 // ---- router backward
+// dX = bf16(unpermute-reduce of dX_perm + dL W_r) in one pass, E <= 64.
+cudaError_t launch_permute_router_bwd(const __nv_bfloat16* dx_perm, const int32_t* row_map,
+                                      const float* dw, const float* probs, const int32_t* idx,
+                                      const __nv_bfloat16* w_r, int T, int d, int E, int k,
+                                      bool renorm, __nv_bfloat16* dx, cudaStream_t st);
 int router_bwd_blocks(int num_sms);
 cudaError_t launch_router_bwd_dl(const float* dw, const float* probs, const int32_t* idx,
                                  const __nv_bfloat16* w_r, int T, int d, int E, int k, bool renorm,
                                  bool fuse_dx, float* dl_f32, __nv_bfloat16* dl_bf16,
                                  float* dx_router, float* db_partial, int nblocks,
                                  DeviceCtl* ctl, cudaStream_t st);
-int router_dw_small_chunk();
-cudaError_t launch_router_dw_small(const float* dl, const __nv_bfloat16* x, int T, int d, int E,
-                                   float* partial, cudaStream_t st);
-cudaError_t launch_reduce_partials_bf16(const float* partial, int n_part, int64_t n,
-                                        __nv_bfloat16* out, cudaStream_t st);
-cudaError_t launch_reduce_rows_f32(const float* partial, int n_part, int E, float* out,
-                                   cudaStream_t st);
+// dW_r partial rows [n_chunks][E*d] over token chunks (E <= 64);
+// router_dw_chunks picks the chunking.
+int router_dw_chunks(int num_sms, int T, int d, int E, int* group_len);
+cudaError_t launch_router_dw(const float* dl, const __nv_bfloat16* x, int T, int d, int E,
+                             int n_chunks, int group_len, float* partial, cudaStream_t st);
+// dw_out = bf16(sum of the n_part partial rows of n_w floats); when db_out
+// is given also db_out = sum of the n_db rows of E floats in db_part.
+cudaError_t launch_reduce_dw(const float* partial, int n_part, int64_t n_w, const float* db_part,
+                             int n_db, int E, __nv_bfloat16* dw_out, float* db_out,
+                             cudaStream_t st);
+
 
 // ---- MXFP8
 cudaError_t launch_mxfp8_quantize(const __nv_bfloat16* in, int64_t rows, int64_t cols, int axis,

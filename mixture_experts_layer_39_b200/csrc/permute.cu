@@ -186,18 +186,6 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
 }
 
-__device__ __forceinline__ void unpack8(const uint4& q, float* f) {
-  f[0] = bf16_lo(q.x); f[1] = bf16_hi(q.x);
-  f[2] = bf16_lo(q.y); f[3] = bf16_hi(q.y);
-  f[4] = bf16_lo(q.z); f[5] = bf16_hi(q.z);
-  f[6] = bf16_lo(q.w); f[7] = bf16_hi(q.w);
-}
-
-__device__ __forceinline__ uint4 pack8(const float* f) {
-  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                    pack_bf16x2(f[6], f[7]));
-}
-
 // y[t] = bf16(sum_j w[t,j] * O[row_map[t,j]]), fp32 in slot order.
 __global__ void __launch_bounds__(kWarps * 32)
     combine_kernel(const uint4* __restrict__ o, const int32_t* __restrict__ row_map,

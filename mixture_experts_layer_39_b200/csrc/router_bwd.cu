@@ -15,6 +15,75 @@ namespace {
 
 constexpr int kWarps = 8;
 
+// dL[t, e] = p[t,e] (dp[t,e] - <p[t], dp[t]>) of one token, held by the warp
+// in the lane layout e = lane + 32 i (i < NPL); dp is the gate-weight
+// gradient scattered to the chosen experts (after the renormalisation's
+// backward when the gate weights were renormalised).  Ids outside [0, E)
+// carry no gradient.  Every lane must call it (one warp reduction).
+template <int NPL>
+__device__ __forceinline__ void token_dlogits(const float* __restrict__ dw,
+                                              const float* __restrict__ probs,
+                                              const int32_t* __restrict__ idx, int64_t t, int E,
+                                              int k, int renorm, int lane, float (&dl)[NPL]) {
+  int id[8];
+  float g[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    id[j] = j < k ? __ldg(idx + t * k + j) : -1;
+    g[j] = j < k ? __ldg(dw + t * k + j) : 0.f;
+    if (id[j] < 0 || id[j] >= E) id[j] = -1;
+  }
+  if (renorm) {
+    float ps[8];
+    float psel_sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      ps[j] = id[j] >= 0 ? __ldg(probs + t * E + id[j]) : 0.f;
+      psel_sum += ps[j];
+    }
+    const float inv = 1.0f / psel_sum;
+    float dot = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) dot += g[j] * ps[j] * inv;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) g[j] = (g[j] - dot) * inv;
+  }
+  float p[NPL], dp[NPL];
+  float pdp = 0.f;
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int e = lane + 32 * i;
+    p[i] = e < E ? __ldg(probs + t * E + e) : 0.f;
+    dp[i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) if (id[j] == e) dp[i] += g[j];
+    pdp += p[i] * dp[i];
+  }
+  pdp = warp_sum(pdp);
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) dl[i] = p[i] * (dp[i] - pdp);
+}
+
+// dX_router[t, 8v .. 8v+7] = sum_e dL[e] W_r[e, 8v .. 8v+7], experts in
+// increasing order from zero (every caller sums in this same order).
+template <int NE>
+__device__ __forceinline__ void router_dx_slice(const uint4* __restrict__ wv, int nvec, int E, int v,
+                                                const float (&dle)[NE], float (&acc)[8]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+#pragma unroll
+  for (int e = 0; e < NE; ++e) {
+    if (e < E) {
+      const uint4 q = wv[static_cast<int64_t>(e) * nvec + v];
+      const float g = dle[e];
+      acc[0] = fmaf(g, bf16_lo(q.x), acc[0]); acc[1] = fmaf(g, bf16_hi(q.x), acc[1]);
+      acc[2] = fmaf(g, bf16_lo(q.y), acc[2]); acc[3] = fmaf(g, bf16_hi(q.y), acc[3]);
+      acc[4] = fmaf(g, bf16_lo(q.z), acc[4]); acc[5] = fmaf(g, bf16_hi(q.z), acc[5]);
+      acc[6] = fmaf(g, bf16_lo(q.w), acc[6]); acc[7] = fmaf(g, bf16_hi(q.w), acc[7]);
+    }
+  }
+}
+
 // NE: compile-time bound on E for the fused dX_router loop (E <= NE <= 32*NPL).
 template <int NPL, bool FUSE_DX, int NE = 32 * NPL>
 __global__ void __launch_bounds__(kWarps * 32)
@@ -41,46 +110,11 @@ __global__ void __launch_bounds__(kWarps * 32)
   const int nvec = d >> 3;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kWarps;
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + warp; t < T; t += stride) {
-    int id[8];
-    float g[8];
-    float psel_sum = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      id[j] = j < k ? __ldg(idx + t * k + j) : -1;
-      g[j] = j < k ? __ldg(dw + t * k + j) : 0.f;
-      if (id[j] < 0 || id[j] >= E) id[j] = -1;
-    }
-    if (renorm) {
-      float ps[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        ps[j] = id[j] >= 0 ? __ldg(probs + t * E + id[j]) : 0.f;
-        psel_sum += ps[j];
-      }
-      const float inv = 1.0f / psel_sum;
-      float dot = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) dot += g[j] * ps[j] * inv;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) g[j] = (g[j] - dot) * inv;
-    }
-    float p[NPL], dp[NPL];
-    float pdp = 0.f;
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      const int e = lane + 32 * i;
-      p[i] = e < E ? __ldg(probs + t * E + e) : 0.f;
-      dp[i] = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) if (id[j] == e) dp[i] += g[j];
-      pdp += p[i] * dp[i];
-    }
-    pdp = warp_sum(pdp);
     float dl[NPL];
+    token_dlogits<NPL>(dw, probs, idx, t, E, k, renorm, lane, dl);
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
       const int e = lane + 32 * i;
-      dl[i] = p[i] * (dp[i] - pdp);
       if (e < E) {
         db[i] += dl[i];
         if (dl_f32 != nullptr) dl_f32[t * E + e] = dl[i];
@@ -97,25 +131,14 @@ __global__ void __launch_bounds__(kWarps * 32)
       float4* out = reinterpret_cast<float4*>(dx_router + t * d);
       for (int v = lane; v < nvec; v += 32) {
         float acc[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-#pragma unroll
-        for (int e = 0; e < NE; ++e) {
-          if (e < E) {
-            const uint4 q = wv[static_cast<int64_t>(e) * nvec + v];
-            const float g = dle[e];
-            acc[0] = fmaf(g, bf16_lo(q.x), acc[0]); acc[1] = fmaf(g, bf16_hi(q.x), acc[1]);
-            acc[2] = fmaf(g, bf16_lo(q.y), acc[2]); acc[3] = fmaf(g, bf16_hi(q.y), acc[3]);
-            acc[4] = fmaf(g, bf16_lo(q.z), acc[4]); acc[5] = fmaf(g, bf16_hi(q.z), acc[5]);
-            acc[6] = fmaf(g, bf16_lo(q.w), acc[6]); acc[7] = fmaf(g, bf16_hi(q.w), acc[7]);
-          }
-        }
+        router_dx_slice<NE>(wv, nvec, E, v, dle, acc);
         out[2 * v] = make_float4(acc[0], acc[1], acc[2], acc[3]);
         out[2 * v + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
       }
     }
   }
   // per-block partial of db (fixed order: warps, then blocks in a later pass)
+  if (db_partial == nullptr) return;
 #pragma unroll
   for (int i = 0; i < NPL; ++i) s_db[warp][lane + 32 * i] = db[i];
   __syncthreads();
@@ -127,109 +150,246 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
 }
 
-// dW_r partial over a chunk of tokens, CUDA cores (E <= 64): each thread
-// owns CPT consecutive columns and all E experts of them; blocks tile
-// (column slice, token chunk).
-constexpr int kChunk = 64;
-constexpr int kDwThreads = 128;
+// dX[t] = bf16(sum_j dX_perm[row_map[t,j]] + dX_router[t]) with dX_router[t]
+// = dL[t] W_r formed on the fly (E <= 64), so that the [T, d] fp32 dX_router
+// never goes through HBM.  dL is recomputed per token from the gate-weight
+// gradient (a few hundred bytes per token).  A warp takes TPW tokens so that
+// every W_r vector it reads (through L1; W_r is at most 256 KB) serves TPW
+// tokens; the dX_perm gathers bypass L1.  KMAX bounds k at compile time.  Sums run in the same order as the
+// two-kernel path (router dX, then unpermute-reduce), so both give the same
+// bits.
+template <int NE, int TPW, int KMAX>
+__global__ void __launch_bounds__(kWarps * 32, 2)
+    permute_router_bwd_kernel(const uint4* __restrict__ dxp, const int32_t* __restrict__ row_map,
+                              const float* __restrict__ dw, const float* __restrict__ probs,
+                              const int32_t* __restrict__ idx, const __nv_bfloat16* __restrict__ w_r,
+                              int T, int d, int E, int k, int renorm, uint4* __restrict__ dx) {
+  constexpr int NPL = (NE + 31) / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t t0 = (static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5)) * TPW;
+  if (t0 >= T) return;
+  const int nvec = d >> 3;
+  float dle[TPW][NE];
+  int rows[TPW][KMAX];
+#pragma unroll
+  for (int h = 0; h < TPW; ++h) {
+    const int64_t t = t0 + h < T ? t0 + h : t0;  // a missing second token repeats the first
+    float dl[NPL];
+    token_dlogits<NPL>(dw, probs, idx, t, E, k, renorm, lane, dl);
+#pragma unroll
+    for (int e = 0; e < NE; ++e) dle[h][e] = __shfl_sync(0xffffffffu, dl[e >> 5], e & 31);
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) rows[h][j] = j < k ? __ldg(row_map + t * k + j) : -1;
+  }
+  const uint4* wv = reinterpret_cast<const uint4*>(w_r);
+  for (int v = lane; v < nvec; v += 32) {
+    uint4 q[TPW][KMAX];
+#pragma unroll
+    for (int h = 0; h < TPW; ++h)
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (rows[h][j] >= 0) q[h][j] = ld_stream16(dxp + static_cast<int64_t>(rows[h][j]) * nvec + v);
+    float r[TPW][8];
+#pragma unroll
+    for (int h = 0; h < TPW; ++h) router_dx_slice<NE>(wv, nvec, E, v, dle[h], r[h]);
+#pragma unroll
+    for (int h = 0; h < TPW; ++h) {
+      if (t0 + h >= T) break;
+      float acc[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        if (rows[h][j] < 0) continue;
+        float f[8];
+        unpack8(q[h][j], f);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] += f[c];
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] += r[h][c];
+      dx[(t0 + h) * nvec + v] = pack8(acc);
+    }
+  }
+}
+
+// dW_r partial sums over a chunk of tokens, CUDA cores (E <= 64).  Each
+// thread owns CPT consecutive columns of x and all E experts of them;
+// blocks tile (column slice, token chunk) and a grid holds about as many
+// blocks as the GPU keeps resident, so every partial row stands for a large
+// chunk of tokens.  dL is staged kDwStage tokens at a time; x is read kDwBatch
+// tokens at a time, all loads issued before the FMAs that use them.  Tokens
+// are accumulated in increasing order.
+constexpr int kDwThreads = 256;
+constexpr int kDwStage = 64;
+constexpr int kDwBatch = 16;
+
+// CPT consecutive bf16 columns, kept packed (two per 32-bit word) until use.
+template <int CPT>
+struct PackedCols {
+  uint32_t w[(CPT + 1) / 2];
+};
+
+template <int CPT>
+__device__ __forceinline__ PackedCols<CPT> load_cols(const __nv_bfloat16* p) {
+  PackedCols<CPT> r;
+  if constexpr (CPT == 4) {
+    const uint2 q = __ldg(reinterpret_cast<const uint2*>(p));
+    r.w[0] = q.x;
+    r.w[1] = q.y;
+  } else if constexpr (CPT == 2) {
+    r.w[0] = __ldg(reinterpret_cast<const unsigned int*>(p));
+  } else {
+    r.w[0] = static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(p)));
+  }
+  return r;
+}
+
+template <int CPT>
+__device__ __forceinline__ float col_value(const PackedCols<CPT>& r, int c) {
+  return (c & 1) ? bf16_hi(r.w[c >> 1]) : bf16_lo(r.w[c >> 1]);
+}
 
 template <int NE, int CPT>
-__global__ void __launch_bounds__(kDwThreads)
-    router_dw_small_kernel(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ x, int T,
-                           int d, int E, float* __restrict__ partial) {
-  __shared__ float s_dl[kChunk * NE];  // 16 KB at NE = 64
-  const int64_t t0 = static_cast<int64_t>(blockIdx.y) * kChunk;
-  const int nt = T - t0 < kChunk ? static_cast<int>(T - t0) : kChunk;
-  for (int i = threadIdx.x; i < nt * E; i += blockDim.x) {
-    const int tt = i / E, e = i - tt * E;
-    s_dl[tt * NE + e] = dl[(t0 + tt) * E + e];
-  }
-  __syncthreads();
+__global__ void __launch_bounds__(kDwThreads, NE <= 8 ? 4 : NE <= 16 ? 3 : 2)
+    router_dw_kernel(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ x, int T,
+                     int d, int E, int group_len, int64_t row_stride, float* __restrict__ partial) {
+  __shared__ float s_dl[kDwStage * NE];  // 16 KB at NE = 64
+  const int64_t g0 = static_cast<int64_t>(blockIdx.y) * group_len;
+  const int64_t g1 = g0 + group_len < T ? g0 + group_len : T;
   const int64_t col = (static_cast<int64_t>(blockIdx.x) * kDwThreads + threadIdx.x) * CPT;
-  if (col >= d) return;
+  const bool active = col < d;
   float acc[NE][CPT];
 #pragma unroll
   for (int e = 0; e < NE; ++e)
 #pragma unroll
     for (int c = 0; c < CPT; ++c) acc[e][c] = 0.f;
-#pragma unroll 4
-  for (int tt = 0; tt < nt; ++tt) {
-    float xv[CPT];
-    const __nv_bfloat16* xr = x + (t0 + tt) * d + col;
-    if constexpr (CPT == 4) {
-      const uint2 q = __ldg(reinterpret_cast<const uint2*>(xr));
-      xv[0] = bf16_lo(q.x); xv[1] = bf16_hi(q.x); xv[2] = bf16_lo(q.y); xv[3] = bf16_hi(q.y);
-    } else if constexpr (CPT == 2) {
-      const uint32_t q = __ldg(reinterpret_cast<const unsigned int*>(xr));
-      xv[0] = bf16_lo(q); xv[1] = bf16_hi(q);
-    } else {
-#pragma unroll
-      for (int c = 0; c < CPT; ++c) xv[c] = __bfloat162float(xr[c]);
+  for (int64_t s0 = g0; s0 < g1; s0 += kDwStage) {
+    const int nt = g1 - s0 < kDwStage ? static_cast<int>(g1 - s0) : kDwStage;
+    __syncthreads();  // the previous stage has been consumed
+    for (int i = threadIdx.x; i < nt * E; i += kDwThreads) {
+      const int tt = i / E, e = i - tt * E;
+      s_dl[tt * NE + e] = __ldg(dl + s0 * E + i);
     }
+    __syncthreads();
+    if (!active) continue;
+    for (int b = 0; b < nt; b += kDwBatch) {
+      const __nv_bfloat16* xr = x + (s0 + b) * d + col;
+      PackedCols<CPT> xq[kDwBatch];
 #pragma unroll
-    for (int e = 0; e < NE; ++e) {
-      if (e < E) {
-        const float g = s_dl[tt * NE + e];
+      for (int u = 0; u < kDwBatch; ++u)
+        if (b + u < nt) xq[u] = load_cols<CPT>(xr + static_cast<int64_t>(u) * d);
 #pragma unroll
-        for (int c = 0; c < CPT; ++c) acc[e][c] = fmaf(g, xv[c], acc[e][c]);
+      for (int u = 0; u < kDwBatch; ++u) {
+        if (b + u < nt) {
+          float xv[CPT];
+#pragma unroll
+          for (int c = 0; c < CPT; ++c) xv[c] = col_value<CPT>(xq[u], c);
+#pragma unroll
+          for (int e = 0; e < NE; ++e) {
+            if (e < E) {
+              const float g = s_dl[(b + u) * NE + e];
+#pragma unroll
+              for (int c = 0; c < CPT; ++c) acc[e][c] = fmaf(g, xv[c], acc[e][c]);
+            }
+          }
+        }
       }
     }
   }
-  float* out = partial + static_cast<int64_t>(blockIdx.y) * E * d;
+  if (!active) return;
+  float* out = partial + static_cast<int64_t>(blockIdx.y) * row_stride;
 #pragma unroll
   for (int e = 0; e < NE; ++e)
-    if (e < E)
+    if (e < E) {
+      if constexpr (CPT == 4) {
+        *reinterpret_cast<float4*>(out + static_cast<int64_t>(e) * d + col) =
+            make_float4(acc[e][0], acc[e][1], acc[e][2], acc[e][3]);
+      } else {
 #pragma unroll
-      for (int c = 0; c < CPT; ++c) out[static_cast<int64_t>(e) * d + col + c] = acc[e][c];
+        for (int c = 0; c < CPT; ++c) out[static_cast<int64_t>(e) * d + col + c] = acc[e][c];
+      }
+    }
 }
 
-// out[i] = bf16(sum_p partial[p][i]).  A block owns 32 float4 columns; its
-// 8 warps take the partials p = w, w+8, ... and are summed in a fixed order.
-__global__ void __launch_bounds__(256)
-    reduce_partials_bf16_kernel(const float4* __restrict__ partial, int n_part, int64_t n4,
-                                __nv_bfloat16* __restrict__ out) {
-  __shared__ float4 s_part[8][32];
+// dw_out[i] = bf16(sum_p partial[p][i]) over n4_w float4 columns, and, when
+// db_out is given, db_out[e] = sum_p db_part[p][e] over n_db rows of E
+// floats (the extra columns of the last blocks).  A block owns 32 columns;
+// its 32 warps take the rows p = w, w+32, ... and their sums are added in
+// warp order, so the result does not depend on timing.
+constexpr int kRedWarps = 32;
+
+__global__ void __launch_bounds__(kRedWarps * 32)
+    reduce_dw_kernel(const float4* __restrict__ partial, int n_part, int64_t stride4, int64_t n4_w,
+                     const float* __restrict__ db_part, int n_db, int E,
+                     __nv_bfloat16* __restrict__ dw_out, float* __restrict__ db_out) {
+  __shared__ float4 s_part[kRedWarps][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t i = static_cast<int64_t>(blockIdx.x) * 32 + lane;
+  const int64_t n4 = n4_w + (db_out != nullptr ? (E + 3) / 4 : 0);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (i < n4) {
+  if (i < n4_w) {
 #pragma unroll 4
-    for (int p = warp; p < n_part; p += 8) {
-      const float4 v = __ldg(partial + static_cast<int64_t>(p) * n4 + i);
+    for (int p = warp; p < n_part; p += kRedWarps) {
+      const float4 v = __ldg(partial + static_cast<int64_t>(p) * stride4 + i);
       acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
+  } else if (i < n4) {
+    const int e0 = static_cast<int>(i - n4_w) * 4;
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int p = warp; p < n_db; p += kRedWarps)
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (e0 + c < E) a[c] += __ldg(db_part + static_cast<int64_t>(p) * E + e0 + c);
+    acc = make_float4(a[0], a[1], a[2], a[3]);
   }
   s_part[warp][lane] = acc;
   __syncthreads();
-  if (warp == 0 && i < n4) {
-    float4 r = s_part[0][lane];
+  if (warp != 0 || i >= n4) return;
+  float4 r = s_part[0][lane];
 #pragma unroll
-    for (int w = 1; w < 8; ++w) {
-      r.x += s_part[w][lane].x; r.y += s_part[w][lane].y;
-      r.z += s_part[w][lane].z; r.w += s_part[w][lane].w;
-    }
-    uint2 packed = make_uint2(pack_bf16x2(r.x, r.y), pack_bf16x2(r.z, r.w));
-    reinterpret_cast<uint2*>(out)[i] = packed;
+  for (int w = 1; w < kRedWarps; ++w) {
+    const float4 u = s_part[w][lane];
+    r.x += u.x; r.y += u.y; r.z += u.z; r.w += u.w;
   }
-}
-
-// out[e] = sum_p partial[p][e]: one warp per e, lanes stride over p, then a
-// fixed-order butterfly.
-__global__ void reduce_rows_f32_kernel(const float* __restrict__ partial, int n_part, int E,
-                                       float* __restrict__ out) {
-  const int lane = threadIdx.x & 31;
-  const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (e >= E) return;
-  float s = 0.f;
-  for (int p = lane; p < n_part; p += 32) s += partial[static_cast<int64_t>(p) * E + e];
-  s = warp_sum(s);
-  if (lane == 0) out[e] = s;
+  if (i < n4_w) {
+    reinterpret_cast<uint2*>(dw_out)[i] = make_uint2(pack_bf16x2(r.x, r.y), pack_bf16x2(r.z, r.w));
+  } else {
+    const int e0 = static_cast<int>(i - n4_w) * 4;
+    const float v[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      if (e0 + c < E) db_out[e0 + c] = v[c];
+  }
 }
 
 }  // namespace
 
+cudaError_t launch_permute_router_bwd(const __nv_bfloat16* dx_perm, const int32_t* row_map,
+                                      const float* dw, const float* probs, const int32_t* idx,
+                                      const __nv_bfloat16* w_r, int T, int d, int E, int k,
+                                      bool renorm, __nv_bfloat16* dx, cudaStream_t st) {
+  auto go = [&](auto kern, int tpw) {
+    const unsigned grid = static_cast<unsigned>(ceil_div64(T, static_cast<int64_t>(kWarps) * tpw));
+    kern<<<grid, kWarps * 32, 0, st>>>(reinterpret_cast<const uint4*>(dx_perm), row_map, dw, probs,
+                                       idx, w_r, T, d, E, k, renorm ? 1 : 0,
+                                       reinterpret_cast<uint4*>(dx));
+    return cudaGetLastError();
+  };
+  if (k <= 4) {
+    if (E <= 8) return go(permute_router_bwd_kernel<8, 2, 4>, 2);
+    if (E <= 16) return go(permute_router_bwd_kernel<16, 2, 4>, 2);
+    if (E <= 32) return go(permute_router_bwd_kernel<32, 1, 4>, 1);
+    if (E <= 64) return go(permute_router_bwd_kernel<64, 1, 4>, 1);
+  } else {
+    if (E <= 16) return go(permute_router_bwd_kernel<16, 1, 8>, 1);
+    if (E <= 32) return go(permute_router_bwd_kernel<32, 1, 8>, 1);
+    if (E <= 64) return go(permute_router_bwd_kernel<64, 1, 8>, 1);
+  }
+  return cudaErrorInvalidValue;
+}
+
 int router_bwd_blocks(int num_sms) { return num_sms * 4; }
-int router_dw_small_chunk() { return kChunk; }
 
 cudaError_t launch_router_bwd_dl(const float* dw, const float* probs, const int32_t* idx,
                                  const __nv_bfloat16* w_r, int T, int d, int E, int k, bool renorm,
@@ -264,34 +424,51 @@ cudaError_t launch_router_bwd_dl(const float* dw, const float* probs, const int3
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_router_dw_small(const float* dl, const __nv_bfloat16* x, int T, int d, int E,
-                                   float* partial, cudaStream_t st) {
-  const unsigned gy = static_cast<unsigned>(ceil_div64(T, kChunk));
+namespace {
+int dw_cols_per_thread(int E) { return E <= 32 ? 2 : 1; }
+int dw_blocks_per_sm(int E) { return E <= 8 ? 4 : E <= 16 ? 3 : 2; }
+}  // namespace
+
+int router_dw_chunks(int num_sms, int T, int d, int E, int* group_len) {
+  const int64_t col_blocks = ceil_div64(d, static_cast<int64_t>(kDwThreads) * dw_cols_per_thread(E));
+  // as many blocks as stay resident, over all column blocks; at least 8
+  // tokens per chunk
+  int64_t n = ceil_div64(static_cast<int64_t>(dw_blocks_per_sm(E)) * num_sms, col_blocks);
+  const int64_t most = ceil_div64(T, 8);
+  if (n > most) n = most;
+  if (n < 1) n = 1;
+  const int64_t len = ceil_div64(T, n);
+  *group_len = static_cast<int>(len);
+  return static_cast<int>(ceil_div64(T, len));
+}
+
+cudaError_t launch_router_dw(const float* dl, const __nv_bfloat16* x, int T, int d, int E,
+                             int n_chunks, int group_len, float* partial, cudaStream_t st) {
+  const int64_t stride = static_cast<int64_t>(E) * d;
   auto go = [&](auto kern, int cpt) {
-    const unsigned gx = static_cast<unsigned>(ceil_div64(d, kDwThreads * cpt));
-    kern<<<dim3(gx, gy), kDwThreads, 0, st>>>(dl, x, T, d, E, partial);
+    const unsigned gx = static_cast<unsigned>(ceil_div64(d, static_cast<int64_t>(kDwThreads) * cpt));
+    kern<<<dim3(gx, static_cast<unsigned>(n_chunks)), kDwThreads, 0, st>>>(dl, x, T, d, E,
+                                                                           group_len, stride,
+                                                                           partial);
     return cudaGetLastError();
   };
-  if (E <= 8) return go(router_dw_small_kernel<8, 4>, 4);
-  if (E <= 16) return go(router_dw_small_kernel<16, 2>, 2);
-  if (E <= 32) return go(router_dw_small_kernel<32, 1>, 1);
-  if (E <= 64) return go(router_dw_small_kernel<64, 1>, 1);
+  if (E <= 8) return go(router_dw_kernel<8, 2>, 2);
+  if (E <= 16) return go(router_dw_kernel<16, 2>, 2);
+  if (E <= 32) return go(router_dw_kernel<32, 2>, 2);
+  if (E <= 64) return go(router_dw_kernel<64, 1>, 1);
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_reduce_partials_bf16(const float* partial, int n_part, int64_t n,
-                                        __nv_bfloat16* out, cudaStream_t st) {
-  const int64_t n4 = n / 4;  // n = E * d, a multiple of 256
-  reduce_partials_bf16_kernel<<<static_cast<unsigned>(ceil_div64(n4, 32)), 256, 0, st>>>(
-      reinterpret_cast<const float4*>(partial), n_part, n4, out);
+cudaError_t launch_reduce_dw(const float* partial, int n_part, int64_t n_w, const float* db_part,
+                             int n_db, int E, __nv_bfloat16* dw_out, float* db_out,
+                             cudaStream_t st) {
+  // n_w = E * d is a multiple of 4 (d is a multiple of 256)
+  const int64_t n4 = n_w / 4 + (db_out != nullptr ? (E + 3) / 4 : 0);
+  reduce_dw_kernel<<<static_cast<unsigned>(ceil_div64(n4, 32)), kRedWarps * 32, 0, st>>>(
+      reinterpret_cast<const float4*>(partial), n_part, n_w / 4, n_w / 4, db_part, n_db, E, dw_out,
+      db_out);
   return cudaGetLastError();
 }
 
-cudaError_t launch_reduce_rows_f32(const float* partial, int n_part, int E, float* out,
-                                   cudaStream_t st) {
-  reduce_rows_f32_kernel<<<static_cast<unsigned>(ceil_div64(E, 8)), 256, 0, st>>>(partial, n_part,
-                                                                                 E, out);
-  return cudaGetLastError();
-}
 
 }  // namespace moe

@@ -7,7 +7,10 @@ in order on the current stream:
   forward : moe_router_topk -> moe_permute -> moe_grouped_swiglu_fwd
             -> moe_unpermute_combine
   backward: moe_unpermute_combine_bwd -> moe_router_topk_bwd
-            -> moe_grouped_swiglu_bwd -> moe_permute_bwd
+            -> moe_grouped_swiglu_bwd -> moe_permute_router_bwd  (E <= 64)
+            or, for E a multiple of 128 (router products on the tensor
+            cores), moe_router_topk_bwd writes dX_router and
+            moe_permute_bwd adds it.
 
 Nothing in a step copies to the host or synchronises.
 """
@@ -25,9 +28,13 @@ F32 = torch.float32
 
 class MoELayer:
     def __init__(self, T, d, f, E, k, device="cuda", renorm=False, keep_logits=False,
-                 handle: ops.Handle | None = None, dtype: str = "bf16"):
+                 handle: ops.Handle | None = None, dtype: str = "bf16",
+                 fuse_router_dx: bool | None = None):
         """dtype: "bf16", or "mxfp8" for E4M3/E8M0 expert GEMM operands (the
-        library then also aligns expert segments to 128 rows)."""
+        library then also aligns expert segments to 128 rows).
+        fuse_router_dx: add the router's input gradient inside the permute
+        backward (default, and only possible, for E <= 64); False keeps the
+        separate [T, d] fp32 dX_router buffer."""
         self.T, self.d, self.f, self.E, self.k = T, d, f, E, k
         dev = torch.device(device)
         self.device = dev
@@ -51,7 +58,13 @@ class MoELayer:
         self.do_perm, self.dw = z(M, d), z(T, k, dt=F32)
         self.dau, self.dx_perm = z(M, 2 * f), z(M, d)
         self.dw_gu, self.dw_d = z(E, 2 * f, d), z(E, d, f)
-        self.dx_router, self.dw_r = z(T, d, dt=F32), z(E, d)
+        if fuse_router_dx is None:
+            fuse_router_dx = E <= 64
+        if fuse_router_dx and E > 64:
+            raise ValueError("the fused router input gradient needs E <= 64")
+        self.fuse_router_dx = fuse_router_dx
+        self.dx_router = None if fuse_router_dx else z(T, d, dt=F32)
+        self.dw_r = z(E, d)
         self.db = z(E, dt=F32)
         self.dx = z(T, d)
 
@@ -94,15 +107,21 @@ class MoELayer:
                                    self.h, self.offsets, w_gu, w_d, self.dau, self.dx_perm,
                                    self.dw_gu, self.dw_d, self.ws, stream)
 
-    def permute_bwd(self, stream=None):
-        ops.moe_permute_bwd(self.handle, self.shape, self.dx_perm, self.row_map, self.dx_router,
-                            self.dx, stream)
+    def permute_bwd(self, w_r=None, stream=None):
+        if self.fuse_router_dx:
+            if w_r is None:
+                raise ValueError("the fused permute backward needs w_r")
+            ops.moe_permute_router_bwd(self.handle, self.shape, self.dx_perm, self.row_map,
+                                       self.dw, self.probs, self.idx, w_r, self.dx, stream)
+        else:
+            ops.moe_permute_bwd(self.handle, self.shape, self.dx_perm, self.row_map,
+                                self.dx_router, self.dx, stream)
 
     def backward(self, dy, x, w_r, w_gu, w_d, stream=None):
         self.combine_bwd(dy, stream)
         self.router_bwd(x, w_r, stream)
         self.experts_bwd(w_gu, w_d, stream)
-        self.permute_bwd(stream)
+        self.permute_bwd(w_r, stream)
         return self.dx
 
     def step(self, x, w_r, w_gu, w_d, dy, bias=None, route=None, stream=None):

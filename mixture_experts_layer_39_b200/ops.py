@@ -137,6 +137,12 @@ def moe_permute_bwd(h, shape, dx_perm, row_map, dx_router, dx, stream=None):
           _ptr(dx_router), _ptr(dx), _stream(stream))
 
 
+def moe_permute_router_bwd(h, shape, dx_perm, row_map, d_topk_w, probs, topk_idx, w_router, dx,
+                           stream=None):
+    _call("moe_permute_router_bwd", h.ptr, ctypes.byref(shape), _ptr(dx_perm), _ptr(row_map),
+          _ptr(d_topk_w), _ptr(probs), _ptr(topk_idx), _ptr(w_router), _ptr(dx), _stream(stream))
+
+
 def moe_router_topk_bwd(h, shape, d_topk_w, probs, topk_idx, x, w_router, dx_router, dw_router,
                         dbias, ws, stream=None):
     _call("moe_router_topk_bwd", h.ptr, ctypes.byref(shape), _ptr(d_topk_w), _ptr(probs),

@@ -24,8 +24,9 @@ def _to(inp, dev):
     return {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
 
 
-def _run(cfg, inp_dev, renorm=False):
-    L = MoELayer(cfg.T, cfg.d, cfg.f, cfg.E, cfg.k, device="cuda", renorm=renorm, keep_logits=True)
+def _run(cfg, inp_dev, renorm=False, fuse_router_dx=None):
+    L = MoELayer(cfg.T, cfg.d, cfg.f, cfg.E, cfg.k, device="cuda", renorm=renorm, keep_logits=True,
+                 fuse_router_dx=fuse_router_dx)
     g = inp_dev
     L.step(g["x"], g["w_r"], g["w_gu"], g["w_d"], g["dy"], g["bias"], g["route"])
     torch.cuda.synchronize()
@@ -117,12 +118,15 @@ def _check_full(cfg, inp, L, renorm=False):
 
     # router backward on the GPU's d(gate weights)
     rb = R.router_bwd(np64(L.dw), probs, idx, x, w_r, renorm)
-    assert_close("dX_router", np64(L.dx_router), rb["dx_router"], 1e-2)
+    if L.dx_router is not None:
+        assert_close("dX_router", np64(L.dx_router), rb["dx_router"], 1e-2)
     assert_close("dW_r", np64(L.dw_r), rb["dw_r"])
     assert_close("db", np64(L.db), rb["db"], 1e-3)
 
-    # permute backward
-    assert_close("dx", np64(L.dx), R.permute_bwd(dxp, rm, np64(L.dx_router)))
+    # permute backward (with the router's input gradient added in the same
+    # kernel when the layer fuses them)
+    dxr = np64(L.dx_router) if L.dx_router is not None else rb["dx_router"]
+    assert_close("dx", np64(L.dx), R.permute_bwd(dxp, rm, dxr))
 
 
 def test_tiny_workload_every_stage(cuda_ok):
@@ -163,6 +167,8 @@ SMALL_CASES = [
     (384, 256, 256, 12, 3, "random"),      # caller-given ids (random routing)
     (3072, 256, 256, 8, 4, "learned"),     # long segments: 256-row CTA-pair tiles
     (2080, 512, 256, 1, 1, "learned"),     # one expert, pair tiles with a ragged tail
+    (500, 768, 256, 7, 2, "renorm"),       # odd E, d not a multiple of 512
+    (257, 256, 256, 13, 5, "bias"),        # second expert tile of the router partly empty
 ]
 
 
@@ -179,6 +185,33 @@ def test_small_shapes_every_stage(cuda_ok, case):
     _check_full(cfg, inp, L, renorm=(mode == "renorm"))
     if mode == "skewed":
         assert (np64(L.counts) == 0).any()
+
+
+FUSION_CASES = [
+    # T, d, f, E, k, mode
+    (4097, 256, 256, 8, 4, "learned"),   # odd T: the last warp has one token
+    (300, 768, 256, 13, 5, "renorm"),    # k > 4, renormalised gate weights
+    (333, 256, 256, 64, 8, "learned"),   # the largest E of the fused path
+    (130, 256, 256, 1, 1, "learned"),    # one expert
+]
+
+
+@pytest.mark.parametrize("case", FUSION_CASES, ids=lambda c: "T%d_d%d_f%d_E%d_k%d_%s" % c)
+def test_fused_router_dx_same_bits(cuda_ok, case):
+    """moe_permute_router_bwd forms dL W_r inside the unpermute-reduce; it
+    must give exactly the bits of moe_router_topk_bwd (dX_router written)
+    followed by moe_permute_bwd on the same inputs."""
+    T, d, f, E, k, mode = case
+    cfg = custom_config(T, d, f, E, k)
+    inp = _to(make_inputs(cfg, seed=T + k, device="cpu"), "cuda")
+    renorm = mode == "renorm"
+    fused = _run(cfg, inp, renorm=renorm, fuse_router_dx=True)
+    split = _run(cfg, inp, renorm=renorm, fuse_router_dx=False)
+    assert fused.dx_router is None and split.dx_router is not None
+    Mp = int(split.offsets[-1])  # rows past the last segment are never written
+    assert torch.equal(fused.dx_perm[:Mp], split.dx_perm[:Mp])
+    assert torch.equal(fused.dx, split.dx)
+    assert torch.equal(fused.dw_r, split.dw_r)
 
 
 # ---------------------------------------------------------------- full sizes
@@ -266,7 +299,14 @@ def test_full_size_sampled(cuda_ok, name):
                        for i, t in enumerate(toks)])
     assert_close("d gate weights (sampled)", np64(L.dw[toks]), dw_ref, 1e-4)
     dxp_rows = {int(r): np64(L.dx_perm[int(r)]) for r in np.unique(rows)}
-    dxr = np64(L.dx_router[toks])
+    # router backward: dL from the GPU's gate-weight gradient, sampled rows
+    rb_rows = R.router_bwd(np64(L.dw[toks]), np64(L.probs[toks]), idx[toks], np64(inp["x"][toks]),
+                           np64(inp["w_r"]))
+    if L.dx_router is not None:
+        dxr = np64(L.dx_router[toks])
+        assert_close("dX_router (sampled)", dxr, rb_rows["dx_router"], 1e-2)
+    else:
+        dxr = rb_rows["dx_router"]
     dx_ref = np.stack([R.bf16_round(sum(dxp_rows[int(rm[t, j])] for j in range(k)) + dxr[i])
                        for i, t in enumerate(toks)])
     assert_close("dx (sampled)", np64(L.dx[toks]), dx_ref)
@@ -279,10 +319,6 @@ def test_full_size_sampled(cuda_ok, name):
     for e in sorted(pick):
         _seg_check(L, inp, e, off, cnt)
 
-    # router backward: dL from the GPU's gate-weight gradient, sampled rows
-    rb_rows = R.router_bwd(np64(L.dw[toks]), np64(L.probs[toks]), idx[toks], np64(inp["x"][toks]),
-                           np64(inp["w_r"]))
-    assert_close("dX_router (sampled)", dxr, rb_rows["dx_router"], 1e-2)
 
 
 def test_mxfp8_quantize_matches_oracle(cuda_ok):
