@@ -53,10 +53,8 @@ def parse_args():
 
 
 def dist_env():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return ws, rank, local
+    from mixture_experts_layer_39_b200.replicas import world
+    return world()
 
 
 def load_peaks():
@@ -284,11 +282,8 @@ def run_ours(args):
                                 device_id=dev)
 
     def max_over_ranks(v):
-        if ws == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        from mixture_experts_layer_39_b200.replicas import max_over_ranks as mor
+        return mor(v, dev)
 
     def barrier():
         if ws > 1:

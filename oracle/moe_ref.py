@@ -279,11 +279,12 @@ def expert_ffn_bwd(dO, x_perm, AU, H, offsets, counts, w_gu, w_d,
     return {"dAU": dAU, "dX_perm": dX, "dW_gu": dW_gu, "dW_d": dW_d}
 
 
-def router_bwd(dw, probs, idx, x, w_r, renorm=False, rnd=bf16_round):
+def router_bwd(dw, probs, idx, x, w_r, renorm=False, rnd=bf16_round, dprob_aux=None):
     """Gradient through the selected probabilities (top-k itself is
     piecewise constant).
         renorm: w_j = p_j / S, S = sum_j p_j  =>  g_j = (dw_j - sum_i dw_i w_i) / S
         dp[t, idx[t, j]] = g[t, j], zero elsewhere
+        dp[t, e] += dprob_aux[e]          (load-balancing loss, when given)
         dL = p * (dp - sum_e p dp)                   softmax backward
         dX_router = dL W_r     (kept unrounded; added into dX before rounding)
         dW_r = bf16(dL^T x),  db = sum_t dL
@@ -300,11 +301,52 @@ def router_bwd(dw, probs, idx, x, w_r, renorm=False, rnd=bf16_round):
         g = (dw - np.sum(dw * wv, axis=1, keepdims=True)) / S
     dp = np.zeros((T, E), F64)
     np.put_along_axis(dp, idx, g, axis=1)
+    if dprob_aux is not None:
+        dp = dp + np.asarray(dprob_aux, F64)[None, :]
     dL = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
     dx_router = dL @ np.asarray(w_r, F64)
     dw_r = _r(rnd)(dL.T @ np.asarray(x, F64))
     db = dL.sum(axis=0)
     return {"dL": dL, "dx_router": dx_router, "dw_r": dw_r, "db": db}
+
+
+# --------------------------------------------------------------------------
+# Load balancing.  The pages say that every engineered MoE framework adds a
+# load-balancing auxiliary loss (or a capacity limit) so that a few hot
+# experts do not take most tokens, that its weight should start small
+# (e.g. 0.001) and be tuned from the spread of expert load (discosf.com
+# article on Olmo-core 3, sections 2.2 and 4.3), and that the v2 router
+# balances load over the global batch (Olmo-core 3 introduction page,
+# meetcoding.cn, section 4 "production-friendly details").  They give no
+# formula; the reading here is the Switch-Transformer loss over the k routed
+# slots, with the statistics kept as sums so that they can be added over
+# micro-batches and ranks before the loss is formed.
+
+def router_load_stats(probs, counts):
+    """Per-expert statistics of one batch:
+        n[e]    = counts[e]          routed (token, slot) pairs of expert e
+        psum[e] = sum_t p[t, e]      router probability mass of expert e
+    Returned as one float64 vector [n | psum] of length 2E."""
+    p = np.asarray(probs, F64)
+    return np.concatenate([np.asarray(counts, F64), p.sum(axis=0)])
+
+
+def router_aux_loss(stats, n_tokens, k, alpha):
+    """Load-balancing loss from (possibly summed) statistics [n | psum]:
+        f_e = n[e] / (n_tokens k)      share of the routed slots
+        P_e = psum[e] / n_tokens       mean router probability
+        loss = alpha E sum_e f_e P_e
+    f_e is piecewise constant in the router logits, so the gradient reaches
+    the probabilities only:  d loss / d p[t, e] = alpha E f_e / n_tokens, the
+    same for every token (returned as the per-expert vector `dprob`)."""
+    stats = np.asarray(stats, F64)
+    E = stats.size // 2
+    n, psum = stats[:E], stats[E:]
+    f = n / (n_tokens * k)
+    P = psum / n_tokens
+    loss = alpha * E * float(np.sum(f * P))
+    dprob = alpha * E * f / n_tokens
+    return loss, dprob
 
 
 def permute_bwd(dX_perm, row_map, dx_router=None, rnd=bf16_round):
