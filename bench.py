@@ -44,6 +44,8 @@ def parse_args():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-ratio", action="store_true", help="skip the E=128 vs E=8 measurement")
     ap.add_argument("--no-mxfp8", action="store_true", help="skip the MXFP8 workload measurement")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the layer variants (load-balancing loss, ...) on the main workload")
     ap.add_argument("--dtype", choices=["bf16", "mxfp8"], default="bf16",
                     help="expert GEMM operands of the main workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -294,9 +296,9 @@ def run_ours(args):
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     sampler = ClockSampler(local)
 
-    def bench_cfg(c, steps, warmup, with_e2e, dtype="bf16"):
+    def bench_cfg(c, steps, warmup, with_e2e, dtype="bf16", **layer_kw):
         g = make_inputs(c, seed=rank, device=dev)
-        L = MoELayer(c.T, c.d, c.f, c.E, c.k, device=dev, dtype=dtype)
+        L = MoELayer(c.T, c.d, c.f, c.E, c.k, device=dev, dtype=dtype, **layer_kw)
         barrier()
         step_ms, gemm_ms, launches = measure(L, g, steps, warmup, flush, dev)
         barrier()
@@ -315,6 +317,10 @@ def run_ours(args):
 
     sampler.start()
     main = bench_cfg(cfg, args.steps, args.warmup, True, dtype=args.dtype)
+    # variants right after the main workload, on the same warm GPU
+    variants = {}
+    if not args.no_variants and args.dtype == "bf16":
+        variants["aux_loss"] = bench_cfg(cfg, args.steps, args.warmup, False, aux_alpha=0.01)
     ratio = None
     if not args.no_ratio and cfg.name == "e8":
         ratio = bench_cfg(CONFIGS["e128"], args.steps, args.warmup, False)
@@ -362,6 +368,17 @@ def run_ours(args):
         line["e128"] = {"value": r_value, "unit": UNIT, "vs_e8": r_value / value,
                         "grouped_gemm_tflops": CONFIGS["e128"].gemm_flops_fwd_bwd()
                         / (statistics.mean(ratio["gemm_ms"]) / 1e3) / 1e12}
+    if variants:
+        base_ms = main["total_ms"] / K
+        line["variants"] = {}
+        for name, v in variants.items():
+            ms = v["total_ms"] / K
+            line["variants"][name] = {
+                "value": cfg.T * K * ws / (v["total_ms"] / 1e3), "unit": UNIT, "ms_per_step": ms,
+                "overhead_ms": ms - base_ms, "launches_per_step": v["launches"] / K}
+        line["variants"]["aux_loss"]["what"] = (
+            "the same step plus the load-balancing loss (alpha 0.01): load statistics, loss and "
+            "its probability gradient in the router backward")
     if mx is not None:
         mc = CONFIGS["mxfp8"]
         line["mxfp8"] = {

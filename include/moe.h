@@ -233,10 +233,10 @@ MOE_API moe_status_t moe_permute_bwd(moe_handle_t h, const moe_shape_t* s, const
                              moe_stream_t stream);
 
 /* Backward of the permute with the router's share of the input gradient
- * added in the same pass (the two contributions of step a14/a15 of the
- * layer: the pages name only the steps, the formulas are the plain
- * backward of the router and of the permute):
- *   dL[t]  = as in moe_router_topk_bwd, from d_topk_w, probs and topk_idx
+ * added in the same pass (the pages name only the steps; the formulas are
+ * the plain backward of the router and of the permute):
+ *   dL[t]  = as in moe_router_topk_bwd, from d_topk_w, probs, topk_idx and
+ *            d_probs_aux (nullable)
  *   dx[t]  = bf16( sum_j dx_perm[row_map[t,j]] + dL[t] w_router ), fp32,
  *            rounded once; dL[t] w_router sums experts in increasing order.
  * Gives the same bits as moe_router_topk_bwd (with dx_router) followed by
@@ -244,18 +244,21 @@ MOE_API moe_status_t moe_permute_bwd(moe_handle_t h, const moe_shape_t* s, const
  * (MOE_ERR_UNSUPPORTED otherwise: for n_experts a multiple of 128 that
  * product runs on the tensor cores inside moe_router_topk_bwd).
  * In : dx_perm [M_cap,d] bf16, row_map [T,k], d_topk_w [T,k] fp32,
- *      probs [T,E] fp32, topk_idx [T,k], w_router [E,d] bf16.
+ *      probs [T,E] fp32, topk_idx [T,k], d_probs_aux [E] fp32 or NULL,
+ *      w_router [E,d] bf16.
  * Out: dx [T,d] bf16.  All pointers device, caller-owned; no workspace. */
 MOE_API moe_status_t moe_permute_router_bwd(moe_handle_t h, const moe_shape_t* s,
                                             const void* dx_perm, const int32_t* row_map,
                                             const float* d_topk_w, const float* probs,
-                                            const int32_t* topk_idx, const void* w_router,
-                                            void* dx, moe_stream_t stream);
+                                            const int32_t* topk_idx, const float* d_probs_aux,
+                                            const void* w_router, void* dx, moe_stream_t stream);
 
 /* Router backward (through the selected probabilities; top-k itself has no
  * gradient):
  *   g = d_topk_w, or with MOE_FLAG_RENORM g_j = (dw_j - sum_i dw_i w_i) / S
  *   dp[t, topk_idx[t,j]] = g[t,j], 0 elsewhere
+ *   dp[t, e] += d_probs_aux[e] for every t, when d_probs_aux is non-NULL
+ *               (the load-balancing loss: moe_router_aux_loss)
  *   dL = probs * (dp - sum_e probs dp)
  *   dx_router = dL w_router            [T,d] fp32 (fed to moe_permute_bwd),
  *                                      written when non-NULL
@@ -264,12 +267,41 @@ MOE_API moe_status_t moe_permute_router_bwd(moe_handle_t h, const moe_shape_t* s
  * With dx_router NULL the call leaves the input gradient to
  * moe_permute_router_bwd (n_experts <= 64), which forms dL w_router on the
  * fly instead of passing [T,d] fp32 through device memory.
- * In : d_topk_w [T,k] fp32, probs [T,E] fp32, topk_idx [T,k], x [T,d] bf16,
- *      w_router [E,d] bf16. */
+ * In : d_topk_w [T,k] fp32, probs [T,E] fp32, topk_idx [T,k],
+ *      d_probs_aux [E] fp32 or NULL, x [T,d] bf16, w_router [E,d] bf16. */
 MOE_API moe_status_t moe_router_topk_bwd(moe_handle_t h, const moe_shape_t* s, const float* d_topk_w,
-                                 const float* probs, const int32_t* topk_idx, const void* x,
+                                 const float* probs, const int32_t* topk_idx,
+                                 const float* d_probs_aux, const void* x,
                                  const void* w_router, float* dx_router, void* dw_router,
                                  float* dbias, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Router load statistics of one batch, for the load-balancing loss.  The
+ * pages call for a load-balancing auxiliary loss (discosf.com article on
+ * Olmo-core 3, sections 2.2 and 4.3) and for balancing over the global
+ * batch (Olmo-core 3 introduction page, section 4); they give no formula,
+ * and the reading is the Switch-Transformer loss over the k routed slots.
+ *   stats[e]     = counts[e]            routed (token, slot) pairs, as fp32
+ *   stats[E + e] = sum_t probs[t, e]    router probability mass
+ * accumulate != 0 adds into stats instead of overwriting it, so that the
+ * sums of several micro-batches (and, summed over ranks by the caller, of
+ * several GPUs) make the global batch's statistics.  Sums in a fixed order.
+ * In : probs [T,E] fp32, counts [E] int32 (from moe_permute).
+ * Out: stats [2E] fp32.  Uses the workspace. */
+MOE_API moe_status_t moe_router_load_stats(moe_handle_t h, const moe_shape_t* s, const float* probs,
+                                           const int32_t* counts, int accumulate, float* stats,
+                                           void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Load-balancing loss of (possibly summed) statistics over n_tokens tokens:
+ *   f_e = stats[e] / (n_tokens k),  P_e = stats[E+e] / n_tokens
+ *   loss = alpha E sum_e f_e P_e        (alpha at balance, alpha E at collapse)
+ *   d_probs_aux[e] = alpha E f_e / n_tokens = d loss / d probs[t, e] for every
+ *                    token (f_e is piecewise constant in the logits)
+ * Feed d_probs_aux to moe_router_topk_bwd / moe_permute_router_bwd.
+ * In : stats [2E] fp32, n_tokens >= 1, alpha >= 0.
+ * Out: loss [1] fp32 and d_probs_aux [E] fp32 (either may be NULL, not both). */
+MOE_API moe_status_t moe_router_aux_loss(moe_handle_t h, const moe_shape_t* s, const float* stats,
+                                         int64_t n_tokens, float alpha, float* loss,
+                                         float* d_probs_aux, moe_stream_t stream);
 
 /* MXFP8 quantisation of a bf16 matrix [rows, cols] (OCP MX v1.0 reading of
  * the pages' "MXFP8"): blocks of 32 consecutive elements, along each row

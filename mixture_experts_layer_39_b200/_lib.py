@@ -43,8 +43,10 @@ SIGNATURES = {
     "moe_unpermute_combine_bwd": [P, SP, P, P, P, P, P, P, P, P, P],
     "moe_grouped_swiglu_bwd": [P, SP, P, P, P, P, P, P, P, P, P, P, P, P, c_size_t, P],
     "moe_permute_bwd": [P, SP, P, P, P, P, P],
-    "moe_permute_router_bwd": [P, SP, P, P, P, P, P, P, P, P],
-    "moe_router_topk_bwd": [P, SP, P, P, P, P, P, P, P, P, P, c_size_t, P],
+    "moe_permute_router_bwd": [P, SP, P, P, P, P, P, P, P, P, P],
+    "moe_router_topk_bwd": [P, SP, P, P, P, P, P, P, P, P, P, P, c_size_t, P],
+    "moe_router_load_stats": [P, SP, P, P, c_int, P, P, c_size_t, P],
+    "moe_router_aux_loss": [P, SP, P, c_int64, ctypes.c_float, P, P, P],
     "moe_mxfp8_quantize": [P, P, c_int64, c_int64, c_int, P, P, P],
     "moe_get_status": [P, ctypes.POINTER(c_int)],
     "moe_get_launch_count": [P, ctypes.POINTER(ctypes.c_uint64)],

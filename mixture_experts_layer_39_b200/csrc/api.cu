@@ -393,7 +393,8 @@ moe_status_t moe_permute_bwd(moe_handle_t h, const moe_shape_t* s, const void* d
 moe_status_t moe_permute_router_bwd(moe_handle_t h, const moe_shape_t* s, const void* dx_perm,
                                     const int32_t* row_map, const float* d_topk_w,
                                     const float* probs, const int32_t* topk_idx,
-                                    const void* w_router, void* dx, moe_stream_t stream) {
+                                    const float* d_probs_aux, const void* w_router, void* dx,
+                                    moe_stream_t stream) {
   MOE_CHECK_HANDLE(h, s);
   MOE_TRY(check_router_shape(s));
   if (s->n_experts > 64) return MOE_ERR_UNSUPPORTED;
@@ -404,14 +405,15 @@ moe_status_t moe_permute_router_bwd(moe_handle_t h, const moe_shape_t* s, const 
   MOE_GUARD(h);
   h->launches += 1;
   return cuda_status(moe::launch_permute_router_bwd(
-      static_cast<const __nv_bfloat16*>(dx_perm), row_map, d_topk_w, probs, topk_idx,
+      static_cast<const __nv_bfloat16*>(dx_perm), row_map, d_topk_w, probs, topk_idx, d_probs_aux,
       static_cast<const __nv_bfloat16*>(w_router), s->T, s->d_model, s->n_experts, s->top_k,
       (s->flags & MOE_FLAG_RENORM) != 0, static_cast<__nv_bfloat16*>(dx),
       static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_router_topk_bwd(moe_handle_t h, const moe_shape_t* s, const float* d_topk_w,
-                                 const float* probs, const int32_t* topk_idx, const void* x,
+                                 const float* probs, const int32_t* topk_idx,
+                                 const float* d_probs_aux, const void* x,
                                  const void* w_router, float* dx_router, void* dw_router,
                                  float* dbias, void* ws, size_t ws_bytes, moe_stream_t stream) {
   MOE_CHECK_HANDLE(h, s);
@@ -436,8 +438,9 @@ moe_status_t moe_router_topk_bwd(moe_handle_t h, const moe_shape_t* s, const flo
     // partial rows in one pass over x, then one reduction for dW_r and db
     h->launches += 3;
     auto* dl = reinterpret_cast<float*>(base + L.dl);
-    MOE_TRY(cuda_status(moe::launch_router_bwd_dl(d_topk_w, probs, topk_idx, wb, T, d, E, k, renorm,
-                                                  want_dx, dl, nullptr, dx_router, db_part,
+    MOE_TRY(cuda_status(moe::launch_router_bwd_dl(d_topk_w, probs, topk_idx, d_probs_aux, wb, T, d,
+                                                  E, k, renorm, want_dx, dl, nullptr, dx_router,
+                                                  db_part,
                                                   L.nblocks, h->ctl, st)));
     MOE_TRY(cuda_status(moe::launch_router_dw(dl, xb, T, d, E, L.n_part, L.group_len, part, st)));
     return cuda_status(moe::launch_reduce_dw(part, L.n_part, static_cast<int64_t>(E) * d, db_part,
@@ -447,15 +450,43 @@ moe_status_t moe_router_topk_bwd(moe_handle_t h, const moe_shape_t* s, const flo
   // E a multiple of 128: dL in bf16, both products on the tensor cores
   h->launches += want_dx ? 4 : 3;
   auto* dl = reinterpret_cast<__nv_bfloat16*>(base + L.dl);
-  MOE_TRY(cuda_status(moe::launch_router_bwd_dl(d_topk_w, probs, topk_idx, wb, T, d, E, k, renorm,
-                                                false, nullptr, dl, nullptr, db_part, L.nblocks,
-                                                h->ctl, st)));
+  MOE_TRY(cuda_status(moe::launch_router_bwd_dl(d_topk_w, probs, topk_idx, d_probs_aux, wb, T, d, E,
+                                                k, renorm, false, nullptr, dl, nullptr, db_part,
+                                                L.nblocks, h->ctl, st)));
   moe::GemmCtx c{h->num_sms, h->ctl};
   if (want_dx) MOE_TRY(moe::gemm_router_dx(c, dl, w_router, dx_router, T, d, E, st));
   MOE_TRY(moe::gemm_router_dw_partial(c, dl, x, part, T, d, E, L.n_part, L.group_len, st));
   return cuda_status(moe::launch_reduce_dw(part, L.n_part, static_cast<int64_t>(E) * d, db_part,
                                            L.nblocks, E, static_cast<__nv_bfloat16*>(dw_router),
                                            dbias, st));
+}
+
+moe_status_t moe_router_load_stats(moe_handle_t h, const moe_shape_t* s, const float* probs,
+                                   const int32_t* counts, int accumulate, float* stats, void* ws,
+                                   size_t ws_bytes, moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  if (!all_nonnull(probs, counts, stats)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(h, s, ws, ws_bytes));
+  const int nb = moe::router_stats_blocks(h->num_sms, s->T);
+  if (static_cast<size_t>(nb) * s->n_experts * 4 > ws_bytes) return MOE_ERR_WORKSPACE;
+  MOE_GUARD(h);
+  h->launches += 2;
+  return cuda_status(moe::launch_router_load_stats(probs, counts, s->T, s->n_experts, nb,
+                                                   accumulate != 0, static_cast<float*>(ws), stats,
+                                                   static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_router_aux_loss(moe_handle_t h, const moe_shape_t* s, const float* stats,
+                                 int64_t n_tokens, float alpha, float* loss, float* d_probs_aux,
+                                 moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  if (stats == nullptr || (loss == nullptr && d_probs_aux == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (n_tokens < 1 || !(alpha >= 0.f)) return MOE_ERR_INVALID_ARG;
+  MOE_GUARD(h);
+  h->launches += 1;
+  return cuda_status(moe::launch_router_aux_loss(stats, s->n_experts, s->top_k,
+                                                 static_cast<float>(n_tokens), alpha, loss,
+                                                 d_probs_aux, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_mxfp8_quantize(moe_handle_t h, const void* in, int64_t rows, int64_t cols,

@@ -21,6 +21,15 @@ cudaError_t launch_softmax_topk(const float* logits_in, const float* bias, const
                                 int T, int E, int k, bool renorm, int32_t* idx, float* w,
                                 float* probs, float* logits_out, DeviceCtl* ctl, cudaStream_t st);
 
+// ---- router load statistics and load-balancing loss
+int router_stats_blocks(int num_sms, int T);
+// partial: router_stats_blocks() x E floats of scratch
+cudaError_t launch_router_load_stats(const float* probs, const int32_t* counts, int T, int E,
+                                     int n_blocks, bool accumulate, float* partial, float* stats,
+                                     cudaStream_t st);
+cudaError_t launch_router_aux_loss(const float* stats, int E, int k, float n_tokens, float alpha,
+                                   float* loss, float* dprob, cudaStream_t st);
+
 // ---- routing metadata + permute
 cudaError_t launch_route_hist(const int32_t* idx, int T, int k, int E, int32_t* sub_counts,
                               DeviceCtl* ctl, cudaStream_t st);
@@ -47,11 +56,13 @@ cudaError_t launch_permute_bwd(const __nv_bfloat16* dx_perm, const int32_t* row_
 // dX = bf16(unpermute-reduce of dX_perm + dL W_r) in one pass, E <= 64.
 cudaError_t launch_permute_router_bwd(const __nv_bfloat16* dx_perm, const int32_t* row_map,
                                       const float* dw, const float* probs, const int32_t* idx,
-                                      const __nv_bfloat16* w_r, int T, int d, int E, int k,
-                                      bool renorm, __nv_bfloat16* dx, cudaStream_t st);
+                                      const float* dprob_aux, const __nv_bfloat16* w_r, int T,
+                                      int d, int E, int k, bool renorm, __nv_bfloat16* dx,
+                                      cudaStream_t st);
 int router_bwd_blocks(int num_sms);
 cudaError_t launch_router_bwd_dl(const float* dw, const float* probs, const int32_t* idx,
-                                 const __nv_bfloat16* w_r, int T, int d, int E, int k, bool renorm,
+                                 const float* dprob_aux, const __nv_bfloat16* w_r, int T, int d,
+                                 int E, int k, bool renorm,
                                  bool fuse_dx, float* dl_f32, __nv_bfloat16* dl_bf16,
                                  float* dx_router, float* db_partial, int nblocks,
                                  DeviceCtl* ctl, cudaStream_t st);

@@ -18,13 +18,17 @@ constexpr int kWarps = 8;
 // dL[t, e] = p[t,e] (dp[t,e] - <p[t], dp[t]>) of one token, held by the warp
 // in the lane layout e = lane + 32 i (i < NPL); dp is the gate-weight
 // gradient scattered to the chosen experts (after the renormalisation's
-// backward when the gate weights were renormalised).  Ids outside [0, E)
-// carry no gradient.  Every lane must call it (one warp reduction).
+// backward when the gate weights were renormalised), plus dprob_aux[e] for
+// every expert when given (the load-balancing loss's gradient, the same for
+// all tokens).  Ids outside [0, E) carry no gradient.  Every lane must call
+// it (one warp reduction).
 template <int NPL>
 __device__ __forceinline__ void token_dlogits(const float* __restrict__ dw,
                                               const float* __restrict__ probs,
-                                              const int32_t* __restrict__ idx, int64_t t, int E,
-                                              int k, int renorm, int lane, float (&dl)[NPL]) {
+                                              const int32_t* __restrict__ idx,
+                                              const float* __restrict__ dprob_aux, int64_t t,
+                                              int E, int k, int renorm, int lane,
+                                              float (&dl)[NPL]) {
   int id[8];
   float g[8];
 #pragma unroll
@@ -57,6 +61,7 @@ __device__ __forceinline__ void token_dlogits(const float* __restrict__ dw,
     dp[i] = 0.f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) if (id[j] == e) dp[i] += g[j];
+    if (dprob_aux != nullptr && e < E) dp[i] += __ldg(dprob_aux + e);
     pdp += p[i] * dp[i];
   }
   pdp = warp_sum(pdp);
@@ -88,7 +93,8 @@ __device__ __forceinline__ void router_dx_slice(const uint4* __restrict__ wv, in
 template <int NPL, bool FUSE_DX, int NE = 32 * NPL>
 __global__ void __launch_bounds__(kWarps * 32)
     router_bwd_dl_kernel(const float* __restrict__ dw, const float* __restrict__ probs,
-                         const int32_t* __restrict__ idx, const __nv_bfloat16* __restrict__ w_r,
+                         const int32_t* __restrict__ idx, const float* __restrict__ dprob_aux,
+                         const __nv_bfloat16* __restrict__ w_r,
                          int T, int d, int E, int k, int renorm, float* __restrict__ dl_f32,
                          __nv_bfloat16* __restrict__ dl_bf16, float* __restrict__ dx_router,
                          float* __restrict__ db_partial, int stage_w) {
@@ -111,7 +117,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kWarps;
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + warp; t < T; t += stride) {
     float dl[NPL];
-    token_dlogits<NPL>(dw, probs, idx, t, E, k, renorm, lane, dl);
+    token_dlogits<NPL>(dw, probs, idx, dprob_aux, t, E, k, renorm, lane, dl);
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
       const int e = lane + 32 * i;
@@ -162,7 +168,9 @@ template <int NE, int TPW, int KMAX>
 __global__ void __launch_bounds__(kWarps * 32, 2)
     permute_router_bwd_kernel(const uint4* __restrict__ dxp, const int32_t* __restrict__ row_map,
                               const float* __restrict__ dw, const float* __restrict__ probs,
-                              const int32_t* __restrict__ idx, const __nv_bfloat16* __restrict__ w_r,
+                              const int32_t* __restrict__ idx,
+                              const float* __restrict__ dprob_aux,
+                              const __nv_bfloat16* __restrict__ w_r,
                               int T, int d, int E, int k, int renorm, uint4* __restrict__ dx) {
   constexpr int NPL = (NE + 31) / 32;
   const int lane = threadIdx.x & 31;
@@ -175,7 +183,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   for (int h = 0; h < TPW; ++h) {
     const int64_t t = t0 + h < T ? t0 + h : t0;  // a missing second token repeats the first
     float dl[NPL];
-    token_dlogits<NPL>(dw, probs, idx, t, E, k, renorm, lane, dl);
+    token_dlogits<NPL>(dw, probs, idx, dprob_aux, t, E, k, renorm, lane, dl);
 #pragma unroll
     for (int e = 0; e < NE; ++e) dle[h][e] = __shfl_sync(0xffffffffu, dl[e >> 5], e & 31);
 #pragma unroll
@@ -213,103 +221,105 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   }
 }
 
-// dW_r partial sums over a chunk of tokens, CUDA cores (E <= 64).  Each
-// thread owns CPT consecutive columns of x and all E experts of them;
-// blocks tile (column slice, token chunk) and a grid holds about as many
-// blocks as the GPU keeps resident, so every partial row stands for a large
-// chunk of tokens.  dL is staged kDwStage tokens at a time; x is read kDwBatch
-// tokens at a time, all loads issued before the FMAs that use them.  Tokens
-// are accumulated in increasing order.
+// dW_r partial sums over a chunk of tokens, CUDA cores (E <= 64).  A block
+// owns a slice of kDwCols columns of x and a chunk of tokens (a multiple of
+// kDwTok); it streams the chunk through shared memory in stages of kDwTok
+// tokens (the x slice and the matching dL rows), double-buffered with
+// cp.async so that the next stage is in flight while this one is reduced.
+// Each thread owns 2 consecutive columns and all E experts of them; tokens
+// are accumulated in increasing order.  The grid holds about as many blocks
+// as stay resident, so every partial row stands for a large chunk of tokens.
 constexpr int kDwThreads = 256;
-constexpr int kDwStage = 64;
-constexpr int kDwBatch = 16;
+constexpr int kDwCols = 2 * kDwThreads;      // 512 columns = 1 KB of a bf16 row
+constexpr int kDwTok = 32;                   // tokens per stage
+constexpr int kDwStageX = kDwTok * kDwCols * 2;  // 32 KB of x per stage
 
-// CPT consecutive bf16 columns, kept packed (two per 32-bit word) until use.
-template <int CPT>
-struct PackedCols {
-  uint32_t w[(CPT + 1) / 2];
-};
-
-template <int CPT>
-__device__ __forceinline__ PackedCols<CPT> load_cols(const __nv_bfloat16* p) {
-  PackedCols<CPT> r;
-  if constexpr (CPT == 4) {
-    const uint2 q = __ldg(reinterpret_cast<const uint2*>(p));
-    r.w[0] = q.x;
-    r.w[1] = q.y;
-  } else if constexpr (CPT == 2) {
-    r.w[0] = __ldg(reinterpret_cast<const unsigned int*>(p));
-  } else {
-    r.w[0] = static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(p)));
-  }
-  return r;
+__device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(sdst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
 }
 
-template <int CPT>
-__device__ __forceinline__ float col_value(const PackedCols<CPT>& r, int c) {
-  return (c & 1) ? bf16_hi(r.w[c >> 1]) : bf16_lo(r.w[c >> 1]);
+__device__ __forceinline__ void cp_async4b(void* sdst, const void* gsrc) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(sdst));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(gsrc) : "memory");
 }
 
-template <int NE, int CPT>
-__global__ void __launch_bounds__(kDwThreads, NE <= 8 ? 4 : NE <= 16 ? 3 : 2)
+template <int NE>
+__global__ void __launch_bounds__(kDwThreads)
     router_dw_kernel(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ x, int T,
-                     int d, int E, int group_len, int64_t row_stride, float* __restrict__ partial) {
-  __shared__ float s_dl[kDwStage * NE];  // 16 KB at NE = 64
+                     int d, int E, int group_len, float* __restrict__ partial) {
+  extern __shared__ __align__(16) uint8_t s_raw[];
+  uint8_t* s_x = s_raw;                                              // [2][kDwTok][kDwCols] bf16
+  float* s_dl = reinterpret_cast<float*>(s_raw + 2 * kDwStageX);      // [2][kDwTok][NE]
+  const int64_t col0 = static_cast<int64_t>(blockIdx.x) * kDwCols;
+  const int width = d - col0 < kDwCols ? static_cast<int>(d - col0) : kDwCols;  // 256 or 512
+  const int pieces = width / 8;                                       // 16-byte pieces per row
   const int64_t g0 = static_cast<int64_t>(blockIdx.y) * group_len;
   const int64_t g1 = g0 + group_len < T ? g0 + group_len : T;
-  const int64_t col = (static_cast<int64_t>(blockIdx.x) * kDwThreads + threadIdx.x) * CPT;
-  const bool active = col < d;
-  float acc[NE][CPT];
-#pragma unroll
-  for (int e = 0; e < NE; ++e)
-#pragma unroll
-    for (int c = 0; c < CPT; ++c) acc[e][c] = 0.f;
-  for (int64_t s0 = g0; s0 < g1; s0 += kDwStage) {
-    const int nt = g1 - s0 < kDwStage ? static_cast<int>(g1 - s0) : kDwStage;
-    __syncthreads();  // the previous stage has been consumed
+  const int n_stages = g1 > g0 ? static_cast<int>(ceil_div64(g1 - g0, kDwTok)) : 0;
+
+  auto issue = [&](int sidx) {
+    const int64_t s0 = g0 + static_cast<int64_t>(sidx) * kDwTok;
+    const int nt = g1 - s0 < kDwTok ? static_cast<int>(g1 - s0) : kDwTok;
+    uint8_t* bx = s_x + (sidx & 1) * kDwStageX;
+    for (int i = threadIdx.x; i < nt * pieces; i += kDwThreads) {
+      const int tt = i / pieces, q = i - tt * pieces;
+      cp_async16(bx + tt * (kDwCols * 2) + q * 16, x + (s0 + tt) * d + col0 + q * 8);
+    }
+    float* bd = s_dl + (sidx & 1) * (kDwTok * NE);
     for (int i = threadIdx.x; i < nt * E; i += kDwThreads) {
       const int tt = i / E, e = i - tt * E;
-      s_dl[tt * NE + e] = __ldg(dl + s0 * E + i);
+      cp_async4b(bd + tt * NE + e, dl + s0 * E + i);
     }
-    __syncthreads();
-    if (!active) continue;
-    for (int b = 0; b < nt; b += kDwBatch) {
-      const __nv_bfloat16* xr = x + (s0 + b) * d + col;
-      PackedCols<CPT> xq[kDwBatch];
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+
+  const int c = threadIdx.x * 2;  // this thread's first column in the slice
+  const bool active = c < width;
+  float acc[NE][2];
 #pragma unroll
-      for (int u = 0; u < kDwBatch; ++u)
-        if (b + u < nt) xq[u] = load_cols<CPT>(xr + static_cast<int64_t>(u) * d);
+  for (int e = 0; e < NE; ++e) acc[e][0] = acc[e][1] = 0.f;
+  if (n_stages > 0) issue(0);
+  for (int sidx = 0; sidx < n_stages; ++sidx) {
+    if (sidx + 1 < n_stages) {
+      issue(sidx + 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncthreads();  // every thread's copies of this stage have landed
+    const int64_t s0 = g0 + static_cast<int64_t>(sidx) * kDwTok;
+    const int nt = g1 - s0 < kDwTok ? static_cast<int>(g1 - s0) : kDwTok;
+    const uint8_t* bx = s_x + (sidx & 1) * kDwStageX;
+    const float* bd = s_dl + (sidx & 1) * (kDwTok * NE);
+    if (active) {
+#pragma unroll 4
+      for (int tt = 0; tt < nt; ++tt) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(bx + tt * (kDwCols * 2) + c * 2);
+        const float x0 = bf16_lo(w), x1 = bf16_hi(w);
 #pragma unroll
-      for (int u = 0; u < kDwBatch; ++u) {
-        if (b + u < nt) {
-          float xv[CPT];
-#pragma unroll
-          for (int c = 0; c < CPT; ++c) xv[c] = col_value<CPT>(xq[u], c);
-#pragma unroll
-          for (int e = 0; e < NE; ++e) {
-            if (e < E) {
-              const float g = s_dl[(b + u) * NE + e];
-#pragma unroll
-              for (int c = 0; c < CPT; ++c) acc[e][c] = fmaf(g, xv[c], acc[e][c]);
-            }
+        for (int e = 0; e < NE; ++e) {
+          if (e < E) {
+            const float g = bd[tt * NE + e];
+            acc[e][0] = fmaf(g, x0, acc[e][0]);
+            acc[e][1] = fmaf(g, x1, acc[e][1]);
           }
         }
       }
     }
+    __syncthreads();  // this buffer is refilled two stages later
   }
   if (!active) return;
-  float* out = partial + static_cast<int64_t>(blockIdx.y) * row_stride;
+  float* out = partial + static_cast<int64_t>(blockIdx.y) * E * d + col0 + c;
 #pragma unroll
   for (int e = 0; e < NE; ++e)
-    if (e < E) {
-      if constexpr (CPT == 4) {
-        *reinterpret_cast<float4*>(out + static_cast<int64_t>(e) * d + col) =
-            make_float4(acc[e][0], acc[e][1], acc[e][2], acc[e][3]);
-      } else {
-#pragma unroll
-        for (int c = 0; c < CPT; ++c) out[static_cast<int64_t>(e) * d + col + c] = acc[e][c];
-      }
-    }
+    if (e < E)
+      *reinterpret_cast<float2*>(out + static_cast<int64_t>(e) * d) = make_float2(acc[e][0], acc[e][1]);
+}
+
+template <int NE>
+constexpr size_t dw_smem_bytes() {
+  return 2 * kDwStageX + 2 * kDwTok * NE * sizeof(float);
 }
 
 // dw_out[i] = bf16(sum_p partial[p][i]) over n4_w float4 columns, and, when
@@ -367,12 +377,13 @@ __global__ void __launch_bounds__(kRedWarps * 32)
 
 cudaError_t launch_permute_router_bwd(const __nv_bfloat16* dx_perm, const int32_t* row_map,
                                       const float* dw, const float* probs, const int32_t* idx,
-                                      const __nv_bfloat16* w_r, int T, int d, int E, int k,
-                                      bool renorm, __nv_bfloat16* dx, cudaStream_t st) {
+                                      const float* dprob_aux, const __nv_bfloat16* w_r, int T,
+                                      int d, int E, int k, bool renorm, __nv_bfloat16* dx,
+                                      cudaStream_t st) {
   auto go = [&](auto kern, int tpw) {
     const unsigned grid = static_cast<unsigned>(ceil_div64(T, static_cast<int64_t>(kWarps) * tpw));
     kern<<<grid, kWarps * 32, 0, st>>>(reinterpret_cast<const uint4*>(dx_perm), row_map, dw, probs,
-                                       idx, w_r, T, d, E, k, renorm ? 1 : 0,
+                                       idx, dprob_aux, w_r, T, d, E, k, renorm ? 1 : 0,
                                        reinterpret_cast<uint4*>(dx));
     return cudaGetLastError();
   };
@@ -392,7 +403,8 @@ cudaError_t launch_permute_router_bwd(const __nv_bfloat16* dx_perm, const int32_
 int router_bwd_blocks(int num_sms) { return num_sms * 4; }
 
 cudaError_t launch_router_bwd_dl(const float* dw, const float* probs, const int32_t* idx,
-                                 const __nv_bfloat16* w_r, int T, int d, int E, int k, bool renorm,
+                                 const float* dprob_aux, const __nv_bfloat16* w_r, int T, int d,
+                                 int E, int k, bool renorm,
                                  bool fuse_dx, float* dl_f32, __nv_bfloat16* dl_bf16,
                                  float* dx_router, float* db_partial, int nblocks,
                                  DeviceCtl* ctl, cudaStream_t st) {
@@ -405,7 +417,8 @@ cudaError_t launch_router_bwd_dl(const float* dw, const float* probs, const int3
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return cudaErrorInvalidValue;
-    kern<<<nblocks, kWarps * 32, smem, st>>>(dw, probs, idx, w_r, T, d, E, k, renorm ? 1 : 0,
+    kern<<<nblocks, kWarps * 32, smem, st>>>(dw, probs, idx, dprob_aux, w_r, T, d, E, k,
+                                             renorm ? 1 : 0,
                                              dl_f32, dl_bf16, dx_router, db_partial,
                                              stage ? 1 : 0);
     return cudaGetLastError();
@@ -425,37 +438,40 @@ cudaError_t launch_router_bwd_dl(const float* dw, const float* probs, const int3
 }
 
 namespace {
-int dw_cols_per_thread(int E) { return E <= 32 ? 2 : 1; }
-int dw_blocks_per_sm(int E) { return E <= 8 ? 4 : E <= 16 ? 3 : 2; }
+int dw_blocks_per_sm(int E) { return E <= 16 ? 3 : 2; }
 }  // namespace
 
 int router_dw_chunks(int num_sms, int T, int d, int E, int* group_len) {
-  const int64_t col_blocks = ceil_div64(d, static_cast<int64_t>(kDwThreads) * dw_cols_per_thread(E));
-  // as many blocks as stay resident, over all column blocks; at least 8
-  // tokens per chunk
+  const int64_t col_blocks = ceil_div64(d, kDwCols);
+  // as many blocks as stay resident, over all column blocks; chunks are
+  // whole stages
   int64_t n = ceil_div64(static_cast<int64_t>(dw_blocks_per_sm(E)) * num_sms, col_blocks);
-  const int64_t most = ceil_div64(T, 8);
+  const int64_t most = ceil_div64(T, kDwTok);
   if (n > most) n = most;
   if (n < 1) n = 1;
-  const int64_t len = ceil_div64(T, n);
+  const int64_t len = ceil_div64(ceil_div64(T, n), kDwTok) * kDwTok;
   *group_len = static_cast<int>(len);
   return static_cast<int>(ceil_div64(T, len));
 }
 
 cudaError_t launch_router_dw(const float* dl, const __nv_bfloat16* x, int T, int d, int E,
                              int n_chunks, int group_len, float* partial, cudaStream_t st) {
-  const int64_t stride = static_cast<int64_t>(E) * d;
-  auto go = [&](auto kern, int cpt) {
-    const unsigned gx = static_cast<unsigned>(ceil_div64(d, static_cast<int64_t>(kDwThreads) * cpt));
-    kern<<<dim3(gx, static_cast<unsigned>(n_chunks)), kDwThreads, 0, st>>>(dl, x, T, d, E,
-                                                                           group_len, stride,
-                                                                           partial);
+  auto go = [&](auto kern, size_t smem) {
+    // several 66-80 KB blocks per SM only fit with the largest shared-memory carve-out
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+      return cudaErrorInvalidValue;
+    const unsigned gx = static_cast<unsigned>(ceil_div64(d, kDwCols));
+    kern<<<dim3(gx, static_cast<unsigned>(n_chunks)), kDwThreads, smem, st>>>(dl, x, T, d, E,
+                                                                              group_len, partial);
     return cudaGetLastError();
   };
-  if (E <= 8) return go(router_dw_kernel<8, 2>, 2);
-  if (E <= 16) return go(router_dw_kernel<16, 2>, 2);
-  if (E <= 32) return go(router_dw_kernel<32, 2>, 2);
-  if (E <= 64) return go(router_dw_kernel<64, 1>, 1);
+  if (E <= 8) return go(router_dw_kernel<8>, dw_smem_bytes<8>());
+  if (E <= 16) return go(router_dw_kernel<16>, dw_smem_bytes<16>());
+  if (E <= 32) return go(router_dw_kernel<32>, dw_smem_bytes<32>());
+  if (E <= 64) return go(router_dw_kernel<64>, dw_smem_bytes<64>());
   return cudaErrorInvalidValue;
 }
 

@@ -12,9 +12,15 @@ in order on the current stream:
             cores), moe_router_topk_bwd writes dX_router and
             moe_permute_bwd adds it.
 
+With aux_alpha > 0 the forward also forms the router's load statistics and
+the load-balancing loss (moe_router_load_stats -> moe_router_aux_loss) and
+the backward adds the loss's gradient in the router backward.
+
 Nothing in a step copies to the host or synchronises.
 """
 from __future__ import annotations
+
+from typing import Callable
 
 import torch
 
@@ -29,12 +35,17 @@ F32 = torch.float32
 class MoELayer:
     def __init__(self, T, d, f, E, k, device="cuda", renorm=False, keep_logits=False,
                  handle: ops.Handle | None = None, dtype: str = "bf16",
-                 fuse_router_dx: bool | None = None):
+                 fuse_router_dx: bool | None = None, aux_alpha: float = 0.0,
+                 aux_reduce: Callable | None = None):
         """dtype: "bf16", or "mxfp8" for E4M3/E8M0 expert GEMM operands (the
         library then also aligns expert segments to 128 rows).
         fuse_router_dx: add the router's input gradient inside the permute
         backward (default, and only possible, for E <= 64); False keeps the
-        separate [T, d] fp32 dX_router buffer."""
+        separate [T, d] fp32 dX_router buffer.
+        aux_alpha: weight of the load-balancing loss (0: none).  aux_reduce:
+        optional callable(stats) -> n_tokens that sums the statistics over
+        ranks in place and returns the global batch's token count
+        (replicas.global_stats_reducer), for balancing over the global batch."""
         self.T, self.d, self.f, self.E, self.k = T, d, f, E, k
         dev = torch.device(device)
         self.device = dev
@@ -67,6 +78,12 @@ class MoELayer:
         self.dw_r = z(E, d)
         self.db = z(E, dt=F32)
         self.dx = z(T, d)
+        # load-balancing loss
+        self.aux_alpha = float(aux_alpha)
+        self.aux_reduce = aux_reduce
+        self.stats = z(2 * E, dt=F32)
+        self.aux_loss = z(1, dt=F32)
+        self.dprob_aux = z(E, dt=F32) if self.aux_alpha > 0 else None
 
     # ------------------------------------------------------------- forward
     def router(self, x, w_r, bias=None, route=None, stream=None):
@@ -85,9 +102,27 @@ class MoELayer:
         ops.moe_unpermute_combine(self.handle, self.shape, self.o_perm, self.row_map, self.w,
                                   self.y, stream)
 
+    def load_stats(self, accumulate=False, stream=None):
+        """[counts | sum_t probs] of this batch into self.stats (added when
+        accumulate)."""
+        ops.moe_router_load_stats(self.handle, self.shape, self.probs, self.counts, accumulate,
+                                  self.stats, self.ws, stream)
+
+    def balance_loss(self, stats=None, n_tokens=None, stream=None):
+        """Load-balancing loss of `stats` (default self.stats) over n_tokens
+        tokens (default T) into self.aux_loss, and its per-expert
+        probability gradient into self.dprob_aux."""
+        ops.moe_router_aux_loss(self.handle, self.shape, self.stats if stats is None else stats,
+                                self.T if n_tokens is None else n_tokens, self.aux_alpha,
+                                self.aux_loss, self.dprob_aux, stream)
+
     def forward(self, x, w_r, w_gu, w_d, bias=None, route=None, stream=None):
         self.router(x, w_r, bias, route, stream)
         self.permute(x, stream)
+        if self.aux_alpha > 0:
+            self.load_stats(False, stream)
+            n = self.aux_reduce(self.stats) if self.aux_reduce is not None else self.T
+            self.balance_loss(None, n, stream)
         self.experts_fwd(w_gu, w_d, stream)
         self.combine(stream)
         return self.y
@@ -99,8 +134,9 @@ class MoELayer:
                                       stream)
 
     def router_bwd(self, x, w_r, stream=None):
-        ops.moe_router_topk_bwd(self.handle, self.shape, self.dw, self.probs, self.idx, x, w_r,
-                                self.dx_router, self.dw_r, self.db, self.ws, stream)
+        ops.moe_router_topk_bwd(self.handle, self.shape, self.dw, self.probs, self.idx,
+                                self.dprob_aux, x, w_r, self.dx_router, self.dw_r, self.db,
+                                self.ws, stream)
 
     def experts_bwd(self, w_gu, w_d, stream=None):
         ops.moe_grouped_swiglu_bwd(self.handle, self.shape, self.do_perm, self.x_perm, self.au,
@@ -112,7 +148,8 @@ class MoELayer:
             if w_r is None:
                 raise ValueError("the fused permute backward needs w_r")
             ops.moe_permute_router_bwd(self.handle, self.shape, self.dx_perm, self.row_map,
-                                       self.dw, self.probs, self.idx, w_r, self.dx, stream)
+                                       self.dw, self.probs, self.idx, self.dprob_aux, w_r,
+                                       self.dx, stream)
         else:
             ops.moe_permute_bwd(self.handle, self.shape, self.dx_perm, self.row_map,
                                 self.dx_router, self.dx, stream)

@@ -137,17 +137,28 @@ def moe_permute_bwd(h, shape, dx_perm, row_map, dx_router, dx, stream=None):
           _ptr(dx_router), _ptr(dx), _stream(stream))
 
 
-def moe_permute_router_bwd(h, shape, dx_perm, row_map, d_topk_w, probs, topk_idx, w_router, dx,
-                           stream=None):
+def moe_permute_router_bwd(h, shape, dx_perm, row_map, d_topk_w, probs, topk_idx, d_probs_aux,
+                           w_router, dx, stream=None):
     _call("moe_permute_router_bwd", h.ptr, ctypes.byref(shape), _ptr(dx_perm), _ptr(row_map),
-          _ptr(d_topk_w), _ptr(probs), _ptr(topk_idx), _ptr(w_router), _ptr(dx), _stream(stream))
+          _ptr(d_topk_w), _ptr(probs), _ptr(topk_idx), _ptr(d_probs_aux), _ptr(w_router), _ptr(dx),
+          _stream(stream))
 
 
-def moe_router_topk_bwd(h, shape, d_topk_w, probs, topk_idx, x, w_router, dx_router, dw_router,
-                        dbias, ws, stream=None):
+def moe_router_topk_bwd(h, shape, d_topk_w, probs, topk_idx, d_probs_aux, x, w_router, dx_router,
+                        dw_router, dbias, ws, stream=None):
     _call("moe_router_topk_bwd", h.ptr, ctypes.byref(shape), _ptr(d_topk_w), _ptr(probs),
-          _ptr(topk_idx), _ptr(x), _ptr(w_router), _ptr(dx_router), _ptr(dw_router), _ptr(dbias),
-          _ptr(ws), ws.numel(), _stream(stream))
+          _ptr(topk_idx), _ptr(d_probs_aux), _ptr(x), _ptr(w_router), _ptr(dx_router),
+          _ptr(dw_router), _ptr(dbias), _ptr(ws), ws.numel(), _stream(stream))
+
+
+def moe_router_load_stats(h, shape, probs, counts, accumulate, stats, ws, stream=None):
+    _call("moe_router_load_stats", h.ptr, ctypes.byref(shape), _ptr(probs), _ptr(counts),
+          1 if accumulate else 0, _ptr(stats), _ptr(ws), ws.numel(), _stream(stream))
+
+
+def moe_router_aux_loss(h, shape, stats, n_tokens, alpha, loss, d_probs_aux, stream=None):
+    _call("moe_router_aux_loss", h.ptr, ctypes.byref(shape), _ptr(stats), int(n_tokens),
+          ctypes.c_float(alpha), _ptr(loss), _ptr(d_probs_aux), _stream(stream))
 
 
 def moe_mxfp8_quantize(h, inp, axis, q, scales, stream=None):

@@ -19,6 +19,7 @@ the host) and are no-ops without an initialised process group.
 from __future__ import annotations
 
 import os
+from typing import Callable
 
 import torch
 import torch.distributed as dist
@@ -51,3 +52,13 @@ def sum_load_stats(stats: torch.Tensor) -> torch.Tensor:
     if _active():
         dist.all_reduce(stats, op=dist.ReduceOp.SUM)
     return stats
+
+
+def global_stats_reducer(tokens_per_rank: int) -> Callable[[torch.Tensor], int]:
+    """For MoELayer(aux_reduce=...): sums the statistics over ranks and
+    returns the global batch's token count (every rank the same T)."""
+    def reduce(stats: torch.Tensor) -> int:
+        sum_load_stats(stats)
+        ws = dist.get_world_size() if _active() else 1
+        return tokens_per_rank * ws
+    return reduce
