@@ -205,14 +205,17 @@ def expert_ffn_fwd(x_perm, offsets, counts, w_gu, w_d, rnd=bf16_round,
 # --------------------------------------------------------------------------
 # Combine (unpermute x gate weight)
 # --------------------------------------------------------------------------
-def combine(O, row_map, w, rnd=bf16_round):
-    """y[t] = bf16( sum_j w[t, j] * O[row_map[t, j]] ), summed in slot order."""
+def combine(O, row_map, w, rnd=bf16_round, shared=None):
+    """y[t] = bf16( sum_j w[t, j] * O[row_map[t, j]] + shared[t] ), summed in
+    slot order, the shared expert's output (when given) last."""
     O = np.asarray(O, F64)
     w = np.asarray(w, F64)
     T, k = row_map.shape
     acc = np.zeros((T, O.shape[1]), F64)
     for j in range(k):
         acc = acc + w[:, j:j + 1] * O[row_map[:, j]]
+    if shared is not None:
+        acc = acc + np.asarray(shared, F64)
     return _r(rnd)(acc)
 
 
@@ -349,8 +352,9 @@ def router_aux_loss(stats, n_tokens, k, alpha):
     return loss, dprob
 
 
-def permute_bwd(dX_perm, row_map, dx_router=None, rnd=bf16_round):
-    """dX[t] = bf16( sum_j dX_perm[row_map[t, j]] + dX_router[t] ), slot order."""
+def permute_bwd(dX_perm, row_map, dx_router=None, rnd=bf16_round, dx_shared=None):
+    """dX[t] = bf16( sum_j dX_perm[row_map[t, j]] + dX_router[t] + dX_shared[t] ),
+    slot order, then the router's and the shared expert's terms (when given)."""
     dX_perm = np.asarray(dX_perm, F64)
     T, k = row_map.shape
     acc = np.zeros((T, dX_perm.shape[1]), F64)
@@ -358,35 +362,74 @@ def permute_bwd(dX_perm, row_map, dx_router=None, rnd=bf16_round):
         acc = acc + dX_perm[row_map[:, j]]
     if dx_router is not None:
         acc = acc + np.asarray(dx_router, F64)
+    if dx_shared is not None:
+        acc = acc + np.asarray(dx_shared, F64)
     return _r(rnd)(acc)
+
+
+# --------------------------------------------------------------------------
+# Shared expert.  The pages list shared experts among the v2 router's
+# features (Olmo-core 3 introduction page, meetcoding.cn, section 4,
+# configuration templates) without defining them.  Reading: one more SwiGLU
+# expert with its own weights W_gu_s [2 f_s, d], W_d_s [d, f_s] that every
+# token passes through, its output added to the routed experts' combine with
+# weight one (so its output gradient is dY itself).  It is the expert FFN
+# above applied to one group holding all T tokens in token order.
+
+def shared_expert_fwd(x, w_gu_s, w_d_s, rnd=bf16_round):
+    """AU_s, H_s, O_s of the shared expert over all tokens."""
+    x = np.asarray(x, F64)
+    T = x.shape[0]
+    return expert_ffn_fwd(x, np.array([0, T]), np.array([T]), np.asarray(w_gu_s)[None],
+                          np.asarray(w_d_s)[None], rnd)
+
+
+def shared_expert_bwd(dy, x, AU_s, H_s, w_gu_s, w_d_s, rnd=bf16_round):
+    """dAU_s, dX_s (= bf16(dAU_s W_gu_s)), dW_gu_s, dW_d_s from dO_s = dY."""
+    x = np.asarray(x, F64)
+    T = x.shape[0]
+    fb = expert_ffn_bwd(dy, x, AU_s, H_s, np.array([0, T]), np.array([T]),
+                        np.asarray(w_gu_s)[None], np.asarray(w_d_s)[None], rnd)
+    return {"dAU_s": fb["dAU"], "dX_s": fb["dX_perm"], "dW_gu_s": fb["dW_gu"][0],
+            "dW_d_s": fb["dW_d"][0]}
 
 
 # --------------------------------------------------------------------------
 # Whole layer
 # --------------------------------------------------------------------------
 def layer_fwd(x, w_r, w_gu, w_d, k, bias=None, renorm=False, route=None,
-              rnd=bf16_round, expert_fn=None):
+              rnd=bf16_round, expert_fn=None, w_gu_s=None, w_d_s=None):
     E = w_r.shape[0]
     r = router_topk(x, w_r, k, bias, renorm, route)
     m = routing_metadata(r["idx"], E)
     x_perm = permute(x, m["row_map"], m["M_pad"], rnd)
     ffn = expert_ffn_fwd(x_perm, m["offsets"], m["counts"], w_gu, w_d, rnd,
                          expert_fn)
-    y = combine(ffn["O"], m["row_map"], r["w"], rnd)
+    sh = shared_expert_fwd(x, w_gu_s, w_d_s, rnd) if w_gu_s is not None else None
+    y = combine(ffn["O"], m["row_map"], r["w"], rnd, None if sh is None else sh["O"])
     out = dict(r)
     out.update(m)
     out.update({"x_perm": x_perm, "AU": ffn["AU"], "H": ffn["H"],
                 "O": ffn["O"], "y": y})
+    if sh is not None:
+        out.update({"AU_s": sh["AU"], "H_s": sh["H"], "O_s": sh["O"]})
     return out
 
 
-def layer_bwd(fwd, dy, x, w_r, w_gu, w_d, renorm=False, rnd=bf16_round):
+def layer_bwd(fwd, dy, x, w_r, w_gu, w_d, renorm=False, rnd=bf16_round, w_gu_s=None,
+              w_d_s=None):
     cb = combine_bwd(dy, fwd["O"], fwd["row_map"], fwd["w"], fwd["M_pad"], rnd)
     fb = expert_ffn_bwd(cb["dO"], fwd["x_perm"], fwd["AU"], fwd["H"],
                         fwd["offsets"], fwd["counts"], w_gu, w_d, rnd)
     rb = router_bwd(cb["dw"], fwd["probs"], fwd["idx"], x, w_r, renorm, rnd)
-    dx = permute_bwd(fb["dX_perm"], fwd["row_map"], rb["dx_router"], rnd)
+    sb = None
+    if w_gu_s is not None:
+        sb = shared_expert_bwd(dy, x, fwd["AU_s"], fwd["H_s"], w_gu_s, w_d_s, rnd)
+    dx = permute_bwd(fb["dX_perm"], fwd["row_map"], rb["dx_router"], rnd,
+                     None if sb is None else sb["dX_s"])
     out = {"dO": cb["dO"], "dw": cb["dw"], "dx": dx}
+    if sb is not None:
+        out.update(sb)
     out.update(fb)
     out.update({"dL": rb["dL"], "dx_router": rb["dx_router"],
                 "dw_r": rb["dw_r"], "db": rb["db"]})

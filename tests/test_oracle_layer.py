@@ -140,3 +140,50 @@ def test_rounding_points_are_bf16():
     # and close to the unrounded layer
     ex = R.layer_fwd(x, w_r, w_gu, w_d, k, rnd=None)
     assert np.max(np.abs(fwd["y"] - ex["y"])) / np.max(np.abs(ex["y"])) < 2e-2
+
+
+# ---------------------------------------------------------------- shared expert
+def test_shared_expert_alone_is_dense_swiglu():
+    """With every routed expert's down projection zero, the layer's output
+    and input gradient are those of the shared expert alone: a dense SwiGLU
+    over all tokens, checked against torch float64 ops and autograd."""
+    T, d, f, E, k, fs = 11, 16, 8, 4, 2, 12
+    x, w_r, w_gu, w_d, dy = _draw(T, d, f, E, 20)
+    w_d = np.zeros_like(w_d)
+    rng = np.random.default_rng(21)
+    w_gu_s = rng.standard_normal((2 * fs, d)) / np.sqrt(d)
+    w_d_s = rng.standard_normal((d, fs)) / np.sqrt(fs)
+    fwd = R.layer_fwd(x, w_r, w_gu, w_d, k, rnd=None, w_gu_s=w_gu_s, w_d_s=w_d_s)
+    xt = torch.tensor(x, requires_grad=True)
+    wg = torch.tensor(w_gu_s[:fs], requires_grad=True)
+    wu = torch.tensor(w_gu_s[fs:], requires_grad=True)
+    wd = torch.tensor(w_d_s, requires_grad=True)
+    y = (F.silu(xt @ wg.T) * (xt @ wu.T)) @ wd.T
+    np.testing.assert_allclose(fwd["y"], y.detach().numpy(), rtol=1e-12, atol=1e-13)
+    (y * torch.tensor(dy)).sum().backward()
+    bwd = R.layer_bwd(fwd, dy, x, w_r, w_gu, w_d, rnd=None, w_gu_s=w_gu_s, w_d_s=w_d_s)
+    np.testing.assert_allclose(bwd["dx"], xt.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(bwd["dW_gu_s"][:fs], wg.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(bwd["dW_gu_s"][fs:], wu.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(bwd["dW_d_s"], wd.grad.numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_shared_expert_backward_matches_finite_differences():
+    T, d, f, E, k, fs = 6, 6, 4, 4, 2, 5
+    x, w_r, w_gu, w_d, dy = _draw(T, d, f, E, 30)
+    rng = np.random.default_rng(31)
+    w_gu_s = rng.standard_normal((2 * fs, d)) / np.sqrt(d)
+    w_d_s = rng.standard_normal((d, fs)) / np.sqrt(fs)
+
+    def L():
+        fwd = R.layer_fwd(x, w_r, w_gu, w_d, k, rnd=None, w_gu_s=w_gu_s, w_d_s=w_d_s)
+        return float(np.sum(fwd["y"] * dy))
+
+    fwd = R.layer_fwd(x, w_r, w_gu, w_d, k, rnd=None, w_gu_s=w_gu_s, w_d_s=w_d_s)
+    assert _margin_ok(fwd, k)
+    bwd = R.layer_bwd(fwd, dy, x, w_r, w_gu, w_d, rnd=None, w_gu_s=w_gu_s, w_d_s=w_d_s)
+    for arr, g in [(x, bwd["dx"]), (w_gu_s, bwd["dW_gu_s"]), (w_d_s, bwd["dW_d_s"]),
+                   (w_gu, bwd["dW_gu"]), (w_r, bwd["dw_r"])]:
+        num = _fd(L, arr)
+        err = np.max(np.abs(num - g)) / max(np.max(np.abs(num)), 1e-30)
+        assert err < 1e-6, err
