@@ -196,16 +196,25 @@ def measure(L, g, steps, warmup, flush, dev, with_gemm_events=True):
     stream = torch.cuda.current_stream()
 
     def one_step(ev=None):
+        # MoELayer.forward / .backward call by call, with events around the
+        # expert GEMMs (the shared expert's included)
         L.router(g["x"], g["w_r"], g["bias"], g["route"])
         L.permute(g["x"])
+        if L.aux_alpha > 0:
+            L.load_stats()
+            L.balance_loss()
         if ev: ev[0].record(stream)
         L.experts_fwd(g["w_gu"], g["w_d"])
+        if L.shared_ff > 0:
+            L.shared_fwd(g["x"], g["w_gu_s"], g["w_d_s"])
         if ev: ev[1].record(stream)
         L.combine()
         L.combine_bwd(g["dy"])
         L.router_bwd(g["x"], g["w_r"])
         if ev: ev[2].record(stream)
         L.experts_bwd(g["w_gu"], g["w_d"])
+        if L.shared_ff > 0:
+            L.shared_bwd(g["dy"], g["x"], g["w_gu_s"], g["w_d_s"])
         if ev: ev[3].record(stream)
         L.permute_bwd(g["w_r"])
 
@@ -321,6 +330,9 @@ def run_ours(args):
     variants = {}
     if not args.no_variants and args.dtype == "bf16":
         variants["aux_loss"] = bench_cfg(cfg, args.steps, args.warmup, False, aux_alpha=0.01)
+        if cfg.name == "e8":
+            variants["shared_expert"] = bench_cfg(CONFIGS["e8_shared"], args.steps, args.warmup,
+                                                  False, shared_ff=CONFIGS["e8_shared"].shared_ff)
     ratio = None
     if not args.no_ratio and cfg.name == "e8":
         ratio = bench_cfg(CONFIGS["e128"], args.steps, args.warmup, False)
@@ -379,6 +391,13 @@ def run_ours(args):
         line["variants"]["aux_loss"]["what"] = (
             "the same step plus the load-balancing loss (alpha 0.01): load statistics, loss and "
             "its probability gradient in the router backward")
+        if "shared_expert" in variants:
+            sc = CONFIGS["e8_shared"]
+            v = variants["shared_expert"]
+            line["variants"]["shared_expert"].update({
+                "what": f"the same step plus a shared expert of d_ff {sc.shared_ff} on every token",
+                "grouped_gemm_tflops": (sc.gemm_flops_fwd_bwd() + sc.shared_flops_fwd_bwd())
+                / (statistics.mean(v["gemm_ms"]) / 1e3) / 1e12})
     if mx is not None:
         mc = CONFIGS["mxfp8"]
         line["mxfp8"] = {

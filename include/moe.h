@@ -186,13 +186,14 @@ MOE_API moe_status_t moe_grouped_swiglu_fwd(moe_handle_t h, const moe_shape_t* s
                                     void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Weighted unpermute-combine ("restore"):
- *   y[t] = bf16( sum_j topk_w[t,j] * o_perm[row_map[t,j]] ), fp32 sum in
- *   slot order.
- * In : o_perm [M_cap,d] bf16, row_map [T,k] int32, topk_w [T,k] fp32.
+ *   y[t] = bf16( sum_j topk_w[t,j] * o_perm[row_map[t,j]] + shared_out[t] ),
+ *   fp32 sum in slot order, the shared expert's output (when non-NULL) last.
+ * In : o_perm [M_cap,d] bf16, row_map [T,k] int32, topk_w [T,k] fp32,
+ *      shared_out [T,d] bf16 or NULL (moe_shared_expert_fwd).
  * Out: y [T,d] bf16. */
 MOE_API moe_status_t moe_unpermute_combine(moe_handle_t h, const moe_shape_t* s, const void* o_perm,
-                                   const int32_t* row_map, const float* topk_w, void* y,
-                                   moe_stream_t stream);
+                                   const int32_t* row_map, const float* topk_w,
+                                   const void* shared_out, void* y, moe_stream_t stream);
 
 /* Backward of the combine:
  *   do_perm[row_map[t,j]] = bf16(topk_w[t,j] * dy[t]); pad rows = 0;
@@ -224,34 +225,64 @@ MOE_API moe_status_t moe_grouped_swiglu_bwd(moe_handle_t h, const moe_shape_t* s
                                     moe_stream_t stream);
 
 /* Backward of the permute:
- *   dx[t] = bf16( sum_j dx_perm[row_map[t,j]] + dx_router[t] ), fp32 sum,
- *   rounded once.  dx_router may be NULL.
- * In : dx_perm [M_cap,d] bf16, row_map [T,k], dx_router [T,d] fp32 or NULL.
+ *   dx[t] = bf16( sum_j dx_perm[row_map[t,j]] + dx_router[t] + dx_shared[t] ),
+ *   fp32 sum, rounded once.  dx_router and dx_shared may be NULL.
+ * In : dx_perm [M_cap,d] bf16, row_map [T,k], dx_router [T,d] fp32 or NULL,
+ *      dx_shared [T,d] bf16 or NULL (moe_shared_expert_bwd).
  * Out: dx [T,d] bf16. */
 MOE_API moe_status_t moe_permute_bwd(moe_handle_t h, const moe_shape_t* s, const void* dx_perm,
-                             const int32_t* row_map, const float* dx_router, void* dx,
-                             moe_stream_t stream);
+                             const int32_t* row_map, const float* dx_router,
+                             const void* dx_shared, void* dx, moe_stream_t stream);
 
 /* Backward of the permute with the router's share of the input gradient
  * added in the same pass (the pages name only the steps; the formulas are
  * the plain backward of the router and of the permute):
  *   dL[t]  = as in moe_router_topk_bwd, from d_topk_w, probs, topk_idx and
  *            d_probs_aux (nullable)
- *   dx[t]  = bf16( sum_j dx_perm[row_map[t,j]] + dL[t] w_router ), fp32,
- *            rounded once; dL[t] w_router sums experts in increasing order.
+ *   dx[t]  = bf16( sum_j dx_perm[row_map[t,j]] + dL[t] w_router
+ *                  + dx_shared[t] ), fp32, rounded once; dL[t] w_router sums
+ *            experts in increasing order; dx_shared may be NULL.
  * Gives the same bits as moe_router_topk_bwd (with dx_router) followed by
  * moe_permute_bwd, but never stores dL w_router.  n_experts <= 64 only
  * (MOE_ERR_UNSUPPORTED otherwise: for n_experts a multiple of 128 that
  * product runs on the tensor cores inside moe_router_topk_bwd).
  * In : dx_perm [M_cap,d] bf16, row_map [T,k], d_topk_w [T,k] fp32,
  *      probs [T,E] fp32, topk_idx [T,k], d_probs_aux [E] fp32 or NULL,
- *      w_router [E,d] bf16.
+ *      w_router [E,d] bf16, dx_shared [T,d] bf16 or NULL.
  * Out: dx [T,d] bf16.  All pointers device, caller-owned; no workspace. */
 MOE_API moe_status_t moe_permute_router_bwd(moe_handle_t h, const moe_shape_t* s,
                                             const void* dx_perm, const int32_t* row_map,
                                             const float* d_topk_w, const float* probs,
                                             const int32_t* topk_idx, const float* d_probs_aux,
-                                            const void* w_router, void* dx, moe_stream_t stream);
+                                            const void* w_router, const void* dx_shared, void* dx,
+                                            moe_stream_t stream);
+
+/* Shared expert (the pages list shared experts among the v2 router's
+ * features -- Olmo-core 3 introduction page, section 4 -- without defining
+ * them; reading: one more SwiGLU expert every token passes through, its
+ * output added to the combine with weight one).  Forward, over all T tokens
+ * in place (no permute):
+ *   AU_s = bf16([x W_g^T, x W_u^T]),  H_s = bf16(silu(A) U),  O_s = bf16(H_s W_d^T)
+ * with W_gu_s [2 f_s, d] (gate rows first) and W_d_s [d, f_s]; s->T and
+ * s->d_model as for the layer, s->d_ff = f_s (n_experts, top_k unused).
+ * bf16 only.  Feed o_s to moe_unpermute_combine's shared_out.
+ * In : x [T,d], w_gu_s [2f_s,d], w_d_s [d,f_s] bf16.
+ * Out: au_s [T,2f_s], h_s [T,f_s], o_s [T,d] bf16.  No workspace. */
+MOE_API moe_status_t moe_shared_expert_fwd(moe_handle_t h, const moe_shape_t* s, const void* x,
+                                           const void* w_gu_s, const void* w_d_s, void* au_s,
+                                           void* h_s, void* o_s, moe_stream_t stream);
+
+/* Shared expert backward, from its output gradient dY (weight one):
+ *   dAU_s = SwiGLU backward of dY W_d_s (as moe_grouped_swiglu_bwd),
+ *   dW_d_s = bf16(dY^T H_s), dx_s = bf16(dAU_s W_gu_s), dW_gu_s = bf16(dAU_s^T x).
+ * Feed dx_s to moe_permute_bwd / moe_permute_router_bwd's dx_shared.
+ * In : dy [T,d], x [T,d], au_s, h_s, w_gu_s, w_d_s bf16.
+ * Out: dau_s [T,2f_s], dx_s [T,d], dw_gu_s [2f_s,d], dw_d_s [d,f_s] bf16. */
+MOE_API moe_status_t moe_shared_expert_bwd(moe_handle_t h, const moe_shape_t* s, const void* dy,
+                                           const void* x, const void* au_s, const void* h_s,
+                                           const void* w_gu_s, const void* w_d_s, void* dau_s,
+                                           void* dx_s, void* dw_gu_s, void* dw_d_s,
+                                           moe_stream_t stream);
 
 /* Router backward (through the selected probabilities; top-k itself has no
  * gradient):

@@ -39,11 +39,13 @@ SIGNATURES = {
     "moe_permute": [P, SP, P, P, P, P, P, P, P, c_size_t, P],
     "moe_permute_noalloc": [P, SP, P, P, P, P, P, P, P],
     "moe_grouped_swiglu_fwd": [P, SP, P, P, P, P, P, P, P, P, c_size_t, P],
-    "moe_unpermute_combine": [P, SP, P, P, P, P, P],
+    "moe_unpermute_combine": [P, SP, P, P, P, P, P, P],
     "moe_unpermute_combine_bwd": [P, SP, P, P, P, P, P, P, P, P, P],
     "moe_grouped_swiglu_bwd": [P, SP, P, P, P, P, P, P, P, P, P, P, P, P, c_size_t, P],
-    "moe_permute_bwd": [P, SP, P, P, P, P, P],
-    "moe_permute_router_bwd": [P, SP, P, P, P, P, P, P, P, P, P],
+    "moe_permute_bwd": [P, SP, P, P, P, P, P, P],
+    "moe_permute_router_bwd": [P, SP, P, P, P, P, P, P, P, P, P, P],
+    "moe_shared_expert_fwd": [P, SP, P, P, P, P, P, P, P],
+    "moe_shared_expert_bwd": [P, SP, P, P, P, P, P, P, P, P, P, P, P],
     "moe_router_topk_bwd": [P, SP, P, P, P, P, P, P, P, P, P, P, c_size_t, P],
     "moe_router_load_stats": [P, SP, P, P, c_int, P, P, c_size_t, P],
     "moe_router_aux_loss": [P, SP, P, c_int64, ctypes.c_float, P, P, P],

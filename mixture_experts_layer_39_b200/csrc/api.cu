@@ -288,15 +288,17 @@ moe_status_t moe_grouped_swiglu_fwd(moe_handle_t h, const moe_shape_t* s, const 
 }
 
 moe_status_t moe_unpermute_combine(moe_handle_t h, const moe_shape_t* s, const void* o_perm,
-                                   const int32_t* row_map, const float* topk_w, void* y,
-                                   moe_stream_t stream) {
+                                   const int32_t* row_map, const float* topk_w,
+                                   const void* shared_out, void* y, moe_stream_t stream) {
   MOE_CHECK_HANDLE(h, s);
   if (!all_nonnull(o_perm, row_map, topk_w, y)) return MOE_ERR_INVALID_ARG;
-  if (!aligned(o_perm, 16) || !aligned(y, 16)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(o_perm, 16) || !aligned(y, 16) || !aligned(shared_out, 16))
+    return MOE_ERR_INVALID_ARG;
   MOE_GUARD(h);
   h->launches += 1;
   return cuda_status(moe::launch_combine(static_cast<const __nv_bfloat16*>(o_perm), row_map, topk_w,
-                                         s->T, s->d_model, s->top_k,
+                                         static_cast<const __nv_bfloat16*>(shared_out), s->T,
+                                         s->d_model, s->top_k,
                                          static_cast<__nv_bfloat16*>(y),
                                          static_cast<cudaStream_t>(stream)));
 }
@@ -375,17 +377,65 @@ moe_status_t moe_grouped_swiglu_bwd(moe_handle_t h, const moe_shape_t* s, const 
   return moe::gemm_wgrad_gate_up(c, dau, x_perm, offsets, dw_gu, E, d, f, m_cap, st);
 }
 
+// Shared expert: the routed experts' GEMMs over one group of all T tokens,
+// read in place from x / dY (no permute); tensor maps are exactly T rows
+// tall, so a ragged last tile reads zeros.
+moe_status_t moe_shared_expert_fwd(moe_handle_t h, const moe_shape_t* s, const void* x,
+                                   const void* w_gu_s, const void* w_d_s, void* au_s, void* h_s,
+                                   void* o_s, moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  if (s->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (!all_nonnull(x, w_gu_s, w_d_s, au_s, h_s, o_s)) return MOE_ERR_INVALID_ARG;
+  for (const void* p : {x, w_gu_s, w_d_s, static_cast<const void*>(au_s),
+                        static_cast<const void*>(h_s), static_cast<const void*>(o_s)})
+    if (!aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  const moe_shape_t one{s->T, s->d_model, s->d_ff, 1, 1, MOE_DTYPE_BF16, 0};
+  auto st = static_cast<cudaStream_t>(stream);
+  MOE_GUARD(h);
+  moe::GemmCtx c{h->num_sms, h->ctl, pair_tiles(&one)};
+  h->launches += 2;
+  MOE_TRY(moe::gemm_fwd_gate_up(c, x, nullptr, w_gu_s, au_s, h_s, 1, s->d_model, s->d_ff, s->T, st));
+  return moe::gemm_fwd_down(c, h_s, nullptr, w_d_s, o_s, 1, s->d_model, s->d_ff, s->T, st);
+}
+
+moe_status_t moe_shared_expert_bwd(moe_handle_t h, const moe_shape_t* s, const void* dy,
+                                   const void* x, const void* au_s, const void* h_s,
+                                   const void* w_gu_s, const void* w_d_s, void* dau_s, void* dx_s,
+                                   void* dw_gu_s, void* dw_d_s, moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  if (s->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (!all_nonnull(dy, x, au_s, h_s, w_gu_s, w_d_s, dau_s, dx_s, dw_gu_s, dw_d_s))
+    return MOE_ERR_INVALID_ARG;
+  for (const void* p : {dy, x, au_s, h_s, w_gu_s, w_d_s, static_cast<const void*>(dau_s),
+                        static_cast<const void*>(dx_s), static_cast<const void*>(dw_gu_s),
+                        static_cast<const void*>(dw_d_s)})
+    if (!aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  const moe_shape_t one{s->T, s->d_model, s->d_ff, 1, 1, MOE_DTYPE_BF16, 0};
+  const int d = s->d_model, f = s->d_ff, T = s->T;
+  auto st = static_cast<cudaStream_t>(stream);
+  MOE_GUARD(h);
+  moe::GemmCtx c{h->num_sms, h->ctl, pair_tiles(&one)};
+  h->launches += 4;
+  MOE_TRY(moe::gemm_dgrad_down_swiglu(c, dy, nullptr, w_d_s, au_s, dau_s, 1, d, f, T, st));
+  MOE_TRY(moe::gemm_wgrad_down(c, dy, h_s, nullptr, dw_d_s, 1, d, f, T, st));
+  MOE_TRY(moe::gemm_dgrad_gate_up(c, dau_s, nullptr, w_gu_s, dx_s, 1, d, f, T, st));
+  return moe::gemm_wgrad_gate_up(c, dau_s, x, nullptr, dw_gu_s, 1, d, f, T, st);
+}
+
 moe_status_t moe_permute_bwd(moe_handle_t h, const moe_shape_t* s, const void* dx_perm,
-                             const int32_t* row_map, const float* dx_router, void* dx,
-                             moe_stream_t stream) {
+                             const int32_t* row_map, const float* dx_router, const void* dx_shared,
+                             void* dx, moe_stream_t stream) {
   MOE_CHECK_HANDLE(h, s);
   if (!all_nonnull(dx_perm, row_map, dx)) return MOE_ERR_INVALID_ARG;
-  if (!aligned(dx_perm, 16) || !aligned(dx, 16) || !aligned(dx_router, 16))
+  if (!aligned(dx_perm, 16) || !aligned(dx, 16) || !aligned(dx_router, 16) ||
+      !aligned(dx_shared, 16))
     return MOE_ERR_INVALID_ARG;
   MOE_GUARD(h);
   h->launches += 1;
   return cuda_status(moe::launch_permute_bwd(static_cast<const __nv_bfloat16*>(dx_perm), row_map,
-                                             dx_router, s->T, s->d_model, s->top_k,
+                                             dx_router,
+                                             static_cast<const __nv_bfloat16*>(dx_shared), s->T,
+                                             s->d_model, s->top_k,
                                              static_cast<__nv_bfloat16*>(dx),
                                              static_cast<cudaStream_t>(stream)));
 }
@@ -393,20 +443,22 @@ moe_status_t moe_permute_bwd(moe_handle_t h, const moe_shape_t* s, const void* d
 moe_status_t moe_permute_router_bwd(moe_handle_t h, const moe_shape_t* s, const void* dx_perm,
                                     const int32_t* row_map, const float* d_topk_w,
                                     const float* probs, const int32_t* topk_idx,
-                                    const float* d_probs_aux, const void* w_router, void* dx,
-                                    moe_stream_t stream) {
+                                    const float* d_probs_aux, const void* w_router,
+                                    const void* dx_shared, void* dx, moe_stream_t stream) {
   MOE_CHECK_HANDLE(h, s);
   MOE_TRY(check_router_shape(s));
   if (s->n_experts > 64) return MOE_ERR_UNSUPPORTED;
   if (!all_nonnull(dx_perm, row_map, d_topk_w, probs, topk_idx, w_router, dx))
     return MOE_ERR_INVALID_ARG;
-  if (!aligned(dx_perm, 16) || !aligned(dx, 16) || !aligned(w_router, 16))
+  if (!aligned(dx_perm, 16) || !aligned(dx, 16) || !aligned(w_router, 16) ||
+      !aligned(dx_shared, 16))
     return MOE_ERR_INVALID_ARG;
   MOE_GUARD(h);
   h->launches += 1;
   return cuda_status(moe::launch_permute_router_bwd(
       static_cast<const __nv_bfloat16*>(dx_perm), row_map, d_topk_w, probs, topk_idx, d_probs_aux,
-      static_cast<const __nv_bfloat16*>(w_router), s->T, s->d_model, s->n_experts, s->top_k,
+      static_cast<const __nv_bfloat16*>(w_router), static_cast<const __nv_bfloat16*>(dx_shared),
+      s->T, s->d_model, s->n_experts, s->top_k,
       (s->flags & MOE_FLAG_RENORM) != 0, static_cast<__nv_bfloat16*>(dx),
       static_cast<cudaStream_t>(stream)));
 }

@@ -125,6 +125,7 @@ moe_status_t gemm_fwd_gate_up(const GemmCtx& c, const void* x_perm, const int32_
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
+  a.uniform_len = static_cast<int>(m_cap);  // one group of m_cap rows when offsets is null
   a.m_cap = m_cap;
   a.out = au;
   a.ldo = 2ll * f;
@@ -148,6 +149,7 @@ moe_status_t gemm_fwd_down(const GemmCtx& c, const void* h, const int32_t* offse
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
+  a.uniform_len = static_cast<int>(m_cap);  // one group of m_cap rows when offsets is null
   a.m_cap = m_cap;
   a.out = o_perm;
   a.ldo = d;
@@ -168,6 +170,7 @@ moe_status_t gemm_dgrad_down_swiglu(const GemmCtx& c, const void* do_perm, const
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
+  a.uniform_len = static_cast<int>(m_cap);  // one group of m_cap rows when offsets is null
   a.m_cap = m_cap;
   a.out = dau;
   a.ldo = 2ll * f;
@@ -191,6 +194,7 @@ moe_status_t gemm_dgrad_gate_up(const GemmCtx& c, const void* dau, const int32_t
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
+  a.uniform_len = static_cast<int>(m_cap);  // one group of m_cap rows when offsets is null
   a.m_cap = m_cap;
   a.out = dx_perm;
   a.ldo = d;
@@ -211,6 +215,7 @@ moe_status_t gemm_wgrad_down(const GemmCtx& c, const void* do_perm, const void* 
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
+  a.uniform_len = static_cast<int>(m_cap);  // one group of m_cap rows when offsets is null
   a.out = dw_d;
   a.ldo = f;
   a.out_gstride = static_cast<int64_t>(d) * f;
@@ -232,6 +237,7 @@ moe_status_t gemm_wgrad_gate_up(const GemmCtx& c, const void* dau, const void* x
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
+  a.uniform_len = static_cast<int>(m_cap);  // one group of m_cap rows when offsets is null
   a.out = dw_gu;
   a.ldo = d;
   a.out_gstride = 2ll * f * d;
@@ -328,6 +334,7 @@ moe_status_t gemm_mx_fwd_gate_up(const GemmCtx& c, const MxOperand& x, const int
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
+  a.uniform_len = static_cast<int>(m_cap);  // one group of m_cap rows when offsets is null
   a.m_cap = m_cap;
   a.out = au;
   a.ldo = 2ll * f;
@@ -351,6 +358,7 @@ moe_status_t gemm_mx_fwd_down(const GemmCtx& c, const MxOperand& h, const int32_
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
+  a.uniform_len = static_cast<int>(m_cap);  // one group of m_cap rows when offsets is null
   a.m_cap = m_cap;
   a.out = o_perm;
   a.ldo = d;
@@ -372,6 +380,7 @@ moe_status_t gemm_mx_dgrad_down_swiglu(const GemmCtx& c, const MxOperand& dO, co
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
+  a.uniform_len = static_cast<int>(m_cap);  // one group of m_cap rows when offsets is null
   a.m_cap = m_cap;
   a.out = dau;
   a.ldo = 2ll * f;
@@ -395,6 +404,7 @@ moe_status_t gemm_mx_dgrad_gate_up(const GemmCtx& c, const MxOperand& dau, const
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
+  a.uniform_len = static_cast<int>(m_cap);  // one group of m_cap rows when offsets is null
   a.m_cap = m_cap;
   a.out = dx_perm;
   a.ldo = d;
@@ -417,6 +427,7 @@ moe_status_t gemm_mx_wgrad(const GemmCtx& c, const MxOperand& a_col, int M, cons
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
+  a.uniform_len = static_cast<int>(m_cap);  // one group of m_cap rows when offsets is null
   a.out = dw;
   a.ldo = N;
   a.out_gstride = static_cast<int64_t>(M) * N;

@@ -43,22 +43,23 @@ cudaError_t launch_permute_scatter(const __nv_bfloat16* x, const int32_t* row_ma
 
 // ---- combine and backwards
 cudaError_t launch_combine(const __nv_bfloat16* o_perm, const int32_t* row_map, const float* w,
-                           int T, int d, int k, __nv_bfloat16* y, cudaStream_t st);
+                           const __nv_bfloat16* shared, int T, int d, int k, __nv_bfloat16* y,
+                           cudaStream_t st);
 cudaError_t launch_combine_bwd(const __nv_bfloat16* dy, const __nv_bfloat16* o_perm,
                                const int32_t* row_map, const float* w, const int32_t* offsets,
                                const int32_t* counts, int T, int d, int k, int E,
                                __nv_bfloat16* do_perm, float* dw, cudaStream_t st);
 cudaError_t launch_permute_bwd(const __nv_bfloat16* dx_perm, const int32_t* row_map,
-                               const float* dx_router, int T, int d, int k, __nv_bfloat16* dx,
-                               cudaStream_t st);
+                               const float* dx_router, const __nv_bfloat16* dx_shared, int T, int d,
+                               int k, __nv_bfloat16* dx, cudaStream_t st);
 
 // ---- router backward
 // dX = bf16(unpermute-reduce of dX_perm + dL W_r) in one pass, E <= 64.
 cudaError_t launch_permute_router_bwd(const __nv_bfloat16* dx_perm, const int32_t* row_map,
                                       const float* dw, const float* probs, const int32_t* idx,
-                                      const float* dprob_aux, const __nv_bfloat16* w_r, int T,
-                                      int d, int E, int k, bool renorm, __nv_bfloat16* dx,
-                                      cudaStream_t st);
+                                      const float* dprob_aux, const __nv_bfloat16* w_r,
+                                      const __nv_bfloat16* dx_shared, int T, int d, int E, int k,
+                                      bool renorm, __nv_bfloat16* dx, cudaStream_t st);
 int router_bwd_blocks(int num_sms);
 cudaError_t launch_router_bwd_dl(const float* dw, const float* probs, const int32_t* idx,
                                  const float* dprob_aux, const __nv_bfloat16* w_r, int T, int d,

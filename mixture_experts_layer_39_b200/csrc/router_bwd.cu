@@ -171,7 +171,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
                               const int32_t* __restrict__ idx,
                               const float* __restrict__ dprob_aux,
                               const __nv_bfloat16* __restrict__ w_r,
-                              int T, int d, int E, int k, int renorm, uint4* __restrict__ dx) {
+                              const uint4* __restrict__ dxs, int T, int d, int E, int k,
+                              int renorm, uint4* __restrict__ dx) {
   constexpr int NPL = (NE + 31) / 32;
   const int lane = threadIdx.x & 31;
   const int64_t t0 = (static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5)) * TPW;
@@ -216,6 +217,12 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
       }
 #pragma unroll
       for (int c = 0; c < 8; ++c) acc[c] += r[h][c];
+      if (dxs != nullptr) {  // the shared expert's input gradient, added last
+        float f[8];
+        unpack8(__ldg(dxs + (t0 + h) * nvec + v), f);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] += f[c];
+      }
       dx[(t0 + h) * nvec + v] = pack8(acc);
     }
   }
@@ -377,13 +384,15 @@ __global__ void __launch_bounds__(kRedWarps * 32)
 
 cudaError_t launch_permute_router_bwd(const __nv_bfloat16* dx_perm, const int32_t* row_map,
                                       const float* dw, const float* probs, const int32_t* idx,
-                                      const float* dprob_aux, const __nv_bfloat16* w_r, int T,
-                                      int d, int E, int k, bool renorm, __nv_bfloat16* dx,
-                                      cudaStream_t st) {
+                                      const float* dprob_aux, const __nv_bfloat16* w_r,
+                                      const __nv_bfloat16* dx_shared, int T, int d, int E, int k,
+                                      bool renorm, __nv_bfloat16* dx, cudaStream_t st) {
   auto go = [&](auto kern, int tpw) {
     const unsigned grid = static_cast<unsigned>(ceil_div64(T, static_cast<int64_t>(kWarps) * tpw));
     kern<<<grid, kWarps * 32, 0, st>>>(reinterpret_cast<const uint4*>(dx_perm), row_map, dw, probs,
-                                       idx, dprob_aux, w_r, T, d, E, k, renorm ? 1 : 0,
+                                       idx, dprob_aux, w_r,
+                                       reinterpret_cast<const uint4*>(dx_shared), T, d, E, k,
+                                       renorm ? 1 : 0,
                                        reinterpret_cast<uint4*>(dx));
     return cudaGetLastError();
   };

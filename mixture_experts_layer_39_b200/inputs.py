@@ -12,6 +12,7 @@ Workloads (shapes and value distributions):
   skew   T=32768 d=2048 f=1024 E=128 k=4  router bias b_e = 2*ln(1/(e+1))
   mxfp8  T=32768 d=4096 f=1536 E=128 k=4  uniform random expert ids,
                                           drawn without replacement
+  e8_shared  e8 plus one shared expert of d_ff 1024 (every token)
 
 Values: x ~ N(0,1); router weight, gate/up and down weights ~ N(0, 1/d);
 upstream gradient dY ~ N(0,1); everything rounded to bf16 (round to
@@ -30,6 +31,8 @@ Layouts (row-major):
   dy     [T, d]        bf16   upstream gradient of y
   bias   [E]           fp32 or None
   route  [T, k]        int32 or None (random-routing expert ids)
+  w_gu_s [2fs, d]      bf16   shared expert gate/up (only with shared_ff = fs > 0)
+  w_d_s  [d, fs]       bf16   shared expert down projection
 """
 from __future__ import annotations
 
@@ -50,6 +53,7 @@ class MoEConfig:
     skew_bias: bool = False
     random_routing: bool = False
     mxfp8: bool = False
+    shared_ff: int = 0
 
     @property
     def routed_rows(self) -> int:
@@ -64,6 +68,10 @@ class MoEConfig:
         # gate/up 4dfM + down 2dfM forward, twice that backward
         return 18.0 * self.d * self.f * self.T * self.k
 
+    def shared_flops_fwd_bwd(self) -> float:
+        # the same for the shared expert over all T tokens
+        return 18.0 * self.d * self.shared_ff * self.T
+
 
 CONFIGS = {
     "tiny": MoEConfig("tiny", 512, 256, 512, 8, 4),
@@ -72,12 +80,13 @@ CONFIGS = {
     "skew": MoEConfig("skew", 32768, 2048, 1024, 128, 4, skew_bias=True),
     "mxfp8": MoEConfig("mxfp8", 32768, 4096, 1536, 128, 4,
                        random_routing=True, mxfp8=True),
+    "e8_shared": MoEConfig("e8_shared", 16384, 2048, 1024, 8, 4, shared_ff=1024),
 }
 
 
 def custom_config(T, d, f, E, k, name="custom", skew_bias=False,
-                  random_routing=False, mxfp8=False) -> MoEConfig:
-    return MoEConfig(name, T, d, f, E, k, skew_bias, random_routing, mxfp8)
+                  random_routing=False, mxfp8=False, shared_ff=0) -> MoEConfig:
+    return MoEConfig(name, T, d, f, E, k, skew_bias, random_routing, mxfp8, shared_ff)
 
 
 def _randn(shape, std, gen, device):
@@ -113,4 +122,7 @@ def make_inputs(cfg: MoEConfig, seed: int = 0, device="cpu") -> dict:
     if cfg.random_routing:
         noise = torch.rand((cfg.T, cfg.E), generator=gen, device=dev)
         out["route"] = noise.argsort(dim=1)[:, : cfg.k].to(torch.int32).contiguous()
+    if cfg.shared_ff > 0:  # drawn last: the other tensors do not change
+        out["w_gu_s"] = _randn((2 * cfg.shared_ff, cfg.d), std_w, gen, dev)
+        out["w_d_s"] = _randn((cfg.d, cfg.shared_ff), std_w, gen, dev)
     return out

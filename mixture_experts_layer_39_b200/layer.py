@@ -12,6 +12,10 @@ in order on the current stream:
             cores), moe_router_topk_bwd writes dX_router and
             moe_permute_bwd adds it.
 
+With shared_ff > 0 a shared expert runs on every token
+(moe_shared_expert_fwd / _bwd); its output joins the combine and its input
+gradient the permute backward.
+
 With aux_alpha > 0 the forward also forms the router's load statistics and
 the load-balancing loss (moe_router_load_stats -> moe_router_aux_loss) and
 the backward adds the loss's gradient in the router backward.
@@ -36,7 +40,7 @@ class MoELayer:
     def __init__(self, T, d, f, E, k, device="cuda", renorm=False, keep_logits=False,
                  handle: ops.Handle | None = None, dtype: str = "bf16",
                  fuse_router_dx: bool | None = None, aux_alpha: float = 0.0,
-                 aux_reduce: Callable | None = None):
+                 aux_reduce: Callable | None = None, shared_ff: int = 0):
         """dtype: "bf16", or "mxfp8" for E4M3/E8M0 expert GEMM operands (the
         library then also aligns expert segments to 128 rows).
         fuse_router_dx: add the router's input gradient inside the permute
@@ -45,7 +49,10 @@ class MoELayer:
         aux_alpha: weight of the load-balancing loss (0: none).  aux_reduce:
         optional callable(stats) -> n_tokens that sums the statistics over
         ranks in place and returns the global batch's token count
-        (replicas.global_stats_reducer), for balancing over the global batch."""
+        (replicas.global_stats_reducer), for balancing over the global batch.
+        shared_ff: hidden size of a shared expert every token passes through
+        (0: none); its weights are passed to forward/backward/step as
+        w_gu_s [2*shared_ff, d] and w_d_s [d, shared_ff]."""
         self.T, self.d, self.f, self.E, self.k = T, d, f, E, k
         dev = torch.device(device)
         self.device = dev
@@ -84,6 +91,16 @@ class MoELayer:
         self.stats = z(2 * E, dt=F32)
         self.aux_loss = z(1, dt=F32)
         self.dprob_aux = z(E, dt=F32) if self.aux_alpha > 0 else None
+        # shared expert
+        self.shared_ff = int(shared_ff)
+        if self.shared_ff > 0:
+            fs = self.shared_ff
+            self.shared_shape = ops.make_shape(T, d, fs, 1, 1, MOE_DTYPE_BF16, False)
+            self.au_s, self.h_s, self.o_s = z(T, 2 * fs), z(T, fs), z(T, d)
+            self.dau_s, self.dx_s = z(T, 2 * fs), z(T, d)
+            self.dw_gu_s, self.dw_d_s = z(2 * fs, d), z(d, fs)
+        else:
+            self.o_s = self.dx_s = None
 
     # ------------------------------------------------------------- forward
     def router(self, x, w_r, bias=None, route=None, stream=None):
@@ -98,9 +115,13 @@ class MoELayer:
         ops.moe_grouped_swiglu_fwd(self.handle, self.shape, self.x_perm, self.offsets, w_gu, w_d,
                                    self.au, self.h, self.o_perm, self.ws, stream)
 
+    def shared_fwd(self, x, w_gu_s, w_d_s, stream=None):
+        ops.moe_shared_expert_fwd(self.handle, self.shared_shape, x, w_gu_s, w_d_s, self.au_s,
+                                  self.h_s, self.o_s, stream)
+
     def combine(self, stream=None):
         ops.moe_unpermute_combine(self.handle, self.shape, self.o_perm, self.row_map, self.w,
-                                  self.y, stream)
+                                  self.o_s, self.y, stream)
 
     def load_stats(self, accumulate=False, stream=None):
         """[counts | sum_t probs] of this batch into self.stats (added when
@@ -116,7 +137,13 @@ class MoELayer:
                                 self.T if n_tokens is None else n_tokens, self.aux_alpha,
                                 self.aux_loss, self.dprob_aux, stream)
 
-    def forward(self, x, w_r, w_gu, w_d, bias=None, route=None, stream=None):
+    def _need_shared(self, w_gu_s, w_d_s):
+        if self.shared_ff > 0 and (w_gu_s is None or w_d_s is None):
+            raise ValueError("this layer has a shared expert: pass w_gu_s and w_d_s")
+
+    def forward(self, x, w_r, w_gu, w_d, bias=None, route=None, stream=None, w_gu_s=None,
+                w_d_s=None):
+        self._need_shared(w_gu_s, w_d_s)
         self.router(x, w_r, bias, route, stream)
         self.permute(x, stream)
         if self.aux_alpha > 0:
@@ -124,6 +151,8 @@ class MoELayer:
             n = self.aux_reduce(self.stats) if self.aux_reduce is not None else self.T
             self.balance_loss(None, n, stream)
         self.experts_fwd(w_gu, w_d, stream)
+        if self.shared_ff > 0:
+            self.shared_fwd(x, w_gu_s, w_d_s, stream)
         self.combine(stream)
         return self.y
 
@@ -149,18 +178,27 @@ class MoELayer:
                 raise ValueError("the fused permute backward needs w_r")
             ops.moe_permute_router_bwd(self.handle, self.shape, self.dx_perm, self.row_map,
                                        self.dw, self.probs, self.idx, self.dprob_aux, w_r,
-                                       self.dx, stream)
+                                       self.dx_s, self.dx, stream)
         else:
             ops.moe_permute_bwd(self.handle, self.shape, self.dx_perm, self.row_map,
-                                self.dx_router, self.dx, stream)
+                                self.dx_router, self.dx_s, self.dx, stream)
 
-    def backward(self, dy, x, w_r, w_gu, w_d, stream=None):
+    def shared_bwd(self, dy, x, w_gu_s, w_d_s, stream=None):
+        ops.moe_shared_expert_bwd(self.handle, self.shared_shape, dy, x, self.au_s, self.h_s,
+                                  w_gu_s, w_d_s, self.dau_s, self.dx_s, self.dw_gu_s,
+                                  self.dw_d_s, stream)
+
+    def backward(self, dy, x, w_r, w_gu, w_d, stream=None, w_gu_s=None, w_d_s=None):
+        self._need_shared(w_gu_s, w_d_s)
         self.combine_bwd(dy, stream)
         self.router_bwd(x, w_r, stream)
         self.experts_bwd(w_gu, w_d, stream)
+        if self.shared_ff > 0:
+            self.shared_bwd(dy, x, w_gu_s, w_d_s, stream)
         self.permute_bwd(w_r, stream)
         return self.dx
 
-    def step(self, x, w_r, w_gu, w_d, dy, bias=None, route=None, stream=None):
-        self.forward(x, w_r, w_gu, w_d, bias, route, stream)
-        self.backward(dy, x, w_r, w_gu, w_d, stream)
+    def step(self, x, w_r, w_gu, w_d, dy, bias=None, route=None, stream=None, w_gu_s=None,
+             w_d_s=None):
+        self.forward(x, w_r, w_gu, w_d, bias, route, stream, w_gu_s, w_d_s)
+        self.backward(dy, x, w_r, w_gu, w_d, stream, w_gu_s, w_d_s)

@@ -112,9 +112,9 @@ def moe_grouped_swiglu_fwd(h, shape, x_perm, offsets, w_gu, w_down, au, hbuf, o_
           ws.numel() if ws is not None else 0, _stream(stream))
 
 
-def moe_unpermute_combine(h, shape, o_perm, row_map, topk_w, y, stream=None):
+def moe_unpermute_combine(h, shape, o_perm, row_map, topk_w, shared_out, y, stream=None):
     _call("moe_unpermute_combine", h.ptr, ctypes.byref(shape), _ptr(o_perm), _ptr(row_map),
-          _ptr(topk_w), _ptr(y), _stream(stream))
+          _ptr(topk_w), _ptr(shared_out), _ptr(y), _stream(stream))
 
 
 def moe_unpermute_combine_bwd(h, shape, dy, o_perm, row_map, topk_w, offsets, counts, do_perm,
@@ -132,16 +132,28 @@ def moe_grouped_swiglu_bwd(h, shape, do_perm, x_perm, au, hbuf, offsets, w_gu, w
           ws.numel() if ws is not None else 0, _stream(stream))
 
 
-def moe_permute_bwd(h, shape, dx_perm, row_map, dx_router, dx, stream=None):
+def moe_permute_bwd(h, shape, dx_perm, row_map, dx_router, dx_shared, dx, stream=None):
     _call("moe_permute_bwd", h.ptr, ctypes.byref(shape), _ptr(dx_perm), _ptr(row_map),
-          _ptr(dx_router), _ptr(dx), _stream(stream))
+          _ptr(dx_router), _ptr(dx_shared), _ptr(dx), _stream(stream))
+
+
+def moe_shared_expert_fwd(h, shape, x, w_gu_s, w_d_s, au_s, h_s, o_s, stream=None):
+    _call("moe_shared_expert_fwd", h.ptr, ctypes.byref(shape), _ptr(x), _ptr(w_gu_s), _ptr(w_d_s),
+          _ptr(au_s), _ptr(h_s), _ptr(o_s), _stream(stream))
+
+
+def moe_shared_expert_bwd(h, shape, dy, x, au_s, h_s, w_gu_s, w_d_s, dau_s, dx_s, dw_gu_s, dw_d_s,
+                          stream=None):
+    _call("moe_shared_expert_bwd", h.ptr, ctypes.byref(shape), _ptr(dy), _ptr(x), _ptr(au_s),
+          _ptr(h_s), _ptr(w_gu_s), _ptr(w_d_s), _ptr(dau_s), _ptr(dx_s), _ptr(dw_gu_s),
+          _ptr(dw_d_s), _stream(stream))
 
 
 def moe_permute_router_bwd(h, shape, dx_perm, row_map, d_topk_w, probs, topk_idx, d_probs_aux,
-                           w_router, dx, stream=None):
+                           w_router, dx_shared, dx, stream=None):
     _call("moe_permute_router_bwd", h.ptr, ctypes.byref(shape), _ptr(dx_perm), _ptr(row_map),
-          _ptr(d_topk_w), _ptr(probs), _ptr(topk_idx), _ptr(d_probs_aux), _ptr(w_router), _ptr(dx),
-          _stream(stream))
+          _ptr(d_topk_w), _ptr(probs), _ptr(topk_idx), _ptr(d_probs_aux), _ptr(w_router),
+          _ptr(dx_shared), _ptr(dx), _stream(stream))
 
 
 def moe_router_topk_bwd(h, shape, d_topk_w, probs, topk_idx, d_probs_aux, x, w_router, dx_router,

@@ -56,12 +56,15 @@ class HostStepper:
                 self.route[b].copy_(route_h, non_blocking=True)
             self.in_ready[b].record(self.copy_in)
 
-    def run(self, steps, w_r, w_gu, w_d, bias=None, after: torch.cuda.Event | None = None):
+    def run(self, steps, w_r, w_gu, w_d, bias=None, after: torch.cuda.Event | None = None,
+            shared=None):
         """steps: list of dicts with pinned host tensors "x", "dy", "y", "dx"
         (and "route" in random-routing mode).  Results land in each step's
         "y" and "dx" host tensors; the call returns after enqueuing
         everything (synchronise the device to read them).  `after`: an event
-        that the first copy waits for."""
+        that the first copy waits for.  `shared`: (w_gu_s, w_d_s) for a layer
+        with a shared expert."""
+        ws = {} if shared is None else {"w_gu_s": shared[0], "w_d_s": shared[1]}
         L = self.L
         n = len(steps)
         if n == 0:
@@ -83,9 +86,9 @@ class HostStepper:
                 c.wait_event(self.dx_out[b])
             L.y, L.dx = self.y[b], self.dx[b]
             x, dy, route = self.x[b], self.dy[b], self.route[b]
-            L.forward(x, w_r, w_gu, w_d, bias, route)
+            L.forward(x, w_r, w_gu, w_d, bias, route, **ws)
             self.fwd_done[b].record(c)
-            L.backward(dy, x, w_r, w_gu, w_d)
+            L.backward(dy, x, w_r, w_gu, w_d, **ws)
             self.bwd_done[b].record(c)
             self.in_free[b].record(c)
             with torch.cuda.stream(self.copy_out):
