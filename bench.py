@@ -330,6 +330,7 @@ def run_ours(args):
     variants = {}
     if not args.no_variants and args.dtype == "bf16":
         variants["aux_loss"] = bench_cfg(cfg, args.steps, args.warmup, False, aux_alpha=0.01)
+        variants["recompute"] = bench_cfg(cfg, args.steps, args.warmup, False, recompute=True)
         if cfg.name == "e8":
             variants["shared_expert"] = bench_cfg(CONFIGS["e8_shared"], args.steps, args.warmup,
                                                   False, shared_ff=CONFIGS["e8_shared"].shared_ff)
@@ -391,6 +392,13 @@ def run_ours(args):
         line["variants"]["aux_loss"]["what"] = (
             "the same step plus the load-balancing loss (alpha 0.01): load statistics, loss and "
             "its probability gradient in the router backward")
+        if "recompute" in variants:
+            M = cfg.T * cfg.k
+            line["variants"]["recompute"]["what"] = (
+                "activation recompute: the forward keeps no [A|U], the backward recomputes the "
+                f"gate/up GEMM (+{4 * cfg.d * cfg.f * M / 1e9:.0f} GFLOP/step); activations "
+                f"kept from forward to backward shrink by {(2 * cfg.f + cfg.f) * 2 * M / 2**20:.0f} "
+                "MiB of [A|U] and H")
         if "shared_expert" in variants:
             sc = CONFIGS["e8_shared"]
             v = variants["shared_expert"]

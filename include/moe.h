@@ -177,13 +177,29 @@ MOE_API moe_status_t moe_permute_noalloc(moe_handle_t h, const moe_shape_t* s, c
  *   o_perm = bf16(h W_down[e]^T)
  * In : x_perm [M_cap,d] bf16, offsets [E+1] int32 (from moe_permute),
  *      w_gu [E,2f,d] bf16, w_down [E,d,f] bf16.
- * Out: au [M_cap,2f] bf16, h [M_cap,f] bf16, o_perm [M_cap,d] bf16.
+ * Out: au [M_cap,2f] bf16 (or NULL: not kept, for activation recompute),
+ *      h [M_cap,f] bf16, o_perm [M_cap,d] bf16.
  * Persistent tcgen05/TMEM kernels fed by TMA; the tile schedule is decoded
  * from `offsets` on the device. */
 MOE_API moe_status_t moe_grouped_swiglu_fwd(moe_handle_t h, const moe_shape_t* s, const void* x_perm,
                                     const int32_t* offsets, const void* w_gu,
                                     const void* w_down, void* au, void* hbuf, void* o_perm,
                                     void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Activation recompute (the pages: recomputing activations in the backward
+ * cuts about two thirds of activation memory for about a fifth of
+ * throughput -- Olmo-core 3 introduction page, section 4).  Recomputes the
+ * forward's gate/up GEMM and SwiGLU for the backward: the same au and h, bit
+ * for bit, as moe_grouped_swiglu_fwd on the same inputs (MXFP8 mode
+ * re-quantises x_perm and w_gu in the workspace first).  With it the
+ * forward can run with au = NULL and h as a transient buffer, and only
+ * x_perm and o_perm need to live from the forward to the backward.
+ * In : x_perm [M_cap,d] bf16, offsets [E+1], w_gu [E,2f,d] bf16.
+ * Out: au [M_cap,2f] bf16, h [M_cap,f] bf16. */
+MOE_API moe_status_t moe_grouped_swiglu_recompute(moe_handle_t h, const moe_shape_t* s,
+                                                  const void* x_perm, const int32_t* offsets,
+                                                  const void* w_gu, void* au, void* hbuf, void* ws,
+                                                  size_t ws_bytes, moe_stream_t stream);
 
 /* Weighted unpermute-combine ("restore"):
  *   y[t] = bf16( sum_j topk_w[t,j] * o_perm[row_map[t,j]] + shared_out[t] ),

@@ -39,6 +39,7 @@ SIGNATURES = {
     "moe_permute": [P, SP, P, P, P, P, P, P, P, c_size_t, P],
     "moe_permute_noalloc": [P, SP, P, P, P, P, P, P, P],
     "moe_grouped_swiglu_fwd": [P, SP, P, P, P, P, P, P, P, P, c_size_t, P],
+    "moe_grouped_swiglu_recompute": [P, SP, P, P, P, P, P, P, c_size_t, P],
     "moe_unpermute_combine": [P, SP, P, P, P, P, P, P],
     "moe_unpermute_combine_bwd": [P, SP, P, P, P, P, P, P, P, P, P],
     "moe_grouped_swiglu_bwd": [P, SP, P, P, P, P, P, P, P, P, P, P, P, P, c_size_t, P],

@@ -255,7 +255,7 @@ moe_status_t moe_grouped_swiglu_fwd(moe_handle_t h, const moe_shape_t* s, const 
                                     void* au, void* hbuf, void* o_perm, void* ws, size_t ws_bytes,
                                     moe_stream_t stream) {
   MOE_CHECK_HANDLE(h, s);
-  if (!all_nonnull(x_perm, offsets, w_gu, w_down, au, hbuf, o_perm)) return MOE_ERR_INVALID_ARG;
+  if (!all_nonnull(x_perm, offsets, w_gu, w_down, hbuf, o_perm)) return MOE_ERR_INVALID_ARG;
   for (const void* p : {x_perm, w_gu, w_down, static_cast<const void*>(au),
                         static_cast<const void*>(hbuf), static_cast<const void*>(o_perm)})
     if (!aligned(p, 16)) return MOE_ERR_INVALID_ARG;
@@ -285,6 +285,36 @@ moe_status_t moe_grouped_swiglu_fwd(moe_handle_t h, const moe_shape_t* s, const 
   h->launches += 2;
   MOE_TRY(moe::gemm_fwd_gate_up(c, x_perm, offsets, w_gu, au, hbuf, E, d, f, m_cap, st));
   return moe::gemm_fwd_down(c, hbuf, offsets, w_down, o_perm, E, d, f, m_cap, st);
+}
+
+moe_status_t moe_grouped_swiglu_recompute(moe_handle_t h, const moe_shape_t* s, const void* x_perm,
+                                          const int32_t* offsets, const void* w_gu, void* au,
+                                          void* hbuf, void* ws, size_t ws_bytes,
+                                          moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  if (!all_nonnull(x_perm, offsets, w_gu, au, hbuf)) return MOE_ERR_INVALID_ARG;
+  for (const void* p : {x_perm, w_gu, static_cast<const void*>(au), static_cast<const void*>(hbuf)})
+    if (!aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  const int d = s->d_model, f = s->d_ff, E = s->n_experts;
+  const int64_t m_cap = max_rows(s);
+  auto st = static_cast<cudaStream_t>(stream);
+  MOE_GUARD(h);
+  moe::GemmCtx c{h->num_sms, h->ctl, pair_tiles(s)};
+  if (s->dtype == MOE_DTYPE_MXFP8) {
+    // the forward's operand quantisation and gate/up GEMM, again
+    MOE_TRY(check_ws(h, s, ws, ws_bytes));
+    const MxWs L = mx_layout(s);
+    auto* b = static_cast<uint8_t*>(ws);
+    auto bf = [](const void* p) { return static_cast<const __nv_bfloat16*>(p); };
+    h->launches += 3;
+    MOE_TRY(cuda_status(moe::launch_mxfp8_quantize(bf(x_perm), m_cap, d, 1, b + L.xq, b + L.xs, st)));
+    MOE_TRY(cuda_status(
+        moe::launch_mxfp8_quantize(bf(w_gu), 2ll * E * f, d, 1, b + L.wguq, b + L.wgus, st)));
+    return moe::gemm_mx_fwd_gate_up(c, {b + L.xq, b + L.xs}, offsets, {b + L.wguq, b + L.wgus}, au,
+                                    hbuf, E, d, f, m_cap, st);
+  }
+  h->launches += 1;
+  return moe::gemm_fwd_gate_up(c, x_perm, offsets, w_gu, au, hbuf, E, d, f, m_cap, st);
 }
 
 moe_status_t moe_unpermute_combine(moe_handle_t h, const moe_shape_t* s, const void* o_perm,

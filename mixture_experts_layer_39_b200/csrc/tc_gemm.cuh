@@ -916,7 +916,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if constexpr (EPI == EPI_SWIGLU_FWD) {
         constexpr int BNH = BN / 2;
         const int64_t col0 = static_cast<int64_t>(tl.n_tile) * BNH;
-        auto* au = static_cast<__nv_bfloat16*>(args.out) + row_first * args.ldo + col0;
+        auto* au = args.out != nullptr
+                       ? static_cast<__nv_bfloat16*>(args.out) + row_first * args.ldo + col0
+                       : nullptr;
         auto* hh = static_cast<__nv_bfloat16*>(args.out2) + row_first * args.ldo2 + col0;
 #pragma unroll 1
         for (int c = 0; c < BNH; c += 64) {
@@ -944,8 +946,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                             pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
             }
           }
-          store_rows(ebuf, lane, vg, reinterpret_cast<uint8_t*>(au + c), args.ldo * 2, vrows);
-          store_rows(ebuf, lane, vu, reinterpret_cast<uint8_t*>(au + args.f + c), args.ldo * 2, vrows);
+          if (args.out != nullptr) {  // [A | U] is not kept when the backward recomputes it
+            store_rows(ebuf, lane, vg, reinterpret_cast<uint8_t*>(au + c), args.ldo * 2, vrows);
+            store_rows(ebuf, lane, vu, reinterpret_cast<uint8_t*>(au + args.f + c), args.ldo * 2,
+                       vrows);
+          }
           store_rows(ebuf, lane, vh, reinterpret_cast<uint8_t*>(hh + c), args.ldo2 * 2, vrows);
         }
       } else {  // EPI_SWIGLU_BWD

@@ -16,6 +16,11 @@ With shared_ff > 0 a shared expert runs on every token
 (moe_shared_expert_fwd / _bwd); its output joins the combine and its input
 gradient the permute backward.
 
+With recompute=True the forward keeps no [A | U] (H is only a transient
+input to the down projection) and the backward first recomputes both
+(moe_grouped_swiglu_recompute): only x_perm and O_perm live from the forward
+to the backward.
+
 With aux_alpha > 0 the forward also forms the router's load statistics and
 the load-balancing loss (moe_router_load_stats -> moe_router_aux_loss) and
 the backward adds the loss's gradient in the router backward.
@@ -40,7 +45,8 @@ class MoELayer:
     def __init__(self, T, d, f, E, k, device="cuda", renorm=False, keep_logits=False,
                  handle: ops.Handle | None = None, dtype: str = "bf16",
                  fuse_router_dx: bool | None = None, aux_alpha: float = 0.0,
-                 aux_reduce: Callable | None = None, shared_ff: int = 0):
+                 aux_reduce: Callable | None = None, shared_ff: int = 0,
+                 recompute: bool = False):
         """dtype: "bf16", or "mxfp8" for E4M3/E8M0 expert GEMM operands (the
         library then also aligns expert segments to 128 rows).
         fuse_router_dx: add the router's input gradient inside the permute
@@ -52,7 +58,11 @@ class MoELayer:
         (replicas.global_stats_reducer), for balancing over the global batch.
         shared_ff: hidden size of a shared expert every token passes through
         (0: none); its weights are passed to forward/backward/step as
-        w_gu_s [2*shared_ff, d] and w_d_s [d, shared_ff]."""
+        w_gu_s [2*shared_ff, d] and w_d_s [d, shared_ff].
+        recompute: activation recompute of the expert gate/up GEMM (self.au
+        and self.h then only hold values between the recompute and the end
+        of the backward, and can be shared between layers)."""
+        self.recompute = bool(recompute)
         self.T, self.d, self.f, self.E, self.k = T, d, f, E, k
         dev = torch.device(device)
         self.device = dev
@@ -113,7 +123,8 @@ class MoELayer:
 
     def experts_fwd(self, w_gu, w_d, stream=None):
         ops.moe_grouped_swiglu_fwd(self.handle, self.shape, self.x_perm, self.offsets, w_gu, w_d,
-                                   self.au, self.h, self.o_perm, self.ws, stream)
+                                   None if self.recompute else self.au, self.h, self.o_perm,
+                                   self.ws, stream)
 
     def shared_fwd(self, x, w_gu_s, w_d_s, stream=None):
         ops.moe_shared_expert_fwd(self.handle, self.shared_shape, x, w_gu_s, w_d_s, self.au_s,
@@ -168,6 +179,9 @@ class MoELayer:
                                 self.ws, stream)
 
     def experts_bwd(self, w_gu, w_d, stream=None):
+        if self.recompute:
+            ops.moe_grouped_swiglu_recompute(self.handle, self.shape, self.x_perm, self.offsets,
+                                             w_gu, self.au, self.h, self.ws, stream)
         ops.moe_grouped_swiglu_bwd(self.handle, self.shape, self.do_perm, self.x_perm, self.au,
                                    self.h, self.offsets, w_gu, w_d, self.dau, self.dx_perm,
                                    self.dw_gu, self.dw_d, self.ws, stream)

@@ -112,6 +112,12 @@ def moe_grouped_swiglu_fwd(h, shape, x_perm, offsets, w_gu, w_down, au, hbuf, o_
           ws.numel() if ws is not None else 0, _stream(stream))
 
 
+def moe_grouped_swiglu_recompute(h, shape, x_perm, offsets, w_gu, au, hbuf, ws, stream=None):
+    _call("moe_grouped_swiglu_recompute", h.ptr, ctypes.byref(shape), _ptr(x_perm), _ptr(offsets),
+          _ptr(w_gu), _ptr(au), _ptr(hbuf), _ptr(ws), ws.numel() if ws is not None else 0,
+          _stream(stream))
+
+
 def moe_unpermute_combine(h, shape, o_perm, row_map, topk_w, shared_out, y, stream=None):
     _call("moe_unpermute_combine", h.ptr, ctypes.byref(shape), _ptr(o_perm), _ptr(row_map),
           _ptr(topk_w), _ptr(shared_out), _ptr(y), _stream(stream))
