@@ -188,7 +188,8 @@ __global__ void __launch_bounds__(kWarps * 32)
 
 // y[t] = bf16(sum_j w[t,j] * O[row_map[t,j]] + shared[t]), fp32 in slot order, the
 // shared expert's output (when given) last.
-__global__ void __launch_bounds__(kWarps * 32)
+template <bool SHARED>
+__global__ void __launch_bounds__(kWarps * 32, 2)
     combine_kernel(const uint4* __restrict__ o, const int32_t* __restrict__ row_map,
                    const float* __restrict__ w, const uint4* __restrict__ shared, int T, int nvec,
                    int k, uint4* __restrict__ y) {
@@ -224,7 +225,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         for (int c = 0; c < 8; ++c) acc[u][c] = fmaf(wt[j], f[c], acc[u][c]);
       }
       if (v0 + 32 * u >= nvec) continue;
-      if (shared != nullptr) {  // the shared expert's output, added last
+      if constexpr (SHARED) {  // the shared expert's output, added last
         float f[8];
         unpack8(__ldg(shared + t * nvec + v0 + 32 * u), f);
 #pragma unroll
@@ -293,6 +294,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
 
 // dX[t] = bf16(sum_j dX_perm[row_map[t,j]] + dX_router[t] + dX_shared[t]), fp32,
 // rounded once (the last two terms when given).
+template <bool SHARED>
 __global__ void __launch_bounds__(kWarps * 32)
     permute_bwd_kernel(const uint4* __restrict__ dxp, const int32_t* __restrict__ row_map,
                        const float4* __restrict__ dxr, const uint4* __restrict__ dxs, int T,
@@ -325,7 +327,7 @@ __global__ void __launch_bounds__(kWarps * 32)
       acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
       acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
     }
-    if (dxs != nullptr) {  // the shared expert's input gradient, added last
+    if constexpr (SHARED) {  // the shared expert's input gradient, added last
       float f[8];
       unpack8(__ldg(dxs + t * nvec + v), f);
 #pragma unroll
@@ -375,9 +377,10 @@ cudaError_t launch_combine(const __nv_bfloat16* o_perm, const int32_t* row_map, 
                            const __nv_bfloat16* shared, int T, int d, int k, __nv_bfloat16* y,
                            cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>(ceil_div64(T, kWarps));
-  combine_kernel<<<grid, kWarps * 32, 0, st>>>(reinterpret_cast<const uint4*>(o_perm), row_map, w,
-                                               reinterpret_cast<const uint4*>(shared), T, d / 8, k,
-                                               reinterpret_cast<uint4*>(y));
+  auto kern = shared != nullptr ? combine_kernel<true> : combine_kernel<false>;
+  kern<<<grid, kWarps * 32, 0, st>>>(reinterpret_cast<const uint4*>(o_perm), row_map, w,
+                                     reinterpret_cast<const uint4*>(shared), T, d / 8, k,
+                                     reinterpret_cast<uint4*>(y));
   return cudaGetLastError();
 }
 
@@ -396,7 +399,8 @@ cudaError_t launch_permute_bwd(const __nv_bfloat16* dx_perm, const int32_t* row_
                                const float* dx_router, const __nv_bfloat16* dx_shared, int T, int d,
                                int k, __nv_bfloat16* dx, cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>(ceil_div64(T, kWarps));
-  permute_bwd_kernel<<<grid, kWarps * 32, 0, st>>>(
+  auto kern = dx_shared != nullptr ? permute_bwd_kernel<true> : permute_bwd_kernel<false>;
+  kern<<<grid, kWarps * 32, 0, st>>>(
       reinterpret_cast<const uint4*>(dx_perm), row_map, reinterpret_cast<const float4*>(dx_router),
       reinterpret_cast<const uint4*>(dx_shared), T, d / 8, k, reinterpret_cast<uint4*>(dx));
   return cudaGetLastError();

@@ -8,6 +8,8 @@
 // For small E these run on CUDA cores; for E a multiple of 128 the two
 // products run on the tcgen05 grouped GEMM (see gemm.cu) and this file only
 // produces dL (bf16) and the db partial sums.
+#include <type_traits>
+
 #include "kernels.cuh"
 
 namespace moe {
@@ -164,7 +166,7 @@ __global__ void __launch_bounds__(kWarps * 32)
 // tokens; the dX_perm gathers bypass L1.  KMAX bounds k at compile time.  Sums run in the same order as the
 // two-kernel path (router dX, then unpermute-reduce), so both give the same
 // bits.
-template <int NE, int TPW, int KMAX>
+template <int NE, int TPW, int KMAX, bool SHARED>
 __global__ void __launch_bounds__(kWarps * 32, 2)
     permute_router_bwd_kernel(const uint4* __restrict__ dxp, const int32_t* __restrict__ row_map,
                               const float* __restrict__ dw, const float* __restrict__ probs,
@@ -217,7 +219,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
       }
 #pragma unroll
       for (int c = 0; c < 8; ++c) acc[c] += r[h][c];
-      if (dxs != nullptr) {  // the shared expert's input gradient, added last
+      if constexpr (SHARED) {  // the shared expert's input gradient, added last
         float f[8];
         unpack8(__ldg(dxs + (t0 + h) * nvec + v), f);
 #pragma unroll
@@ -396,17 +398,21 @@ cudaError_t launch_permute_router_bwd(const __nv_bfloat16* dx_perm, const int32_
                                        reinterpret_cast<uint4*>(dx));
     return cudaGetLastError();
   };
-  if (k <= 4) {
-    if (E <= 8) return go(permute_router_bwd_kernel<8, 2, 4>, 2);
-    if (E <= 16) return go(permute_router_bwd_kernel<16, 2, 4>, 2);
-    if (E <= 32) return go(permute_router_bwd_kernel<32, 1, 4>, 1);
-    if (E <= 64) return go(permute_router_bwd_kernel<64, 1, 4>, 1);
-  } else {
-    if (E <= 16) return go(permute_router_bwd_kernel<16, 1, 8>, 1);
-    if (E <= 32) return go(permute_router_bwd_kernel<32, 1, 8>, 1);
-    if (E <= 64) return go(permute_router_bwd_kernel<64, 1, 8>, 1);
-  }
-  return cudaErrorInvalidValue;
+  auto pick = [&](auto shared_tag) -> cudaError_t {
+    constexpr bool S = decltype(shared_tag)::value;
+    if (k <= 4) {
+      if (E <= 8) return go(permute_router_bwd_kernel<8, 2, 4, S>, 2);
+      if (E <= 16) return go(permute_router_bwd_kernel<16, 2, 4, S>, 2);
+      if (E <= 32) return go(permute_router_bwd_kernel<32, 1, 4, S>, 1);
+      if (E <= 64) return go(permute_router_bwd_kernel<64, 1, 4, S>, 1);
+    } else {
+      if (E <= 16) return go(permute_router_bwd_kernel<16, 1, 8, S>, 1);
+      if (E <= 32) return go(permute_router_bwd_kernel<32, 1, 8, S>, 1);
+      if (E <= 64) return go(permute_router_bwd_kernel<64, 1, 8, S>, 1);
+    }
+    return cudaErrorInvalidValue;
+  };
+  return dx_shared != nullptr ? pick(std::true_type{}) : pick(std::false_type{});
 }
 
 int router_bwd_blocks(int num_sms) { return num_sms * 4; }
