@@ -331,6 +331,7 @@ def run_ours(args):
     if not args.no_variants and args.dtype == "bf16":
         variants["aux_loss"] = bench_cfg(cfg, args.steps, args.warmup, False, aux_alpha=0.01)
         variants["recompute"] = bench_cfg(cfg, args.steps, args.warmup, False, recompute=True)
+        variants["gather"] = bench_cfg(cfg, args.steps, args.warmup, False, gather=True)
         if cfg.name == "e8":
             variants["shared_expert"] = bench_cfg(CONFIGS["e8_shared"], args.steps, args.warmup,
                                                   False, shared_ff=CONFIGS["e8_shared"].shared_ff)
@@ -399,6 +400,10 @@ def run_ours(args):
                 f"gate/up GEMM (+{4 * cfg.d * cfg.f * M / 1e9:.0f} GFLOP/step); activations "
                 f"kept from forward to backward shrink by {(2 * cfg.f + cfg.f) * 2 * M / 2**20:.0f} "
                 "MiB of [A|U] and H")
+        if "gather" in variants:
+            line["variants"]["gather"]["what"] = (
+                "no permuted copy of x: the gate/up GEMM and its weight gradient gather the routed "
+                "rows from x with TMA tile::gather4 (moe_route + *_gather entry points)")
         if "shared_expert" in variants:
             sc = CONFIGS["e8_shared"]
             v = variants["shared_expert"]

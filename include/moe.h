@@ -201,6 +201,49 @@ MOE_API moe_status_t moe_grouped_swiglu_recompute(moe_handle_t h, const moe_shap
                                                   const void* w_gu, void* au, void* hbuf, void* ws,
                                                   size_t ws_bytes, moe_stream_t stream);
 
+/* ---- Gather forms: the routed copies of x are never written.  Instead of
+ * a materialised x_perm, the two expert GEMMs that read routed rows of x
+ * (gate/up forward and its recompute; gate/up weight gradient) gather them
+ * from x with TMA tile::gather4 loads through row_src.  The pages describe
+ * routing data straight into each expert's input buffer (Olmo-core 3
+ * introduction page, section 2, rowwise expert parallelism); this goes one
+ * step further on one GPU and skips that buffer.  bf16 only
+ * (MOE_ERR_UNSUPPORTED for MXFP8); results equal the x_perm forms bit for
+ * bit.
+ *
+ * moe_route: moe_permute without x_perm.
+ * Out: counts, offsets, row_map as moe_permute; row_src [M_cap] int32 =
+ *      the token whose copy routed row r holds, T for pad rows and rows past
+ *      offsets[E]. */
+MOE_API moe_status_t moe_route(moe_handle_t h, const moe_shape_t* s, const int32_t* topk_idx,
+                               int32_t* counts, int32_t* offsets, int32_t* row_map,
+                               int32_t* row_src, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_grouped_swiglu_fwd with x [T,d] and row_src in place of x_perm (au may
+ * be NULL as there).  No workspace. */
+MOE_API moe_status_t moe_grouped_swiglu_fwd_gather(moe_handle_t h, const moe_shape_t* s,
+                                                   const void* x, const int32_t* row_src,
+                                                   const int32_t* offsets, const void* w_gu,
+                                                   const void* w_down, void* au, void* hbuf,
+                                                   void* o_perm, moe_stream_t stream);
+
+/* moe_grouped_swiglu_recompute with x [T,d] and row_src in place of x_perm. */
+MOE_API moe_status_t moe_grouped_swiglu_recompute_gather(moe_handle_t h, const moe_shape_t* s,
+                                                         const void* x, const int32_t* row_src,
+                                                         const int32_t* offsets, const void* w_gu,
+                                                         void* au, void* hbuf,
+                                                         moe_stream_t stream);
+
+/* moe_grouped_swiglu_bwd with x [T,d] and row_src in place of x_perm (only
+ * the gate/up weight gradient reads it).  No workspace. */
+MOE_API moe_status_t moe_grouped_swiglu_bwd_gather(moe_handle_t h, const moe_shape_t* s,
+                                                   const void* do_perm, const void* x,
+                                                   const int32_t* row_src, const void* au,
+                                                   const void* hbuf, const int32_t* offsets,
+                                                   const void* w_gu, const void* w_down, void* dau,
+                                                   void* dx_perm, void* dw_gu, void* dw_down,
+                                                   moe_stream_t stream);
+
 /* Weighted unpermute-combine ("restore"):
  *   y[t] = bf16( sum_j topk_w[t,j] * o_perm[row_map[t,j]] + shared_out[t] ),
  *   fp32 sum in slot order, the shared expert's output (when non-NULL) last.

@@ -38,6 +38,10 @@ SIGNATURES = {
     "moe_router_topk": [P, SP, P, P, P, P, P, P, P, P, P, c_size_t, P],
     "moe_permute": [P, SP, P, P, P, P, P, P, P, c_size_t, P],
     "moe_permute_noalloc": [P, SP, P, P, P, P, P, P, P],
+    "moe_route": [P, SP, P, P, P, P, P, P, c_size_t, P],
+    "moe_grouped_swiglu_fwd_gather": [P, SP, P, P, P, P, P, P, P, P, P],
+    "moe_grouped_swiglu_recompute_gather": [P, SP, P, P, P, P, P, P, P],
+    "moe_grouped_swiglu_bwd_gather": [P, SP, P, P, P, P, P, P, P, P, P, P, P, P, P],
     "moe_grouped_swiglu_fwd": [P, SP, P, P, P, P, P, P, P, P, c_size_t, P],
     "moe_grouped_swiglu_recompute": [P, SP, P, P, P, P, P, P, c_size_t, P],
     "moe_unpermute_combine": [P, SP, P, P, P, P, P, P],

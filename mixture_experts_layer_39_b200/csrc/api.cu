@@ -250,6 +250,93 @@ moe_status_t moe_permute(moe_handle_t h, const moe_shape_t* s, const void* x,
                                                  static_cast<__nv_bfloat16*>(x_perm), st));
 }
 
+// ---- gather forms (no materialised x_perm; bf16)
+moe_status_t moe_route(moe_handle_t h, const moe_shape_t* s, const int32_t* topk_idx,
+                       int32_t* counts, int32_t* offsets, int32_t* row_map, int32_t* row_src,
+                       void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  if (!all_nonnull(topk_idx, counts, offsets, row_map, row_src)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(h, s, ws, ws_bytes));
+  const int T = s->T, E = s->n_experts, k = s->top_k;
+  auto st = static_cast<cudaStream_t>(stream);
+  MOE_GUARD(h);
+  auto* sub = static_cast<int32_t*>(ws);
+  h->launches += 4;
+  MOE_TRY(cuda_status(moe::launch_route_hist(topk_idx, T, k, E, sub, h->ctl, st)));
+  MOE_TRY(cuda_status(
+      moe::launch_route_scan(sub, moe::n_subchunks(T, k), E, moe::seg_align(s), counts, offsets, st)));
+  MOE_TRY(cuda_status(moe::launch_route_rank(topk_idx, T, k, E, sub, offsets, row_map, st)));
+  return cuda_status(
+      moe::launch_route_src(row_map, offsets, counts, T, k, E, max_rows(s), row_src, st));
+}
+
+moe_status_t moe_grouped_swiglu_fwd_gather(moe_handle_t h, const moe_shape_t* s, const void* x,
+                                           const int32_t* row_src, const int32_t* offsets,
+                                           const void* w_gu, const void* w_down, void* au,
+                                           void* hbuf, void* o_perm, moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  if (s->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (!all_nonnull(x, row_src, offsets, w_gu, w_down, hbuf, o_perm)) return MOE_ERR_INVALID_ARG;
+  for (const void* p : {x, w_gu, w_down, static_cast<const void*>(au),
+                        static_cast<const void*>(hbuf), static_cast<const void*>(o_perm)})
+    if (!aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  const int d = s->d_model, f = s->d_ff, E = s->n_experts;
+  const int64_t m_cap = max_rows(s);
+  auto st = static_cast<cudaStream_t>(stream);
+  MOE_GUARD(h);
+  moe::GemmCtx c{h->num_sms, h->ctl, pair_tiles(s)};
+  h->launches += 2;
+  MOE_TRY(moe::gemm_fwd_gate_up_gather(c, x, s->T, row_src, offsets, w_gu, au, hbuf, E, d, f,
+                                       m_cap, st));
+  return moe::gemm_fwd_down(c, hbuf, offsets, w_down, o_perm, E, d, f, m_cap, st);
+}
+
+moe_status_t moe_grouped_swiglu_recompute_gather(moe_handle_t h, const moe_shape_t* s,
+                                                 const void* x, const int32_t* row_src,
+                                                 const int32_t* offsets, const void* w_gu,
+                                                 void* au, void* hbuf, moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  if (s->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (!all_nonnull(x, row_src, offsets, w_gu, au, hbuf)) return MOE_ERR_INVALID_ARG;
+  for (const void* p : {x, w_gu, static_cast<const void*>(au), static_cast<const void*>(hbuf)})
+    if (!aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  auto st = static_cast<cudaStream_t>(stream);
+  MOE_GUARD(h);
+  moe::GemmCtx c{h->num_sms, h->ctl, pair_tiles(s)};
+  h->launches += 1;
+  return moe::gemm_fwd_gate_up_gather(c, x, s->T, row_src, offsets, w_gu, au, hbuf, s->n_experts,
+                                      s->d_model, s->d_ff, max_rows(s), st);
+}
+
+moe_status_t moe_grouped_swiglu_bwd_gather(moe_handle_t h, const moe_shape_t* s,
+                                           const void* do_perm, const void* x,
+                                           const int32_t* row_src, const void* au,
+                                           const void* hbuf, const int32_t* offsets,
+                                           const void* w_gu, const void* w_down, void* dau,
+                                           void* dx_perm, void* dw_gu, void* dw_down,
+                                           moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  if (s->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (!all_nonnull(do_perm, x, row_src, au, hbuf, offsets, w_gu, w_down, dau, dx_perm, dw_gu,
+                   dw_down))
+    return MOE_ERR_INVALID_ARG;
+  for (const void* p : {do_perm, x, au, hbuf, w_gu, w_down, static_cast<const void*>(dau),
+                        static_cast<const void*>(dx_perm), static_cast<const void*>(dw_gu),
+                        static_cast<const void*>(dw_down)})
+    if (!aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  const int d = s->d_model, f = s->d_ff, E = s->n_experts;
+  const int64_t m_cap = max_rows(s);
+  auto st = static_cast<cudaStream_t>(stream);
+  MOE_GUARD(h);
+  moe::GemmCtx c{h->num_sms, h->ctl, pair_tiles(s)};
+  h->launches += 4;
+  MOE_TRY(moe::gemm_dgrad_down_swiglu(c, do_perm, offsets, w_down, au, dau, E, d, f, m_cap, st));
+  MOE_TRY(moe::gemm_wgrad_down(c, do_perm, hbuf, offsets, dw_down, E, d, f, m_cap, st));
+  MOE_TRY(moe::gemm_dgrad_gate_up(c, dau, offsets, w_gu, dx_perm, E, d, f, m_cap, st));
+  return moe::gemm_wgrad_gate_up_gather(c, dau, x, s->T, row_src, offsets, dw_gu, E, d, f, m_cap,
+                                        st);
+}
+
 moe_status_t moe_grouped_swiglu_fwd(moe_handle_t h, const moe_shape_t* s, const void* x_perm,
                                     const int32_t* offsets, const void* w_gu, const void* w_down,
                                     void* au, void* hbuf, void* o_perm, void* ws, size_t ws_bytes,

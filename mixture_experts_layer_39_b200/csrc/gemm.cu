@@ -64,7 +64,8 @@ bool tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, bool FP8 = false, bool PAIR = false>
+template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, bool FP8 = false, bool PAIR = false,
+          bool GATHER = false>
 moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const tc::GemmArgs& args, int grid,
                     cudaStream_t st) {
   // the SwiGLU-backward epilogue's landing buffers take one stage's room;
@@ -73,7 +74,7 @@ moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const tc::GemmAr
   constexpr int STAGES = FP8    ? (EPI == tc::EPI_SWIGLU_BWD ? 5 : 6)
                          : PAIR ? (EPI == tc::EPI_SWIGLU_BWD ? 5 : 6)
                                 : (BN == 256 ? (EPI == tc::EPI_SWIGLU_BWD ? 3 : 4) : 6);
-  auto kern = tc::grouped_gemm_kernel<BN, A_MN, B_MN, EPI, KGROUP, STAGES, FP8, PAIR>;
+  auto kern = tc::grouped_gemm_kernel<BN, A_MN, B_MN, EPI, KGROUP, STAGES, FP8, PAIR, GATHER>;
   const size_t smem = tc::SmemPlan<BN, STAGES, EPI, FP8, PAIR>::bytes(args.n_groups);
   static size_t configured = 0;  // largest size this instantiation was opened for
   if (smem > configured) {
@@ -245,6 +246,62 @@ moe_status_t gemm_wgrad_gate_up(const GemmCtx& c, const void* dau, const void* x
   const int64_t tiles = static_cast<int64_t>(E) * a.m_tiles_fixed * a.n_tiles_n;
   const int grid = static_cast<int>(2 * tiles < c.num_sms ? 2 * tiles : c.num_sms);
   return launch<256, true, true, tc::EPI_BF16, true, false, true>(ta, tb, a, grid, st);
+}
+
+// Gather forms: the routed rows are read from x (T rows) through row_src
+// (tile::gather4 loads; the tensor map's box is one row of 64 columns).
+moe_status_t gemm_fwd_gate_up_gather(const GemmCtx& c, const void* x, int T,
+                                     const int32_t* row_src, const int32_t* offsets,
+                                     const void* w_gu, void* au, void* h, int E, int d, int f,
+                                     int64_t m_cap, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, x, d, T, 2ull * d, 64, 1)) return MOE_ERR_CUDA;
+  if (!tmap_3d(&tb, w_gu, d, 2ull * f, E, 2ull * d, 4ull * f * d, 64, 128)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  a.n_tiles_n = f / 128;
+  a.k_blocks = d / tc::BK;
+  a.n_groups = E;
+  a.offsets = offsets;
+  a.total_len = static_cast<int>(m_cap);
+  a.uniform_len = static_cast<int>(m_cap);
+  a.m_cap = m_cap;
+  a.out = au;
+  a.ldo = 2ll * f;
+  a.out2 = h;
+  a.ldo2 = f;
+  a.f = f;
+  a.row_src = row_src;
+  a.src_oob = T;
+  if (c.pair_m)
+    return launch<256, false, false, tc::EPI_SWIGLU_FWD, false, false, true, true>(ta, tb, a,
+                                                                                   c.num_sms, st);
+  return launch<256, false, false, tc::EPI_SWIGLU_FWD, false, false, false, true>(ta, tb, a,
+                                                                                  c.num_sms, st);
+}
+
+moe_status_t gemm_wgrad_gate_up_gather(const GemmCtx& c, const void* dau, const void* x, int T,
+                                       const int32_t* row_src, const int32_t* offsets,
+                                       void* dw_gu, int E, int d, int f, int64_t m_cap,
+                                       cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, dau, 2ull * f, m_cap, 4ull * f, 64, 64)) return MOE_ERR_CUDA;
+  if (!tmap_2d(&tb, x, d, T, 2ull * d, 64, 1)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  a.n_tiles_n = d / 256;
+  a.n_groups = E;
+  a.offsets = offsets;
+  a.total_len = static_cast<int>(m_cap);
+  a.uniform_len = static_cast<int>(m_cap);
+  a.m_cap = m_cap;
+  a.out = dw_gu;
+  a.ldo = d;
+  a.out_gstride = 2ll * f * d;
+  a.m_tiles_fixed = 2 * f / (2 * tc::BM);  // CTA pairs: 256-row tiles
+  a.row_src = row_src;
+  a.src_oob = T;
+  const int64_t tiles = static_cast<int64_t>(E) * a.m_tiles_fixed * a.n_tiles_n;
+  const int grid = static_cast<int>(2 * tiles < c.num_sms ? 2 * tiles : c.num_sms);
+  return launch<256, true, true, tc::EPI_BF16, true, false, true, true>(ta, tb, a, grid, st);
 }
 
 moe_status_t gemm_router_logits(const GemmCtx& c, const void* x, const void* w_r, float* logits,

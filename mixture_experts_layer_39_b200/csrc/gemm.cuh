@@ -37,6 +37,16 @@ moe_status_t gemm_wgrad_down(const GemmCtx& c, const void* do_perm, const void* 
 moe_status_t gemm_wgrad_gate_up(const GemmCtx& c, const void* dau, const void* x_perm,
                                 const int32_t* offsets, void* dw_gu, int E, int d, int f,
                                 int64_t m_cap, cudaStream_t st);
+// Gather forms of the two GEMMs that read routed copies of x: row r of the
+// routed operand is x[row_src[r]] (T rows; row T and beyond read as zeros).
+moe_status_t gemm_fwd_gate_up_gather(const GemmCtx& c, const void* x, int T,
+                                     const int32_t* row_src, const int32_t* offsets,
+                                     const void* w_gu, void* au, void* h, int E, int d, int f,
+                                     int64_t m_cap, cudaStream_t st);
+moe_status_t gemm_wgrad_gate_up_gather(const GemmCtx& c, const void* dau, const void* x, int T,
+                                       const int32_t* row_src, const int32_t* offsets,
+                                       void* dw_gu, int E, int d, int f, int64_t m_cap,
+                                       cudaStream_t st);
 moe_status_t gemm_router_logits(const GemmCtx& c, const void* x, const void* w_r, float* logits,
                                 int T, int d, int E, cudaStream_t st);
 moe_status_t gemm_router_dx(const GemmCtx& c, const void* dl_bf16, const void* w_r,

@@ -37,6 +37,11 @@ cudaError_t launch_route_scan(int32_t* sub_counts, int64_t n_sub, int E, int ali
                               int32_t* offsets, cudaStream_t st);
 cudaError_t launch_route_rank(const int32_t* idx, int T, int k, int E, const int32_t* sub_base,
                               const int32_t* offsets, int32_t* row_map, cudaStream_t st);
+// row_src [m_cap]: source token of every routed row, T for pad rows and rows
+// past the last segment.
+cudaError_t launch_route_src(const int32_t* row_map, const int32_t* offsets, const int32_t* counts,
+                             int T, int k, int E, int64_t m_cap, int32_t* row_src,
+                             cudaStream_t st);
 cudaError_t launch_permute_scatter(const __nv_bfloat16* x, const int32_t* row_map,
                                    const int32_t* offsets, const int32_t* counts, int T, int d,
                                    int k, int E, __nv_bfloat16* x_perm, cudaStream_t st);

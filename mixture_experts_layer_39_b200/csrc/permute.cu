@@ -149,6 +149,36 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
 }
 
+// row_src[r] = the token whose copy routed row r holds, for the expert GEMMs
+// that gather their rows from x instead of reading x_perm.  Threads [0, T k)
+// take one (token, slot) each; threads [T k, T k + m_cap) take routed row
+// r = i - T k and write oob (a row index past x, which the gather loads read
+// as zeros) when r is a pad row or lies past the last segment.  The two sets
+// of rows are disjoint, so the kernel needs no ordering.
+__global__ void __launch_bounds__(256)
+    route_src_kernel(const int32_t* __restrict__ row_map, const int32_t* __restrict__ offsets,
+                     const int32_t* __restrict__ counts, int T, int k, int E, int64_t m_cap,
+                     int32_t oob, int32_t* __restrict__ row_src) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t tk = static_cast<int64_t>(T) * k;
+  if (i < tk) {
+    row_src[__ldg(row_map + i)] = static_cast<int32_t>(i / k);
+    return;
+  }
+  const int64_t r = i - tk;
+  if (r >= m_cap) return;
+  if (r >= __ldg(offsets + E)) {
+    row_src[r] = oob;
+    return;
+  }
+  int lo = 0, hi = E - 1;  // the segment holding r: the last e with offsets[e] <= r
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(offsets + mid) <= r) lo = mid; else hi = mid - 1;
+  }
+  if (r >= static_cast<int64_t>(__ldg(offsets + lo)) + __ldg(counts + lo)) row_src[r] = oob;
+}
+
 // Warps [0, T): token t, reads x[t] once and writes its k rows.
 // Warps [T, T+E): expert e, zero-fills the pad rows of its segment.
 __global__ void __launch_bounds__(kWarps * 32)
@@ -360,6 +390,15 @@ cudaError_t launch_route_rank(const int32_t* idx, int T, int k, int E, const int
   const unsigned grid = static_cast<unsigned>(ceil_div64(n_sub, kWarps));
   route_rank_kernel<<<grid, kWarps * 32, kWarps * E * sizeof(int), st>>>(
       idx, static_cast<int64_t>(T) * k, E, n_sub, sub_base, offsets, row_map);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_src(const int32_t* row_map, const int32_t* offsets, const int32_t* counts,
+                             int T, int k, int E, int64_t m_cap, int32_t* row_src,
+                             cudaStream_t st) {
+  const int64_t n = static_cast<int64_t>(T) * k + m_cap;
+  route_src_kernel<<<static_cast<unsigned>(ceil_div64(n, 256)), 256, 0, st>>>(
+      row_map, offsets, counts, T, k, E, m_cap, T, row_src);
   return cudaGetLastError();
 }
 

@@ -73,6 +73,11 @@ struct GemmArgs {
   int64_t ld_sfb;
   int64_t sfb_rows;     // rows per group of the B scale array
   int64_t sfb_gstride;  // bytes between groups of B scales (M-grouped)
+  // GATHER: the operand that holds routed rows is read from the unpermuted
+  // matrix (x), routed row r being its row row_src[r]; rows past m_cap and
+  // pad rows use src_oob, a row past the matrix that reads as zeros
+  const int32_t* row_src;
+  int src_oob;
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -201,6 +206,26 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap
       "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
+// Four rows (r0..r3, any order) x one box of columns from c0, into 4
+// consecutive 128-byte rows at dst (the tensor map's box is one row high).
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::"
+      "complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
       : "memory");
 }
 
@@ -520,7 +545,7 @@ struct SmemPlan {
 // the odd CTA's epilogue warps release the accumulator on the leader's
 // barrier.
 template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, int STAGES, bool FP8 = false,
-          bool PAIR = false>
+          bool PAIR = false, bool GATHER = false>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
@@ -528,6 +553,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   static_assert(!(EPI == EPI_SWIGLU_FWD && B_MN), "SwiGLU forward takes K-major weights");
   static_assert(!FP8 || BN == 128, "MXFP8 tiles are 128 x 128 (TMEM holds the scales too)");
   static_assert(!PAIR || (BN == 256 && !FP8), "CTA pairs run bf16 256 x 256 tiles");
+  // GATHER reads routed rows from x: the K-major A of an M-grouped GEMM, or
+  // the MN-major B (rows = routed rows) of a K-grouped one
+  static_assert(!GATHER || (!FP8 && (KGROUP ? B_MN : !A_MN)), "gathered operand");
+  // K-grouped GATHER runs on CTA pairs: one 4-row gather per lane per stage
+  static_assert(!GATHER || !KGROUP || (PAIR && (BN / 2 / (FP8 ? 128 : 64)) * (BK / 4) == 32),
+                "K-grouped gather layout");
   using Plan = SmemPlan<BN, STAGES, EPI, FP8, PAIR>;
   constexpr int MT = PAIR ? 2 * BM : BM;  // tile rows (of the pair)
   constexpr int BNC = PAIR ? BN / 2 : BN;  // B rows held by one CTA
@@ -638,16 +669,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================================================================ producer
     // lane 0 issues the TMA tile loads; with MXFP8 all 32 lanes also copy the
     // stage's scale atoms (cp.async, arriving on the full barrier)
-    if (FP8 || lane == 0) {
+    // GATHER: every lane issues one 4-row gather per 4 routed rows it owns
+    auto src_row = [&](int64_t r) -> int {
+      return r < args.m_cap ? __ldg(args.row_src + r) : args.src_oob;
+    };
+    if (FP8 || GATHER || lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // per-stage: a load is in flight / its phase
       bool ok = true;
       for (int t = unit; t < total_tiles && ok; t += n_units) {
         const Tile tl = decode_tile<KGROUP, BKE, KMMA, MT>(args, s_tile_start, t);
+        // GATHER: x rows of this lane's 4 rows of the stage (M-grouped: the same
+        // rows for the whole tile; K-grouped: loaded one K-block ahead)
+        int gsrc[4] = {0, 0, 0, 0};
+        if constexpr (GATHER && !KGROUP) {
+          const int64_t r = static_cast<int64_t>(tl.row0) + BM * static_cast<int>(rank) + 4 * lane;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) gsrc[i] = src_row(r + i);
+        }
+        constexpr int kGq = BKE / 4;  // 4-row pieces per 64-row K-block chunk
+        if constexpr (GATHER && KGROUP) {
+          const int64_t r = static_cast<int64_t>(tl.k_lo) + 4 * (lane % kGq);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) gsrc[i] = src_row(r + i);
+        }
         for (int kb = 0; kb < tl.k_blocks; ++kb) {
           bool got = mbar_wait(empty_bar(stage), phase ^ 1u, s_abort, true, PAIR);
-          if constexpr (FP8) got = __all_sync(0xffffffffu, got);
+          if constexpr (FP8 || GATHER) got = __all_sync(0xffffffffu, got);
           if (!got) { ok = false; break; }
           const uint32_t sa = smem_base + stage * Plan::kStageBytes;
           const uint32_t sb = sa + Plan::kABytes;
@@ -655,15 +704,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (PAIR) {
             // both CTAs' bytes complete on the leader's full barrier
             const uint32_t fbl = mapa_shared(fb, 0);
-            if (rank == 0) {
+            if (rank == 0 && lane == 0) {
               mbar_arrive_expect_tx(fb, 2 * Plan::kStageBytes);
               armed |= 1u << stage;
               armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
             }
+            if constexpr (GATHER) __syncwarp();
             if constexpr (!KGROUP) {
               const int k0 = kb * BKE;
-              tma_load_2d_pair(sa, &tmA, fbl, k0, tl.row0 + BM * static_cast<int>(rank));
-              if constexpr (EPI == EPI_SWIGLU_FWD) {
+              if constexpr (GATHER) {
+                tma_gather4_pair(sa + lane * 512, &tmA, fbl, k0, gsrc[0], gsrc[1], gsrc[2],
+                                 gsrc[3]);
+              } else {
+                tma_load_2d_pair(sa, &tmA, fbl, k0, tl.row0 + BM * static_cast<int>(rank));
+              }
+              if (lane != 0) {
+              } else if constexpr (EPI == EPI_SWIGLU_FWD) {
                 // the pair's B tile is [gate rows | up rows]: CTA 0 loads gate, CTA 1 up
                 const int nh = tl.n_tile * (BN / 2);
                 tma_load_3d_pair(sb, &tmB, fbl, k0, (rank ? args.f : 0) + nh, tl.group);
@@ -678,24 +734,47 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             } else {
               const int kr = tl.k_lo + kb * BKE;
+              if (lane == 0) {
 #pragma unroll
-              for (int j = 0; j < BM / CH; ++j)
-                tma_load_2d_pair(sa + j * kChunkBytes, &tmA, fbl,
-                                 tl.row0 + BM * static_cast<int>(rank) + CH * j, kr);
+                for (int j = 0; j < BM / CH; ++j)
+                  tma_load_2d_pair(sa + j * kChunkBytes, &tmA, fbl,
+                                   tl.row0 + BM * static_cast<int>(rank) + CH * j, kr);
+              }
+              if constexpr (GATHER) {
+                // B rows are routed rows kr.. of x: lane -> chunk j, rows 4q..4q+3
+                const int j = lane / kGq, q = lane % kGq;
+                tma_gather4_pair(sb + j * kChunkBytes + q * 512, &tmB, fbl,
+                                 tl.n_tile * BN + BNC * static_cast<int>(rank) + CH * j, gsrc[0],
+                                 gsrc[1], gsrc[2], gsrc[3]);
+                if (kb + 1 < tl.k_blocks) {  // the next K-block's rows, in flight during the wait
+                  const int64_t r = static_cast<int64_t>(kr) + BKE + 4 * q;
 #pragma unroll
-              for (int j = 0; j < BNC / CH; ++j)
-                tma_load_3d_pair(sb + j * kChunkBytes, &tmB, fbl,
-                                 tl.n_tile * BN + BNC * static_cast<int>(rank) + CH * j, kr, 0);
+                  for (int i = 0; i < 4; ++i) gsrc[i] = src_row(r + i);
+                }
+              } else if (lane == 0) {
+#pragma unroll
+                for (int j = 0; j < BNC / CH; ++j)
+                  tma_load_3d_pair(sb + j * kChunkBytes, &tmB, fbl,
+                                   tl.n_tile * BN + BNC * static_cast<int>(rank) + CH * j, kr, 0);
+              }
             }
-          } else if (lane == 0) {
-            mbar_arrive_expect_tx(fb, Plan::kStageBytes);
-            armed |= 1u << stage;
-            armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          } else if (GATHER || lane == 0) {
+            if (lane == 0) {
+              mbar_arrive_expect_tx(fb, Plan::kStageBytes);
+              armed |= 1u << stage;
+              armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+            }
+            if constexpr (GATHER) __syncwarp();
             if constexpr (!KGROUP) {
               const int k0 = kb * BKE;
               // A: K-major rows of the group's slice
-              tma_load_2d(sa, &tmA, fb, k0, tl.row0);
-              if constexpr (EPI == EPI_SWIGLU_FWD) {
+              if constexpr (GATHER) {
+                tma_gather4(sa + lane * 512, &tmA, fb, k0, gsrc[0], gsrc[1], gsrc[2], gsrc[3]);
+              } else {
+                tma_load_2d(sa, &tmA, fb, k0, tl.row0);
+              }
+              if (lane != 0) {
+              } else if constexpr (EPI == EPI_SWIGLU_FWD) {
                 const int nh = tl.n_tile * (BN / 2);
                 tma_load_3d(sb, &tmB, fb, k0, nh, tl.group);
                 tma_load_3d(sb + (BN / 2) * 128, &tmB, fb, k0, args.f + nh, tl.group);
@@ -708,12 +787,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             } else {
               const int kr = tl.k_lo + kb * BKE;
+              if (lane == 0) {
 #pragma unroll
-              for (int j = 0; j < BM / CH; ++j)
-                tma_load_2d(sa + j * kChunkBytes, &tmA, fb, tl.row0 + CH * j, kr);
+                for (int j = 0; j < BM / CH; ++j)
+                  tma_load_2d(sa + j * kChunkBytes, &tmA, fb, tl.row0 + CH * j, kr);
+              }
+              if (lane == 0) {
 #pragma unroll
-              for (int j = 0; j < BN / CH; ++j)
-                tma_load_3d(sb + j * kChunkBytes, &tmB, fb, tl.n_tile * BN + CH * j, kr, 0);
+                for (int j = 0; j < BN / CH; ++j)
+                  tma_load_3d(sb + j * kChunkBytes, &tmB, fb, tl.n_tile * BN + CH * j, kr, 0);
+              }
             }
           }
           if constexpr (FP8) {

@@ -16,6 +16,10 @@ With shared_ff > 0 a shared expert runs on every token
 (moe_shared_expert_fwd / _bwd); its output joins the combine and its input
 gradient the permute backward.
 
+With gather=True (bf16) no permuted copy of x is written: moe_route
+produces the routing metadata and row_src, and the expert GEMMs that read
+routed rows of x gather them from x itself (the *_gather entry points).
+
 With recompute=True the forward keeps no [A | U] (H is only a transient
 input to the down projection) and the backward first recomputes both
 (moe_grouped_swiglu_recompute): only x_perm and O_perm live from the forward
@@ -46,7 +50,7 @@ class MoELayer:
                  handle: ops.Handle | None = None, dtype: str = "bf16",
                  fuse_router_dx: bool | None = None, aux_alpha: float = 0.0,
                  aux_reduce: Callable | None = None, shared_ff: int = 0,
-                 recompute: bool = False):
+                 recompute: bool = False, gather: bool = False):
         """dtype: "bf16", or "mxfp8" for E4M3/E8M0 expert GEMM operands (the
         library then also aligns expert segments to 128 rows).
         fuse_router_dx: add the router's input gradient inside the permute
@@ -63,6 +67,10 @@ class MoELayer:
         and self.h then only hold values between the recompute and the end
         of the backward, and can be shared between layers)."""
         self.recompute = bool(recompute)
+        self.gather = bool(gather)
+        if self.gather and dtype != "bf16":
+            raise ValueError("the gather forms are bf16 only")
+        self._x = None  # x of the current step (gather forms read it in the GEMMs)
         self.T, self.d, self.f, self.E, self.k = T, d, f, E, k
         dev = torch.device(device)
         self.device = dev
@@ -80,7 +88,9 @@ class MoELayer:
         self.logits = z(T, E, dt=F32) if keep_logits else None
         self.counts, self.offsets = z(E, dt=I32), z(E + 1, dt=I32)
         self.row_map = z(T, k, dt=I32)
-        self.x_perm, self.au, self.h = z(M, d), z(M, 2 * f), z(M, f)
+        self.x_perm = None if self.gather else z(M, d)
+        self.row_src = z(M, dt=I32) if self.gather else None
+        self.au, self.h = z(M, 2 * f), z(M, f)
         self.o_perm, self.y = z(M, d), z(T, d)
         # backward state
         self.do_perm, self.dw = z(M, d), z(T, k, dt=F32)
@@ -118,13 +128,23 @@ class MoELayer:
                             self.probs, self.logits, self.ws, stream)
 
     def permute(self, x, stream=None):
+        self._x = x
+        if self.gather:
+            ops.moe_route(self.handle, self.shape, self.idx, self.counts, self.offsets,
+                          self.row_map, self.row_src, self.ws, stream)
+            return
         ops.moe_permute(self.handle, self.shape, x, self.idx, self.counts, self.offsets,
                         self.row_map, self.x_perm, self.ws, stream)
 
     def experts_fwd(self, w_gu, w_d, stream=None):
+        au = None if self.recompute else self.au
+        if self.gather:
+            ops.moe_grouped_swiglu_fwd_gather(self.handle, self.shape, self._x, self.row_src,
+                                              self.offsets, w_gu, w_d, au, self.h, self.o_perm,
+                                              stream)
+            return
         ops.moe_grouped_swiglu_fwd(self.handle, self.shape, self.x_perm, self.offsets, w_gu, w_d,
-                                   None if self.recompute else self.au, self.h, self.o_perm,
-                                   self.ws, stream)
+                                   au, self.h, self.o_perm, self.ws, stream)
 
     def shared_fwd(self, x, w_gu_s, w_d_s, stream=None):
         ops.moe_shared_expert_fwd(self.handle, self.shared_shape, x, w_gu_s, w_d_s, self.au_s,
@@ -179,6 +199,16 @@ class MoELayer:
                                 self.ws, stream)
 
     def experts_bwd(self, w_gu, w_d, stream=None):
+        if self.gather:
+            if self.recompute:
+                ops.moe_grouped_swiglu_recompute_gather(self.handle, self.shape, self._x,
+                                                        self.row_src, self.offsets, w_gu, self.au,
+                                                        self.h, stream)
+            ops.moe_grouped_swiglu_bwd_gather(self.handle, self.shape, self.do_perm, self._x,
+                                              self.row_src, self.au, self.h, self.offsets, w_gu,
+                                              w_d, self.dau, self.dx_perm, self.dw_gu, self.dw_d,
+                                              stream)
+            return
         if self.recompute:
             ops.moe_grouped_swiglu_recompute(self.handle, self.shape, self.x_perm, self.offsets,
                                              w_gu, self.au, self.h, self.ws, stream)
@@ -204,6 +234,7 @@ class MoELayer:
 
     def backward(self, dy, x, w_r, w_gu, w_d, stream=None, w_gu_s=None, w_d_s=None):
         self._need_shared(w_gu_s, w_d_s)
+        self._x = x
         self.combine_bwd(dy, stream)
         self.router_bwd(x, w_r, stream)
         self.experts_bwd(w_gu, w_d, stream)

@@ -118,6 +118,31 @@ def moe_grouped_swiglu_recompute(h, shape, x_perm, offsets, w_gu, au, hbuf, ws, 
           _stream(stream))
 
 
+def moe_route(h, shape, topk_idx, counts, offsets, row_map, row_src, ws, stream=None):
+    _call("moe_route", h.ptr, ctypes.byref(shape), _ptr(topk_idx), _ptr(counts), _ptr(offsets),
+          _ptr(row_map), _ptr(row_src), _ptr(ws), ws.numel(), _stream(stream))
+
+
+def moe_grouped_swiglu_fwd_gather(h, shape, x, row_src, offsets, w_gu, w_down, au, hbuf, o_perm,
+                                  stream=None):
+    _call("moe_grouped_swiglu_fwd_gather", h.ptr, ctypes.byref(shape), _ptr(x), _ptr(row_src),
+          _ptr(offsets), _ptr(w_gu), _ptr(w_down), _ptr(au), _ptr(hbuf), _ptr(o_perm),
+          _stream(stream))
+
+
+def moe_grouped_swiglu_recompute_gather(h, shape, x, row_src, offsets, w_gu, au, hbuf,
+                                        stream=None):
+    _call("moe_grouped_swiglu_recompute_gather", h.ptr, ctypes.byref(shape), _ptr(x),
+          _ptr(row_src), _ptr(offsets), _ptr(w_gu), _ptr(au), _ptr(hbuf), _stream(stream))
+
+
+def moe_grouped_swiglu_bwd_gather(h, shape, do_perm, x, row_src, au, hbuf, offsets, w_gu, w_down,
+                                  dau, dx_perm, dw_gu, dw_down, stream=None):
+    _call("moe_grouped_swiglu_bwd_gather", h.ptr, ctypes.byref(shape), _ptr(do_perm), _ptr(x),
+          _ptr(row_src), _ptr(au), _ptr(hbuf), _ptr(offsets), _ptr(w_gu), _ptr(w_down),
+          _ptr(dau), _ptr(dx_perm), _ptr(dw_gu), _ptr(dw_down), _stream(stream))
+
+
 def moe_unpermute_combine(h, shape, o_perm, row_map, topk_w, shared_out, y, stream=None):
     _call("moe_unpermute_combine", h.ptr, ctypes.byref(shape), _ptr(o_perm), _ptr(row_map),
           _ptr(topk_w), _ptr(shared_out), _ptr(y), _stream(stream))
