@@ -338,9 +338,11 @@ def run_ours(args):
     ratio = None
     if not args.no_ratio and cfg.name == "e8":
         ratio = bench_cfg(CONFIGS["e128"], args.steps, args.warmup, False)
-    mx = None
+    mx = mx_bf16 = None
     if not args.no_mxfp8 and cfg.name == "e8":
         mx = bench_cfg(CONFIGS["mxfp8"], args.steps, args.warmup, False, dtype="mxfp8")
+        # the same workload with bf16 expert GEMMs, for the MXFP8-vs-BF16 comparison
+        mx_bf16 = bench_cfg(CONFIGS["mxfp8"], args.steps, args.warmup, False, dtype="bf16")
     clocks = sampler.stop()
 
     K = args.steps
@@ -421,6 +423,12 @@ def run_ours(args):
             "expert_calls_tflops": mc.gemm_flops_fwd_bwd() / (statistics.mean(mx["gemm_ms"]) / 1e3) / 1e12,
             "expert_calls_note": "18*d*f*T*k GEMM FLOPs over the two expert calls, MXFP8 "
                                  "quantisation kernels included"}
+        if mx_bf16 is not None:
+            bf_value = mc.T * K * ws / (mx_bf16["total_ms"] / 1e3)
+            line["mxfp8"].update({
+                "bf16_value": bf_value, "bf16_ms_per_step": mx_bf16["total_ms"] / K,
+                "vs_bf16": line["mxfp8"]["value"] / bf_value,
+                "bf16_note": "the same workload and routing with bf16 expert GEMM operands"})
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = {k: v for k, v in cpu_baseline(cfg, args.cpu_seconds).items()
                                 if k in ("value", "unit", "cores", "kind", "sample")}
