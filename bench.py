@@ -361,7 +361,8 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if args.dtype == "bf16" else "mxfp8 (e4m3 + e8m0/32)",
         "data": "synthetic (seeded N(0,1) activations, N(0,1/d) weights, learned-style routing)",
         "config": {"workload": f"{cfg.name}: T={cfg.T} d_model={cfg.d} d_ff={cfg.f} E={cfg.E} "
-                               f"top_k={cfg.k} (4x4096 tokens)",
+                               f"top_k={cfg.k}"
+                               + (f" ({cfg.T // 4096}x4096 tokens)" if cfg.T % 4096 == 0 else ""),
                    "global_batch": cfg.T * ws, "parallelism": f"replicas{ws}" if ws > 1 else "1 GPU",
                    "l2": "flushed between timed steps (512 MiB write outside the step events)"},
         "roofline": {"bound": "tensor", "kernel": "grouped_gemm_kernel (6 launches per step)",

@@ -13,6 +13,7 @@ Workloads (shapes and value distributions):
   mxfp8  T=32768 d=4096 f=1536 E=128 k=4  uniform random expert ids,
                                           drawn without replacement
   e8_shared  e8 plus one shared expert of d_ff 1024 (every token)
+  mxfp8_small T=8192 d=4096 f=1536 E=32 k=4, as mxfp8 (1024 rows per expert)
 
 Values: x ~ N(0,1); router weight, gate/up and down weights ~ N(0, 1/d);
 upstream gradient dY ~ N(0,1); everything rounded to bf16 (round to
@@ -81,6 +82,10 @@ CONFIGS = {
     "mxfp8": MoEConfig("mxfp8", 32768, 4096, 1536, 128, 4,
                        random_routing=True, mxfp8=True),
     "e8_shared": MoEConfig("e8_shared", 16384, 2048, 1024, 8, 4, shared_ff=1024),
+    # the mxfp8 workload's d, f and rows per expert (1024) at a quarter of its
+    # tokens and experts: small enough for full profiler captures
+    "mxfp8_small": MoEConfig("mxfp8_small", 8192, 4096, 1536, 32, 4,
+                             random_routing=True, mxfp8=True),
 }
 
 
