@@ -39,7 +39,7 @@
  *     entry, and moe_get_status reports it later.
  *   - Layouts are row-major.  bf16 = bfloat16 (round to nearest even).
  *   - Supported shapes: 1 <= k <= min(E, 8), 1 <= E <= 1024, T >= 1,
- *     d_model and d_ff multiples of 256.
+ *     d_model and d_ff multiples of 128.
  *
  * Routed-row space.  Every expert e owns a segment of rows
  * [offsets[e], offsets[e+1]) in the permuted buffers; segments start at
@@ -303,8 +303,8 @@ MOE_API moe_status_t moe_permute_bwd(moe_handle_t h, const moe_shape_t* s, const
  *            experts in increasing order; dx_shared may be NULL.
  * Gives the same bits as moe_router_topk_bwd (with dx_router) followed by
  * moe_permute_bwd, but never stores dL w_router.  n_experts <= 64 only
- * (MOE_ERR_UNSUPPORTED otherwise: for n_experts a multiple of 128 that
- * product runs on the tensor cores inside moe_router_topk_bwd).
+ * (MOE_ERR_UNSUPPORTED otherwise: above 64 experts that product runs on the
+ * tensor cores inside moe_router_topk_bwd).
  * In : dx_perm [M_cap,d] bf16, row_map [T,k], d_topk_w [T,k] fp32,
  *      probs [T,E] fp32, topk_idx [T,k], d_probs_aux [E] fp32 or NULL,
  *      w_router [E,d] bf16, dx_shared [T,d] bf16 or NULL.

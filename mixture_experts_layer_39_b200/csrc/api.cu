@@ -20,12 +20,9 @@ using moe::max_rows;
 
 bool router_on_tensor_cores(int E) { return E > 64; }
 
-moe_status_t check_router_shape(const moe_shape_t* s) {
-  const int E = s->n_experts;
-  if (E <= 64) return MOE_OK;
-  if (E % 128 == 0) return MOE_OK;
-  return MOE_ERR_UNSUPPORTED;
-}
+// Row stride of the tensor-core router's logits and bf16 dL buffers: E
+// rounded up to whole 128-column tiles.
+int router_ld(int E) { return (E + 127) / 128 * 128; }
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
@@ -48,7 +45,8 @@ RouterBwdWs router_bwd_layout(const moe_context* h, const moe_shape_t* s) {
   w.nblocks = moe::router_bwd_blocks(h->num_sms);
   size_t off = 0;
   w.dl = off;
-  off += align256(static_cast<size_t>(T) * E * (router_on_tensor_cores(E) ? 2 : 4));
+  off += align256(router_on_tensor_cores(E) ? static_cast<size_t>(T) * router_ld(E) * 2
+                                            : static_cast<size_t>(T) * E * 4);
   w.db_part = off;
   off += align256(static_cast<size_t>(w.nblocks) * E * 4);
   w.part = off;
@@ -108,7 +106,7 @@ size_t workspace_bytes(const moe_context* h, const moe_shape_t* s) {
     upd(w.fwd_total);
     upd(w.bwd_total);
   }
-  upd(align256(static_cast<size_t>(T) * E * 4));                                   // router logits
+  upd(align256(static_cast<size_t>(T) * router_ld(static_cast<int>(E)) * 4));       // router logits
   upd(align256(static_cast<size_t>(moe::n_subchunks(s->T, s->top_k)) * E * 4));    // permute
   upd(router_bwd_layout(h, s).total);                                              // router bwd
   return need;
@@ -201,7 +199,6 @@ moe_status_t moe_router_topk(moe_handle_t h, const moe_shape_t* s, const void* x
                              int32_t* topk_idx, float* topk_w, float* probs, float* logits,
                              void* ws, size_t ws_bytes, moe_stream_t stream) {
   MOE_CHECK_HANDLE(h, s);
-  MOE_TRY(check_router_shape(s));
   if (!all_nonnull(x, w_router, topk_idx, topk_w, probs)) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(w_router, 16)) return MOE_ERR_INVALID_ARG;
   const int T = s->T, d = s->d_model, E = s->n_experts, k = s->top_k;
@@ -214,8 +211,12 @@ moe_status_t moe_router_topk(moe_handle_t h, const moe_shape_t* s, const void* x
         static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_router), bias,
         route_in, T, d, E, k, renorm, topk_idx, topk_w, probs, logits, h->ctl, st));
   }
+  // the GEMM writes whole 128-column tiles: straight into `logits` when E
+  // fills them, else into the workspace, from which the softmax copies
+  // the first E columns of each row to `logits`
+  const int ld = router_ld(E);
   float* lg = logits;
-  if (lg == nullptr) {
+  if (lg == nullptr || ld != E) {
     MOE_TRY(check_ws(h, s, ws, ws_bytes));
     lg = static_cast<float*>(ws);
   } else if (!aligned(lg, 16)) {
@@ -223,9 +224,9 @@ moe_status_t moe_router_topk(moe_handle_t h, const moe_shape_t* s, const void* x
   }
   moe::GemmCtx c{h->num_sms, h->ctl};
   h->launches += 2;
-  MOE_TRY(moe::gemm_router_logits(c, x, w_router, lg, T, d, E, st));
-  return cuda_status(moe::launch_softmax_topk(lg, bias, route_in, T, E, k, renorm, topk_idx, topk_w,
-                                              probs, logits, h->ctl, st));
+  MOE_TRY(moe::gemm_router_logits(c, x, w_router, lg, T, d, E, ld, st));
+  return cuda_status(moe::launch_softmax_topk(lg, ld, bias, route_in, T, E, k, renorm, topk_idx,
+                                              topk_w, probs, logits, h->ctl, st));
 }
 
 moe_status_t moe_permute(moe_handle_t h, const moe_shape_t* s, const void* x,
@@ -563,7 +564,6 @@ moe_status_t moe_permute_router_bwd(moe_handle_t h, const moe_shape_t* s, const 
                                     const float* d_probs_aux, const void* w_router,
                                     const void* dx_shared, void* dx, moe_stream_t stream) {
   MOE_CHECK_HANDLE(h, s);
-  MOE_TRY(check_router_shape(s));
   if (s->n_experts > 64) return MOE_ERR_UNSUPPORTED;
   if (!all_nonnull(dx_perm, row_map, d_topk_w, probs, topk_idx, w_router, dx))
     return MOE_ERR_INVALID_ARG;
@@ -586,7 +586,6 @@ moe_status_t moe_router_topk_bwd(moe_handle_t h, const moe_shape_t* s, const flo
                                  const void* w_router, float* dx_router, void* dw_router,
                                  float* dbias, void* ws, size_t ws_bytes, moe_stream_t stream) {
   MOE_CHECK_HANDLE(h, s);
-  MOE_TRY(check_router_shape(s));
   if (!all_nonnull(d_topk_w, probs, topk_idx, x, w_router, dw_router)) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(dx_router, 16))
     return MOE_ERR_INVALID_ARG;
@@ -608,7 +607,7 @@ moe_status_t moe_router_topk_bwd(moe_handle_t h, const moe_shape_t* s, const flo
     h->launches += 3;
     auto* dl = reinterpret_cast<float*>(base + L.dl);
     MOE_TRY(cuda_status(moe::launch_router_bwd_dl(d_topk_w, probs, topk_idx, d_probs_aux, wb, T, d,
-                                                  E, k, renorm, want_dx, dl, nullptr, dx_router,
+                                                  E, k, renorm, want_dx, dl, nullptr, 0, dx_router,
                                                   db_part,
                                                   L.nblocks, h->ctl, st)));
     MOE_TRY(cuda_status(moe::launch_router_dw(dl, xb, T, d, E, L.n_part, L.group_len, part, st)));
@@ -616,15 +615,17 @@ moe_status_t moe_router_topk_bwd(moe_handle_t h, const moe_shape_t* s, const flo
                                              L.nblocks, E, static_cast<__nv_bfloat16*>(dw_router),
                                              dbias, st));
   }
-  // E a multiple of 128: dL in bf16, both products on the tensor cores
+  // E above 64: dL in bf16 (row stride router_ld(E)), both products on the
+  // tensor cores
   h->launches += want_dx ? 4 : 3;
   auto* dl = reinterpret_cast<__nv_bfloat16*>(base + L.dl);
+  const int ld = router_ld(E);
   MOE_TRY(cuda_status(moe::launch_router_bwd_dl(d_topk_w, probs, topk_idx, d_probs_aux, wb, T, d, E,
-                                                k, renorm, false, nullptr, dl, nullptr, db_part,
+                                                k, renorm, false, nullptr, dl, ld, nullptr, db_part,
                                                 L.nblocks, h->ctl, st)));
   moe::GemmCtx c{h->num_sms, h->ctl};
-  if (want_dx) MOE_TRY(moe::gemm_router_dx(c, dl, w_router, dx_router, T, d, E, st));
-  MOE_TRY(moe::gemm_router_dw_partial(c, dl, x, part, T, d, E, L.n_part, L.group_len, st));
+  if (want_dx) MOE_TRY(moe::gemm_router_dx(c, dl, ld, w_router, dx_router, T, d, E, st));
+  MOE_TRY(moe::gemm_router_dw_partial(c, dl, ld, x, part, T, d, E, L.n_part, L.group_len, st));
   return cuda_status(moe::launch_reduce_dw(part, L.n_part, static_cast<int64_t>(E) * d, db_part,
                                            L.nblocks, E, static_cast<__nv_bfloat16*>(dw_router),
                                            dbias, st));

@@ -48,7 +48,7 @@ inline moe_status_t check_shape(const moe_shape_t* s) {
     return MOE_ERR_INVALID_ARG;
   if (s->top_k > s->n_experts) return MOE_ERR_INVALID_ARG;
   if (s->top_k > 8 || s->n_experts > 1024) return MOE_ERR_UNSUPPORTED;
-  if (s->d_model % 256 != 0 || s->d_ff % 256 != 0) return MOE_ERR_UNSUPPORTED;
+  if (s->d_model % 128 != 0 || s->d_ff % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (s->dtype != MOE_DTYPE_BF16 && s->dtype != MOE_DTYPE_MXFP8) return MOE_ERR_INVALID_ARG;
   if (max_rows(s) >= (1ll << 31) - 256) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;

@@ -112,6 +112,18 @@ tc::GemmArgs base_args(const GemmCtx& c) {
   return a;
 }
 
+// N output columns in tiles of bn (the last tile may be partly past N)
+void set_n(tc::GemmArgs& a, int64_t N, int bn) {
+  a.n_cols = static_cast<int>(N);
+  a.n_tiles_n = static_cast<int>(ceil_div64(N, bn));
+}
+
+// K-grouped: M output rows per group in tiles of mt rows
+void set_m(tc::GemmArgs& a, int64_t M, int mt) {
+  a.m_rows = static_cast<int>(M);
+  a.m_tiles_fixed = static_cast<int>(ceil_div64(M, mt));
+}
+
 }  // namespace
 
 moe_status_t gemm_fwd_gate_up(const GemmCtx& c, const void* x_perm, const int32_t* offsets,
@@ -121,7 +133,7 @@ moe_status_t gemm_fwd_gate_up(const GemmCtx& c, const void* x_perm, const int32_
   if (!tmap_2d(&ta, x_perm, d, m_cap, 2ull * d, 64, 128)) return MOE_ERR_CUDA;
   if (!tmap_3d(&tb, w_gu, d, 2ull * f, E, 2ull * d, 4ull * f * d, 64, 128)) return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  a.n_tiles_n = f / 128;
+  set_n(a, 2ll * f, 256);  // 128 columns of A and of U per tile
   a.k_blocks = d / tc::BK;
   a.n_groups = E;
   a.offsets = offsets;
@@ -145,7 +157,7 @@ moe_status_t gemm_fwd_down(const GemmCtx& c, const void* h, const int32_t* offse
   if (!tmap_3d(&tb, w_d, f, d, E, 2ull * f, 2ull * d * f, 64, c.pair_m ? 128 : 256))
     return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  a.n_tiles_n = d / 256;
+  set_n(a, d, 256);
   a.k_blocks = f / tc::BK;
   a.n_groups = E;
   a.offsets = offsets;
@@ -166,7 +178,7 @@ moe_status_t gemm_dgrad_down_swiglu(const GemmCtx& c, const void* do_perm, const
   // W_d[e] is [d (contraction), f (output)]: N-major operand
   if (!tmap_3d(&tb, w_d, f, d, E, 2ull * f, 2ull * d * f, 64, 64)) return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  a.n_tiles_n = f / 256;
+  set_n(a, f, 256);
   a.k_blocks = d / tc::BK;
   a.n_groups = E;
   a.offsets = offsets;
@@ -190,7 +202,7 @@ moe_status_t gemm_dgrad_gate_up(const GemmCtx& c, const void* dau, const int32_t
   // W_gu[e] is [2f (contraction), d (output)]: N-major operand
   if (!tmap_3d(&tb, w_gu, d, 2ull * f, E, 2ull * d, 4ull * f * d, 64, 64)) return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  a.n_tiles_n = d / 256;
+  set_n(a, d, 256);
   a.k_blocks = 2 * f / tc::BK;
   a.n_groups = E;
   a.offsets = offsets;
@@ -211,8 +223,7 @@ moe_status_t gemm_wgrad_down(const GemmCtx& c, const void* do_perm, const void* 
   if (!tmap_2d(&ta, do_perm, d, m_cap, 2ull * d, 64, 64)) return MOE_ERR_CUDA;
   if (!tmap_3d(&tb, h, f, m_cap, 1, 2ull * f, 2ull * f * m_cap, 64, 64)) return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  a.n_tiles_n = f / 256;
-  a.m_tiles_fixed = d / tc::BM;
+  set_n(a, f, 256);
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
@@ -220,7 +231,7 @@ moe_status_t gemm_wgrad_down(const GemmCtx& c, const void* do_perm, const void* 
   a.out = dw_d;
   a.ldo = f;
   a.out_gstride = static_cast<int64_t>(d) * f;
-  a.m_tiles_fixed = d / (2 * tc::BM);  // CTA pairs: 256-row tiles
+  set_m(a, d, 2 * tc::BM);  // CTA pairs: 256-row tiles
   const int64_t tiles = static_cast<int64_t>(E) * a.m_tiles_fixed * a.n_tiles_n;
   const int grid = static_cast<int>(2 * tiles < c.num_sms ? 2 * tiles : c.num_sms);
   return launch<256, true, true, tc::EPI_BF16, true, false, true>(ta, tb, a, grid, st);
@@ -233,8 +244,7 @@ moe_status_t gemm_wgrad_gate_up(const GemmCtx& c, const void* dau, const void* x
   if (!tmap_2d(&ta, dau, 2ull * f, m_cap, 4ull * f, 64, 64)) return MOE_ERR_CUDA;
   if (!tmap_3d(&tb, x_perm, d, m_cap, 1, 2ull * d, 2ull * d * m_cap, 64, 64)) return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  a.n_tiles_n = d / 256;
-  a.m_tiles_fixed = 2 * f / tc::BM;
+  set_n(a, d, 256);
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
@@ -242,7 +252,7 @@ moe_status_t gemm_wgrad_gate_up(const GemmCtx& c, const void* dau, const void* x
   a.out = dw_gu;
   a.ldo = d;
   a.out_gstride = 2ll * f * d;
-  a.m_tiles_fixed = 2 * f / (2 * tc::BM);  // CTA pairs: 256-row tiles
+  set_m(a, 2ll * f, 2 * tc::BM);  // CTA pairs: 256-row tiles
   const int64_t tiles = static_cast<int64_t>(E) * a.m_tiles_fixed * a.n_tiles_n;
   const int grid = static_cast<int>(2 * tiles < c.num_sms ? 2 * tiles : c.num_sms);
   return launch<256, true, true, tc::EPI_BF16, true, false, true>(ta, tb, a, grid, st);
@@ -258,7 +268,7 @@ moe_status_t gemm_fwd_gate_up_gather(const GemmCtx& c, const void* x, int T,
   if (!tmap_2d(&ta, x, d, T, 2ull * d, 64, 1)) return MOE_ERR_CUDA;
   if (!tmap_3d(&tb, w_gu, d, 2ull * f, E, 2ull * d, 4ull * f * d, 64, 128)) return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  a.n_tiles_n = f / 128;
+  set_n(a, 2ll * f, 256);  // 128 columns of A and of U per tile
   a.k_blocks = d / tc::BK;
   a.n_groups = E;
   a.offsets = offsets;
@@ -287,7 +297,7 @@ moe_status_t gemm_wgrad_gate_up_gather(const GemmCtx& c, const void* dau, const 
   if (!tmap_2d(&ta, dau, 2ull * f, m_cap, 4ull * f, 64, 64)) return MOE_ERR_CUDA;
   if (!tmap_2d(&tb, x, d, T, 2ull * d, 64, 1)) return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  a.n_tiles_n = d / 256;
+  set_n(a, d, 256);
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
@@ -296,7 +306,7 @@ moe_status_t gemm_wgrad_gate_up_gather(const GemmCtx& c, const void* dau, const 
   a.out = dw_gu;
   a.ldo = d;
   a.out_gstride = 2ll * f * d;
-  a.m_tiles_fixed = 2 * f / (2 * tc::BM);  // CTA pairs: 256-row tiles
+  set_m(a, 2ll * f, 2 * tc::BM);  // CTA pairs: 256-row tiles
   a.row_src = row_src;
   a.src_oob = T;
   const int64_t tiles = static_cast<int64_t>(E) * a.m_tiles_fixed * a.n_tiles_n;
@@ -305,12 +315,14 @@ moe_status_t gemm_wgrad_gate_up_gather(const GemmCtx& c, const void* dau, const 
 }
 
 moe_status_t gemm_router_logits(const GemmCtx& c, const void* x, const void* w_r, float* logits,
-                                int T, int d, int E, cudaStream_t st) {
+                                int T, int d, int E, int ld, cudaStream_t st) {
   CUtensorMap ta, tb;
   if (!tmap_2d(&ta, x, d, T, 2ull * d, 64, 128)) return MOE_ERR_CUDA;
   if (!tmap_3d(&tb, w_r, d, E, 1, 2ull * d, 2ull * d * E, 64, 128)) return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  a.n_tiles_n = E / 128;
+  // ld = E rounded up to whole 128-column tiles; the columns past E come out
+  // zero (W_r rows past E read as TMA zero fill)
+  set_n(a, ld, 128);
   a.k_blocks = d / tc::BK;
   a.n_groups = 1;
   a.offsets = nullptr;
@@ -318,20 +330,21 @@ moe_status_t gemm_router_logits(const GemmCtx& c, const void* x, const void* w_r
   a.total_len = T;
   a.m_cap = T;
   a.out = logits;
-  a.ldo = E;
+  a.ldo = ld;
   const int64_t tiles = ceil_div64(T, tc::BM) * a.n_tiles_n;
   const int grid = static_cast<int>(tiles < c.num_sms ? tiles : c.num_sms);
   return launch<128, false, false, tc::EPI_F32, false>(ta, tb, a, grid, st);
 }
 
-moe_status_t gemm_router_dx(const GemmCtx& c, const void* dl_bf16, const void* w_r,
+moe_status_t gemm_router_dx(const GemmCtx& c, const void* dl_bf16, int ld, const void* w_r,
                             float* dx_router, int T, int d, int E, cudaStream_t st) {
   CUtensorMap ta, tb;
-  if (!tmap_2d(&ta, dl_bf16, E, T, 2ull * E, 64, 128)) return MOE_ERR_CUDA;
+  // contraction over E, zero-filled past E in both operands
+  if (!tmap_2d(&ta, dl_bf16, E, T, 2ull * ld, 64, 128)) return MOE_ERR_CUDA;
   if (!tmap_3d(&tb, w_r, d, E, 1, 2ull * d, 2ull * d * E, 64, 64)) return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  a.n_tiles_n = d / 256;
-  a.k_blocks = E / tc::BK;
+  set_n(a, d, 256);
+  a.k_blocks = static_cast<int>(ceil_div64(E, tc::BK));
   a.n_groups = 1;
   a.offsets = nullptr;
   a.uniform_len = T;
@@ -345,7 +358,7 @@ moe_status_t gemm_router_dx(const GemmCtx& c, const void* dl_bf16, const void* w
 }
 
 int router_dw_groups(int num_sms, int T, int d, int E, int* group_len) {
-  const int tiles_per_group = (E / tc::BM) * (d / 256);
+  const int tiles_per_group = static_cast<int>(ceil_div64(E, tc::BM) * ceil_div64(d, 256));
   int g = num_sms / (tiles_per_group > 0 ? tiles_per_group : 1);
   if (g < 1) g = 1;
   int64_t len = ceil_div64(ceil_div64(T, g), 64) * 64;
@@ -354,15 +367,15 @@ int router_dw_groups(int num_sms, int T, int d, int E, int* group_len) {
   return g;
 }
 
-moe_status_t gemm_router_dw_partial(const GemmCtx& c, const void* dl_bf16, const void* x,
+moe_status_t gemm_router_dw_partial(const GemmCtx& c, const void* dl_bf16, int ld, const void* x,
                                     float* partial, int T, int d, int E, int n_groups,
                                     int group_len, cudaStream_t st) {
   CUtensorMap ta, tb;
-  if (!tmap_2d(&ta, dl_bf16, E, T, 2ull * E, 64, 64)) return MOE_ERR_CUDA;
+  if (!tmap_2d(&ta, dl_bf16, E, T, 2ull * ld, 64, 64)) return MOE_ERR_CUDA;
   if (!tmap_3d(&tb, x, d, T, 1, 2ull * d, 2ull * d * T, 64, 64)) return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  a.n_tiles_n = d / 256;
-  a.m_tiles_fixed = E / tc::BM;
+  set_n(a, d, 256);
+  set_m(a, E, tc::BM);
   a.n_groups = n_groups;
   a.offsets = nullptr;
   a.uniform_len = group_len;
@@ -386,7 +399,7 @@ moe_status_t gemm_mx_fwd_gate_up(const GemmCtx& c, const MxOperand& x, const int
   if (!tmap_2d(&ta, x.q, d, m_cap, d, 128, 128, true)) return MOE_ERR_CUDA;
   if (!tmap_3d(&tb, w_gu.q, d, 2ull * f, E, d, 2ull * f * d, 128, 64, true)) return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  a.n_tiles_n = f / 64;
+  set_n(a, 2ll * f, 128);  // 64 columns of A and of U per tile
   a.k_blocks = d / 128;
   a.n_groups = E;
   a.offsets = offsets;
@@ -410,7 +423,7 @@ moe_status_t gemm_mx_fwd_down(const GemmCtx& c, const MxOperand& h, const int32_
   if (!tmap_2d(&ta, h.q, f, m_cap, f, 128, 128, true)) return MOE_ERR_CUDA;
   if (!tmap_3d(&tb, w_d.q, f, d, E, f, 1ull * d * f, 128, 128, true)) return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  a.n_tiles_n = d / 128;
+  set_n(a, d, 128);
   a.k_blocks = f / 128;
   a.n_groups = E;
   a.offsets = offsets;
@@ -432,7 +445,7 @@ moe_status_t gemm_mx_dgrad_down_swiglu(const GemmCtx& c, const MxOperand& dO, co
   // W_d[e] is [d (contraction), f (output)]: N-major, quantised along d
   if (!tmap_3d(&tb, w_d_col.q, f, d, E, f, 1ull * d * f, 128, 128, true)) return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  a.n_tiles_n = f / 128;
+  set_n(a, f, 128);
   a.k_blocks = d / 128;
   a.n_groups = E;
   a.offsets = offsets;
@@ -456,7 +469,7 @@ moe_status_t gemm_mx_dgrad_gate_up(const GemmCtx& c, const MxOperand& dau, const
   if (!tmap_2d(&ta, dau.q, 2ull * f, m_cap, 2ull * f, 128, 128, true)) return MOE_ERR_CUDA;
   if (!tmap_3d(&tb, w_gu_col.q, d, 2ull * f, E, d, 2ull * f * d, 128, 128, true)) return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  a.n_tiles_n = d / 128;
+  set_n(a, d, 128);
   a.k_blocks = 2 * f / 128;
   a.n_groups = E;
   a.offsets = offsets;
@@ -479,8 +492,8 @@ moe_status_t gemm_mx_wgrad(const GemmCtx& c, const MxOperand& a_col, int M, cons
   if (!tmap_2d(&ta, a_col.q, M, m_cap, M, 128, 128, true)) return MOE_ERR_CUDA;
   if (!tmap_3d(&tb, b_col.q, N, m_cap, 1, N, 1ull * N * m_cap, 128, 128, true)) return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  a.n_tiles_n = N / 128;
-  a.m_tiles_fixed = M / tc::BM;
+  set_n(a, N, 128);
+  set_m(a, M, tc::BM);
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);

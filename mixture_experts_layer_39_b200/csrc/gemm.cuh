@@ -47,12 +47,14 @@ moe_status_t gemm_wgrad_gate_up_gather(const GemmCtx& c, const void* dau, const 
                                        const int32_t* row_src, const int32_t* offsets,
                                        void* dw_gu, int E, int d, int f, int64_t m_cap,
                                        cudaStream_t st);
+// Router on the tensor cores (any E above 64): the logits buffer and the
+// bf16 dL buffer have row stride ld = E rounded up to a multiple of 128.
 moe_status_t gemm_router_logits(const GemmCtx& c, const void* x, const void* w_r, float* logits,
-                                int T, int d, int E, cudaStream_t st);
-moe_status_t gemm_router_dx(const GemmCtx& c, const void* dl_bf16, const void* w_r,
+                                int T, int d, int E, int ld, cudaStream_t st);
+moe_status_t gemm_router_dx(const GemmCtx& c, const void* dl_bf16, int ld, const void* w_r,
                             float* dx_router, int T, int d, int E, cudaStream_t st);
 int router_dw_groups(int num_sms, int T, int d, int E, int* group_len);
-moe_status_t gemm_router_dw_partial(const GemmCtx& c, const void* dl_bf16, const void* x,
+moe_status_t gemm_router_dw_partial(const GemmCtx& c, const void* dl_bf16, int ld, const void* x,
                                     float* partial, int T, int d, int E, int n_groups,
                                     int group_len, cudaStream_t st);
 

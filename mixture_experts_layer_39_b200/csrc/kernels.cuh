@@ -17,9 +17,11 @@ cudaError_t launch_router_fused(const __nv_bfloat16* x, const __nv_bfloat16* w_r
                                 const int32_t* route_in, int T, int d, int E, int k, bool renorm,
                                 int32_t* idx, float* w, float* probs, float* logits,
                                 DeviceCtl* ctl, cudaStream_t st);
-cudaError_t launch_softmax_topk(const float* logits_in, const float* bias, const int32_t* route_in,
-                                int T, int E, int k, bool renorm, int32_t* idx, float* w,
-                                float* probs, float* logits_out, DeviceCtl* ctl, cudaStream_t st);
+// logits_in has row stride ld_in; logits_out (dense [T, E]) may alias it when ld_in = E
+cudaError_t launch_softmax_topk(const float* logits_in, int ld_in, const float* bias,
+                                const int32_t* route_in, int T, int E, int k, bool renorm,
+                                int32_t* idx, float* w, float* probs, float* logits_out,
+                                DeviceCtl* ctl, cudaStream_t st);
 
 // ---- router load statistics and load-balancing loss
 int router_stats_blocks(int num_sms, int T);
@@ -70,7 +72,7 @@ cudaError_t launch_router_bwd_dl(const float* dw, const float* probs, const int3
                                  const float* dprob_aux, const __nv_bfloat16* w_r, int T, int d,
                                  int E, int k, bool renorm,
                                  bool fuse_dx, float* dl_f32, __nv_bfloat16* dl_bf16,
-                                 float* dx_router, float* db_partial, int nblocks,
+                                 int ld_bf16, float* dx_router, float* db_partial, int nblocks,
                                  DeviceCtl* ctl, cudaStream_t st);
 // dW_r partial rows [n_chunks][E*d] over token chunks (E <= 64);
 // router_dw_chunks picks the chunking.

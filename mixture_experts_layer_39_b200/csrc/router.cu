@@ -396,7 +396,8 @@ __global__ void __launch_bounds__(kMmaWarps * 32, NT == 1 ? 7 : 5)
 // argmax on (logit desc, index asc).
 template <int NPL>
 __global__ void __launch_bounds__(kWarps * 32)
-    softmax_topk_kernel(const float* __restrict__ logits_in, const float* __restrict__ bias,
+    softmax_topk_kernel(const float* __restrict__ logits_in, int ld_in,
+                        const float* __restrict__ bias,
                         const int32_t* __restrict__ route_in, int T, int E, int k, int renorm,
                         int32_t* __restrict__ idx_out, float* __restrict__ w_out,
                         float* __restrict__ probs, float* __restrict__ logits_out,
@@ -410,7 +411,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   for (int i = 0; i < NPL; ++i) {
     const int e = lane + 32 * i;
     if (e < E) {
-      l[i] = logits_in[t * E + e] + (bias != nullptr ? __ldg(bias + e) : 0.f);
+      l[i] = logits_in[t * ld_in + e] + (bias != nullptr ? __ldg(bias + e) : 0.f);
       m = fmaxf(m, l[i]);
     } else {
       l[i] = -FLT_MAX;
@@ -528,12 +529,13 @@ cudaError_t launch_router_fused(const __nv_bfloat16* x, const __nv_bfloat16* w_r
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_softmax_topk(const float* logits_in, const float* bias, const int32_t* route_in,
-                                int T, int E, int k, bool renorm, int32_t* idx, float* w,
-                                float* probs, float* logits_out, DeviceCtl* ctl, cudaStream_t st) {
+cudaError_t launch_softmax_topk(const float* logits_in, int ld_in, const float* bias,
+                                const int32_t* route_in, int T, int E, int k, bool renorm,
+                                int32_t* idx, float* w, float* probs, float* logits_out,
+                                DeviceCtl* ctl, cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>(ceil_div64(T, kWarps));
   auto go = [&](auto kern) {
-    kern<<<grid, kWarps * 32, 0, st>>>(logits_in, bias, route_in, T, E, k, renorm ? 1 : 0, idx, w,
+    kern<<<grid, kWarps * 32, 0, st>>>(logits_in, ld_in, bias, route_in, T, E, k, renorm ? 1 : 0, idx, w,
                                        probs, logits_out, ctl);
     return cudaGetLastError();
   };

@@ -98,7 +98,8 @@ __global__ void __launch_bounds__(kWarps * 32)
                          const int32_t* __restrict__ idx, const float* __restrict__ dprob_aux,
                          const __nv_bfloat16* __restrict__ w_r,
                          int T, int d, int E, int k, int renorm, float* __restrict__ dl_f32,
-                         __nv_bfloat16* __restrict__ dl_bf16, float* __restrict__ dx_router,
+                         __nv_bfloat16* __restrict__ dl_bf16, int ld_bf16,
+                         float* __restrict__ dx_router,
                          float* __restrict__ db_partial, int stage_w) {
   __shared__ float s_db[kWarps][32 * NPL];
   extern __shared__ uint4 s_wdyn[];
@@ -126,7 +127,7 @@ __global__ void __launch_bounds__(kWarps * 32)
       if (e < E) {
         db[i] += dl[i];
         if (dl_f32 != nullptr) dl_f32[t * E + e] = dl[i];
-        if (dl_bf16 != nullptr) dl_bf16[t * E + e] = __float2bfloat16_rn(dl[i]);
+        if (dl_bf16 != nullptr) dl_bf16[t * ld_bf16 + e] = __float2bfloat16_rn(dl[i]);
       }
     }
     if constexpr (FUSE_DX) {
@@ -421,7 +422,7 @@ cudaError_t launch_router_bwd_dl(const float* dw, const float* probs, const int3
                                  const float* dprob_aux, const __nv_bfloat16* w_r, int T, int d,
                                  int E, int k, bool renorm,
                                  bool fuse_dx, float* dl_f32, __nv_bfloat16* dl_bf16,
-                                 float* dx_router, float* db_partial, int nblocks,
+                                 int ld_bf16, float* dx_router, float* db_partial, int nblocks,
                                  DeviceCtl* ctl, cudaStream_t st) {
   (void)ctl;
   const size_t w_bytes = static_cast<size_t>(E) * d * 2;
@@ -434,7 +435,7 @@ cudaError_t launch_router_bwd_dl(const float* dw, const float* probs, const int3
       return cudaErrorInvalidValue;
     kern<<<nblocks, kWarps * 32, smem, st>>>(dw, probs, idx, dprob_aux, w_r, T, d, E, k,
                                              renorm ? 1 : 0,
-                                             dl_f32, dl_bf16, dx_router, db_partial,
+                                             dl_f32, dl_bf16, ld_bf16, dx_router, db_partial,
                                              stage ? 1 : 0);
     return cudaGetLastError();
   };
@@ -493,7 +494,7 @@ cudaError_t launch_router_dw(const float* dl, const __nv_bfloat16* x, int T, int
 cudaError_t launch_reduce_dw(const float* partial, int n_part, int64_t n_w, const float* db_part,
                              int n_db, int E, __nv_bfloat16* dw_out, float* db_out,
                              cudaStream_t st) {
-  // n_w = E * d is a multiple of 4 (d is a multiple of 256)
+  // n_w = E * d is a multiple of 4 (d is a multiple of 128)
   const int64_t n4 = n_w / 4 + (db_out != nullptr ? (E + 3) / 4 : 0);
   reduce_dw_kernel<<<static_cast<unsigned>(ceil_div64(n4, 32)), kRedWarps * 32, 0, st>>>(
       reinterpret_cast<const float4*>(partial), n_part, n_w / 4, n_w / 4, db_part, n_db, E, dw_out,

@@ -49,6 +49,9 @@ enum Epi : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_SWIGLU_FWD = 2, EPI_SWIGLU_BWD =
 
 struct GemmArgs {
   int n_tiles_n;     // tiles along N per (group, m-tile)
+  int n_cols;        // columns of the output (N); the last N tile may run past it
+  int m_rows;        // K-grouped: rows of each group's output (M); the last M tile
+                     // may run past it (operand rows past it read as TMA zero fill)
   int k_blocks;      // M-grouped: contraction length / BK
   int n_groups;
   const int* offsets;  // [n_groups + 1] on the device, or nullptr: uniform groups
@@ -927,7 +930,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     auto quarter_rows = [&](const Tile& tl) -> int {
       if constexpr (KGROUP) {
-        return 32;
+        const int64_t n = args.m_rows - quarter_first(tl);
+        return n <= 0 ? 0 : (n >= 32 ? 32 : static_cast<int>(n));
       } else {
         const int rpw = rows_per_warp(tl);
         int64_t lim = tl.row_end < args.m_cap ? tl.row_end : args.m_cap;
@@ -961,12 +965,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
       const bool zero_acc = KGROUP && tl.k_blocks == 0;
+      // output columns of this tile that exist (a multiple of 64; the SwiGLU
+      // forward tile always lies inside [A | U])
+      const int n_left = args.n_cols - tl.n_tile * BN;
+      const int ncols = n_left < BN ? n_left : BN;
       const int64_t gofs = KGROUP ? static_cast<int64_t>(tl.group) * args.out_gstride : 0;
       if constexpr (EPI == EPI_BF16) {
         auto* base = static_cast<__nv_bfloat16*>(args.out) + gofs + row_first * args.ldo +
                      static_cast<int64_t>(tl.n_tile) * BN;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 64) {
+        for (int c = 0; c < ncols; c += 64) {
           uint32_t r0[32], r1[32];
           tmem_ld32(tbase + c, r0);
           tmem_ld32(tbase + c + 32, r1);
@@ -985,7 +993,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto* base = static_cast<float*>(args.out) + gofs + row_first * args.ldo +
                      static_cast<int64_t>(tl.n_tile) * BN;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
+        for (int c = 0; c < ncols; c += 32) {
           uint32_t r[32];
           tmem_ld32(tbase + c, r);
           tmem_ld_wait();
@@ -1040,14 +1048,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto* dau = static_cast<__nv_bfloat16*>(args.out) + row_first * args.ldo +
                     static_cast<int64_t>(tl.n_tile) * BN;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 64) {
+        for (int c = 0; c < ncols; c += 64) {
           uint4 va[8], vu[8];
           cp_async_wait_all();
           __syncwarp();
           stage_read_row(lbuf_a, lane, va);
           stage_read_row(lbuf_u, lane, vu);
           __syncwarp();
-          if (c + 64 < BN) {  // next chunk lands while this one is computed and stored
+          if (c + 64 < ncols) {  // next chunk lands while this one is computed and stored
             cp_async_rows(lbuf_a, reinterpret_cast<const uint8_t*>(aux + c + 64), args.ld_aux * 2,
                           vrows, lane, args.aux);
             cp_async_rows(lbuf_u, reinterpret_cast<const uint8_t*>(aux + args.f + c + 64),

@@ -8,8 +8,8 @@ in order on the current stream:
             -> moe_unpermute_combine
   backward: moe_unpermute_combine_bwd -> moe_router_topk_bwd
             -> moe_grouped_swiglu_bwd -> moe_permute_router_bwd  (E <= 64)
-            or, for E a multiple of 128 (router products on the tensor
-            cores), moe_router_topk_bwd writes dX_router and
+            or, for E above 64 (router products on the tensor cores),
+            moe_router_topk_bwd writes dX_router and
             moe_permute_bwd adds it.
 
 With shared_ff > 0 a shared expert runs on every token

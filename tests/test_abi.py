@@ -51,15 +51,20 @@ def test_max_rows_and_shape_checks(lib):
     assert lib.moe_max_rows(ctypes.byref(s), ctypes.byref(n)) == 0
     assert n.value == 16384 * 4 + 31 * 128
     bad = [
-        _lib.MoeShape(16, 200, 256, 8, 2, 0, 0),     # d not a multiple of 256 -> unsupported
+        _lib.MoeShape(16, 200, 256, 8, 2, 0, 0),     # d not a multiple of 128 -> unsupported
+        _lib.MoeShape(16, 256, 320, 8, 2, 0, 0),     # d_ff not a multiple of 128 -> unsupported
         _lib.MoeShape(16, 256, 256, 8, 9, 0, 0),     # k > E -> invalid
         _lib.MoeShape(16, 256, 256, 2048, 2, 0, 0),  # E > 1024 -> unsupported
         _lib.MoeShape(0, 256, 256, 8, 2, 0, 0),      # T = 0 -> invalid
         _lib.MoeShape(16, 256, 256, 8, 2, 7, 0),     # unknown dtype -> invalid
     ]
-    want = [2, 1, 2, 1, 1]
+    want = [2, 2, 1, 2, 1, 1]
     for s_, w in zip(bad, want):
         assert lib.moe_max_rows(ctypes.byref(s_), ctypes.byref(n)) == w
+    # multiples of 128 that are not multiples of 256, and any E up to 1024
+    for good in [(16, 384, 640, 8, 2), (16, 128, 128, 200, 8), (3, 256, 384, 1024, 8)]:
+        s_ = _lib.MoeShape(*good, 0, 0)
+        assert lib.moe_max_rows(ctypes.byref(s_), ctypes.byref(n)) == 0
 
 
 def test_null_handle_rejected_before_any_launch(lib):

@@ -45,6 +45,7 @@ CASES = [
     (300, 256, 256, 13, 5, True),      # odd E, renormalised gate weights
     (333, 256, 256, 64, 8, False),     # largest E of the CUDA-core router backward
     (520, 256, 256, 128, 4, False),    # tensor-core router backward (E = 128)
+    (300, 384, 256, 100, 4, True),     # E = 100: padded dL rows, zero-filled contraction tail
 ]
 
 

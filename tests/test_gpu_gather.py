@@ -34,6 +34,7 @@ CASES = [
     (520, 256, 256, 128, 4),
     (3072, 256, 256, 8, 4),
     (2080, 512, 256, 1, 1),
+    (1600, 384, 640, 2, 2),          # half-used last N tiles and wgrad M tiles
 ]
 
 

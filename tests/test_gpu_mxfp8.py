@@ -33,7 +33,7 @@ def _segments(L, E):
 
 
 @pytest.mark.parametrize("T,d,f,E,k", [(384, 256, 256, 4, 2), (700, 512, 256, 6, 3),
-                                       (256, 256, 512, 8, 1)])
+                                       (256, 256, 512, 8, 1), (384, 384, 384, 4, 2)])
 def test_mxfp8_small_every_stage(cuda_ok, T, d, f, E, k):
     cfg = custom_config(T, d, f, E, k, random_routing=True, mxfp8=True)
     inp = make_inputs(cfg, seed=T + d, device="cpu")

@@ -169,6 +169,13 @@ SMALL_CASES = [
     (2080, 512, 256, 1, 1, "learned"),     # one expert, pair tiles with a ragged tail
     (500, 768, 256, 7, 2, "renorm"),       # odd E, d not a multiple of 512
     (257, 256, 256, 13, 5, "bias"),        # second expert tile of the router partly empty
+    (2048, 256, 256, 1024, 8, "learned"),  # the largest E and k
+    (300, 256, 256, 4, 4, "learned"),      # k = E: every token on every expert
+    (1600, 384, 640, 2, 2, "learned"),     # CTA pairs; d, f multiples of 128 but not of 256:
+                                           # half-used last N tiles and wgrad M tiles
+    (600, 384, 384, 8, 2, "bias"),         # single-CTA tiles, half-used last N tiles
+    (700, 256, 256, 200, 6, "learned"),    # E = 200: tensor-core router, padded logits rows
+    (500, 384, 128, 96, 3, "renorm"),      # E = 96, f = 128: one half-used N tile
 ]
 
 

@@ -34,6 +34,7 @@ CASES = [
     (300, 256, 256, 13, 5, "bf16"),
     (520, 256, 256, 128, 4, "bf16"),
     (1024, 256, 256, 8, 4, "mxfp8"),
+    (600, 384, 384, 8, 2, "bf16"),     # half-used last N tiles
 ]
 
 

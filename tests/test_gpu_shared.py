@@ -28,6 +28,7 @@ CASES = [
     (300, 256, 256, 13, 5, 256),     # ragged T (a 44-row last tile), k > 4
     (2080, 512, 256, 8, 4, 768),     # CTA-pair tiles of the shared expert, ragged tail
     (520, 256, 256, 128, 4, 256),    # E = 128: separate router dX plus the shared term
+    (600, 384, 384, 8, 2, 384),      # d, d_ff multiples of 128 only: half-used last tiles
 ]
 
 
