@@ -1,7 +1,6 @@
 // extern "C" entry points of libmoe.so (declared and documented in
 // include/moe.h): argument checks, workspace carving, launch order.
 #include <cstdio>
-#include <cstdlib>
 #include <new>
 
 #include "context.cuh"

@@ -64,16 +64,12 @@ bool tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, bool FP8 = false, bool PAIR = false,
-          bool GATHER = false>
-moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const tc::GemmArgs& args, int grid,
-                    cudaStream_t st) {
-  // the SwiGLU-backward epilogue's landing buffers take one stage's room;
-  // MXFP8 stages are 32 KB of operands plus 1 KB of scale atoms; a CTA of a
-  // pair holds 32 KB of operands per stage
-  constexpr int STAGES = FP8    ? (EPI == tc::EPI_SWIGLU_BWD ? 5 : 6)
-                         : PAIR ? (EPI == tc::EPI_SWIGLU_BWD ? 5 : 6)
-                                : (BN == 256 ? (EPI == tc::EPI_SWIGLU_BWD ? 3 : 4) : 6);
+constexpr size_t kMaxDynSmem = 227 * 1024;  // per block on sm_100
+
+template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, int STAGES, bool FP8, bool PAIR,
+          bool GATHER>
+moe_status_t launch_stages(const CUtensorMap& a, const CUtensorMap& b, const tc::GemmArgs& args,
+                           int grid, cudaStream_t st) {
   auto kern = tc::grouped_gemm_kernel<BN, A_MN, B_MN, EPI, KGROUP, STAGES, FP8, PAIR, GATHER>;
   const size_t smem = tc::SmemPlan<BN, STAGES, EPI, FP8, PAIR>::bytes(args.n_groups);
   static size_t configured = 0;  // largest size this instantiation was opened for
@@ -104,6 +100,44 @@ moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const tc::GemmAr
     kern<<<grid, tc::kThreads, smem, st>>>(a, b, args);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }
+}
+
+// Ring depth: as many stages as fit beside the epilogue buffers.  A stage is
+// 48 KB for single-CTA 128 x 256 tiles and for wide pairs, 32 KB for 256 x 256
+// pairs and 16 KB (+1 KB of scale atoms) for MXFP8 128 x 128 tiles.  The
+// SwiGLU backward's landing buffers take 16 KB more; with more than ~440
+// experts the tile table no longer fits beside a sixth pair stage, and the
+// launch falls back to one stage fewer.
+template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, bool FP8 = false, bool PAIR = false,
+          bool GATHER = false>
+moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const tc::GemmArgs& args, int grid,
+                    cudaStream_t st) {
+  constexpr bool BWD = EPI == tc::EPI_SWIGLU_BWD;
+  constexpr int STAGES = FP8    ? (BWD ? 5 : 6)
+                         : PAIR ? (BN == 512 ? (BWD ? 3 : 4) : 6)
+                                : (BN == 256 ? 4 : 6);
+  if constexpr (BWD && !FP8) {
+    if (tc::SmemPlan<BN, STAGES, EPI, FP8, PAIR>::bytes(args.n_groups) > kMaxDynSmem)
+      return launch_stages<BN, A_MN, B_MN, EPI, KGROUP, STAGES - 1, FP8, PAIR, GATHER>(a, b, args,
+                                                                                      grid, st);
+  }
+  return launch_stages<BN, A_MN, B_MN, EPI, KGROUP, STAGES, FP8, PAIR, GATHER>(a, b, args, grid, st);
+}
+
+// Weight gradients run 256 x 512 pair tiles ("wide") when the experts'
+// contraction ranges are long (at least 4096 routed rows on average: the
+// single accumulator's epilogue, which no longer overlaps the next tile, is
+// then a few percent of a tile) and 256 x 256 tiles would not fill the SMs'
+// waves enough better.  A wide tile does twice the work of a narrow one in
+// about 0.87 of twice its time (it reads 25% fewer operand bytes per FLOP);
+// tiles = E x M tiles x N tiles, units = CTA pairs.
+bool wide_wgrad(int num_sms, int64_t E, int64_t M, int64_t N, int64_t rows) {
+  if (rows < 4096 * E) return false;
+  const int64_t units = num_sms / 2 > 0 ? num_sms / 2 : 1;
+  const int64_t mt = ceil_div64(M, 256);
+  const int64_t waves_n = ceil_div64(E * mt * ceil_div64(N, 256), units);
+  const int64_t waves_w = ceil_div64(E * mt * ceil_div64(N, 512), units);
+  return 174 * waves_w <= 100 * waves_n;
 }
 
 tc::GemmArgs base_args(const GemmCtx& c) {
@@ -222,8 +256,9 @@ moe_status_t gemm_wgrad_down(const GemmCtx& c, const void* do_perm, const void* 
   // A = dO^T (M = d along the rows' contiguous axis), B = H (N = f)
   if (!tmap_2d(&ta, do_perm, d, m_cap, 2ull * d, 64, 64)) return MOE_ERR_CUDA;
   if (!tmap_3d(&tb, h, f, m_cap, 1, 2ull * f, 2ull * f * m_cap, 64, 64)) return MOE_ERR_CUDA;
+  const bool wide = wide_wgrad(c.num_sms, E, d, f, m_cap);
   tc::GemmArgs a = base_args(c);
-  set_n(a, f, 256);
+  set_n(a, f, wide ? 512 : 256);
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
@@ -234,6 +269,7 @@ moe_status_t gemm_wgrad_down(const GemmCtx& c, const void* do_perm, const void* 
   set_m(a, d, 2 * tc::BM);  // CTA pairs: 256-row tiles
   const int64_t tiles = static_cast<int64_t>(E) * a.m_tiles_fixed * a.n_tiles_n;
   const int grid = static_cast<int>(2 * tiles < c.num_sms ? 2 * tiles : c.num_sms);
+  if (wide) return launch<512, true, true, tc::EPI_BF16, true, false, true>(ta, tb, a, grid, st);
   return launch<256, true, true, tc::EPI_BF16, true, false, true>(ta, tb, a, grid, st);
 }
 
@@ -243,8 +279,9 @@ moe_status_t gemm_wgrad_gate_up(const GemmCtx& c, const void* dau, const void* x
   CUtensorMap ta, tb;
   if (!tmap_2d(&ta, dau, 2ull * f, m_cap, 4ull * f, 64, 64)) return MOE_ERR_CUDA;
   if (!tmap_3d(&tb, x_perm, d, m_cap, 1, 2ull * d, 2ull * d * m_cap, 64, 64)) return MOE_ERR_CUDA;
+  const bool wide = wide_wgrad(c.num_sms, E, 2ll * f, d, m_cap);
   tc::GemmArgs a = base_args(c);
-  set_n(a, d, 256);
+  set_n(a, d, wide ? 512 : 256);
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
@@ -255,6 +292,7 @@ moe_status_t gemm_wgrad_gate_up(const GemmCtx& c, const void* dau, const void* x
   set_m(a, 2ll * f, 2 * tc::BM);  // CTA pairs: 256-row tiles
   const int64_t tiles = static_cast<int64_t>(E) * a.m_tiles_fixed * a.n_tiles_n;
   const int grid = static_cast<int>(2 * tiles < c.num_sms ? 2 * tiles : c.num_sms);
+  if (wide) return launch<512, true, true, tc::EPI_BF16, true, false, true>(ta, tb, a, grid, st);
   return launch<256, true, true, tc::EPI_BF16, true, false, true>(ta, tb, a, grid, st);
 }
 

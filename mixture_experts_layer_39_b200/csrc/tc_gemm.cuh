@@ -489,17 +489,20 @@ __device__ __forceinline__ void pack64(const float* f, uint4 (&v)[8]) {
                       pack_bf16x2(f[8 * q + 4], f[8 * q + 5]), pack_bf16x2(f[8 * q + 6], f[8 * q + 7]));
 }
 
-// Asynchronous copy of the warp's 32 rows x 128 bytes at `g` into `buf`
-// (staging layout), zero-filling rows past valid_rows; no registers held.
-// (`safe` is any valid global address, used as the source of zero-size copies.)
-__device__ __forceinline__ void cp_async_rows(uint8_t* buf, const uint8_t* g, int64_t ld_bytes,
-                                              int valid_rows, int lane, const void* safe) {
+// SwiGLU backward: 32 columns of the saved A (slots 0-3 of each staging row)
+// and the same 32 columns of U (slots 4-7) for the warp's 32 rows, copied
+// asynchronously; rows past valid_rows are zero-filled.
+__device__ __forceinline__ void cp_async_au(uint8_t* buf, const uint8_t* ga, const uint8_t* gu,
+                                            int64_t ld_bytes, int valid_rows, int lane,
+                                            const void* safe) {
+  const int q = lane & 7;
+  const uint8_t* g = q < 4 ? ga + (q << 4) : gu + ((q - 4) << 4);
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int row = 4 * j + (lane >> 3);
     const bool ok = row < valid_rows;
-    const uint8_t* src = ok ? g + row * ld_bytes + ((lane & 7) << 4) : static_cast<const uint8_t*>(safe);
-    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(stage_slot(buf, row, lane & 7)));
+    const uint8_t* src = ok ? g + row * ld_bytes : static_cast<const uint8_t*>(safe);
+    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(stage_slot(buf, row, q)));
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
                  "r"(ok ? 16 : 0)
                  : "memory");
@@ -533,9 +536,9 @@ struct SmemPlan {
   static constexpr int kBarBytes = (2 * STAGES + 5) * 8;               // full, empty, tfull x2, tempty x2, drain
   static constexpr int kMiscOff = kBarOff + kBarBytes;                 // tmem base, abort flag
   static constexpr int kEpiOff = (kMiscOff + 16 + 127) / 128 * 128;    // 4 epilogue warps' buffers
-  // per warp: the 4 KB staging buffer, plus (SwiGLU backward) an 8 KB landing
-  // buffer that cp.async fills with the next chunk's saved [A | U] rows
-  static constexpr int kWarpEpiBytes = kEpiBufBytes + (EPI == EPI_SWIGLU_BWD ? 2 * kEpiBufBytes : 0);
+  // per warp: the 4 KB staging buffer, plus (SwiGLU backward) a 4 KB landing
+  // buffer that cp.async fills with the next 32 columns of the saved A and U
+  static constexpr int kWarpEpiBytes = kEpiBufBytes + (EPI == EPI_SWIGLU_BWD ? kEpiBufBytes : 0);
   static constexpr int kTileOff = kEpiOff + 4 * kWarpEpiBytes;         // group tile starts
   static constexpr int bytes(int n_groups) { return 1024 + kTileOff + 4 * (n_groups + 1); }
 };
@@ -552,10 +555,10 @@ template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, int STAGES, bool F
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
-  static_assert(BN == 128 || BN == 256, "BN");
+  static_assert(BN == 128 || BN == 256 || (BN == 512 && PAIR), "BN");
   static_assert(!(EPI == EPI_SWIGLU_FWD && B_MN), "SwiGLU forward takes K-major weights");
   static_assert(!FP8 || BN == 128, "MXFP8 tiles are 128 x 128 (TMEM holds the scales too)");
-  static_assert(!PAIR || (BN == 256 && !FP8), "CTA pairs run bf16 256 x 256 tiles");
+  static_assert(!PAIR || (BN >= 256 && !FP8), "CTA pairs run bf16 256 x 256 or 256 x 512 tiles");
   // GATHER reads routed rows from x: the K-major A of an M-grouped GEMM, or
   // the MN-major B (rows = routed rows) of a K-grouped one
   static_assert(!GATHER || (!FP8 && (KGROUP ? B_MN : !A_MN)), "gathered operand");
@@ -571,8 +574,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int CH = FP8 ? 128 : 64;
   constexpr uint32_t kChunkBytes = BKE * 128;      // one MN chunk of an MN-major stage
   constexpr uint32_t kSfCols = 4 + 4 * (BN / 128); // TMEM columns of one scale buffer
-  constexpr uint32_t kTmemCols = FP8 ? 512 : 2 * BN;
-  constexpr uint32_t kIdesc = FP8 ? idesc_mxf8(BM, BN, A_MN, B_MN) : idesc_bf16(MT, BN, A_MN, B_MN);
+  // Wide pairs (BN = 512): two N = 256 MMAs per K step, each reading 128 of
+  // every CTA's 256 B rows, into one accumulator that fills TMEM (the
+  // epilogue of a tile then does not overlap the next tile's MMAs).
+  constexpr int NMMA = BN > 256 ? 256 : BN;  // N of one MMA instruction
+  constexpr int NACC = BN > 256 ? 1 : 2;     // TMEM accumulators
+  constexpr uint32_t kBHalfBytes = (BNC / 2) * 128;  // B rows of one wide-pair MMA, per CTA
+  constexpr uint32_t kTmemCols = FP8 ? 512 : NACC * BN;
+  constexpr uint32_t kIdesc = FP8 ? idesc_mxf8(BM, BN, A_MN, B_MN) : idesc_bf16(MT, NMMA, A_MN, B_MN);
   // M-grouped bf16 tail tiles of <= 64 rows run M = 64 MMAs: rows 16q..16q+15
   // of the accumulator then sit in TMEM lanes 32q..32q+15
   constexpr bool kTail64 = !FP8 && !KGROUP && !A_MN && !PAIR;
@@ -862,7 +871,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile tl = decode_tile<KGROUP, BKE, KMMA, MT>(args, s_tile_start, t);
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, s_abort, true, PAIR)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);  // acc = 0 when NACC = 1
         for (int kb = 0; kb < tl.k_blocks; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, s_abort, true, PAIR)) { ok = false; break; }
           tc_fence_after();
@@ -893,6 +902,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t sid = static_cast<uint32_t>(kk);
               mma_mxf8(d_tmem, ad, bd, kIdesc | (sid << 4) | (sid << 29), sf_col | (sid << 30),
                        (sf_col + 4) | (sid << 30), (kb > 0 || kk > 0) ? 1u : 0u);
+            } else if constexpr (PAIR && BN > 256) {
+              // B rows [0,128) and [128,256) of each CTA: 16 KB apart in both layouts
+              const uint64_t bd1 = B_MN ? smem_desc_sw128(sb + kBHalfBytes + kk * KMMA * 128, kChunkBytes, 1024)
+                                        : smem_desc_sw128(sb + kBHalfBytes + kk * 32, 16, 1024);
+              mma_bf16_pair(d_tmem, ad, bd, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+              mma_bf16_pair(d_tmem + NMMA, ad, bd1, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
             } else if constexpr (PAIR) {
               mma_bf16_pair(d_tmem, ad, bd, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
             } else {
@@ -905,7 +920,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         if constexpr (PAIR) mma_commit_pair(tfull_bar(acc)); else mma_commit(tfull_bar(acc));
-        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
       }
       if (!ok) report(args.ctl, MOE_ERR_TIMEOUT, 2);
       // all MMAs issued by this thread have finished once the drain barrier flips
@@ -915,9 +930,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ================================================================ epilogue
     const int quarter = warp & 3;  // TMEM lanes this warp may access
+    // TMEM column of tile column c (in B-row order).  Wide pairs: CTA p holds
+    // B rows [256p, 256p+256) and MMA h reads rows [128h, 128h+128) of each
+    // CTA, writing TMEM columns [256h, 256h+256) = (CTA 0's, CTA 1's).
+    auto tcol = [](int c) -> uint32_t {
+      if constexpr (BN > 256) {
+        return static_cast<uint32_t>(((c >> 7) & 1) * 256 + (c >> 8) * 128 + (c & 127));
+      } else {
+        return static_cast<uint32_t>(c);
+      }
+    };
     uint8_t* ebuf = smem + Plan::kEpiOff + (warp - 2) * Plan::kWarpEpiBytes;
-    uint8_t* lbuf_a = ebuf + kEpiBufBytes;       // SwiGLU backward: landing buffer for A
-    uint8_t* lbuf_u = ebuf + 2 * kEpiBufBytes;   // ... and for U
+    uint8_t* lbuf = ebuf + kEpiBufBytes;  // SwiGLU backward: landing buffer for [A | U]
     int acc = 0;
     uint32_t acc_phase = 0;
     // rows of this warp's quarter in the tile, and the row prefetch of a tile's
@@ -943,16 +967,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Tile tl = decode_tile<KGROUP, BKE, KMMA, MT>(args, s_tile_start, t);
       const int vrows = quarter_rows(tl);
       const int64_t row_first = quarter_first(tl);  // warp's first row
-      // SwiGLU backward: the saved [A | U] rows of the first 64 columns are
+      // SwiGLU backward: the saved A and U of the first 32 columns are
       // requested before waiting for the accumulator, so their latency
-      // overlaps the main loop; each later chunk is requested one chunk ahead.
+      // overlaps the main loop; each later 32 columns are requested while the
+      // previous ones are computed.
       const __nv_bfloat16* aux = nullptr;
       if constexpr (EPI == EPI_SWIGLU_BWD) {
         aux = args.aux + row_first * args.ld_aux + static_cast<int64_t>(tl.n_tile) * BN;
-        cp_async_rows(lbuf_a, reinterpret_cast<const uint8_t*>(aux), args.ld_aux * 2, vrows, lane,
-                      args.aux);
-        cp_async_rows(lbuf_u, reinterpret_cast<const uint8_t*>(aux + args.f), args.ld_aux * 2, vrows,
-                      lane, args.aux);
+        cp_async_au(lbuf, reinterpret_cast<const uint8_t*>(aux),
+                    reinterpret_cast<const uint8_t*>(aux + args.f), args.ld_aux * 2, vrows, lane,
+                    args.aux);
         cp_async_commit();
       }
       const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull_bar(acc), acc_phase, s_abort, true, PAIR));
@@ -976,8 +1000,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < ncols; c += 64) {
           uint32_t r0[32], r1[32];
-          tmem_ld32(tbase + c, r0);
-          tmem_ld32(tbase + c + 32, r1);
+          tmem_ld32(tbase + tcol(c), r0);
+          tmem_ld32(tbase + tcol(c + 32), r1);
           tmem_ld_wait();
           float f[64];
 #pragma unroll
@@ -995,7 +1019,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < ncols; c += 32) {
           uint32_t r[32];
-          tmem_ld32(tbase + c, r);
+          tmem_ld32(tbase + tcol(c), r);
           tmem_ld_wait();
           uint4 v[8];
 #pragma unroll
@@ -1017,8 +1041,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             uint32_t g[32], u[32];
-            tmem_ld32(tbase + c + 32 * half, g);
-            tmem_ld32(tbase + BNH + c + 32 * half, u);
+            tmem_ld32(tbase + tcol(c + 32 * half), g);
+            tmem_ld32(tbase + tcol(BNH + c + 32 * half), u);
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -1049,28 +1073,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     static_cast<int64_t>(tl.n_tile) * BN;
 #pragma unroll 1
         for (int c = 0; c < ncols; c += 64) {
-          uint4 va[8], vu[8];
-          cp_async_wait_all();
-          __syncwarp();
-          stage_read_row(lbuf_a, lane, va);
-          stage_read_row(lbuf_u, lane, vu);
-          __syncwarp();
-          if (c + 64 < ncols) {  // next chunk lands while this one is computed and stored
-            cp_async_rows(lbuf_a, reinterpret_cast<const uint8_t*>(aux + c + 64), args.ld_aux * 2,
-                          vrows, lane, args.aux);
-            cp_async_rows(lbuf_u, reinterpret_cast<const uint8_t*>(aux + args.f + c + 64),
-                          args.ld_aux * 2, vrows, lane, args.aux);
-            cp_async_commit();
-          }
           uint4 ou[8];  // dU in registers; dA goes straight to the staging buffer
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
+            const int cc = c + 32 * half;
+            uint4 vau[8];  // this lane's row: A in slots 0-3, U in slots 4-7
+            cp_async_wait_all();
+            __syncwarp();
+            stage_read_row(lbuf, lane, vau);
+            __syncwarp();
+            if (cc + 32 < ncols) {  // the next 32 columns land while these are computed
+              cp_async_au(lbuf, reinterpret_cast<const uint8_t*>(aux + cc + 32),
+                          reinterpret_cast<const uint8_t*>(aux + args.f + cc + 32),
+                          args.ld_aux * 2, vrows, lane, args.aux);
+              cp_async_commit();
+            }
             uint32_t r[32];
-            tmem_ld32(tbase + c + 32 * half, r);
+            tmem_ld32(tbase + tcol(cc), r);
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const uint4 qa = va[4 * half + q], qu = vu[4 * half + q];
+              const uint4 qa = vau[q], qu = vau[4 + q];
               const float a[8] = {bf16_lo(qa.x), bf16_hi(qa.x), bf16_lo(qa.y), bf16_hi(qa.y),
                                   bf16_lo(qa.z), bf16_hi(qa.z), bf16_lo(qa.w), bf16_hi(qa.w)};
               const float u[8] = {bf16_lo(qu.x), bf16_hi(qu.x), bf16_lo(qu.y), bf16_hi(qu.y),
@@ -1102,7 +1125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (PAIR && rank != 0) mbar_arrive_remote(mapa_shared(tempty_bar(acc), 0));
         else mbar_arrive(tempty_bar(acc));
       }
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
     }
   }
 
