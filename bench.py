@@ -9,9 +9,11 @@ experts on one GPU and has no exchange step): every rank runs the same
 workload on its own tokens, the timing is the max over ranks and `value`
 is the tokens of all ranks over that time (weak scaling).
 
-Timed region: W untimed warm-up steps, then exactly K steps, each bracketed
-by CUDA events on the stream the library launches on; between steps (and
-outside the events) a 512 MiB buffer is written to flush the 126 MB L2.
+Timed region: W untimed warm-up steps (eager), then exactly K steps, each
+one replay of a CUDA graph captured from the step's library calls and
+bracketed by CUDA events on the stream the library launches on; between
+steps (and outside the events) a 512 MiB buffer is written to flush the
+126 MB L2.
 Rank 0 prints one JSON line.
 """
 from __future__ import annotations
@@ -192,12 +194,17 @@ def gemm_traffic(cfg_name):
 
 
 def measure(L, g, steps, warmup, flush, dev, with_gemm_events=True):
+    """Times `steps` steps of the layer.  After `warmup` eager steps the step
+    (every library call of MoELayer.forward/.backward, in order) is captured
+    once as a CUDA graph and replayed: the library launches on the caller's
+    stream and allocates nothing, so the captured graph holds exactly the
+    step's kernels.  Events around the expert GEMMs are captured as external
+    event nodes; the step events are recorded on the stream around each
+    replay, and the L2 flush runs between steps outside them."""
     import torch
-    stream = torch.cuda.current_stream()
 
     def one_step(ev=None):
-        # MoELayer.forward / .backward call by call, with events around the
-        # expert GEMMs (the shared expert's included)
+        stream = torch.cuda.current_stream()
         L.router(g["x"], g["w_r"], g["bias"], g["route"])
         L.permute(g["x"])
         if L.aux_alpha > 0:
@@ -222,20 +229,33 @@ def measure(L, g, steps, warmup, flush, dev, with_gemm_events=True):
         flush.fill_(1)
         one_step()
     torch.cuda.synchronize(dev)
+    gev = ([torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+           if with_gemm_events else None)
+    graph = torch.cuda.CUDAGraph()
     n0 = L.handle.launch_count()
+    with torch.cuda.graph(graph):
+        one_step(gev)
+    per_step = L.handle.launch_count() - n0  # kernels in the graph
+    stream = torch.cuda.current_stream()
+    for _ in range(2):  # first replays upload the graph
+        flush.fill_(1)
+        graph.replay()
+    torch.cuda.synchronize(dev)
     mk = lambda: torch.cuda.Event(enable_timing=True)
     step_ev = [(mk(), mk()) for _ in range(steps)]
-    gemm_ev = [[mk() for _ in range(4)] for _ in range(steps)] if with_gemm_events else None
+    gemm_ms = [] if gev else None
     for i in range(steps):
         flush.fill_(i & 0xFF)
         step_ev[i][0].record(stream)
-        one_step(gemm_ev[i] if gemm_ev else None)
+        graph.replay()
         step_ev[i][1].record(stream)
+        if gev:  # the graph's events are re-recorded by the next replay
+            step_ev[i][1].synchronize()
+            gemm_ms.append(gev[0].elapsed_time(gev[1]) + gev[2].elapsed_time(gev[3]))
     torch.cuda.synchronize(dev)
-    launches = L.handle.launch_count() - n0
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    gemm_ms = [e[0].elapsed_time(e[1]) + e[2].elapsed_time(e[3]) for e in gemm_ev] if gemm_ev else None
-    return step_ms, gemm_ms, launches
+    del graph
+    return step_ms, gemm_ms, per_step * steps
 
 
 def measure_e2e(L, g, steps, warmup, dev):
