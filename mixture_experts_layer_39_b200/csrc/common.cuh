@@ -26,6 +26,33 @@ __device__ __forceinline__ void report(DeviceCtl* ctl, int code, int detail) {
   if (atomicCAS(&ctl->status, 0, code) == 0) atomicExch(&ctl->detail, detail);
 }
 
+// Programmatic dependent launch.  Every kernel of the library is launched
+// with launch_pdl, so it may be scheduled while the previous kernel in the
+// stream is still finishing.  pdl_wait() returns once that kernel has
+// completed and its writes are visible; each kernel calls it before its
+// first global memory access (no-op when launched without the attribute),
+// then pdl_trigger() lets the next kernel in the stream be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));

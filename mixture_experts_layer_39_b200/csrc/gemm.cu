@@ -88,17 +88,20 @@ moe_status_t launch_stages(const CUtensorMap& a, const CUtensorMap& b, const tc:
     cfg.blockDim = dim3(tc::kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, a, b, args) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   } else {
-    kern<<<grid, tc::kThreads, smem, st>>>(a, b, args);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_pdl(kern, dim3(grid), dim3(tc::kThreads), smem, st, a, b, args) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
   }
 }
 

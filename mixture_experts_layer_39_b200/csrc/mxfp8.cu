@@ -35,6 +35,8 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
 // axis 1: one thread per 32-element block of a row.
 __global__ void mx_rowwise_kernel(const uint4* __restrict__ in, int64_t rows, int64_t cols,
                                   uint4* __restrict__ q, uint8_t* __restrict__ scales) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t nblk = cols / 32;
   const int64_t total = rows * nblk;
   for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < total;
@@ -75,6 +77,8 @@ __global__ void mx_rowwise_kernel(const uint4* __restrict__ in, int64_t rows, in
 __global__ void mx_colwise_kernel(const uint32_t* __restrict__ in, int64_t rows, int64_t cols,
                                   uint16_t* __restrict__ q, uint8_t* __restrict__ scales,
                                   int scale_mode, int64_t rows_per_group) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t cpairs = cols / 2;
   const int64_t total = (rows / 32) * cpairs;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
@@ -117,12 +121,12 @@ cudaError_t launch_mxfp8_quantize(const __nv_bfloat16* in, int64_t rows, int64_t
   if (axis == 1) {
     const int64_t total = rows * (cols / 32);
     const unsigned grid = static_cast<unsigned>(ceil_div64(total, 256) < 65535 ? ceil_div64(total, 256) : 65535);
-    mx_rowwise_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(in), rows, cols,
+    (void)launch_pdl(mx_rowwise_kernel, grid, 256, 0, st, reinterpret_cast<const uint4*>(in), rows, cols,
                                             reinterpret_cast<uint4*>(q), scales);
   } else {
     const int64_t total = (rows / 32) * (cols / 2);
     const unsigned grid = static_cast<unsigned>(ceil_div64(total, 256) < 65535 ? ceil_div64(total, 256) : 65535);
-    mx_colwise_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(in), rows, cols,
+    (void)launch_pdl(mx_colwise_kernel, grid, 256, 0, st, reinterpret_cast<const uint32_t*>(in), rows, cols,
                                             reinterpret_cast<uint16_t*>(q), scales, 0, rows);
   }
   return cudaGetLastError();
@@ -133,7 +137,7 @@ cudaError_t launch_mxfp8_quantize_cols_t(const __nv_bfloat16* in, int64_t rows, 
                                          cudaStream_t st) {
   const int64_t total = (rows / 32) * (cols / 2);
   const unsigned grid = static_cast<unsigned>(ceil_div64(total, 256) < 65535 ? ceil_div64(total, 256) : 65535);
-  mx_colwise_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(in), rows, cols,
+  (void)launch_pdl(mx_colwise_kernel, grid, 256, 0, st, reinterpret_cast<const uint32_t*>(in), rows, cols,
                                           reinterpret_cast<uint16_t*>(q), scales, 1, rows_per_group);
   return cudaGetLastError();
 }

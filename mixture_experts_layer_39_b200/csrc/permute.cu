@@ -32,6 +32,8 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 __global__ void __launch_bounds__(kWarps * 32)
     route_hist_kernel(const int32_t* __restrict__ idx, int64_t n_entries, int E, int64_t n_sub,
                       int32_t* __restrict__ sub_counts, DeviceCtl* ctl) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int s_cnt[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* cnt = s_cnt + warp * E;
@@ -57,6 +59,8 @@ __global__ void __launch_bounds__(kWarps * 32)
 __global__ void __launch_bounds__(1024)
     route_scan_kernel(int32_t* __restrict__ sub, int64_t n_sub, int E, int align,
                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int s_tot[1024];
   __shared__ int s_warp[32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -123,6 +127,8 @@ __global__ void __launch_bounds__(kWarps * 32)
     route_rank_kernel(const int32_t* __restrict__ idx, int64_t n_entries, int E, int64_t n_sub,
                       const int32_t* __restrict__ sub_base, const int32_t* __restrict__ offsets,
                       int32_t* __restrict__ row_map) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int s_base_all[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* base = s_base_all + warp * E;
@@ -159,6 +165,8 @@ __global__ void __launch_bounds__(256)
     route_src_kernel(const int32_t* __restrict__ row_map, const int32_t* __restrict__ offsets,
                      const int32_t* __restrict__ counts, int T, int k, int E, int64_t m_cap,
                      int32_t oob, int32_t* __restrict__ row_src) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t tk = static_cast<int64_t>(T) * k;
   if (i < tk) {
@@ -185,6 +193,8 @@ __global__ void __launch_bounds__(kWarps * 32)
     permute_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ row_map,
                            const int32_t* __restrict__ offsets, const int32_t* __restrict__ counts,
                            int T, int nvec, int k, int E, uint4* __restrict__ x_perm) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
   if (gw < T) {
@@ -223,6 +233,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     combine_kernel(const uint4* __restrict__ o, const int32_t* __restrict__ row_map,
                    const float* __restrict__ w, const uint4* __restrict__ shared, int T, int nvec,
                    int k, uint4* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -274,6 +286,8 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
                        const int32_t* __restrict__ offsets, const int32_t* __restrict__ counts,
                        int T, int nvec, int k, int E, uint4* __restrict__ dO,
                        float* __restrict__ dw) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
   if (gw < T) {
@@ -329,6 +343,8 @@ __global__ void __launch_bounds__(kWarps * 32)
     permute_bwd_kernel(const uint4* __restrict__ dxp, const int32_t* __restrict__ row_map,
                        const float4* __restrict__ dxr, const uint4* __restrict__ dxs, int T,
                        int nvec, int k, uint4* __restrict__ dx) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -373,14 +389,14 @@ cudaError_t launch_route_hist(const int32_t* idx, int T, int k, int E, int32_t* 
                               DeviceCtl* ctl, cudaStream_t st) {
   const int64_t n_sub = n_subchunks(T, k);
   const unsigned grid = static_cast<unsigned>(ceil_div64(n_sub, kWarps));
-  route_hist_kernel<<<grid, kWarps * 32, kWarps * E * sizeof(int), st>>>(
+  (void)launch_pdl(route_hist_kernel, grid, kWarps * 32, kWarps * E * sizeof(int), st,
       idx, static_cast<int64_t>(T) * k, E, n_sub, sub_counts, ctl);
   return cudaGetLastError();
 }
 
 cudaError_t launch_route_scan(int32_t* sub_counts, int64_t n_sub, int E, int align, int32_t* counts,
                               int32_t* offsets, cudaStream_t st) {
-  route_scan_kernel<<<1, 1024, 0, st>>>(sub_counts, n_sub, E, align, counts, offsets);
+  (void)launch_pdl(route_scan_kernel, 1, 1024, 0, st, sub_counts, n_sub, E, align, counts, offsets);
   return cudaGetLastError();
 }
 
@@ -388,7 +404,7 @@ cudaError_t launch_route_rank(const int32_t* idx, int T, int k, int E, const int
                               const int32_t* offsets, int32_t* row_map, cudaStream_t st) {
   const int64_t n_sub = n_subchunks(T, k);
   const unsigned grid = static_cast<unsigned>(ceil_div64(n_sub, kWarps));
-  route_rank_kernel<<<grid, kWarps * 32, kWarps * E * sizeof(int), st>>>(
+  (void)launch_pdl(route_rank_kernel, grid, kWarps * 32, kWarps * E * sizeof(int), st,
       idx, static_cast<int64_t>(T) * k, E, n_sub, sub_base, offsets, row_map);
   return cudaGetLastError();
 }
@@ -397,7 +413,7 @@ cudaError_t launch_route_src(const int32_t* row_map, const int32_t* offsets, con
                              int T, int k, int E, int64_t m_cap, int32_t* row_src,
                              cudaStream_t st) {
   const int64_t n = static_cast<int64_t>(T) * k + m_cap;
-  route_src_kernel<<<static_cast<unsigned>(ceil_div64(n, 256)), 256, 0, st>>>(
+  (void)launch_pdl(route_src_kernel, static_cast<unsigned>(ceil_div64(n, 256)), 256, 0, st,
       row_map, offsets, counts, T, k, E, m_cap, T, row_src);
   return cudaGetLastError();
 }
@@ -406,7 +422,7 @@ cudaError_t launch_permute_scatter(const __nv_bfloat16* x, const int32_t* row_ma
                                    const int32_t* offsets, const int32_t* counts, int T, int d,
                                    int k, int E, __nv_bfloat16* x_perm, cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>(ceil_div64(static_cast<int64_t>(T) + E, kWarps));
-  permute_scatter_kernel<<<grid, kWarps * 32, 0, st>>>(
+  (void)launch_pdl(permute_scatter_kernel, grid, kWarps * 32, 0, st,
       reinterpret_cast<const uint4*>(x), row_map, offsets, counts, T, d / 8, k, E,
       reinterpret_cast<uint4*>(x_perm));
   return cudaGetLastError();
@@ -417,7 +433,7 @@ cudaError_t launch_combine(const __nv_bfloat16* o_perm, const int32_t* row_map, 
                            cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>(ceil_div64(T, kWarps));
   auto kern = shared != nullptr ? combine_kernel<true> : combine_kernel<false>;
-  kern<<<grid, kWarps * 32, 0, st>>>(reinterpret_cast<const uint4*>(o_perm), row_map, w,
+  (void)launch_pdl(kern, grid, kWarps * 32, 0, st, reinterpret_cast<const uint4*>(o_perm), row_map, w,
                                      reinterpret_cast<const uint4*>(shared), T, d / 8, k,
                                      reinterpret_cast<uint4*>(y));
   return cudaGetLastError();
@@ -428,7 +444,7 @@ cudaError_t launch_combine_bwd(const __nv_bfloat16* dy, const __nv_bfloat16* o_p
                                const int32_t* counts, int T, int d, int k, int E,
                                __nv_bfloat16* do_perm, float* dw, cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>(ceil_div64(static_cast<int64_t>(T) + E, kWarps));
-  combine_bwd_kernel<<<grid, kWarps * 32, 0, st>>>(
+  (void)launch_pdl(combine_bwd_kernel, grid, kWarps * 32, 0, st,
       reinterpret_cast<const uint4*>(dy), reinterpret_cast<const uint4*>(o_perm), row_map, w,
       offsets, counts, T, d / 8, k, E, reinterpret_cast<uint4*>(do_perm), dw);
   return cudaGetLastError();
@@ -439,7 +455,7 @@ cudaError_t launch_permute_bwd(const __nv_bfloat16* dx_perm, const int32_t* row_
                                int k, __nv_bfloat16* dx, cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>(ceil_div64(T, kWarps));
   auto kern = dx_shared != nullptr ? permute_bwd_kernel<true> : permute_bwd_kernel<false>;
-  kern<<<grid, kWarps * 32, 0, st>>>(
+  (void)launch_pdl(kern, grid, kWarps * 32, 0, st,
       reinterpret_cast<const uint4*>(dx_perm), row_map, reinterpret_cast<const float4*>(dx_router),
       reinterpret_cast<const uint4*>(dx_shared), T, d / 8, k, reinterpret_cast<uint4*>(dx));
   return cudaGetLastError();

@@ -49,6 +49,8 @@ __global__ void __launch_bounds__(kWarps * 32)
                         int T, int d, int E, int k, int renorm, int32_t* __restrict__ idx_out,
                         float* __restrict__ w_out, float* __restrict__ probs,
                         float* __restrict__ logits, DeviceCtl* ctl) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float4 s_wf[];  // [E][d] fp32 when W_SMEM
   const int lane = threadIdx.x & 31;
   const int nvec = d >> 3;
@@ -240,6 +242,8 @@ __global__ void __launch_bounds__(kMmaWarps * 32, NT == 1 ? 7 : 5)
                       int d, int E, int k, int renorm, int32_t* __restrict__ idx_out,
                       float* __restrict__ w_out, float* __restrict__ probs,
                       float* __restrict__ logits, DeviceCtl* ctl) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float4 s_part[kMmaWarps][NT][32];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -402,6 +406,8 @@ __global__ void __launch_bounds__(kWarps * 32)
                         int32_t* __restrict__ idx_out, float* __restrict__ w_out,
                         float* __restrict__ probs, float* __restrict__ logits_out,
                         DeviceCtl* ctl) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -505,11 +511,11 @@ cudaError_t launch_router_fused(const __nv_bfloat16* x, const __nv_bfloat16* w_r
                                static_cast<int>(w_smem)) != cudaSuccess)
         return cudaErrorInvalidValue;
       const unsigned grid = static_cast<unsigned>(want < 2 * sms ? want : 2 * sms);
-      kern_smem<<<grid, kWarps * 32, w_smem, st>>>(x, w_r, bias, route_in, T, d, E, k,
+      (void)launch_pdl(kern_smem, grid, kWarps * 32, w_smem, st, x, w_r, bias, route_in, T, d, E, k,
                                                    renorm ? 1 : 0, idx, w, probs, logits, ctl);
     } else {
       const unsigned grid = static_cast<unsigned>(want < 8 * sms ? want : 8 * sms);
-      kern_l1<<<grid, kWarps * 32, 0, st>>>(x, w_r, bias, route_in, T, d, E, k, renorm ? 1 : 0,
+      (void)launch_pdl(kern_l1, grid, kWarps * 32, 0, st, x, w_r, bias, route_in, T, d, E, k, renorm ? 1 : 0,
                                             idx, w, probs, logits, ctl);
     }
     return cudaGetLastError();
@@ -517,10 +523,10 @@ cudaError_t launch_router_fused(const __nv_bfloat16* x, const __nv_bfloat16* w_r
   if (E <= 16) {
     const unsigned grid = static_cast<unsigned>(ceil_div64(T, kMmaTokens));
     if (E <= 8)
-      router_mma_kernel<1><<<grid, kMmaWarps * 32, 0, st>>>(x, w_r, bias, route_in, T, d, E, k,
+      (void)launch_pdl(router_mma_kernel<1>, grid, kMmaWarps * 32, 0, st, x, w_r, bias, route_in, T, d, E, k,
                                                             renorm ? 1 : 0, idx, w, probs, logits, ctl);
     else
-      router_mma_kernel<2><<<grid, kMmaWarps * 32, 0, st>>>(x, w_r, bias, route_in, T, d, E, k,
+      (void)launch_pdl(router_mma_kernel<2>, grid, kMmaWarps * 32, 0, st, x, w_r, bias, route_in, T, d, E, k,
                                                             renorm ? 1 : 0, idx, w, probs, logits, ctl);
     return cudaGetLastError();
   }
@@ -535,7 +541,7 @@ cudaError_t launch_softmax_topk(const float* logits_in, int ld_in, const float* 
                                 DeviceCtl* ctl, cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>(ceil_div64(T, kWarps));
   auto go = [&](auto kern) {
-    kern<<<grid, kWarps * 32, 0, st>>>(logits_in, ld_in, bias, route_in, T, E, k, renorm ? 1 : 0, idx, w,
+    (void)launch_pdl(kern, grid, kWarps * 32, 0, st, logits_in, ld_in, bias, route_in, T, E, k, renorm ? 1 : 0, idx, w,
                                        probs, logits_out, ctl);
     return cudaGetLastError();
   };

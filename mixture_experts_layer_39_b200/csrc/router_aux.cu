@@ -26,6 +26,8 @@ template <int NPL>
 __global__ void __launch_bounds__(kStatWarps * 32)
     router_stats_partial_kernel(const float* __restrict__ probs, int T, int E, int chunk,
                                 float* __restrict__ partial) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float s_sum[kStatWarps][32 * NPL];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * chunk;
@@ -57,6 +59,8 @@ __global__ void __launch_bounds__(kStatWarps * 32)
     router_stats_final_kernel(const float* __restrict__ partial, int n_part,
                               const int32_t* __restrict__ counts, int E, int accumulate,
                               float* __restrict__ stats) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int e = blockIdx.x * kStatWarps + (threadIdx.x >> 5);
   if (e >= E) return;
@@ -77,6 +81,8 @@ constexpr int kAuxThreads = 1024;
 __global__ void __launch_bounds__(kAuxThreads)
     router_aux_loss_kernel(const float* __restrict__ stats, int E, int k, float n_tokens,
                            float alpha, float* __restrict__ loss, float* __restrict__ dprob) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float s_prod[kAuxThreads];
   const float slots = n_tokens * static_cast<float>(k);
   for (int e = threadIdx.x; e < E; e += kAuxThreads) {
@@ -106,7 +112,7 @@ cudaError_t launch_router_load_stats(const float* probs, const int32_t* counts, 
                                      cudaStream_t st) {
   const int chunk = static_cast<int>(ceil_div64(T, n_blocks));
   auto go = [&](auto kern) {
-    kern<<<static_cast<unsigned>(n_blocks), kStatWarps * 32, 0, st>>>(probs, T, E, chunk, partial);
+    (void)launch_pdl(kern, static_cast<unsigned>(n_blocks), kStatWarps * 32, 0, st, probs, T, E, chunk, partial);
     return cudaGetLastError();
   };
   cudaError_t e;
@@ -118,15 +124,14 @@ cudaError_t launch_router_load_stats(const float* probs, const int32_t* counts, 
   else if (E <= 1024) e = go(router_stats_partial_kernel<32>);
   else return cudaErrorInvalidValue;
   if (e != cudaSuccess) return e;
-  router_stats_final_kernel<<<static_cast<unsigned>(ceil_div64(E, kStatWarps)), kStatWarps * 32,
-                              0, st>>>(partial, n_blocks, counts, E, accumulate ? 1 : 0, stats);
+  (void)launch_pdl(router_stats_final_kernel, static_cast<unsigned>(ceil_div64(E, kStatWarps)), kStatWarps * 32, 0, st, partial, n_blocks, counts, E, accumulate ? 1 : 0, stats);
   return cudaGetLastError();
 }
 
 cudaError_t launch_router_aux_loss(const float* stats, int E, int k, float n_tokens, float alpha,
                                    float* loss, float* dprob, cudaStream_t st) {
   if (E > kAuxThreads) return cudaErrorInvalidValue;
-  router_aux_loss_kernel<<<1, kAuxThreads, 0, st>>>(stats, E, k, n_tokens, alpha, loss, dprob);
+  (void)launch_pdl(router_aux_loss_kernel, 1, kAuxThreads, 0, st, stats, E, k, n_tokens, alpha, loss, dprob);
   return cudaGetLastError();
 }
 

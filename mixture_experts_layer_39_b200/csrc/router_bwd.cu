@@ -101,6 +101,8 @@ __global__ void __launch_bounds__(kWarps * 32)
                          __nv_bfloat16* __restrict__ dl_bf16, int ld_bf16,
                          float* __restrict__ dx_router,
                          float* __restrict__ db_partial, int stage_w) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float s_db[kWarps][32 * NPL];
   extern __shared__ uint4 s_wdyn[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -176,6 +178,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
                               const __nv_bfloat16* __restrict__ w_r,
                               const uint4* __restrict__ dxs, int T, int d, int E, int k,
                               int renorm, uint4* __restrict__ dx) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int NPL = (NE + 31) / 32;
   const int lane = threadIdx.x & 31;
   const int64_t t0 = (static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5)) * TPW;
@@ -258,6 +262,8 @@ template <int NE>
 __global__ void __launch_bounds__(kDwThreads)
     router_dw_kernel(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ x, int T,
                      int d, int E, int group_len, float* __restrict__ partial) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) uint8_t s_raw[];
   uint8_t* s_x = s_raw;                                              // [2][kDwTok][kDwCols] bf16
   float* s_dl = reinterpret_cast<float*>(s_raw + 2 * kDwStageX);      // [2][kDwTok][NE]
@@ -343,6 +349,8 @@ __global__ void __launch_bounds__(kRedWarps * 32)
     reduce_dw_kernel(const float4* __restrict__ partial, int n_part, int64_t stride4, int64_t n4_w,
                      const float* __restrict__ db_part, int n_db, int E,
                      __nv_bfloat16* __restrict__ dw_out, float* __restrict__ db_out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float4 s_part[kRedWarps][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t i = static_cast<int64_t>(blockIdx.x) * 32 + lane;
@@ -392,7 +400,7 @@ cudaError_t launch_permute_router_bwd(const __nv_bfloat16* dx_perm, const int32_
                                       bool renorm, __nv_bfloat16* dx, cudaStream_t st) {
   auto go = [&](auto kern, int tpw) {
     const unsigned grid = static_cast<unsigned>(ceil_div64(T, static_cast<int64_t>(kWarps) * tpw));
-    kern<<<grid, kWarps * 32, 0, st>>>(reinterpret_cast<const uint4*>(dx_perm), row_map, dw, probs,
+    (void)launch_pdl(kern, grid, kWarps * 32, 0, st, reinterpret_cast<const uint4*>(dx_perm), row_map, dw, probs,
                                        idx, dprob_aux, w_r,
                                        reinterpret_cast<const uint4*>(dx_shared), T, d, E, k,
                                        renorm ? 1 : 0,
@@ -433,7 +441,7 @@ cudaError_t launch_router_bwd_dl(const float* dw, const float* probs, const int3
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return cudaErrorInvalidValue;
-    kern<<<nblocks, kWarps * 32, smem, st>>>(dw, probs, idx, dprob_aux, w_r, T, d, E, k,
+    (void)launch_pdl(kern, nblocks, kWarps * 32, smem, st, dw, probs, idx, dprob_aux, w_r, T, d, E, k,
                                              renorm ? 1 : 0,
                                              dl_f32, dl_bf16, ld_bf16, dx_router, db_partial,
                                              stage ? 1 : 0);
@@ -480,7 +488,7 @@ cudaError_t launch_router_dw(const float* dl, const __nv_bfloat16* x, int T, int
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return cudaErrorInvalidValue;
     const unsigned gx = static_cast<unsigned>(ceil_div64(d, kDwCols));
-    kern<<<dim3(gx, static_cast<unsigned>(n_chunks)), kDwThreads, smem, st>>>(dl, x, T, d, E,
+    (void)launch_pdl(kern, dim3(gx, static_cast<unsigned>(n_chunks)), kDwThreads, smem, st, dl, x, T, d, E,
                                                                               group_len, partial);
     return cudaGetLastError();
   };
@@ -496,7 +504,7 @@ cudaError_t launch_reduce_dw(const float* partial, int n_part, int64_t n_w, cons
                              cudaStream_t st) {
   // n_w = E * d is a multiple of 4 (d is a multiple of 128)
   const int64_t n4 = n_w / 4 + (db_out != nullptr ? (E + 3) / 4 : 0);
-  reduce_dw_kernel<<<static_cast<unsigned>(ceil_div64(n4, 32)), kRedWarps * 32, 0, st>>>(
+  (void)launch_pdl(reduce_dw_kernel, static_cast<unsigned>(ceil_div64(n4, 32)), kRedWarps * 32, 0, st,
       reinterpret_cast<const float4*>(partial), n_part, n_w / 4, n_w / 4, db_part, n_db, E, dw_out,
       db_out);
   return cudaGetLastError();

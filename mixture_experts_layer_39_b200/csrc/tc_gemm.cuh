@@ -642,6 +642,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
   }
+  // everything above touched only shared memory, TMEM and kernel parameters;
+  // the previous kernel's outputs (offsets, operands) are read from here on
+  pdl_wait();
+  pdl_trigger();
   int total_tiles;
   if constexpr (!KGROUP) {
     // tiles per group, then an exclusive scan by warp 2
