@@ -609,7 +609,8 @@ moe_status_t moe_router_topk_bwd(moe_handle_t h, const moe_shape_t* s, const flo
                                                   E, k, renorm, want_dx, dl, nullptr, 0, dx_router,
                                                   db_part,
                                                   L.nblocks, h->ctl, st)));
-    MOE_TRY(cuda_status(moe::launch_router_dw(dl, xb, T, d, E, L.n_part, L.group_len, part, st)));
+    MOE_TRY(cuda_status(
+        moe::launch_router_dw(dl, xb, T, d, E, L.n_part, L.group_len, part, h->ctl, st)));
     return cuda_status(moe::launch_reduce_dw(part, L.n_part, static_cast<int64_t>(E) * d, db_part,
                                              L.nblocks, E, static_cast<__nv_bfloat16*>(dw_router),
                                              dbias, st));

@@ -74,11 +74,13 @@ cudaError_t launch_router_bwd_dl(const float* dw, const float* probs, const int3
                                  bool fuse_dx, float* dl_f32, __nv_bfloat16* dl_bf16,
                                  int ld_bf16, float* dx_router, float* db_partial, int nblocks,
                                  DeviceCtl* ctl, cudaStream_t st);
-// dW_r partial rows [n_chunks][E*d] over token chunks (E <= 64);
+// dW_r partial rows [n_chunks][E*d] over token chunks (E <= 64; E <= 16 streamed
+// with bulk copies, the dL buffer padded to a multiple of 256 bytes);
 // router_dw_chunks picks the chunking.
 int router_dw_chunks(int num_sms, int T, int d, int E, int* group_len);
 cudaError_t launch_router_dw(const float* dl, const __nv_bfloat16* x, int T, int d, int E,
-                             int n_chunks, int group_len, float* partial, cudaStream_t st);
+                             int n_chunks, int group_len, float* partial, DeviceCtl* ctl,
+                             cudaStream_t st);
 // dw_out = bf16(sum of the n_part partial rows of n_w floats); when db_out
 // is given also db_out = sum of the n_db rows of E floats in db_part.
 cudaError_t launch_reduce_dw(const float* partial, int n_part, int64_t n_w, const float* db_part,

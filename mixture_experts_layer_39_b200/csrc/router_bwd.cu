@@ -333,6 +333,217 @@ __global__ void __launch_bounds__(kDwThreads)
       *reinterpret_cast<float2*>(out + static_cast<int64_t>(e) * d) = make_float2(acc[e][0], acc[e][1]);
 }
 
+// dW_r partial sums for E <= 16 on the tensor cores.  dW_r^T[col][e] =
+// sum_t x[t][col] dL[t][e] is a product with M = columns, K = tokens and
+// N = experts: bf16 mma.sync m16n8k16, x^T fragments loaded from shared
+// memory with ldmatrix.trans, fp32 accumulation.  x is exact in bf16; dL is
+// split into bf16 hi + lo parts (two MMAs), which keeps about 16 of its 24
+// mantissa bits.  A block owns kDsCols (or d) columns and a chunk of tokens;
+// a 3-deep ring of stages, each the chunk's next kDsTok rows of x (one
+// cp.async.bulk per row, rows padded by 16 bytes so that ldmatrix is free of
+// bank conflicts) and their dL rows, is filled by thread 0 and completes on
+// an mbarrier per stage.  Warp w owns columns [256w, 256w + 256); tokens are
+// accumulated in increasing order, so the result does not depend on timing.
+constexpr int kDsThreads = 256;
+constexpr int kDsCols = 2048;
+constexpr int kDsTok = 16;  // tokens per stage = one MMA K step
+constexpr int kDsStages = 3;
+constexpr int kDsRow = kDsCols * 2 + 16;            // padded smem row, bytes
+constexpr int kDsStageX = kDsTok * kDsRow;          // 65792 bytes
+constexpr int kDsStageDl = kDsTok * 16 * 4;         // dL rows of up to 16 experts
+constexpr size_t kDsSmem = kDsStages * (kDsStageX + kDsStageDl) + kDsStages * 8;
+
+__device__ __forceinline__ void ds_mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void ds_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+// global -> shared bulk copy completing on `bar` (16-byte aligned, size a multiple of 16)
+__device__ __forceinline__ void ds_bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// bounded wait on a phase of `bar`; false after kDsWaitNs
+constexpr uint64_t kDsWaitNs = 2000000000ull;
+__device__ __forceinline__ bool ds_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok = 0;
+  uint64_t t0 = 0;
+  for (int i = 0;; ++i) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if (i == 0) t0 = globaltimer_ns();
+    else if (globaltimer_ns() - t0 > kDsWaitNs) return false;
+  }
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// bf16 hi part of v, and the bf16 of what is left
+__device__ __forceinline__ void split_bf16(float v, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(v);
+  lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+}
+
+template <int NE>
+__global__ void __launch_bounds__(kDsThreads, 1)
+    router_dw_stream_kernel(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ x,
+                            int T, int d, int E, int group_len, float* __restrict__ partial,
+                            DeviceCtl* ctl) {
+  static_assert(NE == 8 || NE == 16, "experts per n-tile");
+  constexpr int NT = NE / 8;  // MMA n-tiles of 8 experts
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ __align__(128) uint8_t s_raw[];
+  uint8_t* s_x = s_raw;  // [stages][kDsTok][kDsRow]
+  float* s_dl = reinterpret_cast<float*>(s_raw + kDsStages * kDsStageX);  // [stages][kDsTok][E]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_raw + kDsStages * (kDsStageX + kDsStageDl));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, q = lane & 3;
+  const int64_t col0 = static_cast<int64_t>(blockIdx.x) * kDsCols;
+  const int cols = d - col0 < kDsCols ? static_cast<int>(d - col0) : kDsCols;  // multiple of 128
+  const int wcol = warp * 256;                    // this warp's first column
+  const int mtiles = cols - wcol >= 256 ? 16 : (cols > wcol ? (cols - wcol) / 16 : 0);
+  const int64_t g0 = static_cast<int64_t>(blockIdx.y) * group_len;
+  const int64_t g1 = g0 + group_len < T ? g0 + group_len : T;
+  const int n_stages = g1 > g0 ? static_cast<int>(ceil_div64(g1 - g0, kDsTok)) : 0;
+  auto bar = [&](int st) { return static_cast<uint32_t>(__cvta_generic_to_shared(bars + st)); };
+  auto issue = [&](int sidx) {  // thread 0
+    const int st = sidx % kDsStages;
+    const int64_t s0 = g0 + static_cast<int64_t>(sidx) * kDsTok;
+    const int nt = g1 - s0 < kDsTok ? static_cast<int>(g1 - s0) : kDsTok;
+    // dL rows: 16-byte multiples (the dL buffer is padded to 256 bytes)
+    const uint32_t dl_bytes = (static_cast<uint32_t>(nt * E * 4) + 15u) & ~15u;
+    ds_expect_tx(bar(st), static_cast<uint32_t>(nt * cols * 2) + dl_bytes);
+    const uint32_t sx = static_cast<uint32_t>(__cvta_generic_to_shared(s_x + st * kDsStageX));
+    for (int tt = 0; tt < nt; ++tt)
+      ds_bulk_g2s(sx + tt * kDsRow, x + (s0 + tt) * d + col0, static_cast<uint32_t>(cols * 2),
+                  bar(st));
+    ds_bulk_g2s(static_cast<uint32_t>(__cvta_generic_to_shared(s_dl + st * (kDsStageDl / 4))),
+                dl + s0 * E, dl_bytes, bar(st));
+  };
+  // rows a short last stage does not fill must hold finite values (their dL is 0)
+  for (int i = tid; i < kDsStages * kDsStageX / 16; i += kDsThreads)
+    reinterpret_cast<uint4*>(s_x)[i] = make_uint4(0, 0, 0, 0);
+  if (tid == 0) {
+    for (int st = 0; st < kDsStages; ++st) ds_mbar_init(bar(st), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // zeros before the bulk writes
+  __syncthreads();
+  if (tid == 0)
+    for (int sidx = 0; sidx < kDsStages && sidx < n_stages; ++sidx) issue(sidx);
+
+  float acc[16][NT][4];
+#pragma unroll
+  for (int m = 0; m < 16; ++m)
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[m][n][i] = 0.f;
+  // ldmatrix: lane l addresses row (l & 7) of 8x8 matrix l >> 3:
+  // matrices (cols 0-7, tokens 0-7), (cols 8-15, tokens 0-7), (0-7, 8-15), (8-15, 8-15)
+  const int lm = lane >> 3, lr = lane & 7;
+  const uint32_t lofs = static_cast<uint32_t>(((lm >> 1) * 8 + lr) * kDsRow + (wcol + (lm & 1) * 8) * 2);
+  int done = 0;
+  bool ok = true;
+  for (int sidx = 0; sidx < n_stages; ++sidx) {
+    const int st = sidx % kDsStages;
+    ok = __syncthreads_and(ds_wait(bar(st), static_cast<uint32_t>((sidx / kDsStages) & 1)));
+    if (!ok) break;
+    const int64_t s0 = g0 + static_cast<int64_t>(sidx) * kDsTok;
+    const int nt = g1 - s0 < kDsTok ? static_cast<int>(g1 - s0) : kDsTok;
+    const float* bd = s_dl + st * (kDsStageDl / 4);
+    // B fragments (K = tokens x N = experts): b0 = dL[2q, 2q+1][e], b1 = dL[2q+8, 2q+9][e],
+    // e = 8n + g; hi and lo parts
+    uint32_t bhi[NT][2], blo[NT][2];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const int e = 8 * n + g;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int t0 = 2 * q + 8 * h;
+        const float v0 = (e < E && t0 < nt) ? bd[t0 * E + e] : 0.f;
+        const float v1 = (e < E && t0 + 1 < nt) ? bd[(t0 + 1) * E + e] : 0.f;
+        __nv_bfloat16 h0, l0, h1, l1;
+        split_bf16(v0, h0, l0);
+        split_bf16(v1, h1, l1);
+        bhi[n][h] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                    (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+        blo[n][h] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
+                    (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+      }
+    }
+    const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(s_x + st * kDsStageX)) + lofs;
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      if (m < mtiles) {
+        uint32_t a[4];
+        ldsm_x4_trans(sbase + m * 32, a);
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          mma_16816(acc[m][n], a, bhi[n][0], bhi[n][1]);
+          mma_16816(acc[m][n], a, blo[n][0], blo[n][1]);
+        }
+      }
+    }
+    done = sidx + 1;
+    __syncthreads();  // every warp is done with this stage's buffers
+    if (tid == 0 && sidx + kDsStages < n_stages) issue(sidx + kDsStages);
+  }
+  if (!ok) {
+    // let this block's copies in flight land before it exits
+    if (tid == 0) {
+      report(ctl, MOE_ERR_TIMEOUT, 6);
+      for (int sidx = done; sidx < n_stages && sidx < done + kDsStages; ++sidx)
+        ds_wait(bar(sidx % kDsStages), static_cast<uint32_t>((sidx / kDsStages) & 1));
+    }
+    return;
+  }
+  // C fragments: c0 = (col g, expert 2q), c1 = (g, 2q+1), c2 = (g+8, 2q), c3 = (g+8, 2q+1)
+  float* out = partial + static_cast<int64_t>(blockIdx.y) * E * d + col0 + wcol;
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    if (m < mtiles) {
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int e = 8 * n + 2 * q + (i & 1);
+          const int c = 16 * m + g + 8 * (i >> 1);
+          if (e < E) out[static_cast<int64_t>(e) * d + c] = acc[m][n][i];
+        }
+      }
+    }
+  }
+}
+
 template <int NE>
 constexpr size_t dw_smem_bytes() {
   return 2 * kDwStageX + 2 * kDwTok * NE * sizeof(float);
@@ -466,6 +677,16 @@ int dw_blocks_per_sm(int E) { return E <= 16 ? 3 : 2; }
 }  // namespace
 
 int router_dw_chunks(int num_sms, int T, int d, int E, int* group_len) {
+  if (E <= 16) {  // streamed: one block per SM over all column slices, whole stages
+    const int64_t col_blocks = ceil_div64(d, kDsCols);
+    int64_t n = ceil_div64(num_sms, col_blocks);
+    const int64_t most = ceil_div64(T, kDsTok);
+    if (n > most) n = most;
+    if (n < 1) n = 1;
+    const int64_t len = ceil_div64(ceil_div64(T, n), kDsTok) * kDsTok;
+    *group_len = static_cast<int>(len);
+    return static_cast<int>(ceil_div64(T, len));
+  }
   const int64_t col_blocks = ceil_div64(d, kDwCols);
   // as many blocks as stay resident, over all column blocks; chunks are
   // whole stages
@@ -479,7 +700,18 @@ int router_dw_chunks(int num_sms, int T, int d, int E, int* group_len) {
 }
 
 cudaError_t launch_router_dw(const float* dl, const __nv_bfloat16* x, int T, int d, int E,
-                             int n_chunks, int group_len, float* partial, cudaStream_t st) {
+                             int n_chunks, int group_len, float* partial, DeviceCtl* ctl,
+                             cudaStream_t st) {
+  if (E <= 16) {
+    auto kern = E <= 8 ? router_dw_stream_kernel<8> : router_dw_stream_kernel<16>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kDsSmem)) != cudaSuccess)
+      return cudaErrorInvalidValue;
+    const unsigned gx = static_cast<unsigned>(ceil_div64(d, kDsCols));
+    (void)launch_pdl(kern, dim3(gx, static_cast<unsigned>(n_chunks)), kDsThreads, kDsSmem, st, dl,
+                     x, T, d, E, group_len, partial, ctl);
+    return cudaGetLastError();
+  }
   auto go = [&](auto kern, size_t smem) {
     // several 66-80 KB blocks per SM only fit with the largest shared-memory carve-out
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -492,8 +724,6 @@ cudaError_t launch_router_dw(const float* dl, const __nv_bfloat16* x, int T, int
                                                                               group_len, partial);
     return cudaGetLastError();
   };
-  if (E <= 8) return go(router_dw_kernel<8>, dw_smem_bytes<8>());
-  if (E <= 16) return go(router_dw_kernel<16>, dw_smem_bytes<16>());
   if (E <= 32) return go(router_dw_kernel<32>, dw_smem_bytes<32>());
   if (E <= 64) return go(router_dw_kernel<64>, dw_smem_bytes<64>());
   return cudaErrorInvalidValue;
