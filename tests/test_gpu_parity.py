@@ -176,6 +176,9 @@ SMALL_CASES = [
     (600, 384, 384, 8, 2, "bias"),         # single-CTA tiles, half-used last N tiles
     (700, 256, 256, 200, 6, "learned"),    # E = 200: tensor-core router, padded logits rows
     (500, 384, 128, 96, 3, "renorm"),      # E = 96, f = 128: one half-used N tile
+    (1024, 256, 256, 8, 4, "learned"),     # ~512 rows per expert: several 128-row tiles
+    (700, 384, 512, 4, 2, "renorm"),       # ~350 rows per expert, d an odd multiple of 128
+    (1600, 256, 256, 6, 2, "skewed"),      # empty experts next to one long segment
 ]
 
 
