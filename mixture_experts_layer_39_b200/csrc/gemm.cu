@@ -7,7 +7,7 @@
 //             dgrad-gu   : dAU x W_gu[e]    -> dX_perm
 //             wgrad-down : dO_e^T H_e       -> dW_d[e]   (contraction over e's rows)
 //             wgrad-gu   : dAU_e^T X_e      -> dW_gu[e]
-//   router    logits  : x W_r^T (E multiple of 128), dX_router = dL W_r,
+//   router    logits  : x W_r^T (E > 64), dX_router = dL W_r,
 //             dW_r partials = dL^T x over token chunks
 #include <cudaTypedefs.h>
 

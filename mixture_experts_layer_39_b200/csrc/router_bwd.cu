@@ -5,9 +5,10 @@
 // optional renormalisation), dp[t, idx[t,j]] = g[t,j] and the softmax
 // backward gives dL = p * (dp - <p, dp>).  Then
 //   dX_router = dL W_r,  dW_r = dL^T x,  db = sum_t dL.
-// For small E these run on CUDA cores; for E a multiple of 128 the two
-// products run on the tcgen05 grouped GEMM (see gemm.cu) and this file only
-// produces dL (bf16) and the db partial sums.
+// For E <= 64 this file forms them: dX_router inside the permute backward,
+// dW_r with mma.sync (E <= 16) or on CUDA cores (E <= 64).  Above 64 experts
+// the two products run on the tcgen05 grouped GEMM (see gemm.cu) and this
+// file only produces dL (bf16) and the db partial sums.
 #include <type_traits>
 
 #include "kernels.cuh"
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   }
 }
 
-// dW_r partial sums over a chunk of tokens, CUDA cores (E <= 64).  A block
+// dW_r partial sums over a chunk of tokens, CUDA cores (16 < E <= 64).  A block
 // owns a slice of kDwCols columns of x and a chunk of tokens (a multiple of
 // kDwTok); it streams the chunk through shared memory in stages of kDwTok
 // tokens (the x slice and the matching dL rows), double-buffered with
