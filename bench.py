@@ -258,6 +258,50 @@ def measure(L, g, steps, warmup, flush, dev, with_gemm_events=True):
     return step_ms, gemm_ms, per_step * steps
 
 
+def measure_memory_bound(L, g, flush, reps=10):
+    """HBM-bound calls of the step, each timed alone with CUDA events after an
+    L2 flush (median of `reps`), against its algorithmic bytes: useful rows
+    only, no pad rows, metadata and router outputs counted where they are
+    written.  The layer holds a completed step, so every call sees the inputs
+    it has in the step."""
+    import torch
+    T, d, k, E = L.T, L.d, L.k, L.E
+    rows = T * k * d * 2  # the T*k routed bf16 rows
+    tok = T * d * 2       # one bf16 row per token
+    fused = L.fuse_router_dx
+    calls = {
+        "router": (lambda: L.router(g["x"], g["w_r"], g["bias"], g["route"]),
+                   tok + T * E * 4 + T * k * 8, "read x; write probs, ids, gate weights"),
+        "permute": (lambda: L.permute(g["x"]), tok + rows,
+                    "routing metadata + read x, write the T*k routed rows"),
+        "combine": (lambda: L.combine(), rows + tok, "read the routed rows, write y"),
+        "combine_bwd": (lambda: L.combine_bwd(g["dy"]), tok + 2 * rows,
+                        "read dY and the routed rows of O, write dO"),
+        "permute_bwd": (lambda: L.permute_bwd(g["w_r"]),
+                        rows + tok + (0 if fused else T * d * 4),
+                        "read dX_perm" + ("" if fused else " and dX_router (fp32)") + ", write dX"
+                        + (" (router input gradient formed in the same pass)" if fused else "")),
+    }
+    stream = torch.cuda.current_stream()
+    out = {}
+    for name, (fn, nbytes, what) in calls.items():
+        fn()  # warm
+        ts = []
+        for _ in range(reps):
+            flush.fill_(3)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        ts.sort()
+        ms = ts[len(ts) // 2]
+        out[name] = {"ms": ms, "bytes": nbytes, "gb_s": nbytes / (ms / 1e3) / 1e9, "what": what}
+    return out
+
+
 def measure_e2e(L, g, steps, warmup, dev):
     """The same step through the public API with host buffers: every step's
     inputs (x, dY and, in random-routing mode, the expert ids) are copied in
@@ -334,6 +378,8 @@ def run_ours(args):
         out = {"total_ms": max_over_ranks(sum(step_ms)), "step_ms": step_ms,
                "gemm_ms": gemm_ms, "launches": launches, "counts": L.counts.cpu().numpy()}
         if with_e2e:
+            out["memory_bound"] = measure_memory_bound(L, g, flush)
+            barrier()
             e2e_ms, h2d, d2h = measure_e2e(L, g, steps, min(warmup, 3), dev)
             barrier()
             out.update({"e2e_total_ms": max_over_ranks(e2e_ms), "h2d": h2d, "d2h": d2h})
@@ -398,6 +444,10 @@ def run_ours(args):
                          "share_of_step": gemm_ms / (main["total_ms"] / K)},
         "routing": {"max_over_mean_load": float(counts.max() / counts.mean()),
                     "zero_experts": int((counts == 0).sum())},
+        "memory_bound": {
+            "peak_gb_s": peaks["hbm_gbs"], "peak_source": f"{peak_kind} copy",
+            "timing": "each call alone, CUDA events, L2 flushed before it, median of 10 (rank 0)",
+            **{n: {**v, "frac": v["gb_s"] / peaks["hbm_gbs"]} for n, v in main["memory_bound"].items()}},
         "clocks": clocks,
     }
     if ratio is not None:
