@@ -179,6 +179,8 @@ SMALL_CASES = [
     (1024, 256, 256, 8, 4, "learned"),     # ~512 rows per expert: several 128-row tiles
     (700, 384, 512, 4, 2, "renorm"),       # ~350 rows per expert, d an odd multiple of 128
     (1600, 256, 256, 6, 2, "skewed"),      # empty experts next to one long segment
+    (300, 2304, 256, 8, 2, "learned"),     # d > 2048: router dW over two column slices
+    (200, 4096, 128, 16, 4, "bias"),       # d = 4096, E = 16 (router dW: two n-tiles of experts)
 ]
 
 
