@@ -12,6 +12,8 @@
 // conversion (cvt with .satfinite through cuda_fp8.h).
 #include <cuda_fp8.h>
 
+#include <type_traits>
+
 #include "kernels.cuh"
 
 namespace moe {
@@ -25,6 +27,18 @@ __device__ __forceinline__ int mx_scale_exp(float amax) {
 
 __device__ __forceinline__ float pow2_neg(int e) {  // 2^-e for e in [-127, 126]
   return __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+}
+
+__device__ __forceinline__ __nv_bfloat162 as_bf162(uint32_t v) {
+  __nv_bfloat162 r;
+  memcpy(&r, &v, sizeof(r));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t as_u32(__nv_bfloat162 v) {
+  uint32_t r;
+  memcpy(&r, &v, sizeof(r));
+  return r;
 }
 
 __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
@@ -70,48 +84,102 @@ __global__ void mx_rowwise_kernel(const uint4* __restrict__ in, int64_t rows, in
   }
 }
 
-// axis 0: one thread per (32-row block, pair of adjacent columns).  Scales go
-// to [rows/32, cols] (scale_mode 0) or, for the GEMM operand layout, to
+// axis 0: one thread per (32-row block, W adjacent columns), W = 4 where the
+// row width and the buffers' alignment allow 8-byte loads, else 2.  Each row
+// of the block is one vector load and one vector store of W codes; the two
+// columns of a bf16 pair are converted by one paired E4M3 conversion (each
+// element rounds on its own, so pairing changes no code).  Scales go to
+// [rows/32, cols] (scale_mode 0) or, for the GEMM operand layout, to
 // [groups, cols, rows_per_group/32] (scale_mode 1: a column's scales along
 // the contraction axis are contiguous inside each group of rows).
-__global__ void mx_colwise_kernel(const uint32_t* __restrict__ in, int64_t rows, int64_t cols,
-                                  uint16_t* __restrict__ q, uint8_t* __restrict__ scales,
+template <int W>
+__global__ void mx_colwise_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_t cols,
+                                  uint8_t* __restrict__ q, uint8_t* __restrict__ scales,
                                   int scale_mode, int64_t rows_per_group) {
+  static_assert(W == 2 || W == 4, "two or four columns per thread");
+  constexpr int NP = W / 2;  // bf16 pairs per row slice
+  using In = typename std::conditional<NP == 2, uint2, uint32_t>::type;
+  using Out = typename std::conditional<NP == 2, uint32_t, uint16_t>::type;
   pdl_wait();
   pdl_trigger();
-  const int64_t cpairs = cols / 2;
-  const int64_t total = (rows / 32) * cpairs;
+  const int64_t cgroups = cols / W;
+  const int64_t total = (rows / 32) * cgroups;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t rb = i / cpairs, cp = i - rb * cpairs;
-    float a[32], b[32];
-    float am0 = 0.f, am1 = 0.f;
+    const int64_t rb = i / cgroups, cg = i - rb * cgroups;
+    const In* src = reinterpret_cast<const In*>(in) + rb * 32 * cgroups + cg;
+    uint32_t w[32][NP];
 #pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      const uint32_t w = __ldg(in + (rb * 32 + r) * cpairs + cp);
-      a[r] = bf16_lo(w);
-      b[r] = bf16_hi(w);
-      am0 = fmaxf(am0, fabsf(a[r]));
-      am1 = fmaxf(am1, fabsf(b[r]));
+    for (int r = 0; r < 32; ++r, src += cgroups) {
+      const In v = __ldg(src);
+      if constexpr (NP == 2) {
+        w[r][0] = v.x;
+        w[r][1] = v.y;
+      } else {
+        w[r][0] = v;
+      }
     }
-    const int e0 = mx_scale_exp(am0), e1 = mx_scale_exp(am1);
-    const float i0 = pow2_neg(e0), i1 = pow2_neg(e1);
+    // amax on the packed pairs: a max is exact in bf16, and like fmaxf
+    // __hmax2 returns the other operand when one is NaN.
+    __nv_bfloat162 m[NP];
 #pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      const uint16_t lo = e4m3x2(a[r] * i0, 0.f) & 0xFF;
-      const uint16_t hi = e4m3x2(b[r] * i1, 0.f) & 0xFF;
-      q[(rb * 32 + r) * cpairs + cp] = static_cast<uint16_t>(lo | (hi << 8));
+    for (int j = 0; j < NP; ++j) m[j] = __float2bfloat162_rn(0.f);
+#pragma unroll
+    for (int r = 0; r < 32; ++r)
+#pragma unroll
+      for (int j = 0; j < NP; ++j) m[j] = __hmax2(m[j], __habs2(as_bf162(w[r][j])));
+    int e[W];
+    float inv[W];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+      const uint32_t mb = as_u32(m[j]);
+      e[2 * j] = mx_scale_exp(bf16_lo(mb));
+      e[2 * j + 1] = mx_scale_exp(bf16_hi(mb));
+    }
+#pragma unroll
+    for (int c = 0; c < W; ++c) inv[c] = pow2_neg(e[c]);
+    Out* dst = reinterpret_cast<Out*>(q) + rb * 32 * cgroups + cg;
+#pragma unroll
+    for (int r = 0; r < 32; ++r, dst += cgroups) {
+      uint32_t p = 0;
+#pragma unroll
+      for (int j = 0; j < NP; ++j)
+        p |= static_cast<uint32_t>(e4m3x2(bf16_lo(w[r][j]) * inv[2 * j],
+                                          bf16_hi(w[r][j]) * inv[2 * j + 1]))
+             << (16 * j);
+      *dst = static_cast<Out>(p);
     }
     if (scale_mode == 0) {
-      reinterpret_cast<uint16_t*>(scales)[rb * cpairs + cp] =
-          static_cast<uint16_t>((e0 + 127) | ((e1 + 127) << 8));
+      uint32_t s = 0;
+#pragma unroll
+      for (int c = 0; c < W; ++c) s |= static_cast<uint32_t>(e[c] + 127) << (8 * c);
+      reinterpret_cast<Out*>(scales)[rb * cgroups + cg] = static_cast<Out>(s);
     } else {
       const int64_t bpg = rows_per_group / 32;  // scale blocks per group
       const int64_t g = rb / bpg, rl = rb - g * bpg;
-      scales[(g * cols + 2 * cp) * bpg + rl] = static_cast<uint8_t>(e0 + 127);
-      scales[(g * cols + 2 * cp + 1) * bpg + rl] = static_cast<uint8_t>(e1 + 127);
+#pragma unroll
+      for (int c = 0; c < W; ++c)
+        scales[(g * cols + W * cg + c) * bpg + rl] = static_cast<uint8_t>(e[c] + 127);
     }
   }
+}
+
+// Picks four columns per thread when every vector access stays aligned.
+cudaError_t launch_colwise(const __nv_bfloat16* in, int64_t rows, int64_t cols, uint8_t* q,
+                           uint8_t* scales, int scale_mode, int64_t rows_per_group,
+                           cudaStream_t st) {
+  const bool wide = cols % 4 == 0 && (reinterpret_cast<uintptr_t>(in) & 7) == 0 &&
+                    (reinterpret_cast<uintptr_t>(q) & 3) == 0 &&
+                    (scale_mode != 0 || (reinterpret_cast<uintptr_t>(scales) & 3) == 0);
+  const int64_t total = (rows / 32) * (cols / (wide ? 4 : 2));
+  const unsigned grid = static_cast<unsigned>(ceil_div64(total, 256) < 65535 ? ceil_div64(total, 256) : 65535);
+  if (wide)
+    (void)launch_pdl(mx_colwise_kernel<4>, grid, 256, 0, st, in, rows, cols, q, scales, scale_mode,
+                     rows_per_group);
+  else
+    (void)launch_pdl(mx_colwise_kernel<2>, grid, 256, 0, st, in, rows, cols, q, scales, scale_mode,
+                     rows_per_group);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -123,23 +191,15 @@ cudaError_t launch_mxfp8_quantize(const __nv_bfloat16* in, int64_t rows, int64_t
     const unsigned grid = static_cast<unsigned>(ceil_div64(total, 256) < 65535 ? ceil_div64(total, 256) : 65535);
     (void)launch_pdl(mx_rowwise_kernel, grid, 256, 0, st, reinterpret_cast<const uint4*>(in), rows, cols,
                                             reinterpret_cast<uint4*>(q), scales);
-  } else {
-    const int64_t total = (rows / 32) * (cols / 2);
-    const unsigned grid = static_cast<unsigned>(ceil_div64(total, 256) < 65535 ? ceil_div64(total, 256) : 65535);
-    (void)launch_pdl(mx_colwise_kernel, grid, 256, 0, st, reinterpret_cast<const uint32_t*>(in), rows, cols,
-                                            reinterpret_cast<uint16_t*>(q), scales, 0, rows);
+    return cudaGetLastError();
   }
-  return cudaGetLastError();
+  return launch_colwise(in, rows, cols, q, scales, 0, rows, st);
 }
 
 cudaError_t launch_mxfp8_quantize_cols_t(const __nv_bfloat16* in, int64_t rows, int64_t cols,
                                          int64_t rows_per_group, uint8_t* q, uint8_t* scales,
                                          cudaStream_t st) {
-  const int64_t total = (rows / 32) * (cols / 2);
-  const unsigned grid = static_cast<unsigned>(ceil_div64(total, 256) < 65535 ? ceil_div64(total, 256) : 65535);
-  (void)launch_pdl(mx_colwise_kernel, grid, 256, 0, st, reinterpret_cast<const uint32_t*>(in), rows, cols,
-                                          reinterpret_cast<uint16_t*>(q), scales, 1, rows_per_group);
-  return cudaGetLastError();
+  return launch_colwise(in, rows, cols, q, scales, 1, rows_per_group, st);
 }
 
 }  // namespace moe

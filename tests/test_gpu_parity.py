@@ -356,3 +356,27 @@ def test_mxfp8_quantize_matches_oracle(cuda_ok):
         qo, so = M.quantize_blocks(a.double().numpy(), axis)
         np.testing.assert_array_equal(s.cpu().numpy(), so)
         np.testing.assert_array_equal(q.cpu().numpy(), qo)
+
+
+@pytest.mark.parametrize("rows,cols", [(64, 130), (96, 132), (32, 2)])
+def test_mxfp8_quantize_columnwise_widths(cuda_ok, rows, cols):
+    """Column-wise blocks where a thread takes two columns (cols % 4 == 2) and
+    four (cols % 4 == 0), each column with its own magnitude, so every lane of
+    a vector access has its own scale; bit-exact against the oracle."""
+    from mixture_experts_layer_39_b200 import ops
+    from oracle import mxfp8_ref as M
+    h = ops.Handle(0)
+    g = torch.Generator().manual_seed(rows + cols)
+    a = torch.randn(rows, cols, generator=g) * torch.exp(torch.randn(1, cols, generator=g) * 5)
+    a[:, 0] = 0.0
+    if cols > 3:
+        a[:32, 3] = -1e-30
+        a[1, 2] = 4e5
+    a = a.to(torch.bfloat16)
+    q = torch.empty(rows, cols, dtype=torch.uint8, device="cuda")
+    s = torch.empty(rows // 32, cols, dtype=torch.uint8, device="cuda")
+    ops.moe_mxfp8_quantize(h, a.cuda(), 0, q, s)
+    torch.cuda.synchronize()
+    qo, so = M.quantize_blocks(a.double().numpy(), 0)
+    np.testing.assert_array_equal(s.cpu().numpy(), so)
+    np.testing.assert_array_equal(q.cpu().numpy(), qo)
