@@ -83,3 +83,23 @@ def test_create_without_device_fails_cleanly(lib):
     h = ctypes.c_void_p()
     assert lib.moe_create(ctypes.byref(h), 0) != 0
     assert not h.value
+
+
+def test_max_rows_mxfp8_and_row_limit(lib):
+    """MXFP8 segments start at multiples of 128 rows, so the cap is the
+    routed rows plus 127 per expert, rounded up to 128; shapes whose cap
+    reaches 2^31 rows are refused (row indices are int32)."""
+    n = ctypes.c_int64()
+    s = _lib.MoeShape(32768, 4096, 1536, 128, 4, 1, 0)
+    assert lib.moe_max_rows(ctypes.byref(s), ctypes.byref(n)) == 0
+    r = 32768 * 4 + 127 * 128
+    assert n.value == (r + 127) // 128 * 128
+    s = _lib.MoeShape(3, 128, 128, 5, 2, 1, 0)
+    assert lib.moe_max_rows(ctypes.byref(s), ctypes.byref(n)) == 0
+    assert n.value == (6 + 127 * 5 + 127) // 128 * 128
+    assert n.value % 128 == 0
+    s = _lib.MoeShape(1 << 28, 128, 128, 8, 8, 0, 0)   # 2^31 routed rows
+    assert lib.moe_max_rows(ctypes.byref(s), ctypes.byref(n)) == 2
+    s = _lib.MoeShape((1 << 28) - 64, 128, 128, 8, 8, 0, 0)  # just under the limit
+    assert lib.moe_max_rows(ctypes.byref(s), ctypes.byref(n)) == 0
+    assert n.value == ((1 << 28) - 64) * 8 + 31 * 8
