@@ -163,3 +163,26 @@ def test_bf16_round_matches_torch():
     ours = R.bf16_round(v)
     ref = torch.tensor(v.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
     np.testing.assert_array_equal(ours, ref)
+
+
+def test_bf16_round_exact_ties_go_to_even():
+    """fp32 words whose dropped half is exactly 0x8000 lie halfway between
+    two bf16 values (random values almost never do). They must round to the
+    neighbour with an even upper half, as torch's cast does. Words one below
+    and one above the tie round down and up."""
+    rng = np.random.default_rng(8)
+    hi = rng.integers(0, 0x7F80, 4000).astype(np.uint32)    # finite upper halves
+    hi = np.concatenate([hi, hi | 0x8000, [0, 1, 2, 3, 0x7F7E, 0x7F7F]]).astype(np.uint32)
+    for low in (0x8000, 0x7FFF, 0x8001):
+        v = ((hi << 16) | low).view(np.float32).astype(np.float64)
+        ours = R.bf16_round(v)
+        ref = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+        np.testing.assert_array_equal(ours, ref)
+        up = ours.astype(np.float32).view(np.uint32) >> 16
+        mag = (hi & 0x7FFF).astype(np.int64)
+        got = (up & 0x7FFF).astype(np.int64)
+        if low == 0x8000:
+            want = np.where(mag % 2 == 0, mag, mag + 1)        # ties to the even neighbour
+        else:
+            want = mag + (1 if low == 0x8001 else 0)
+        np.testing.assert_array_equal(got, want)
