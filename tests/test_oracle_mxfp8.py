@@ -54,12 +54,15 @@ def test_e4m3_encode_saturates():
 def test_scale_rule_brute_force():
     rng = np.random.default_rng(1)
     amax = np.concatenate([rng.standard_normal(2000) ** 2 * 2.0 ** rng.integers(-60, 60, 2000),
-                           2.0 ** np.arange(-100, 100, dtype=np.float64), [448.0, 512.0, 511.9]])
+                           2.0 ** np.arange(-133, 140, dtype=np.float64), [448.0, 512.0, 511.9],
+                           # both clamps: bf16 subnormals reach e < -127 (2^-133 is the
+                           # smallest), huge float64 values e > 127
+                           [1.5 * 2.0 ** -119, 1.9 * 2.0 ** -120, 1e-40, 3.0 * 2.0 ** 135]])
     amax = np.abs(amax)
     got = M.scale_exponent(amax)
     for a, e in zip(amax, got):
         # the unique e with 2^8 <= a / 2^e < 2^9
-        cand = [s for s in range(-140, 141) if 256.0 <= a / 2.0 ** s < 512.0]
+        cand = [s for s in range(-160, 161) if 256.0 <= a / 2.0 ** s < 512.0]
         assert len(cand) == 1 and e == max(-127, min(127, cand[0]))
     assert M.scale_exponent(np.array([0.0]))[0] == -127
 
