@@ -103,3 +103,14 @@ def test_max_rows_mxfp8_and_row_limit(lib):
     s = _lib.MoeShape((1 << 28) - 64, 128, 128, 8, 8, 0, 0)  # just under the limit
     assert lib.moe_max_rows(ctypes.byref(s), ctypes.byref(n)) == 0
     assert n.value == ((1 << 28) - 64) * 8 + 31 * 8
+
+
+def test_every_entry_point_is_documented():
+    """Each declaration in include/moe.h follows its own comment block
+    (macros it defines may sit between the two)."""
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    for m in re.finditer(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text):
+        before = text[:m.start()].rstrip().splitlines()
+        while before and before[-1].startswith("#define"):
+            before.pop()
+        assert before and before[-1].rstrip().endswith("*/"), m.group(1)
