@@ -21,8 +21,16 @@ class MoeError(RuntimeError):
 
 
 def _ptr(t):
+    """Data pointer of a tensor for the C ABI, which takes dense row-major
+    buffers in device memory: a strided view or a host tensor is refused
+    here rather than read with the wrong layout."""
     if t is None:
         return None
+    if not t.is_contiguous():
+        raise ValueError(f"expected a contiguous tensor, got strides {tuple(t.stride())} "
+                         f"for shape {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"expected a CUDA tensor, got one on {t.device}")
     return ctypes.c_void_p(t.data_ptr())
 
 

@@ -114,3 +114,17 @@ def test_every_entry_point_is_documented():
         while before and before[-1].startswith("#define"):
             before.pop()
         assert before and before[-1].rstrip().endswith("*/"), m.group(1)
+
+
+def test_binding_refuses_strided_and_host_tensors():
+    """The binding passes raw pointers; a layout it cannot express is an
+    error before any call into the library."""
+    import torch
+    from mixture_experts_layer_39_b200 import ops
+    assert ops._ptr(None) is None
+    with pytest.raises(ValueError, match="contiguous"):
+        ops._ptr(torch.zeros(4, 6).t())
+    with pytest.raises(ValueError, match="contiguous"):
+        ops._ptr(torch.zeros(8)[::2])
+    with pytest.raises(ValueError, match="CUDA"):
+        ops._ptr(torch.zeros(4, 6))
