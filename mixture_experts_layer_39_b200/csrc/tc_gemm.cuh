@@ -517,10 +517,6 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 // ---------------------------------------------------------------- the kernel
 template <int BN, int STAGES, int EPI, bool FP8 = false, bool PAIR = false>
 struct SmemPlan {
