@@ -68,3 +68,19 @@ def test_c_program_links_and_calls_host_entry_points(tmp_path, libdir):
     assert run.returncode == 0, (run.returncode, run.stderr)
     unsupported, unknown = run.stdout.strip().split("|")
     assert unsupported and "unknown" in unknown
+
+
+def test_readme_c_example_compiles(tmp_path):
+    """The C example in the README is code against the real header."""
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    import re
+    text = open(os.path.join(ROOT, "README.md")).read()
+    blocks = re.findall(r"```c\n(.*?)```", text, re.S)
+    assert blocks
+    src = tmp_path / "example.c"
+    src.write_text(blocks[0])
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        "-c", str(src), "-o", str(tmp_path / "example.o")],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
