@@ -435,12 +435,3 @@ def layer_bwd(fwd, dy, x, w_r, w_gu, w_d, renorm=False, rnd=bf16_round, w_gu_s=N
                 "dw_r": rb["dw_r"], "db": rb["db"]})
     return out
 
-
-def token_ffn(x_t, e, w_gu, w_d):
-    """Dense SwiGLU of one token through expert e, float64, no rounding
-    (used by sampled checks at full size)."""
-    f = w_gu.shape[1] // 2
-    x_t = np.asarray(x_t, F64)
-    A = np.asarray(w_gu[e, :f], F64) @ x_t
-    U = np.asarray(w_gu[e, f:], F64) @ x_t
-    return np.asarray(w_d[e], F64) @ (silu(A) * U)
