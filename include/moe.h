@@ -99,21 +99,30 @@ typedef struct moe_context* moe_handle_t;
 typedef void* moe_stream_t; /* a cudaStream_t */
 
 /* Creates a handle bound to CUDA device `device`: caches the SM count and
- * allocates the device status word.  *h receives the handle. */
+ * allocates the device status word.  *h receives the handle.
+ * (Library plumbing: the pages have no counterpart.) */
 MOE_API moe_status_t moe_create(moe_handle_t* h, int device);
 
-/* Frees the handle's control block.  Pending work must have finished. */
+/* Frees the handle's control block.  Pending work must have finished.
+ * (Library plumbing: the pages have no counterpart.) */
 MOE_API moe_status_t moe_destroy(moe_handle_t h);
 
 /* Bytes of scratch every step call of this shape may use, in one buffer
  * shared by all calls (calls on one stream run in order, so they can share
- * it).  Must be 256-byte aligned. */
+ * it).  Must be 256-byte aligned.
+ * (Library plumbing: the pages have no counterpart.) */
 MOE_API moe_status_t moe_workspace_size(moe_handle_t h, const moe_shape_t* s, size_t* bytes);
 
-/* M_cap: rows of every buffer in the routed-row space (see above). */
+/* M_cap: rows of every buffer in the routed-row space (see above).
+ * (Library plumbing: the pages have no counterpart.) */
 MOE_API moe_status_t moe_max_rows(const moe_shape_t* s, int64_t* rows);
 
-/* Router forward (top-k softmax).
+/* Router forward (top-k softmax).  The pages: a router network scores each
+ * token over the experts and the k highest are kept (discosf.com article on
+ * Olmo-core 3, sections 1.1 and 2.1); the trillion-scale runs route at
+ * random (Olmo-core 3 introduction page, key-numbers caveats), which
+ * route_in serves.  Softmax before top-k, no renormalisation and the tie
+ * rule are readings (the pages give no formula).
  *   L[t,e] = sum_i x[t,i] * w_router[e,i] (+ bias[e]), fp32 accumulate;
  *   probs  = softmax over all E experts, fp32;
  *   topk_idx[t, 0..k-1] = the k largest L[t,:], ties to the lower expert
@@ -132,7 +141,14 @@ MOE_API moe_status_t moe_router_topk(moe_handle_t h, const moe_shape_t* s,
                              float* probs, float* logits, void* ws, size_t ws_bytes,
                              moe_stream_t stream);
 
-/* Routing metadata + rowwise permute, all on the device.
+/* Routing metadata + rowwise permute, all on the device.  The pages: the
+ * routing metadata stays on the GPU so the host never waits for a copy back,
+ * and routed tokens are written straight into each expert's input buffer
+ * (Olmo-core 3 introduction page, section 2, GPU-resident routing and
+ * rowwise expert parallelism); the routing result becomes a permutation
+ * index that regroups tokens per expert (discosf.com article on Olmo-core 3,
+ * section 2.1).  Expert-major stable order and 32-row segment padding are
+ * readings.
  *   counts[e]   = number of (t,j) with topk_idx[t,j] == e;
  *   offsets[e]  = sum_{e'<e} roundup(counts[e'], A); offsets[E] = M_pad
  *                 (A = 32, or 128 in MXFP8 mode);
@@ -161,7 +177,9 @@ MOE_API moe_status_t moe_permute(moe_handle_t h, const moe_shape_t* s, const voi
  * otherwise MOE_ERR_WORKSPACE is returned before any launch.  The first call
  * on a device looks up the array's device address (a host-side step, done
  * once per device with that device current); make that first call before
- * any stream capture.  All calls share the array: calls whose work can
+ * any stream capture.  The address is kept per CUDA context: after a device
+ * reset the next call looks it up again, so make that call before any
+ * capture too.  All calls share the array: calls whose work can
  * overlap on the GPU (unordered streams, several host threads) race on it.
  * Nothing is allocated or freed by this call. */
 #define MOE_NOALLOC_SCRATCH_INTS (1 << 18)
@@ -170,7 +188,13 @@ MOE_API moe_status_t moe_permute_noalloc(moe_handle_t h, const moe_shape_t* s, c
                                          int32_t* offsets, int32_t* row_map, void* x_perm,
                                          moe_stream_t stream);
 
-/* Grouped SwiGLU expert FFN, forward.  For the rows of expert e:
+/* Grouped SwiGLU expert FFN, forward.  The pages: all experts' small GEMMs
+ * run as one grouped GEMM whose schedule is read on the device (Olmo-core 3
+ * introduction page, section 2, grouped GEMM and device-scheduled grouped
+ * GEMM), and no token is dropped when an expert is over-subscribed
+ * (vibecoding.ru news item on Olmo-core 3, paragraph on grouped_gemm and
+ * dropless MoE).  The SwiGLU form without biases is a reading.
+ * For the rows of expert e:
  *   A = X W_gu[e][0:f]^T, U = X W_gu[e][f:2f]^T   (fp32 accumulate)
  *   au[:, 0:f] = bf16(A), au[:, f:2f] = bf16(U)   (saved for the backward)
  *   h = bf16(silu(A) * U), silu(z) = z / (1 + exp(-z))
@@ -220,14 +244,17 @@ MOE_API moe_status_t moe_route(moe_handle_t h, const moe_shape_t* s, const int32
                                int32_t* row_src, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* moe_grouped_swiglu_fwd with x [T,d] and row_src in place of x_perm (au may
- * be NULL as there).  No workspace. */
+ * be NULL as there).  No workspace.  Same passages as moe_grouped_swiglu_fwd
+ * and moe_route (Olmo-core 3 introduction page, section 2). */
 MOE_API moe_status_t moe_grouped_swiglu_fwd_gather(moe_handle_t h, const moe_shape_t* s,
                                                    const void* x, const int32_t* row_src,
                                                    const int32_t* offsets, const void* w_gu,
                                                    const void* w_down, void* au, void* hbuf,
                                                    void* o_perm, moe_stream_t stream);
 
-/* moe_grouped_swiglu_recompute with x [T,d] and row_src in place of x_perm. */
+/* moe_grouped_swiglu_recompute with x [T,d] and row_src in place of x_perm.
+ * Same passages as moe_grouped_swiglu_recompute (Olmo-core 3 introduction
+ * page, section 4) and moe_route (same page, section 2). */
 MOE_API moe_status_t moe_grouped_swiglu_recompute_gather(moe_handle_t h, const moe_shape_t* s,
                                                          const void* x, const int32_t* row_src,
                                                          const int32_t* offsets, const void* w_gu,
@@ -235,7 +262,9 @@ MOE_API moe_status_t moe_grouped_swiglu_recompute_gather(moe_handle_t h, const m
                                                          moe_stream_t stream);
 
 /* moe_grouped_swiglu_bwd with x [T,d] and row_src in place of x_perm (only
- * the gate/up weight gradient reads it).  No workspace. */
+ * the gate/up weight gradient reads it).  No workspace.  Same passages as
+ * moe_grouped_swiglu_bwd and moe_route (Olmo-core 3 introduction page,
+ * section 2). */
 MOE_API moe_status_t moe_grouped_swiglu_bwd_gather(moe_handle_t h, const moe_shape_t* s,
                                                    const void* do_perm, const void* x,
                                                    const int32_t* row_src, const void* au,
@@ -244,7 +273,10 @@ MOE_API moe_status_t moe_grouped_swiglu_bwd_gather(moe_handle_t h, const moe_sha
                                                    void* dx_perm, void* dw_gu, void* dw_down,
                                                    moe_stream_t stream);
 
-/* Weighted unpermute-combine ("restore"):
+/* Weighted unpermute-combine ("restore").  The pages: expert outputs are
+ * put back in the tokens' original order (discosf.com article on Olmo-core 3,
+ * section 2.1); weighting by the gate weights and the slot-order fp32 sum
+ * are readings.
  *   y[t] = bf16( sum_j topk_w[t,j] * o_perm[row_map[t,j]] + shared_out[t] ),
  *   fp32 sum in slot order, the shared expert's output (when non-NULL) last.
  * In : o_perm [M_cap,d] bf16, row_map [T,k] int32, topk_w [T,k] fp32,
@@ -254,7 +286,9 @@ MOE_API moe_status_t moe_unpermute_combine(moe_handle_t h, const moe_shape_t* s,
                                    const int32_t* row_map, const float* topk_w,
                                    const void* shared_out, void* y, moe_stream_t stream);
 
-/* Backward of the combine:
+/* Backward of the combine: the plain backward of moe_unpermute_combine
+ * (restore step: discosf.com article on Olmo-core 3, section 2.1; the
+ * pages train the layer but give no backward formula).
  *   do_perm[row_map[t,j]] = bf16(topk_w[t,j] * dy[t]); pad rows = 0;
  *   d_topk_w[t,j] = sum_i dy[t,i] * o_perm[row_map[t,j], i]  (fp32).
  * In : dy [T,d] bf16, o_perm, row_map, topk_w, offsets [E+1], counts [E].
@@ -265,7 +299,10 @@ MOE_API moe_status_t moe_unpermute_combine_bwd(moe_handle_t h, const moe_shape_t
                                        const int32_t* counts, void* do_perm, float* d_topk_w,
                                        moe_stream_t stream);
 
-/* Grouped SwiGLU expert FFN, backward (dgrad and wgrad).  Per expert e:
+/* Grouped SwiGLU expert FFN, backward (dgrad and wgrad).  The same grouped,
+ * device-scheduled GEMMs as the forward (Olmo-core 3 introduction page,
+ * section 2); the formulas are the plain backward of the SwiGLU reading.
+ * Per expert e:
  *   dH = do_perm W_down[e]                       (fp32 accumulate)
  *   s = sigmoid(A), A and U read from au
  *   dau[:,0:f] = bf16(dH U s (1 + A (1 - s))),  dau[:,f:2f] = bf16(dH silu(A))
@@ -283,7 +320,9 @@ MOE_API moe_status_t moe_grouped_swiglu_bwd(moe_handle_t h, const moe_shape_t* s
                                     void* dw_down, void* ws, size_t ws_bytes,
                                     moe_stream_t stream);
 
-/* Backward of the permute:
+/* Backward of the permute: the plain backward of moe_permute's copy
+ * (permutation index and restore: discosf.com article on Olmo-core 3,
+ * section 2.1), each token's k routed gradients summed back to it.
  *   dx[t] = bf16( sum_j dx_perm[row_map[t,j]] + dx_router[t] + dx_shared[t] ),
  *   fp32 sum, rounded once.  dx_router and dx_shared may be NULL.
  * In : dx_perm [M_cap,d] bf16, row_map [T,k], dx_router [T,d] fp32 or NULL,
@@ -294,8 +333,10 @@ MOE_API moe_status_t moe_permute_bwd(moe_handle_t h, const moe_shape_t* s, const
                              const void* dx_shared, void* dx, moe_stream_t stream);
 
 /* Backward of the permute with the router's share of the input gradient
- * added in the same pass (the pages name only the steps; the formulas are
- * the plain backward of the router and of the permute):
+ * added in the same pass (the pages name only the steps -- the router:
+ * discosf.com article on Olmo-core 3, sections 1.1 and 2.1; the permutation
+ * and restore: same article, section 2.1 -- and the formulas are the plain
+ * backward of the router and of the permute):
  *   dL[t]  = as in moe_router_topk_bwd, from d_topk_w, probs, topk_idx and
  *            d_probs_aux (nullable)
  *   dx[t]  = bf16( sum_j dx_perm[row_map[t,j]] + dL[t] w_router
@@ -331,7 +372,9 @@ MOE_API moe_status_t moe_shared_expert_fwd(moe_handle_t h, const moe_shape_t* s,
                                            const void* w_gu_s, const void* w_d_s, void* au_s,
                                            void* h_s, void* o_s, moe_stream_t stream);
 
-/* Shared expert backward, from its output gradient dY (weight one):
+/* Shared expert backward (shared experts: Olmo-core 3 introduction page,
+ * section 4; the plain backward of the reading above), from its output
+ * gradient dY (weight one):
  *   dAU_s = SwiGLU backward of dY W_d_s (as moe_grouped_swiglu_bwd),
  *   dW_d_s = bf16(dY^T H_s), dx_s = bf16(dAU_s W_gu_s), dW_gu_s = bf16(dAU_s^T x).
  * Feed dx_s to moe_permute_bwd / moe_permute_router_bwd's dx_shared.
@@ -344,7 +387,8 @@ MOE_API moe_status_t moe_shared_expert_bwd(moe_handle_t h, const moe_shape_t* s,
                                            moe_stream_t stream);
 
 /* Router backward (through the selected probabilities; top-k itself has no
- * gradient):
+ * gradient).  The plain backward of the router of moe_router_topk
+ * (discosf.com article on Olmo-core 3, sections 1.1 and 2.1):
  *   g = d_topk_w, or with MOE_FLAG_RENORM g_j = (dw_j - sum_i dw_i w_i) / S
  *   dp[t, topk_idx[t,j]] = g[t,j], 0 elsewhere
  *   dp[t, e] += d_probs_aux[e] for every t, when d_probs_aux is non-NULL
@@ -381,7 +425,9 @@ MOE_API moe_status_t moe_router_load_stats(moe_handle_t h, const moe_shape_t* s,
                                            const int32_t* counts, int accumulate, float* stats,
                                            void* ws, size_t ws_bytes, moe_stream_t stream);
 
-/* Load-balancing loss of (possibly summed) statistics over n_tokens tokens:
+/* Load-balancing loss (discosf.com article on Olmo-core 3, sections 2.2 and
+ * 4.3; the Switch-Transformer reading of moe_router_load_stats) of
+ * (possibly summed) statistics over n_tokens tokens:
  *   f_e = stats[e] / (n_tokens k),  P_e = stats[E+e] / n_tokens
  *   loss = alpha E sum_e f_e P_e        (alpha at balance, alpha E at collapse)
  *   d_probs_aux[e] = alpha E f_e / n_tokens = d loss / d probs[t, e] for every
@@ -394,7 +440,9 @@ MOE_API moe_status_t moe_router_aux_loss(moe_handle_t h, const moe_shape_t* s, c
                                          float* d_probs_aux, moe_stream_t stream);
 
 /* MXFP8 quantisation of a bf16 matrix [rows, cols] (OCP MX v1.0 reading of
- * the pages' "MXFP8"): blocks of 32 consecutive elements, along each row
+ * the pages' "MXFP8", offered for selected operations, its gain coming from
+ * the FFN and expert data movement: Olmo-core 3 introduction page, section 3
+ * "MXFP8"): blocks of 32 consecutive elements, along each row
  * (axis = 1) or down each column (axis = 0); per block the E8M0 scale code
  * is clamp(floor(log2(amax)) - 8, -127, 127) + 127 (code 0 for an all-zero
  * block) and each element is the E4M3 code of round-to-nearest-even
@@ -407,14 +455,28 @@ MOE_API moe_status_t moe_mxfp8_quantize(moe_handle_t h, const void* in, int64_t 
 
 /* Waits for the device, then returns the status word recorded by kernels
  * (MOE_OK if none) in *device_status and clears it.  The only call that
- * synchronises; not meant for use inside a step. */
+ * synchronises; not meant for use inside a step.
+ * (Library plumbing: the pages have no counterpart.) */
 MOE_API moe_status_t moe_get_status(moe_handle_t h, int* device_status);
 
 /* Number of kernels this handle has launched since it was created (a host
- * counter: it costs nothing on the device and does not synchronise). */
+ * counter: it costs nothing on the device and does not synchronise).
+ * (Library plumbing: the pages have no counterpart.) */
 MOE_API moe_status_t moe_get_launch_count(moe_handle_t h, uint64_t* launches);
 
-/* Static description of a status code. */
+/* Time limit, in nanoseconds, of the bounded waits in the main loops of the
+ * grouped-GEMM kernels this handle launches from now on (default 2 s).  A
+ * wait that runs out records MOE_ERR_TIMEOUT in the status word; the kernel
+ * then waits for its own copies and MMAs in flight (those drain waits keep
+ * the 2 s bound), frees its tensor memory and returns, so the context stays
+ * usable.  ns = 0 makes every such wait give up unless its first test finds
+ * it complete: a test uses that to check the timeout path without faulting
+ * the GPU.  Host-only; launches nothing.
+ * (Library plumbing: the pages have no counterpart.) */
+MOE_API moe_status_t moe_set_wait_limit(moe_handle_t h, uint64_t ns);
+
+/* Static description of a status code.
+ * (Library plumbing: the pages have no counterpart.) */
 MOE_API const char* moe_status_string(moe_status_t s);
 
 #ifdef __cplusplus

@@ -57,6 +57,7 @@ SIGNATURES = {
     "moe_mxfp8_quantize": [P, P, c_int64, c_int64, c_int, P, P, P],
     "moe_get_status": [P, ctypes.POINTER(c_int)],
     "moe_get_launch_count": [P, ctypes.POINTER(ctypes.c_uint64)],
+    "moe_set_wait_limit": [P, ctypes.c_uint64],
     "moe_status_string": [c_int],
 }
 

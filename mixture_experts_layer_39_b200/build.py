@@ -35,6 +35,19 @@ def _headers():
     return glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(ROOT, "include", "*.h"))
 
 
+STAMP = os.path.join(BUILD, "flags.txt")
+
+
+def _flags_stamp():
+    """The compiler and flags the objects are built with: objects built with
+    another compiler or other flags are stale whatever their times."""
+    try:
+        ver = subprocess.run([NVCC, "--version"], capture_output=True, text=True).stdout.strip()
+    except OSError:
+        ver = "nvcc not found"
+    return "\n".join([NVCC, ver, *FLAGS]) + "\n"
+
+
 def _stale(obj, src, headers):
     if not os.path.exists(obj):
         return True
@@ -55,6 +68,9 @@ def build(jobs: int = 8, force: bool = False, verbose: bool = False) -> str:
     headers = _headers()
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     objs = [os.path.join(BUILD, os.path.basename(s)[:-3] + ".o") for s in sources]
+    stamp = _flags_stamp()
+    if not os.path.exists(STAMP) or open(STAMP).read() != stamp:
+        force = True
     todo = [(s, o) for s, o in zip(sources, objs) if force or _stale(o, s, headers)]
     if todo:
         with cf.ThreadPoolExecutor(max_workers=jobs) as ex:
@@ -70,6 +86,8 @@ def build(jobs: int = 8, force: bool = False, verbose: bool = False) -> str:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
         if verbose:
             print("linked", os.path.relpath(LIB, ROOT))
+    with open(STAMP, "w") as fh:
+        fh.write(stamp)
     return LIB
 
 

@@ -116,6 +116,49 @@ def test_every_entry_point_is_documented():
         assert before and before[-1].rstrip().endswith("*/"), m.group(1)
 
 
+PAGES = re.compile(r"Olmo-core 3 introduction page|discosf\.com article|vibecoding\.ru news item"
+                   r"|bigchange\.ai article")
+NO_COUNTERPART = re.compile(r"the pages have no counterpart|The pages describe no such call")
+
+
+def _blocks():
+    """(name, comment block) of every declaration in include/moe.h."""
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    out = []
+    for m in re.finditer(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text):
+        head = text[:m.start()]
+        end = head.rstrip().rfind("*/")
+        start = head.rfind("/*", 0, end)
+        lines = [ln.strip().lstrip("/*").strip() for ln in head[start:end].splitlines()]
+        out.append((m.group(1), " ".join(" ".join(lines).split())))
+    return out
+
+
+def test_every_step_call_cites_its_passage():
+    """Each call that runs a step of the layer names the page and section it
+    follows; each call with no counterpart on the pages (handle plumbing, the
+    no-workspace permute, the wait limit) says so."""
+    for name, block in _blocks():
+        if NO_COUNTERPART.search(block):
+            continue
+        assert PAGES.search(block), f"{name}: no page/section cited in its comment block"
+
+
+def test_binding_checks_dtypes():
+    """The binding refuses a tensor whose element type differs from the one
+    the header states, before any pointer reaches the library."""
+    import torch
+    from mixture_experts_layer_39_b200 import ops
+
+    class _H:
+        device = 0
+    with pytest.raises(TypeError, match="bfloat16"):
+        ops._arg(_H(), torch.zeros(4, dtype=torch.float32), ops.BF16, "x")
+    with pytest.raises(TypeError, match="int32"):
+        ops._arg(_H(), torch.zeros(4, dtype=torch.int64), ops.I32, "topk_idx")
+    assert ops._arg(_H(), None, ops.F32, "bias") is None
+
+
 def test_binding_refuses_strided_and_host_tensors():
     """The binding passes raw pointers; a layout it cannot express is an
     error before any call into the library."""
