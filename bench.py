@@ -47,6 +47,12 @@ def parse_args():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-ratio", action="store_true", help="skip the E=128 vs E=8 measurement")
     ap.add_argument("--no-mxfp8", action="store_true", help="skip the MXFP8 workload measurement")
+    ap.add_argument("--no-skew", action="store_true",
+                    help="skip the skewed-routing workload measurement")
+    ap.add_argument("--api-trace", metavar="JSON",
+                    help="instead of timing: trace --steps eager steps of the workload with the "
+                         "CUDA profiler (CUPTI, through torch.profiler) and write the per-step "
+                         "counts of kernels, copies and synchronising API calls to JSON")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the layer variants (load-balancing loss, ...) on the main workload")
     ap.add_argument("--dtype", choices=["bf16", "mxfp8"], default="bf16",
@@ -421,6 +427,9 @@ def run_ours(args):
     ratio = None
     if not args.no_ratio and cfg.name == "e8":
         ratio = bench_cfg(CONFIGS["e128"], args.steps, args.warmup, False)
+    skew = None
+    if not args.no_skew and cfg.name == "e8":
+        skew = bench_cfg(CONFIGS["skew"], args.steps, args.warmup, False)
     mx = mx_bf16 = None
     if not args.no_mxfp8 and cfg.name == "e8":
         mx = bench_cfg(CONFIGS["mxfp8"], args.steps, args.warmup, False, dtype="mxfp8")
@@ -473,6 +482,19 @@ def run_ours(args):
         line["e128"] = {"value": r_value, "unit": UNIT, "vs_e8": r_value / value,
                         "grouped_gemm_tflops": CONFIGS["e128"].gemm_flops_fwd_bwd()
                         / (statistics.mean(ratio["gemm_ms"]) / 1e3) / 1e12}
+    if skew is not None:
+        sc = CONFIGS["skew"]
+        sk_counts = skew["counts"]
+        line["skew"] = {
+            "workload": f"skew: T={sc.T} d_model={sc.d} d_ff={sc.f} E={sc.E} top_k={sc.k}, router "
+                        "bias 2*ln(1/(e+1)), dropless (no capacity cap)",
+            "value": sc.T * K * ws / (skew["total_ms"] / 1e3), "unit": UNIT,
+            "ms_per_step": skew["total_ms"] / K,
+            "grouped_gemm_tflops": sc.gemm_flops_fwd_bwd()
+            / (statistics.mean(skew["gemm_ms"]) / 1e3) / 1e12,
+            "routing": {"max_over_mean_load": float(sk_counts.max() / sk_counts.mean()),
+                        "max_count": int(sk_counts.max()), "mean_count": float(sk_counts.mean()),
+                        "zero_experts": int((sk_counts == 0).sum())}}
     if variants:
         base_ms = main["total_ms"] / K
         line["variants"] = {}
@@ -528,6 +550,82 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------------ API trace
+SYNC_CALLS = ("Synchronize", "cudaMemcpy", "cuMemcpy", "cudaMemset", "cuMemset",
+              "cudaMalloc", "cuMemAlloc", "cudaFree", "cuMemFree", "cudaStreamQuery",
+              "cudaEventQuery")
+
+
+def run_api_trace(args):
+    """Eager steps of the layer under the CUDA profiler (CUPTI activity
+    records through torch.profiler).  For every step, between its first and
+    last host call: the runtime and driver API calls by name, the calls that
+    copy, allocate or wait (SYNC_CALLS), and on the device timeline the
+    kernels, copies and memsets the step's calls caused."""
+    import torch
+    from torch.profiler import ProfilerActivity, profile, record_function
+    from mixture_experts_layer_39_b200.inputs import CONFIGS, make_inputs
+    from mixture_experts_layer_39_b200.layer import MoELayer
+
+    cfg = CONFIGS[args.workload]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    g = make_inputs(cfg, seed=0, device=dev)
+    L = MoELayer(cfg.T, cfg.d, cfg.f, cfg.E, cfg.k, device=dev, dtype=args.dtype)
+    step = lambda: L.step(g["x"], g["w_r"], g["w_gu"], g["w_d"], g["dy"], g["bias"], g["route"])
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    n0 = L.handle.launch_count()
+    with profile(activities=[ProfilerActivity.CPU, ProfilerActivity.CUDA]) as prof:
+        for i in range(args.steps):
+            with record_function(f"moe_layer_step_{i}"):
+                step()
+        torch.cuda.synchronize(dev)
+    launches = (L.handle.launch_count() - n0) // max(1, args.steps)
+    fd, path = tempfile.mkstemp(suffix=".json")
+    os.close(fd)
+    prof.export_chrome_trace(path)
+    with open(path) as fh:
+        trace = json.load(fh)
+    os.unlink(path)
+    ev = [e for e in trace.get("traceEvents", []) if e.get("ph") == "X"]
+    steps = sorted((e for e in ev if e.get("cat") == "user_annotation"
+                    and e.get("name", "").startswith("moe_layer_step_")), key=lambda e: e["ts"])
+    api = [e for e in ev if e.get("cat") in ("cuda_runtime", "cuda_driver")]
+    dev_ev = [e for e in ev if e.get("cat") in ("kernel", "gpu_memcpy", "gpu_memset")]
+    per_step = []
+    for sev in steps:
+        t0, t1 = sev["ts"], sev["ts"] + sev["dur"]
+        calls = [e for e in api if t0 <= e["ts"] <= t1]
+        corr = {e.get("args", {}).get("correlation") for e in calls}
+        caused = [e for e in dev_ev if e.get("args", {}).get("correlation") in corr]
+        names = {}
+        for e in calls:
+            names[e["name"]] = names.get(e["name"], 0) + 1
+        sync = {n: c for n, c in names.items() if any(k in n for k in SYNC_CALLS)
+                and "Async" not in n}
+        per_step.append({
+            "api_calls": names,
+            "sync_or_alloc_calls": sync,
+            "async_copy_calls": {n: c for n, c in names.items() if "Memcpy" in n and "Async" in n},
+            "device_kernels": sum(1 for e in caused if e["cat"] == "kernel"),
+            "device_copies": [e["name"] for e in caused if e["cat"] == "gpu_memcpy"],
+            "device_memsets": sum(1 for e in caused if e["cat"] == "gpu_memset"),
+            "kernel_names": sorted({e["name"].split("(")[0][:80] for e in caused
+                                    if e["cat"] == "kernel"}),
+        })
+    out = {"workload": cfg.name, "dtype": args.dtype, "steps": args.steps, "warmup": args.warmup,
+           "tool": f"torch.profiler (Kineto/CUPTI) {torch.__version__}", "per_step": per_step,
+           "library_launches_per_step": launches}
+    with open(args.api_trace, "w") as fh:
+        json.dump(out, fh, indent=1)
+    print(json.dumps({"api_trace": args.api_trace,
+                      "steps": [{"kernels": p["device_kernels"], "copies": len(p["device_copies"]),
+                                 "sync_or_alloc": sum(p["sync_or_alloc_calls"].values())}
+                                for p in per_step]}), flush=True)
+
+
 # ------------------------------------------------------------------ reference arm
 def run_reference(args):
     """The oracle, as it stands, on the host cores: each step is the layer's
@@ -564,6 +662,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.api_trace:
+        run_api_trace(args)
     else:
         run_ours(args)
 

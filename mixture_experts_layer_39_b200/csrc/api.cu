@@ -32,6 +32,15 @@ bool pair_tiles(const moe_shape_t* s) {
   return static_cast<int64_t>(s->T) * s->top_k >= 1536ll * s->n_experts;
 }
 
+moe::GemmCtx gemm_ctx(const moe_context* h, bool pair_m) {
+  moe::GemmCtx c;
+  c.num_sms = h->num_sms;
+  c.ctl = h->ctl;
+  c.pair_m = pair_m;
+  c.wait_ns = h->wait_ns;
+  return c;
+}
+
 // Router backward workspace layout.
 struct RouterBwdWs {
   size_t dl, db_part, part, total;
@@ -208,7 +217,7 @@ moe_status_t moe_router_topk(moe_handle_t h, const moe_shape_t* s, const void* x
     h->launches += 1;
     return cuda_status(moe::launch_router_fused(
         static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_router), bias,
-        route_in, T, d, E, k, renorm, topk_idx, topk_w, probs, logits, h->ctl, st));
+        route_in, T, d, E, k, renorm, topk_idx, topk_w, probs, logits, h->ctl, h->num_sms, st));
   }
   // the GEMM writes whole 128-column tiles: straight into `logits` when E
   // fills them, else into the workspace, from which the softmax copies
@@ -221,7 +230,7 @@ moe_status_t moe_router_topk(moe_handle_t h, const moe_shape_t* s, const void* x
   } else if (!aligned(lg, 16)) {
     return MOE_ERR_INVALID_ARG;
   }
-  moe::GemmCtx c{h->num_sms, h->ctl};
+  const moe::GemmCtx c = gemm_ctx(h, false);
   h->launches += 2;
   MOE_TRY(moe::gemm_router_logits(c, x, w_router, lg, T, d, E, ld, st));
   return cuda_status(moe::launch_softmax_topk(lg, ld, bias, route_in, T, E, k, renorm, topk_idx,
@@ -284,7 +293,7 @@ moe_status_t moe_grouped_swiglu_fwd_gather(moe_handle_t h, const moe_shape_t* s,
   const int64_t m_cap = max_rows(s);
   auto st = static_cast<cudaStream_t>(stream);
   MOE_GUARD(h);
-  moe::GemmCtx c{h->num_sms, h->ctl, pair_tiles(s)};
+  const moe::GemmCtx c = gemm_ctx(h, pair_tiles(s));
   h->launches += 2;
   MOE_TRY(moe::gemm_fwd_gate_up_gather(c, x, s->T, row_src, offsets, w_gu, au, hbuf, E, d, f,
                                        m_cap, st));
@@ -302,7 +311,7 @@ moe_status_t moe_grouped_swiglu_recompute_gather(moe_handle_t h, const moe_shape
     if (!aligned(p, 16)) return MOE_ERR_INVALID_ARG;
   auto st = static_cast<cudaStream_t>(stream);
   MOE_GUARD(h);
-  moe::GemmCtx c{h->num_sms, h->ctl, pair_tiles(s)};
+  const moe::GemmCtx c = gemm_ctx(h, pair_tiles(s));
   h->launches += 1;
   return moe::gemm_fwd_gate_up_gather(c, x, s->T, row_src, offsets, w_gu, au, hbuf, s->n_experts,
                                       s->d_model, s->d_ff, max_rows(s), st);
@@ -328,7 +337,7 @@ moe_status_t moe_grouped_swiglu_bwd_gather(moe_handle_t h, const moe_shape_t* s,
   const int64_t m_cap = max_rows(s);
   auto st = static_cast<cudaStream_t>(stream);
   MOE_GUARD(h);
-  moe::GemmCtx c{h->num_sms, h->ctl, pair_tiles(s)};
+  const moe::GemmCtx c = gemm_ctx(h, pair_tiles(s));
   h->launches += 4;
   MOE_TRY(moe::gemm_dgrad_down_swiglu(c, do_perm, offsets, w_down, au, dau, E, d, f, m_cap, st));
   MOE_TRY(moe::gemm_wgrad_down(c, do_perm, hbuf, offsets, dw_down, E, d, f, m_cap, st));
@@ -350,14 +359,14 @@ moe_status_t moe_grouped_swiglu_fwd(moe_handle_t h, const moe_shape_t* s, const 
   const int64_t m_cap = max_rows(s);
   auto st = static_cast<cudaStream_t>(stream);
   MOE_GUARD(h);
-  moe::GemmCtx c{h->num_sms, h->ctl, pair_tiles(s)};
+  const moe::GemmCtx c = gemm_ctx(h, pair_tiles(s));
   if (s->dtype == MOE_DTYPE_MXFP8) {
     MOE_TRY(check_ws(h, s, ws, ws_bytes));
     const MxWs L = mx_layout(s);
     auto* b = static_cast<uint8_t*>(ws);
     auto bf = [](const void* p) { return static_cast<const __nv_bfloat16*>(p); };
     auto rows = [&](const void* in, int64_t r, int64_t cols, size_t q, size_t sc) {
-      return cuda_status(moe::launch_mxfp8_quantize(bf(in), r, cols, 1, b + q, b + sc, st));
+      return cuda_status(moe::launch_mxfp8_quantize_atoms(bf(in), r, cols, b + q, b + sc, st));
     };
     h->launches += 6;
     MOE_TRY(rows(x_perm, m_cap, d, L.xq, L.xs));
@@ -386,7 +395,7 @@ moe_status_t moe_grouped_swiglu_recompute(moe_handle_t h, const moe_shape_t* s, 
   const int64_t m_cap = max_rows(s);
   auto st = static_cast<cudaStream_t>(stream);
   MOE_GUARD(h);
-  moe::GemmCtx c{h->num_sms, h->ctl, pair_tiles(s)};
+  const moe::GemmCtx c = gemm_ctx(h, pair_tiles(s));
   if (s->dtype == MOE_DTYPE_MXFP8) {
     // the forward's operand quantisation and gate/up GEMM, again
     MOE_TRY(check_ws(h, s, ws, ws_bytes));
@@ -394,9 +403,9 @@ moe_status_t moe_grouped_swiglu_recompute(moe_handle_t h, const moe_shape_t* s, 
     auto* b = static_cast<uint8_t*>(ws);
     auto bf = [](const void* p) { return static_cast<const __nv_bfloat16*>(p); };
     h->launches += 3;
-    MOE_TRY(cuda_status(moe::launch_mxfp8_quantize(bf(x_perm), m_cap, d, 1, b + L.xq, b + L.xs, st)));
+    MOE_TRY(cuda_status(moe::launch_mxfp8_quantize_atoms(bf(x_perm), m_cap, d, b + L.xq, b + L.xs, st)));
     MOE_TRY(cuda_status(
-        moe::launch_mxfp8_quantize(bf(w_gu), 2ll * E * f, d, 1, b + L.wguq, b + L.wgus, st)));
+        moe::launch_mxfp8_quantize_atoms(bf(w_gu), 2ll * E * f, d, b + L.wguq, b + L.wgus, st)));
     return moe::gemm_mx_fwd_gate_up(c, {b + L.xq, b + L.xs}, offsets, {b + L.wguq, b + L.wgus}, au,
                                     hbuf, E, d, f, m_cap, st);
   }
@@ -453,14 +462,14 @@ moe_status_t moe_grouped_swiglu_bwd(moe_handle_t h, const moe_shape_t* s, const 
   const int64_t m_cap = max_rows(s);
   auto st = static_cast<cudaStream_t>(stream);
   MOE_GUARD(h);
-  moe::GemmCtx c{h->num_sms, h->ctl, pair_tiles(s)};
+  const moe::GemmCtx c = gemm_ctx(h, pair_tiles(s));
   if (s->dtype == MOE_DTYPE_MXFP8) {
     MOE_TRY(check_ws(h, s, ws, ws_bytes));
     const MxWs L = mx_layout(s);
     auto* b = static_cast<uint8_t*>(ws);
     auto bf = [](const void* p) { return static_cast<const __nv_bfloat16*>(p); };
     auto rows = [&](const void* in, int64_t r, int64_t cols, size_t q, size_t sc) {
-      return cuda_status(moe::launch_mxfp8_quantize(bf(in), r, cols, 1, b + q, b + sc, st));
+      return cuda_status(moe::launch_mxfp8_quantize_atoms(bf(in), r, cols, b + q, b + sc, st));
     };
     auto cols_t = [&](const void* in, int64_t r, int64_t cols, int64_t group, size_t q, size_t sc) {
       return cuda_status(moe::launch_mxfp8_quantize_cols_t(bf(in), r, cols, group, b + q, b + sc, st));
@@ -509,7 +518,7 @@ moe_status_t moe_shared_expert_fwd(moe_handle_t h, const moe_shape_t* s, const v
   const moe_shape_t one{s->T, s->d_model, s->d_ff, 1, 1, MOE_DTYPE_BF16, 0};
   auto st = static_cast<cudaStream_t>(stream);
   MOE_GUARD(h);
-  moe::GemmCtx c{h->num_sms, h->ctl, pair_tiles(&one)};
+  const moe::GemmCtx c = gemm_ctx(h, pair_tiles(&one));
   h->launches += 2;
   MOE_TRY(moe::gemm_fwd_gate_up(c, x, nullptr, w_gu_s, au_s, h_s, 1, s->d_model, s->d_ff, s->T, st));
   return moe::gemm_fwd_down(c, h_s, nullptr, w_d_s, o_s, 1, s->d_model, s->d_ff, s->T, st);
@@ -531,7 +540,7 @@ moe_status_t moe_shared_expert_bwd(moe_handle_t h, const moe_shape_t* s, const v
   const int d = s->d_model, f = s->d_ff, T = s->T;
   auto st = static_cast<cudaStream_t>(stream);
   MOE_GUARD(h);
-  moe::GemmCtx c{h->num_sms, h->ctl, pair_tiles(&one)};
+  const moe::GemmCtx c = gemm_ctx(h, pair_tiles(&one));
   h->launches += 4;
   MOE_TRY(moe::gemm_dgrad_down_swiglu(c, dy, nullptr, w_d_s, au_s, dau_s, 1, d, f, T, st));
   MOE_TRY(moe::gemm_wgrad_down(c, dy, h_s, nullptr, dw_d_s, 1, d, f, T, st));
@@ -623,7 +632,7 @@ moe_status_t moe_router_topk_bwd(moe_handle_t h, const moe_shape_t* s, const flo
   MOE_TRY(cuda_status(moe::launch_router_bwd_dl(d_topk_w, probs, topk_idx, d_probs_aux, wb, T, d, E,
                                                 k, renorm, false, nullptr, dl, ld, nullptr, db_part,
                                                 L.nblocks, h->ctl, st)));
-  moe::GemmCtx c{h->num_sms, h->ctl};
+  const moe::GemmCtx c = gemm_ctx(h, false);
   if (want_dx) MOE_TRY(moe::gemm_router_dx(c, dl, ld, w_router, dx_router, T, d, E, st));
   MOE_TRY(moe::gemm_router_dw_partial(c, dl, ld, x, part, T, d, E, L.n_part, L.group_len, st));
   return cuda_status(moe::launch_reduce_dw(part, L.n_part, static_cast<int64_t>(E) * d, db_part,
@@ -683,6 +692,12 @@ moe_status_t moe_get_status(moe_handle_t h, int* device_status) {
   if (cudaMemset(h->ctl, 0, sizeof(c)) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
   *device_status = c.status;
+  return MOE_OK;
+}
+
+moe_status_t moe_set_wait_limit(moe_handle_t h, uint64_t ns) {
+  if (h == nullptr) return MOE_ERR_INVALID_ARG;
+  h->wait_ns = ns;
   return MOE_OK;
 }
 

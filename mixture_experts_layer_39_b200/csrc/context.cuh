@@ -8,6 +8,7 @@ struct moe_context {
   int num_sms;
   moe::DeviceCtl* ctl;    // device status word
   uint64_t launches = 0;  // kernels launched through this handle
+  uint64_t wait_ns = 2000000000ull;  // GEMM main-loop wait limit (moe_set_wait_limit)
 };
 
 namespace moe {

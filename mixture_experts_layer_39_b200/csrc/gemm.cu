@@ -64,12 +64,29 @@ bool tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 5-D map over MXFP8 scales in the tensor cores' atom order: 512-byte atoms
+// (128 MN indices x 128 contraction elements) indexed (K block, MN block,
+// group); one box is one atom.  Atoms past an operand's MN extent read as
+// zeros (their rows of the operand tile are zero fill too).
+bool tmap_sf(CUtensorMap* m, const void* base, uint64_t n_kb, uint64_t n_rb, uint64_t groups) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[5] = {128, 4, n_kb, n_rb, groups};
+  cuuint64_t strides[4] = {128, 512, 512 * n_kb, 512 * n_kb * n_rb};
+  cuuint32_t box[5] = {128, 4, 1, 1, 1};
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 constexpr size_t kMaxDynSmem = 227 * 1024;  // per block on sm_100
 
 template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, int STAGES, bool FP8, bool PAIR,
           bool GATHER>
-moe_status_t launch_stages(const CUtensorMap& a, const CUtensorMap& b, const tc::GemmArgs& args,
-                           int grid, cudaStream_t st) {
+moe_status_t launch_stages(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& sa,
+                           const CUtensorMap& sb, const tc::GemmArgs& args, int grid,
+                           cudaStream_t st) {
   auto kern = tc::grouped_gemm_kernel<BN, A_MN, B_MN, EPI, KGROUP, STAGES, FP8, PAIR, GATHER>;
   const size_t smem = tc::SmemPlan<BN, STAGES, EPI, FP8, PAIR>::bytes(args.n_groups);
   static size_t configured = 0;  // largest size this instantiation was opened for
@@ -97,9 +114,9 @@ moe_status_t launch_stages(const CUtensorMap& a, const CUtensorMap& b, const tc:
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, kern, a, b, args) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, kern, a, b, sa, sb, args) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   } else {
-    return launch_pdl(kern, dim3(grid), dim3(tc::kThreads), smem, st, a, b, args) == cudaSuccess
+    return launch_pdl(kern, dim3(grid), dim3(tc::kThreads), smem, st, a, b, sa, sb, args) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
   }
@@ -107,24 +124,28 @@ moe_status_t launch_stages(const CUtensorMap& a, const CUtensorMap& b, const tc:
 
 // Ring depth: as many stages as fit beside the epilogue buffers.  A stage is
 // 48 KB for single-CTA 128 x 256 tiles and for wide pairs, 32 KB for 256 x 256
-// pairs and 16 KB (+1 KB of scale atoms) for MXFP8 128 x 128 tiles.  The
-// SwiGLU backward's landing buffers take 16 KB more; with more than ~440
-// experts the tile table no longer fits beside a sixth pair stage, and the
-// launch falls back to one stage fewer.
+// pairs (bf16 or MXFP8; MXFP8 adds 1.5 KB of scale atoms).  The SwiGLU
+// backward's landing buffers take 16 KB more; with more than ~440 experts the
+// tile table no longer fits beside a sixth pair stage, and the launch falls
+// back to one stage fewer.  sa, sb: the MXFP8 scale maps (unused otherwise).
 template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, bool FP8 = false, bool PAIR = false,
           bool GATHER = false>
 moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const tc::GemmArgs& args, int grid,
-                    cudaStream_t st) {
+                    cudaStream_t st, const CUtensorMap* sa = nullptr,
+                    const CUtensorMap* sb = nullptr) {
+  const CUtensorMap& sfa = sa != nullptr ? *sa : a;
+  const CUtensorMap& sfb = sb != nullptr ? *sb : b;
   constexpr bool BWD = EPI == tc::EPI_SWIGLU_BWD;
   constexpr int STAGES = FP8    ? (BWD ? 5 : 6)
                          : PAIR ? (BN == 512 ? (BWD ? 3 : 4) : 6)
                                 : (BN == 256 ? 4 : 6);
-  if constexpr (BWD && !FP8) {
+  if constexpr (BWD || FP8) {
     if (tc::SmemPlan<BN, STAGES, EPI, FP8, PAIR>::bytes(args.n_groups) > kMaxDynSmem)
-      return launch_stages<BN, A_MN, B_MN, EPI, KGROUP, STAGES - 1, FP8, PAIR, GATHER>(a, b, args,
-                                                                                      grid, st);
+      return launch_stages<BN, A_MN, B_MN, EPI, KGROUP, STAGES - 1, FP8, PAIR, GATHER>(
+          a, b, sfa, sfb, args, grid, st);
   }
-  return launch_stages<BN, A_MN, B_MN, EPI, KGROUP, STAGES, FP8, PAIR, GATHER>(a, b, args, grid, st);
+  return launch_stages<BN, A_MN, B_MN, EPI, KGROUP, STAGES, FP8, PAIR, GATHER>(a, b, sfa, sfb, args,
+                                                                              grid, st);
 }
 
 // Weight gradients run 256 x 512 pair tiles ("wide") when the experts'
@@ -146,6 +167,7 @@ bool wide_wgrad(int num_sms, int64_t E, int64_t M, int64_t N, int64_t rows) {
 tc::GemmArgs base_args(const GemmCtx& c) {
   tc::GemmArgs a{};
   a.ctl = c.ctl;
+  a.wait_ns = c.wait_ns;
   return a;
 }
 
@@ -430,111 +452,108 @@ moe_status_t gemm_router_dw_partial(const GemmCtx& c, const void* dl_bf16, int l
 }
 
 // ------------------------------------------------------------------ MXFP8
-// Operands are E4M3 codes with E8M0 scales stored [MN index][K/32]; tiles are
-// 128 x 128 and each stage carries 128 contraction elements (128 bytes).
+// Operands are E4M3 codes with E8M0 scales in atom order (see tmap_sf); the
+// GEMMs run 256 x 256 CTA-pair tiles with 128 contraction elements (128
+// bytes) per stage.
 
-moe_status_t gemm_mx_fwd_gate_up(const GemmCtx& c, const MxOperand& x, const int32_t* offsets,
-                                 const MxOperand& w_gu, void* au, void* h, int E, int d, int f,
-                                 int64_t m_cap, cudaStream_t st) {
-  CUtensorMap ta, tb;
-  if (!tmap_2d(&ta, x.q, d, m_cap, d, 128, 128, true)) return MOE_ERR_CUDA;
-  if (!tmap_3d(&tb, w_gu.q, d, 2ull * f, E, d, 2ull * f * d, 128, 64, true)) return MOE_ERR_CUDA;
+namespace {
+
+tc::GemmArgs mx_m_grouped(const GemmCtx& c, const int32_t* offsets, int E, int64_t N, int K,
+                          int64_t m_cap) {
   tc::GemmArgs a = base_args(c);
-  set_n(a, 2ll * f, 128);  // 64 columns of A and of U per tile
-  a.k_blocks = d / 128;
+  set_n(a, N, 256);
+  a.k_blocks = K / 128;
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
   a.uniform_len = static_cast<int>(m_cap);  // one group of m_cap rows when offsets is null
   a.m_cap = m_cap;
+  return a;
+}
+
+}  // namespace
+
+moe_status_t gemm_mx_fwd_gate_up(const GemmCtx& c, const MxOperand& x, const int32_t* offsets,
+                                 const MxOperand& w_gu, void* au, void* h, int E, int d, int f,
+                                 int64_t m_cap, cudaStream_t st) {
+  CUtensorMap ta, tb, tsa, tsb;
+  if (!tmap_2d(&ta, x.q, d, m_cap, d, 128, 128, true)) return MOE_ERR_CUDA;
+  if (!tmap_3d(&tb, w_gu.q, d, 2ull * f, E, d, 2ull * f * d, 128, 128, true)) return MOE_ERR_CUDA;
+  if (!tmap_sf(&tsa, x.s, d / 128, m_cap / 128, 1)) return MOE_ERR_CUDA;
+  if (!tmap_sf(&tsb, w_gu.s, d / 128, 2ull * f / 128, E)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = mx_m_grouped(c, offsets, E, 2ll * f, d, m_cap);  // 128 of A and of U per tile
   a.out = au;
   a.ldo = 2ll * f;
   a.out2 = h;
   a.ldo2 = f;
   a.f = f;
-  a.sfa = x.s; a.ld_sfa = d / 32; a.sfa_rows = m_cap;
-  a.sfb = w_gu.s; a.ld_sfb = d / 32; a.sfb_rows = 2ll * f; a.sfb_gstride = 2ll * f * (d / 32);
-  return launch<128, false, false, tc::EPI_SWIGLU_FWD, false, true>(ta, tb, a, c.num_sms, st);
+  return launch<256, false, false, tc::EPI_SWIGLU_FWD, false, true, true>(ta, tb, a, c.num_sms, st,
+                                                                        &tsa, &tsb);
 }
 
 moe_status_t gemm_mx_fwd_down(const GemmCtx& c, const MxOperand& h, const int32_t* offsets,
                               const MxOperand& w_d, void* o_perm, int E, int d, int f,
                               int64_t m_cap, cudaStream_t st) {
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tsa, tsb;
   if (!tmap_2d(&ta, h.q, f, m_cap, f, 128, 128, true)) return MOE_ERR_CUDA;
   if (!tmap_3d(&tb, w_d.q, f, d, E, f, 1ull * d * f, 128, 128, true)) return MOE_ERR_CUDA;
-  tc::GemmArgs a = base_args(c);
-  set_n(a, d, 128);
-  a.k_blocks = f / 128;
-  a.n_groups = E;
-  a.offsets = offsets;
-  a.total_len = static_cast<int>(m_cap);
-  a.uniform_len = static_cast<int>(m_cap);  // one group of m_cap rows when offsets is null
-  a.m_cap = m_cap;
+  if (!tmap_sf(&tsa, h.s, f / 128, m_cap / 128, 1)) return MOE_ERR_CUDA;
+  if (!tmap_sf(&tsb, w_d.s, f / 128, d / 128, E)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = mx_m_grouped(c, offsets, E, d, f, m_cap);
   a.out = o_perm;
   a.ldo = d;
-  a.sfa = h.s; a.ld_sfa = f / 32; a.sfa_rows = m_cap;
-  a.sfb = w_d.s; a.ld_sfb = f / 32; a.sfb_rows = d; a.sfb_gstride = 1ll * d * (f / 32);
-  return launch<128, false, false, tc::EPI_BF16, false, true>(ta, tb, a, c.num_sms, st);
+  return launch<256, false, false, tc::EPI_BF16, false, true, true>(ta, tb, a, c.num_sms, st, &tsa,
+                                                                  &tsb);
 }
 
 moe_status_t gemm_mx_dgrad_down_swiglu(const GemmCtx& c, const MxOperand& dO, const int32_t* offsets,
                                        const MxOperand& w_d_col, const void* au, void* dau, int E,
                                        int d, int f, int64_t m_cap, cudaStream_t st) {
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tsa, tsb;
   if (!tmap_2d(&ta, dO.q, d, m_cap, d, 128, 128, true)) return MOE_ERR_CUDA;
   // W_d[e] is [d (contraction), f (output)]: N-major, quantised along d
   if (!tmap_3d(&tb, w_d_col.q, f, d, E, f, 1ull * d * f, 128, 128, true)) return MOE_ERR_CUDA;
-  tc::GemmArgs a = base_args(c);
-  set_n(a, f, 128);
-  a.k_blocks = d / 128;
-  a.n_groups = E;
-  a.offsets = offsets;
-  a.total_len = static_cast<int>(m_cap);
-  a.uniform_len = static_cast<int>(m_cap);  // one group of m_cap rows when offsets is null
-  a.m_cap = m_cap;
+  if (!tmap_sf(&tsa, dO.s, d / 128, m_cap / 128, 1)) return MOE_ERR_CUDA;
+  if (!tmap_sf(&tsb, w_d_col.s, d / 128, f / 128, E)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = mx_m_grouped(c, offsets, E, f, d, m_cap);
   a.out = dau;
   a.ldo = 2ll * f;
   a.aux = static_cast<const __nv_bfloat16*>(au);
   a.ld_aux = 2ll * f;
   a.f = f;
-  a.sfa = dO.s; a.ld_sfa = d / 32; a.sfa_rows = m_cap;
-  a.sfb = w_d_col.s; a.ld_sfb = d / 32; a.sfb_rows = f; a.sfb_gstride = 1ll * f * (d / 32);
-  return launch<128, false, true, tc::EPI_SWIGLU_BWD, false, true>(ta, tb, a, c.num_sms, st);
+  return launch<256, false, true, tc::EPI_SWIGLU_BWD, false, true, true>(ta, tb, a, c.num_sms, st,
+                                                                       &tsa, &tsb);
 }
 
 moe_status_t gemm_mx_dgrad_gate_up(const GemmCtx& c, const MxOperand& dau, const int32_t* offsets,
                                    const MxOperand& w_gu_col, void* dx_perm, int E, int d, int f,
                                    int64_t m_cap, cudaStream_t st) {
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tsa, tsb;
   if (!tmap_2d(&ta, dau.q, 2ull * f, m_cap, 2ull * f, 128, 128, true)) return MOE_ERR_CUDA;
+  // W_gu[e] is [2f (contraction), d (output)]: N-major, quantised along 2f
   if (!tmap_3d(&tb, w_gu_col.q, d, 2ull * f, E, d, 2ull * f * d, 128, 128, true)) return MOE_ERR_CUDA;
-  tc::GemmArgs a = base_args(c);
-  set_n(a, d, 128);
-  a.k_blocks = 2 * f / 128;
-  a.n_groups = E;
-  a.offsets = offsets;
-  a.total_len = static_cast<int>(m_cap);
-  a.uniform_len = static_cast<int>(m_cap);  // one group of m_cap rows when offsets is null
-  a.m_cap = m_cap;
+  if (!tmap_sf(&tsa, dau.s, 2ull * f / 128, m_cap / 128, 1)) return MOE_ERR_CUDA;
+  if (!tmap_sf(&tsb, w_gu_col.s, 2ull * f / 128, d / 128, E)) return MOE_ERR_CUDA;
+  tc::GemmArgs a = mx_m_grouped(c, offsets, E, d, 2 * f, m_cap);
   a.out = dx_perm;
   a.ldo = d;
-  a.sfa = dau.s; a.ld_sfa = 2 * f / 32; a.sfa_rows = m_cap;
-  a.sfb = w_gu_col.s; a.ld_sfb = 2 * f / 32; a.sfb_rows = d; a.sfb_gstride = 1ll * d * (2 * f / 32);
-  return launch<128, false, true, tc::EPI_BF16, false, true>(ta, tb, a, c.num_sms, st);
+  return launch<256, false, true, tc::EPI_BF16, false, true, true>(ta, tb, a, c.num_sms, st, &tsa,
+                                                                 &tsb);
 }
 
 moe_status_t gemm_mx_wgrad(const GemmCtx& c, const MxOperand& a_col, int M, const MxOperand& b_col,
                            int N, const int32_t* offsets, void* dw, int E, int64_t m_cap,
                            cudaStream_t st) {
   // dW[e] (M x N) = A_e^T B_e over e's token rows; both operands are token-major
-  // (MN-major) and quantised along tokens, scales [M or N][m_cap/32]
-  CUtensorMap ta, tb;
+  // (MN-major) and quantised along tokens (scale atoms over 128 tokens)
+  CUtensorMap ta, tb, tsa, tsb;
   if (!tmap_2d(&ta, a_col.q, M, m_cap, M, 128, 128, true)) return MOE_ERR_CUDA;
   if (!tmap_3d(&tb, b_col.q, N, m_cap, 1, N, 1ull * N * m_cap, 128, 128, true)) return MOE_ERR_CUDA;
+  if (!tmap_sf(&tsa, a_col.s, m_cap / 128, M / 128, 1)) return MOE_ERR_CUDA;
+  if (!tmap_sf(&tsb, b_col.s, m_cap / 128, N / 128, 1)) return MOE_ERR_CUDA;
   tc::GemmArgs a = base_args(c);
-  set_n(a, N, 128);
-  set_m(a, M, tc::BM);
+  set_n(a, N, 256);
+  set_m(a, M, 2 * tc::BM);  // CTA pairs: 256-row tiles
   a.n_groups = E;
   a.offsets = offsets;
   a.total_len = static_cast<int>(m_cap);
@@ -542,11 +561,9 @@ moe_status_t gemm_mx_wgrad(const GemmCtx& c, const MxOperand& a_col, int M, cons
   a.out = dw;
   a.ldo = N;
   a.out_gstride = static_cast<int64_t>(M) * N;
-  a.sfa = a_col.s; a.ld_sfa = m_cap / 32; a.sfa_rows = M;
-  a.sfb = b_col.s; a.ld_sfb = m_cap / 32; a.sfb_rows = N; a.sfb_gstride = 0;
   const int64_t tiles = static_cast<int64_t>(E) * a.m_tiles_fixed * a.n_tiles_n;
-  const int grid = static_cast<int>(tiles < c.num_sms ? tiles : c.num_sms);
-  return launch<128, true, true, tc::EPI_BF16, true, true>(ta, tb, a, grid, st);
+  const int grid = static_cast<int>(2 * tiles < c.num_sms ? 2 * tiles : c.num_sms);
+  return launch<256, true, true, tc::EPI_BF16, true, true, true>(ta, tb, a, grid, st, &tsa, &tsb);
 }
 
 }  // namespace moe

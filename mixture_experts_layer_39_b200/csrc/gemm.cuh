@@ -11,6 +11,9 @@ struct GemmCtx {
   // M-grouped bf16 GEMMs run 256-row tiles on CTA pairs (worth it when the
   // experts' row segments are long compared with a tile)
   bool pair_m = false;
+  // time limit of the GEMMs' main-loop waits (the handle's; 0 = give up
+  // unless already complete)
+  uint64_t wait_ns = 2000000000ull;
 };
 
 // An MXFP8 operand: E4M3 codes and E8M0 scales ([MN index][K/32] bytes).

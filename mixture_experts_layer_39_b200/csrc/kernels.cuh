@@ -16,7 +16,7 @@ inline int64_t n_subchunks(int T, int k) { return ceil_div64(static_cast<int64_t
 cudaError_t launch_router_fused(const __nv_bfloat16* x, const __nv_bfloat16* w_r, const float* bias,
                                 const int32_t* route_in, int T, int d, int E, int k, bool renorm,
                                 int32_t* idx, float* w, float* probs, float* logits,
-                                DeviceCtl* ctl, cudaStream_t st);
+                                DeviceCtl* ctl, int num_sms, cudaStream_t st);
 // logits_in has row stride ld_in; logits_out (dense [T, E]) may alias it when ld_in = E
 cudaError_t launch_softmax_topk(const float* logits_in, int ld_in, const float* bias,
                                 const int32_t* route_in, int T, int E, int k, bool renorm,
@@ -91,7 +91,13 @@ cudaError_t launch_reduce_dw(const float* partial, int n_part, int64_t n_w, cons
 // ---- MXFP8
 cudaError_t launch_mxfp8_quantize(const __nv_bfloat16* in, int64_t rows, int64_t cols, int axis,
                                   uint8_t* q, uint8_t* scales, cudaStream_t st);
-// Column-wise (32-row blocks) with scales stored [groups][cols][rows_per_group/32].
+// GEMM operands (scales in the tensor cores' 512-byte atom order; see
+// mxfp8.cu).  Row-wise: [rows, cols] along cols, rows and cols multiples of
+// 128.  Column-wise: 32-row blocks along the rows of each group of
+// rows_per_group rows, the column being the MN index; cols and
+// rows_per_group multiples of 128.
+cudaError_t launch_mxfp8_quantize_atoms(const __nv_bfloat16* in, int64_t rows, int64_t cols,
+                                        uint8_t* q, uint8_t* scales, cudaStream_t st);
 cudaError_t launch_mxfp8_quantize_cols_t(const __nv_bfloat16* in, int64_t rows, int64_t cols,
                                          int64_t rows_per_group, uint8_t* q, uint8_t* scales,
                                          cudaStream_t st);

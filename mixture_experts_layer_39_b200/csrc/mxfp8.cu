@@ -46,9 +46,22 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
       __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
 }
 
-// axis 1: one thread per 32-element block of a row.
+// Byte of the scale of (MN index r, 32-element contraction block kb) in the
+// tensor cores' scale-atom order: atoms of 512 bytes for 128 MN indices x 4
+// blocks (128 contraction elements), atom (r/128, kb/4) at index
+// (r/128) * n_kb4 + kb/4 (n_kb4 = contraction length / 128), and inside an
+// atom byte (r%32)*16 + ((r/32)%4)*4 + kb%4.  The GEMMs copy one atom per
+// stage with one TMA load and hand it to tcgen05.cp unchanged.
+__device__ __forceinline__ int64_t atom_byte(int64_t r, int64_t kb, int64_t n_kb4) {
+  return ((r >> 7) * n_kb4 + (kb >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (kb & 3);
+}
+
+// axis 1: one thread per 32-element block of a row.  Scales go to
+// [rows, cols/32] (atoms = false) or, for the GEMM operands, in atom order
+// (atoms = true; rows and cols multiples of 128).
 __global__ void mx_rowwise_kernel(const uint4* __restrict__ in, int64_t rows, int64_t cols,
-                                  uint4* __restrict__ q, uint8_t* __restrict__ scales) {
+                                  uint4* __restrict__ q, uint8_t* __restrict__ scales,
+                                  bool atoms) {
   pdl_wait();
   pdl_trigger();
   const int64_t nblk = cols / 32;
@@ -80,7 +93,12 @@ __global__ void mx_rowwise_kernel(const uint4* __restrict__ in, int64_t rows, in
     }
     q[b * 2] = make_uint4(p[0], p[1], p[2], p[3]);
     q[b * 2 + 1] = make_uint4(p[4], p[5], p[6], p[7]);
-    scales[b] = static_cast<uint8_t>(e + 127);
+    if (atoms) {
+      const int64_t r = b / nblk;
+      scales[atom_byte(r, b - r * nblk, nblk >> 2)] = static_cast<uint8_t>(e + 127);
+    } else {
+      scales[b] = static_cast<uint8_t>(e + 127);
+    }
   }
 }
 
@@ -89,9 +107,10 @@ __global__ void mx_rowwise_kernel(const uint4* __restrict__ in, int64_t rows, in
 // of the block is one vector load and one vector store of W codes; the two
 // columns of a bf16 pair are converted by one paired E4M3 conversion (each
 // element rounds on its own, so pairing changes no code).  Scales go to
-// [rows/32, cols] (scale_mode 0) or, for the GEMM operand layout, to
-// [groups, cols, rows_per_group/32] (scale_mode 1: a column's scales along
-// the contraction axis are contiguous inside each group of rows).
+// [rows/32, cols] (scale_mode 0) or, for the GEMM operands, per group of
+// rows_per_group rows in atom order with the column as the MN index and the
+// row inside the group as the contraction index (scale_mode 1; cols and
+// rows_per_group multiples of 128).
 template <int W>
 __global__ void mx_colwise_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_t cols,
                                   uint8_t* __restrict__ q, uint8_t* __restrict__ scales,
@@ -157,9 +176,10 @@ __global__ void mx_colwise_kernel(const __nv_bfloat16* __restrict__ in, int64_t 
     } else {
       const int64_t bpg = rows_per_group / 32;  // scale blocks per group
       const int64_t g = rb / bpg, rl = rb - g * bpg;
+      uint8_t* gs = scales + g * cols * bpg;
 #pragma unroll
       for (int c = 0; c < W; ++c)
-        scales[(g * cols + W * cg + c) * bpg + rl] = static_cast<uint8_t>(e[c] + 127);
+        gs[atom_byte(W * cg + c, rl, bpg >> 2)] = static_cast<uint8_t>(e[c] + 127);
     }
   }
 }
@@ -184,16 +204,24 @@ cudaError_t launch_colwise(const __nv_bfloat16* in, int64_t rows, int64_t cols, 
 
 }  // namespace
 
+cudaError_t launch_rowwise(const __nv_bfloat16* in, int64_t rows, int64_t cols, uint8_t* q,
+                           uint8_t* scales, bool atoms, cudaStream_t st) {
+  const int64_t total = rows * (cols / 32);
+  const unsigned grid = static_cast<unsigned>(ceil_div64(total, 256) < 65535 ? ceil_div64(total, 256) : 65535);
+  (void)launch_pdl(mx_rowwise_kernel, grid, 256, 0, st, reinterpret_cast<const uint4*>(in), rows,
+                   cols, reinterpret_cast<uint4*>(q), scales, atoms);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_mxfp8_quantize(const __nv_bfloat16* in, int64_t rows, int64_t cols, int axis,
                                   uint8_t* q, uint8_t* scales, cudaStream_t st) {
-  if (axis == 1) {
-    const int64_t total = rows * (cols / 32);
-    const unsigned grid = static_cast<unsigned>(ceil_div64(total, 256) < 65535 ? ceil_div64(total, 256) : 65535);
-    (void)launch_pdl(mx_rowwise_kernel, grid, 256, 0, st, reinterpret_cast<const uint4*>(in), rows, cols,
-                                            reinterpret_cast<uint4*>(q), scales);
-    return cudaGetLastError();
-  }
+  if (axis == 1) return launch_rowwise(in, rows, cols, q, scales, false, st);
   return launch_colwise(in, rows, cols, q, scales, 0, rows, st);
+}
+
+cudaError_t launch_mxfp8_quantize_atoms(const __nv_bfloat16* in, int64_t rows, int64_t cols,
+                                        uint8_t* q, uint8_t* scales, cudaStream_t st) {
+  return launch_rowwise(in, rows, cols, q, scales, true, st);
 }
 
 cudaError_t launch_mxfp8_quantize_cols_t(const __nv_bfloat16* in, int64_t rows, int64_t cols,

@@ -170,7 +170,10 @@ __global__ void __launch_bounds__(256)
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t tk = static_cast<int64_t>(T) * k;
   if (i < tk) {
-    row_src[__ldg(row_map + i)] = static_cast<int32_t>(i / k);
+    // an entry whose expert id was out of range has row -1 (the rank kernel
+    // skipped it and the histogram recorded MOE_ERR_DEVICE_CHECK): no row
+    const int32_t r = __ldg(row_map + i);
+    if (r >= 0) row_src[r] = static_cast<int32_t>(i / k);
     return;
   }
   const int64_t r = i - tk;

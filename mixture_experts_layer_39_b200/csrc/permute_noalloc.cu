@@ -10,19 +10,26 @@
 // can fail when memory is tight).  This variant keeps its scratch in a
 // fixed array compiled into the library instead.
 //
-// The array: kNoallocScratchInts int32 values (1 MiB), declared below at
-// file scope in device memory.  Every GPU that loads the library holds one
-// copy of it until the process exits.  Host code cannot use the array's name
-// as a device address (on the host it names a placeholder), so the first call
-// on each device, with that device current, looks the address up with
-// cudaGetSymbolAddress and keeps it; later calls on that device reuse it.
-// Make that first call before starting any stream capture.
+// The array: MOE_NOALLOC_SCRATCH_INTS int32 values (1 MiB, the size the
+// header states), declared below at file scope in device memory.  Every GPU
+// that loads the library holds one copy of it until the process exits.  Host
+// code cannot use the array's name as a device address (on the host it names
+// a placeholder), so the first call on each device, with that device
+// current, looks the address up with cudaGetSymbolAddress and keeps it;
+// later calls on that device reuse it.  Make that first call before starting
+// any stream capture.  The address is kept together with the id of the CUDA
+// context it was looked up in: a device reset destroys that context and the
+// module is loaded again elsewhere, so a call that finds another context
+// looks the address up again (before any capture, like the first call).
 //
 // Sharing: every call on a device uses the same array and leaves its
 // contents behind.  Nothing in it has to start at zero (each entry a call
 // reads is written earlier in that same call), but two calls whose work
 // overlaps on the GPU (different streams with no ordering between them, or
 // several host threads) race on the array and corrupt each other's results.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "context.cuh"
@@ -30,23 +37,51 @@
 
 namespace {
 
-constexpr int64_t kNoallocScratchInts = 1 << 18;  // 262144 int32 = 1 MiB
+constexpr int64_t kNoallocScratchInts = MOE_NOALLOC_SCRATCH_INTS;  // 262144 int32 = 1 MiB
+static_assert(kNoallocScratchInts == (1 << 18), "the header documents a 1 MiB array");
 
 static __device__ __align__(256) int32_t g_permute_scratch[kNoallocScratchInts];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 int32_t* g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // context id the address belongs to
+
+// Id of the calling thread's current CUDA context (unique per context
+// created in this process), or 0 when there is none or it cannot be read.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  return get_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
+}
 
 // Device address of the array on `device`, which must be the current device.
 moe_status_t scratch_on_device(int device, int32_t** out) {
   if (device < 0 || device >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[device] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (g_scratch_addr[device] == nullptr || ctx == 0 || ctx != g_scratch_ctx[device]) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_permute_scratch);
     if (e != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
     g_scratch_addr[device] = static_cast<int32_t*>(p);
+    // the lookup made the device's primary context current if it was not
+    g_scratch_ctx[device] = ctx != 0 ? ctx : current_context_id();
   }
   *out = g_scratch_addr[device];
   return MOE_OK;

@@ -497,10 +497,7 @@ __global__ void __launch_bounds__(kWarps * 32)
 cudaError_t launch_router_fused(const __nv_bfloat16* x, const __nv_bfloat16* w_r, const float* bias,
                                 const int32_t* route_in, int T, int d, int E, int k, bool renorm,
                                 int32_t* idx, float* w, float* probs, float* logits,
-                                DeviceCtl* ctl, cudaStream_t st) {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+                                DeviceCtl* ctl, int sms, cudaStream_t st) {
   const size_t w_smem = static_cast<size_t>(E) * d * 4;
   auto go = [&](auto kern_smem, auto kern_l1, int tpw) {
     const int64_t groups = ceil_div64(T, tpw);

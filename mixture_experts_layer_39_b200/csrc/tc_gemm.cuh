@@ -28,9 +28,10 @@
 // MN-major = 64-element chunks along M/N, one 128-byte row per K index (TMA
 // box {64, 64}), chunks 8 KB apart.
 //
-// Every mbarrier wait is bounded (kWaitLimitNs, globaltimer); on expiry the
-// CTA records MOE_ERR_TIMEOUT, drains its own TMA copies and MMAs, frees
-// TMEM and returns.
+// Every mbarrier wait is bounded (globaltimer).  The waits of the main loops
+// give up after GemmArgs::wait_ns (the handle's limit, 2 s unless changed);
+// the CTA then records MOE_ERR_TIMEOUT, drains its own TMA copies and MMAs
+// (those drain waits always allow kWaitLimitNs), frees TMEM and returns.
 #pragma once
 
 #include <cuda.h>
@@ -68,14 +69,7 @@ struct GemmArgs {
   int64_t ld_aux;
   int f;  // SwiGLU: width of one half ([A | U] column offset of U)
   DeviceCtl* ctl;
-  // MXFP8 operands: E8M0 scales stored [MN index][K/32] (bytes), B's per group
-  const uint8_t* sfa;
-  int64_t ld_sfa;       // bytes per A row (M index) = K_total / 32
-  int64_t sfa_rows;     // rows of the A scale array (reads are clamped to it)
-  const uint8_t* sfb;
-  int64_t ld_sfb;
-  int64_t sfb_rows;     // rows per group of the B scale array
-  int64_t sfb_gstride;  // bytes between groups of B scales (M-grouped)
+  uint64_t wait_ns;  // limit of the main loops' waits; 0: give up unless already complete
   // GATHER: the operand that holds routed rows is read from the unpermuted
   // matrix (x), routed row r being its row row_src[r]; rows past m_cap and
   // pad rows use src_oob, a row past the matrix that reads as zeros
@@ -114,22 +108,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait: true when the phase completed; false when another role
-// aborted or the time limit passed (then the abort flag is raised).
+// aborted or `limit_ns` passed (then the abort flag is raised).  A limit of
+// 0 gives up at once unless the first test finds the phase complete.
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity);
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          bool honour_abort = true, bool cluster_scope = false) {
+                                          uint64_t limit_ns, bool honour_abort = true,
+                                          bool cluster_scope = false) {
   auto poll = [&]() {
     return cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
   };
   if (poll()) return true;
+  if (limit_ns == 0) {
+    *abort_flag = 1;
+    return false;
+  }
   const uint64_t t0 = globaltimer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 64; ++i)
       if (poll()) return true;
     if (honour_abort && *abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       return false;
     }
@@ -209,6 +209,18 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap
       "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
+// One 512-byte scale atom (box {128, 4, 1, 1, 1} of a 5-D map over the
+// atom-ordered scales: coordinates (0, 0, K block, MN block, group)); the
+// completion bytes go to `bar`, which may live in either CTA of the pair.
+__device__ __forceinline__ void tma_load_atom_pair(uint32_t dst, const CUtensorMap* map,
+                                                   uint32_t bar, int kb, int rb, int g) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(kb), "r"(rb), "r"(g), "r"(bar)
       : "memory");
 }
 
@@ -296,6 +308,18 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
+__device__ __forceinline__ void mma_mxf8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}\n"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem),
+      "r"(accumulate)
+      : "memory");
+}
+
 // Instruction descriptor of kind::mxf8f6f4 (block-scaled): E4M3 A and B, E8M0
 // scales (bit 23), K = 32 per MMA.  The scale-factor ids (bits 4-5 for B,
 // 29-30 for A) select the byte of each 32-bit scale word and are or-ed in
@@ -305,39 +329,17 @@ __host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, bool a_mn, bool 
          (1u << 23) | ((uint32_t)(M >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %6, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}\n"
-      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem),
-      "r"(accumulate)
-      : "memory");
-}
-
 // One 512-byte scale atom (32 rows x 16 bytes, no swizzle: 8-row groups 128 B
 // apart) from shared memory into 4 TMEM columns, copied to all four lane
-// quarters.
-__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint32_t saddr) {
+// quarters; issued by the pair's leader, each CTA's atom (same shared-memory
+// offset) lands in that CTA's TMEM.
+__device__ __forceinline__ void tmem_cp_sf_pair(uint32_t taddr, uint32_t saddr) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
   d |= static_cast<uint64_t>(512u >> 4) << 16;   // leading byte offset (unused at 16 B width)
   d |= static_cast<uint64_t>(128u >> 4) << 32;   // stride byte offset: 8 rows x 16 B
   d |= static_cast<uint64_t>(1) << 46;           // descriptor version
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
-}
-
-__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc) {
-  const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(gsrc) : "memory");
-}
-
-// Arrives on the mbarrier once all prior cp.async of this thread completed
-// (the arrival is counted in the barrier's expected count).
-__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
 }
 
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -525,7 +527,8 @@ struct SmemPlan {
   static constexpr int kABytes = BM * 128;
   static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * 128;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  // MXFP8: per stage one 512-byte scale atom per 128 rows of A and of B
+  // MXFP8 (CTA pairs): per stage and CTA one 512-byte scale atom for its own
+  // 128 rows of A and one per 128 of the pair's BN rows of B
   static constexpr int kSfStageBytes = FP8 ? 512 * (1 + BN / 128) : 0;
   static constexpr int kSfOff = STAGES * kStageBytes;
   static constexpr int kBarOff = kSfOff + STAGES * kSfStageBytes;      // 1024-aligned stages
@@ -546,15 +549,27 @@ struct SmemPlan {
 // TMEM holds its own 128 accumulator rows, so the epilogue is unchanged, and
 // the odd CTA's epilogue warps release the accumulator on the leader's
 // barrier.
+//
+// MXFP8 (FP8 = true) always runs on CTA pairs with 256 x 256 tiles and 128
+// contraction elements per stage.  The E8M0 scales come from arrays in the
+// tensor cores' 512-byte atom order (tmSA, tmSB: 5-D maps, one atom per
+// (128 MN indices, 128 contraction elements)): each CTA loads the atom of
+// its own 128 A rows and both atoms of the pair's 256 B rows with pair TMA
+// loads that complete on the leader's full barrier; the leader copies them
+// to TMEM (tcgen05.cp.cta_group::2, each CTA's atoms into its own TMEM) and
+// issues block-scaled pair MMAs.  TMEM then holds one 256-column accumulator
+// and two alternating scale buffers.
 template <int BN, bool A_MN, bool B_MN, int EPI, bool KGROUP, int STAGES, bool FP8 = false,
           bool PAIR = false, bool GATHER = false>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmSA,
+                        const __grid_constant__ CUtensorMap tmSB, const GemmArgs args) {
   static_assert(BN == 128 || BN == 256 || (BN == 512 && PAIR), "BN");
   static_assert(!(EPI == EPI_SWIGLU_FWD && B_MN), "SwiGLU forward takes K-major weights");
-  static_assert(!FP8 || BN == 128, "MXFP8 tiles are 128 x 128 (TMEM holds the scales too)");
-  static_assert(!PAIR || (BN >= 256 && !FP8), "CTA pairs run bf16 256 x 256 or 256 x 512 tiles");
+  static_assert(!FP8 || (PAIR && BN == 256), "MXFP8 runs 256 x 256 CTA-pair tiles");
+  static_assert(!PAIR || BN >= 256, "CTA pairs run 256 x 256 or 256 x 512 tiles");
   // GATHER reads routed rows from x: the K-major A of an M-grouped GEMM, or
   // the MN-major B (rows = routed rows) of a K-grouped one
   static_assert(!GATHER || (!FP8 && (KGROUP ? B_MN : !A_MN)), "gathered operand");
@@ -570,14 +585,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int CH = FP8 ? 128 : 64;
   constexpr uint32_t kChunkBytes = BKE * 128;      // one MN chunk of an MN-major stage
   constexpr uint32_t kSfCols = 4 + 4 * (BN / 128); // TMEM columns of one scale buffer
+  constexpr uint32_t kSfTmaBytes = FP8 ? 512 * (1 + BN / 128) : 0;  // scale atoms per stage, per CTA
   // Wide pairs (BN = 512): two N = 256 MMAs per K step, each reading 128 of
   // every CTA's 256 B rows, into one accumulator that fills TMEM (the
-  // epilogue of a tile then does not overlap the next tile's MMAs).
+  // epilogue of a tile then does not overlap the next tile's MMAs).  MXFP8
+  // pairs also keep one accumulator: the scale buffers need TMEM too.
   constexpr int NMMA = BN > 256 ? 256 : BN;  // N of one MMA instruction
-  constexpr int NACC = BN > 256 ? 1 : 2;     // TMEM accumulators
+  constexpr int NACC = (BN > 256 || FP8) ? 1 : 2;  // TMEM accumulators
   constexpr uint32_t kBHalfBytes = (BNC / 2) * 128;  // B rows of one wide-pair MMA, per CTA
   constexpr uint32_t kTmemCols = FP8 ? 512 : NACC * BN;
-  constexpr uint32_t kIdesc = FP8 ? idesc_mxf8(BM, BN, A_MN, B_MN) : idesc_bf16(MT, NMMA, A_MN, B_MN);
+  constexpr uint32_t kIdesc = FP8 ? idesc_mxf8(MT, BN, A_MN, B_MN) : idesc_bf16(MT, NMMA, A_MN, B_MN);
   // M-grouped bf16 tail tiles of <= 64 rows run M = 64 MMAs: rows 16q..16q+15
   // of the accumulator then sit in TMEM lanes 32q..32q+15
   constexpr bool kTail64 = !FP8 && !KGROUP && !A_MN && !PAIR;
@@ -606,8 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- set-up: barriers, TMEM, group tile starts
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      // MXFP8: the 32 producer lanes' scale copies arrive on the full barrier too
-      mbar_init(full_bar(s), FP8 ? 33 : 1);
+      mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -622,6 +638,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    if constexpr (FP8) {
+      prefetch_tmap(&tmSA);
+      prefetch_tmap(&tmSB);
+    }
   }
   if (warp == 1) {
     if constexpr (PAIR) {
@@ -679,13 +699,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ================================================================ producer
-    // lane 0 issues the TMA tile loads; with MXFP8 all 32 lanes also copy the
-    // stage's scale atoms (cp.async, arriving on the full barrier)
+    // lane 0 issues the TMA tile loads (and, MXFP8, the stage's scale atoms)
     // GATHER: every lane issues one 4-row gather per 4 routed rows it owns
     auto src_row = [&](int64_t r) -> int {
       return r < args.m_cap ? __ldg(args.row_src + r) : args.src_oob;
     };
-    if (FP8 || GATHER || lane == 0) {
+    if (GATHER || lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // per-stage: a load is in flight / its phase
@@ -707,8 +726,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 4; ++i) gsrc[i] = src_row(r + i);
         }
         for (int kb = 0; kb < tl.k_blocks; ++kb) {
-          bool got = mbar_wait(empty_bar(stage), phase ^ 1u, s_abort, true, PAIR);
-          if constexpr (FP8 || GATHER) got = __all_sync(0xffffffffu, got);
+          bool got = mbar_wait(empty_bar(stage), phase ^ 1u, s_abort, args.wait_ns, true, PAIR);
+          if constexpr (GATHER) got = __all_sync(0xffffffffu, got);
           if (!got) { ok = false; break; }
           const uint32_t sa = smem_base + stage * Plan::kStageBytes;
           const uint32_t sb = sa + Plan::kABytes;
@@ -717,7 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // both CTAs' bytes complete on the leader's full barrier
             const uint32_t fbl = mapa_shared(fb, 0);
             if (rank == 0 && lane == 0) {
-              mbar_arrive_expect_tx(fb, 2 * Plan::kStageBytes);
+              mbar_arrive_expect_tx(fb, 2 * (Plan::kStageBytes + kSfTmaBytes));
               armed |= 1u << stage;
               armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
             }
@@ -812,54 +831,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if constexpr (FP8) {
-            // scale atoms: byte (r0*16 + r1*4 + s) = scale of row 32*r1 + r0, K-slice s
-            uint8_t* sfa_s = smem + Plan::kSfOff + stage * Plan::kSfStageBytes;
-            uint8_t* sfb_s = sfa_s + 512;
-            const int64_t kbyte = KGROUP ? (static_cast<int64_t>(tl.k_lo) >> 5) + kb * 4
-                                         : static_cast<int64_t>(kb) * 4;
+            // scale atoms (512 bytes each): the one of this CTA's 128 A rows, then
+            // both of the pair's 256 B rows (identical in the two CTAs); their
+            // bytes complete on the leader's full barrier like the tiles
+            if (lane == 0) {
+              const uint32_t fbl = mapa_shared(fb, 0);
+              const uint32_t sfa_s = smem_base + Plan::kSfOff + stage * Plan::kSfStageBytes;
+              const int kbs = KGROUP ? (tl.k_lo >> 7) + kb : kb;  // 128-element K block
+              tma_load_atom_pair(sfa_s, &tmSA, fbl, kbs, (tl.row0 >> 7) + static_cast<int>(rank), 0);
 #pragma unroll
-            for (int r1 = 0; r1 < 4; ++r1) {
-              int64_t row = static_cast<int64_t>(tl.row0) + 32 * r1 + lane;
-              row = row < args.sfa_rows ? row : args.sfa_rows - 1;
-              cp_async4(sfa_s + lane * 16 + r1 * 4, args.sfa + row * args.ld_sfa + kbyte);
-            }
-            const int64_t gofs = KGROUP ? 0 : static_cast<int64_t>(tl.group) * args.sfb_gstride;
-#pragma unroll
-            for (int j = 0; j < BN / 128; ++j) {
-#pragma unroll
-              for (int r1 = 0; r1 < 4; ++r1) {
-                const int local = 128 * j + 32 * r1 + lane;  // row of the B tile
-                int64_t n;
+              for (int j = 0; j < BN / 128; ++j) {
+                int rb;
                 if constexpr (EPI == EPI_SWIGLU_FWD) {
-                  const int nh = tl.n_tile * (BN / 2);
-                  n = local < BN / 2 ? nh + local : args.f + nh + (local - BN / 2);
+                  rb = j == 0 ? tl.n_tile : (args.f >> 7) + tl.n_tile;  // gate rows, then up rows
                 } else {
-                  n = static_cast<int64_t>(tl.n_tile) * BN + local;
+                  rb = tl.n_tile * (BN / 128) + j;
                 }
-                n = n < args.sfb_rows ? n : args.sfb_rows - 1;
-                cp_async4(sfb_s + j * 512 + lane * 16 + r1 * 4,
-                          args.sfb + gofs + n * args.ld_sfb + kbyte);
+                tma_load_atom_pair(sfa_s + 512 + 512 * j, &tmSB, fbl, kbs, rb, KGROUP ? 0 : tl.group);
               }
             }
-            cp_async_arrive_noinc(fb);
           }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
       if (!ok) {
         if (lane == 0) report(args.ctl, MOE_ERR_TIMEOUT, 1);
-        if constexpr (FP8) cp_async_wait_all();
         // let every copy this warp started land before the CTA exits
         if (lane == 0)
           for (int s = 0; s < STAGES; ++s)
-            if (armed & (1u << s)) mbar_wait(full_bar(s), (armed_parity >> s) & 1u, s_abort, false);
+            if (armed & (1u << s))
+              mbar_wait(full_bar(s), (armed_parity >> s) & 1u, s_abort, kWaitLimitNs, false);
       }
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
     if (PAIR && lane == 0 && rank != 0) {
       // the leader issues the pair's MMAs; wait for them before TMEM is freed
-      mbar_wait(drain_bar, 0, s_abort, false, true);
+      mbar_wait(drain_bar, 0, s_abort, kWaitLimitNs, false, true);
     } else if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -869,27 +877,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int t = unit; t < total_tiles && ok; t += n_units) {
         const Tile tl = decode_tile<KGROUP, BKE, KMMA, MT>(args, s_tile_start, t);
-        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, s_abort, true, PAIR)) { ok = false; break; }
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, s_abort, args.wait_ns, true, PAIR)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);  // acc = 0 when NACC = 1
         for (int kb = 0; kb < tl.k_blocks; ++kb) {
-          if (!mbar_wait(full_bar(stage), phase, s_abort, true, PAIR)) { ok = false; break; }
+          if (!mbar_wait(full_bar(stage), phase, s_abort, args.wait_ns, true, PAIR)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t sa = smem_base + stage * Plan::kStageBytes;
           const uint32_t sb = sa + Plan::kABytes;
           const int n16 = (kb == tl.k_blocks - 1) ? tl.last_k16 : 4;
           uint32_t sf_col = 0;
           if constexpr (FP8) {
-            // the atoms were written by cp.async (generic proxy); order them before
-            // the tensor core's reads, then copy them to TMEM (alternating buffers
-            // after the accumulators)
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            sf_col = tmem_base + 2 * BN + sf_buf * kSfCols;
+            // the stage's scale atoms (landed by TMA with the tiles) into TMEM,
+            // alternating buffers after the accumulator; each CTA's own atoms go
+            // to its own TMEM
+            sf_col = tmem_base + NACC * BN + sf_buf * kSfCols;
             sf_buf ^= 1u;
             const uint32_t sfa_s = smem_base + Plan::kSfOff + stage * Plan::kSfStageBytes;
-            tmem_cp_sf(sf_col, sfa_s);
+            tmem_cp_sf_pair(sf_col, sfa_s);
 #pragma unroll
-            for (int j = 0; j < BN / 128; ++j) tmem_cp_sf(sf_col + 4 + 4 * j, sfa_s + 512 + 512 * j);
+            for (int j = 0; j < BN / 128; ++j)
+              tmem_cp_sf_pair(sf_col + 4 + 4 * j, sfa_s + 512 + 512 * j);
           }
           for (int kk = 0; kk < n16; ++kk) {
             // K-major: the next MMA starts 32 bytes further along each 128-byte row;
@@ -900,8 +914,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      : smem_desc_sw128(sb + kk * 32, 16, 1024);
             if constexpr (FP8) {
               const uint32_t sid = static_cast<uint32_t>(kk);
-              mma_mxf8(d_tmem, ad, bd, kIdesc | (sid << 4) | (sid << 29), sf_col | (sid << 30),
-                       (sf_col + 4) | (sid << 30), (kb > 0 || kk > 0) ? 1u : 0u);
+              mma_mxf8_pair(d_tmem, ad, bd, kIdesc | (sid << 4) | (sid << 29), sf_col | (sid << 30),
+                            (sf_col + 4) | (sid << 30), (kb > 0 || kk > 0) ? 1u : 0u);
             } else if constexpr (PAIR && BN > 256) {
               // B rows [0,128) and [128,256) of each CTA: 16 KB apart in both layouts
               const uint64_t bd1 = B_MN ? smem_desc_sw128(sb + kBHalfBytes + kk * KMMA * 128, kChunkBytes, 1024)
@@ -925,7 +939,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) report(args.ctl, MOE_ERR_TIMEOUT, 2);
       // all MMAs issued by this thread have finished once the drain barrier flips
       if constexpr (PAIR) mma_commit_pair(drain_bar); else mma_commit(drain_bar);
-      mbar_wait(drain_bar, 0, s_abort, false, PAIR);
+      mbar_wait(drain_bar, 0, s_abort, kWaitLimitNs, false, PAIR);
     }
   } else {
     // ================================================================ epilogue
@@ -979,7 +993,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     args.aux);
         cp_async_commit();
       }
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull_bar(acc), acc_phase, s_abort, true, PAIR));
+      const bool ok = __all_sync(
+          0xffffffffu, mbar_wait(tfull_bar(acc), acc_phase, s_abort, args.wait_ns, true, PAIR));
       if (!ok) {
         if constexpr (EPI == EPI_SWIGLU_BWD) cp_async_wait_all();  // own copies land first
         if (lane == 0) report(args.ctl, MOE_ERR_TIMEOUT, 3);

@@ -10,6 +10,7 @@ from mixture_experts_layer_39_b200.inputs import CONFIGS, custom_config, make_in
 from mixture_experts_layer_39_b200.layer import MoELayer
 from oracle import moe_ref as R
 from oracle import mxfp8_ref as MX
+from tests import _helpers as H
 from tests._helpers import TOL_MXFP8, assert_close, np64
 
 pytestmark = pytest.mark.gpu
@@ -32,13 +33,64 @@ def _segments(L, E):
     return m
 
 
-@pytest.mark.parametrize("T,d,f,E,k", [(384, 256, 256, 4, 2), (700, 512, 256, 6, 3),
-                                       (256, 256, 512, 8, 1), (384, 384, 384, 4, 2)])
-def test_mxfp8_small_every_stage(cuda_ok, T, d, f, E, k):
-    cfg = custom_config(T, d, f, E, k, random_routing=True, mxfp8=True)
-    inp = make_inputs(cfg, seed=T + d, device="cpu")
+def _edge_inputs(cfg, mode, seed):
+    """Inputs of one small case.  Modes:
+      random     uniform random expert ids (the workload's routing)
+      empty      random ids that never pick expert 1: a zero-count segment,
+                 whose weight gradients must come out zero
+      skewed     router logits plus a bias that sends most tokens to expert
+                 0 and none to experts 1, 3, 5 (dropless: no capacity cap)
+      subnormal  random ids; x holds one 32-element row block of bf16
+                 subnormals (the row-wise scale takes the exponent clamp at
+                 -127) and one column of subnormals (every token-axis block
+                 of that column takes it in the weight gradient)"""
+    inp = make_inputs(cfg, seed=seed, device="cpu")
+    if mode == "empty":
+        g = torch.Generator().manual_seed(seed + 1)
+        noise = torch.rand(cfg.T, cfg.E, generator=g)
+        noise[:, 1] = 2.0  # sorts last, never among the k chosen (k < E)
+        inp["route"] = noise.argsort(dim=1)[:, :cfg.k].to(torch.int32).contiguous()
+    elif mode == "skewed":
+        inp["route"] = None
+        inp["bias"] = torch.tensor([4.0, -30.0, 2.0, -30.0, 0.0, -30.0][:cfg.E], dtype=torch.float32)
+    elif mode == "subnormal":
+        g = torch.Generator().manual_seed(seed + 2)
+        x = inp["x"].float()
+        t0 = cfg.T // 3
+        x[t0, 32:64] = torch.randn(32, generator=g) * 2e-39   # bf16 min normal is 2^-126
+        x[:, 7] = torch.randn(cfg.T, generator=g) * 3e-39
+        xb = x.to(torch.bfloat16)
+        sub = xb[t0, 32:64].float().abs()
+        assert (sub < 2.0 ** -126).all() and int((sub > 0).sum()) >= 16
+        inp["x"] = xb
+    return inp
+
+
+MX_CASES = [
+    # T, d, f, E, k, mode
+    (384, 256, 256, 4, 2, "random"),
+    (700, 512, 256, 6, 3, "random"),
+    (256, 256, 512, 8, 1, "random"),
+    (384, 384, 384, 4, 2, "random"),
+    (500, 256, 256, 6, 2, "empty"),
+    (700, 384, 256, 6, 2, "skewed"),
+    (600, 256, 384, 4, 2, "subnormal"),
+]
+
+
+@pytest.mark.parametrize("case", MX_CASES, ids=lambda c: "T%d_d%d_f%d_E%d_k%d_%s" % c)
+def test_mxfp8_small_every_stage(cuda_ok, case):
+    T, d, f, E, k, mode = case
+    cfg = custom_config(T, d, f, E, k, random_routing=(mode != "skewed"), mxfp8=True)
+    inp = _edge_inputs(cfg, mode, seed=T + d)
     L = _run(cfg, {n: (v.cuda() if v is not None else None) for n, v in inp.items()})
     m = _segments(L, E)
+    if mode in ("empty", "skewed"):
+        assert (m["counts"] == 0).any()
+        for e in np.flatnonzero(m["counts"] == 0):
+            assert torch.count_nonzero(L.dw_gu[e]) == 0 and torch.count_nonzero(L.dw_d[e]) == 0
+    if mode == "skewed":
+        assert m["counts"].max() > 2 * m["counts"].mean()
     Mp, off, cnt, rm = m["M_pad"], m["offsets"], m["counts"], m["row_map"]
     w_gu, w_d = np64(inp["w_gu"]), np64(inp["w_d"])
     xp = np64(L.x_perm[:Mp])
@@ -76,7 +128,10 @@ def test_mxfp8_workload_sampled_experts(cuda_ok):
     L = _run(cfg, g)
     m = _segments(L, cfg.E)
     off, cnt = m["offsets"], m["counts"]
-    for e in (0, int(np.argmax(cnt)), int(np.argmin(cnt))):
+    log0 = len(H.LOG)
+    order = np.argsort(cnt, kind="stable")
+    pick = sorted({0, cfg.E - 1, int(order[-1]), int(order[0]), int(order[len(order) // 2])})
+    for e in pick:
         # the whole padded segment: its pad rows are zero on both sides, and
         # token-axis scale blocks of 32 rows start at the segment start
         r0, r1 = int(off[e]), int(off[e + 1])
@@ -92,3 +147,4 @@ def test_mxfp8_workload_sampled_experts(cuda_ok):
         assert_close(f"dAU[{e}]", np64(L.dau[r0:r1]), bwd["dAU"], TOL_MXFP8)
         assert_close(f"dW_d[{e}]", np64(L.dw_d[e]), bwd["dW_d"][0], TOL_MXFP8)
         assert_close(f"dW_gu[{e}]", np64(L.dw_gu[e]), bwd["dW_gu"][0], TOL_MXFP8)
+    H.report("full-size mxfp8 (sampled experts)", log0)

@@ -15,6 +15,7 @@ import torch
 from mixture_experts_layer_39_b200.inputs import CONFIGS, custom_config, make_inputs
 from mixture_experts_layer_39_b200.layer import MoELayer
 from oracle import moe_ref as R
+from tests import _helpers as H
 from tests._helpers import TAU, assert_close, np64, topk_margin
 
 pytestmark = pytest.mark.gpu
@@ -268,6 +269,7 @@ def test_full_size_sampled(cuda_ok, name):
     inp = make_inputs(cfg, seed=0, device="cuda")
     L = _run(cfg, inp)
     k, E = cfg.k, cfg.E
+    log0 = len(H.LOG)
     rng = np.random.default_rng(1)
     toks = np.unique(np.concatenate([[0, cfg.T - 1], rng.integers(0, cfg.T, 254)]))
 
@@ -330,6 +332,7 @@ def test_full_size_sampled(cuda_ok, name):
     pick |= {int(e) for e in order[cnt[order] == 0][:2]}
     for e in sorted(pick):
         _seg_check(L, inp, e, off, cnt)
+    H.report(f"full-size {name}", log0)
 
 
 
@@ -342,7 +345,10 @@ def test_mxfp8_quantize_matches_oracle(cuda_ok):
     a[3] = 0.0
     a[5, :32] = 1e-30
     a[7, 64:96] = 3e4
+    a[9, 96:128] = torch.randn(32, generator=g) * 2e-39   # bf16 subnormals: scale clamp at -127
+    a[:, 130] = torch.randn(256, generator=g) * 3e-39     # every column-wise block of a column
     a = a.to(torch.bfloat16)
+    assert (a[9, 96:128].float().abs() < 2.0 ** -126).all() and bool(a[9, 96:128].any())
     for axis in (1, 0):
         ad = a.cuda()
         if axis == 1:
