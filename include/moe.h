@@ -53,7 +53,13 @@
  * moe_grouped_swiglu_fwd/bwd quantise every operand along its contraction
  * axis (E4M3 elements, one E8M0 scale per 32) into the workspace and run
  * block-scaled tcgen05 MMAs with fp32 accumulation; their outputs stay
- * bf16.  The router, permute and combine are unchanged.
+ * bf16.  The router, permute and combine are unchanged.  The workspace then
+ * has two parts: a leading scratch region that every call may overwrite,
+ * and a persistent region after it into which moe_grouped_swiglu_fwd writes
+ * the column-wise quantised W_gu, W_down, x_perm and h that
+ * moe_grouped_swiglu_bwd reads.  So in MXFP8 mode the backward must get the
+ * workspace the forward of the same step used, and nothing else may write
+ * past the scratch region in between (no other call of this library does).
  */
 #ifndef MOE_H_
 #define MOE_H_
@@ -173,7 +179,7 @@ MOE_API moe_status_t moe_permute(moe_handle_t h, const moe_shape_t* s, const voi
  * Same arguments, outputs and device-side checks as moe_permute.  Its scratch
  * is a fixed 1 MiB array inside the library (one per GPU that loads it, held
  * until the process exits), so the shape must satisfy
- *   ceil(T*k / 256) * E <= MOE_NOALLOC_SCRATCH_INTS,
+ *   ceil(T / 16) * E <= MOE_NOALLOC_SCRATCH_INTS,
  * otherwise MOE_ERR_WORKSPACE is returned before any launch.  The first call
  * on a device looks up the array's device address (a host-side step, done
  * once per device with that device current); make that first call before
@@ -312,7 +318,10 @@ MOE_API moe_status_t moe_unpermute_combine_bwd(moe_handle_t h, const moe_shape_t
  * Experts with no rows get zero weight gradients.
  * In : do_perm, x_perm, au, hbuf [M_cap,*] bf16, offsets [E+1], w_gu, w_down.
  * Out: dau [M_cap,2f] bf16, dx_perm [M_cap,d] bf16, dw_gu [E,2f,d] bf16,
- *      dw_down [E,d,f] bf16. */
+ *      dw_down [E,d,f] bf16.
+ * MXFP8 mode: x_perm, hbuf, w_gu and w_down enter through the column-wise
+ * copies the forward left in the workspace (see the MXFP8 note above); the
+ * arguments must still be the forward's tensors. */
 MOE_API moe_status_t moe_grouped_swiglu_bwd(moe_handle_t h, const moe_shape_t* s, const void* do_perm,
                                     const void* x_perm, const void* au, const void* hbuf,
                                     const int32_t* offsets, const void* w_gu,

@@ -68,13 +68,21 @@ RouterBwdWs router_bwd_layout(const moe_context* h, const moe_shape_t* s) {
   return w;
 }
 
-// MXFP8 expert GEMMs: quantised operand copies (E4M3 codes + E8M0 scales)
-// carved from the workspace; the forward and the backward call reuse the
-// same bytes.
+// MXFP8 expert GEMMs: quantised operand copies (E4M3 codes + E8M0 scales in
+// the GEMMs' atom order) carved from the workspace.  The forward quantises
+// each of its operands once into both orientations: the row-wise copy it
+// uses itself goes to the transient region (shared with the backward's own
+// copies and with the other calls' scratch), the column-wise copy the
+// backward needs (W_gu and W_d along their output axis, x_perm and H along
+// tokens) goes to the persistent region that follows, which no other call
+// touches.  The backward quantises dO and dAU into both orientations.
 struct MxWs {
+  // transient, forward
   size_t xq, xs, wguq, wgus, hq, hs, wdq, wds, fwd_total;
-  size_t doq, dos, wdq_c, wds_c, dauq, daus, wguq_c, wgus_c, doq_c, dos_c, hq_c, hs_c, dauq_c,
-      daus_c, xq_c, xs_c, bwd_total;
+  // transient, backward
+  size_t doq, dos, dauq, daus, doq_c, dos_c, dauq_c, daus_c, bwd_total;
+  // persistent (offsets from the start of the persistent region)
+  size_t wdq_c, wds_c, wguq_c, wgus_c, xq_c, xs_c, hq_c, hs_c, keep_total;
 };
 
 MxWs mx_layout(const moe_shape_t* s) {
@@ -94,18 +102,22 @@ MxWs mx_layout(const moe_shape_t* s) {
   w.fwd_total = off;
   off = 0;
   w.doq = take(M * d);              w.dos = take(M * d / 32);
-  w.wdq_c = take(E * d * f);        w.wds_c = take(E * f * d / 32);
   w.dauq = take(M * 2 * f);         w.daus = take(M * 2 * f / 32);
-  w.wguq_c = take(E * 2 * f * d);   w.wgus_c = take(E * d * 2 * f / 32);
   w.doq_c = take(M * d);            w.dos_c = take(d * M / 32);
-  w.hq_c = take(M * f);             w.hs_c = take(f * M / 32);
   w.dauq_c = take(M * 2 * f);       w.daus_c = take(2 * f * M / 32);
-  w.xq_c = take(M * d);             w.xs_c = take(d * M / 32);
   w.bwd_total = off;
+  off = 0;
+  w.wdq_c = take(E * d * f);        w.wds_c = take(E * f * d / 32);
+  w.wguq_c = take(E * 2 * f * d);   w.wgus_c = take(E * d * 2 * f / 32);
+  w.xq_c = take(M * d);             w.xs_c = take(d * M / 32);
+  w.hq_c = take(M * f);             w.hs_c = take(f * M / 32);
+  w.keep_total = off;
   return w;
 }
 
-size_t workspace_bytes(const moe_context* h, const moe_shape_t* s) {
+// Bytes of the workspace's leading scratch region, which every call may
+// overwrite (in MXFP8 mode the persistent region follows it).
+size_t scratch_bytes(const moe_context* h, const moe_shape_t* s) {
   const int64_t T = s->T, E = s->n_experts;
   size_t need = 0;
   auto upd = [&](size_t v) { need = v > need ? v : need; };
@@ -118,6 +130,11 @@ size_t workspace_bytes(const moe_context* h, const moe_shape_t* s) {
   upd(align256(static_cast<size_t>(moe::n_subchunks(s->T, s->top_k)) * E * 4));    // permute
   upd(router_bwd_layout(h, s).total);                                              // router bwd
   return need;
+}
+
+size_t workspace_bytes(const moe_context* h, const moe_shape_t* s) {
+  const size_t scratch = scratch_bytes(h, s);
+  return s->dtype == MOE_DTYPE_MXFP8 ? scratch + mx_layout(s).keep_total : scratch;
 }
 
 moe_status_t check_ws(const moe_context* h, const moe_shape_t* s, void* ws, size_t ws_bytes) {
@@ -249,14 +266,12 @@ moe_status_t moe_permute(moe_handle_t h, const moe_shape_t* s, const void* x,
   auto st = static_cast<cudaStream_t>(stream);
   MOE_GUARD(h);
   auto* sub = static_cast<int32_t*>(ws);
-  h->launches += 4;
-  MOE_TRY(cuda_status(moe::launch_route_hist(topk_idx, T, k, E, sub, h->ctl, st)));
-  MOE_TRY(cuda_status(
-      moe::launch_route_scan(sub, moe::n_subchunks(T, k), E, moe::seg_align(s), counts, offsets, st)));
-  MOE_TRY(cuda_status(moe::launch_route_rank(topk_idx, T, k, E, sub, offsets, row_map, st)));
-  return cuda_status(moe::launch_permute_scatter(static_cast<const __nv_bfloat16*>(x), row_map,
-                                                 offsets, counts, T, d, k, E,
-                                                 static_cast<__nv_bfloat16*>(x_perm), st));
+  h->launches += 2;
+  MOE_TRY(cuda_status(moe::launch_route_count(topk_idx, T, k, E, moe::seg_align(s), sub, counts,
+                                              offsets, h->ctl, st)));
+  return cuda_status(moe::launch_route_rank_scatter(
+      topk_idx, static_cast<const __nv_bfloat16*>(x), T, k, E, sub, offsets, counts, d, row_map,
+      static_cast<__nv_bfloat16*>(x_perm), st));
 }
 
 // ---- gather forms (no materialised x_perm; bf16)
@@ -270,11 +285,11 @@ moe_status_t moe_route(moe_handle_t h, const moe_shape_t* s, const int32_t* topk
   auto st = static_cast<cudaStream_t>(stream);
   MOE_GUARD(h);
   auto* sub = static_cast<int32_t*>(ws);
-  h->launches += 4;
-  MOE_TRY(cuda_status(moe::launch_route_hist(topk_idx, T, k, E, sub, h->ctl, st)));
-  MOE_TRY(cuda_status(
-      moe::launch_route_scan(sub, moe::n_subchunks(T, k), E, moe::seg_align(s), counts, offsets, st)));
-  MOE_TRY(cuda_status(moe::launch_route_rank(topk_idx, T, k, E, sub, offsets, row_map, st)));
+  h->launches += 3;
+  MOE_TRY(cuda_status(moe::launch_route_count(topk_idx, T, k, E, moe::seg_align(s), sub, counts,
+                                              offsets, h->ctl, st)));
+  MOE_TRY(cuda_status(moe::launch_route_rank_scatter(topk_idx, nullptr, T, k, E, sub, offsets,
+                                                     counts, s->d_model, row_map, nullptr, st)));
   return cuda_status(
       moe::launch_route_src(row_map, offsets, counts, T, k, E, max_rows(s), row_src, st));
 }
@@ -365,16 +380,20 @@ moe_status_t moe_grouped_swiglu_fwd(moe_handle_t h, const moe_shape_t* s, const 
     const MxWs L = mx_layout(s);
     auto* b = static_cast<uint8_t*>(ws);
     auto bf = [](const void* p) { return static_cast<const __nv_bfloat16*>(p); };
-    auto rows = [&](const void* in, int64_t r, int64_t cols, size_t q, size_t sc) {
-      return cuda_status(moe::launch_mxfp8_quantize_atoms(bf(in), r, cols, b + q, b + sc, st));
+    auto* keep = b + scratch_bytes(h, s);  // read by moe_grouped_swiglu_bwd
+    // row-wise copy for this call, column-wise copy kept for the backward
+    auto both = [&](const void* in, int64_t r, int64_t cols, int64_t group, size_t q, size_t sc,
+                    size_t qc, size_t scc) {
+      return cuda_status(moe::launch_mxfp8_quantize_both(bf(in), r, cols, group, b + q, b + sc,
+                                                         keep + qc, keep + scc, st));
     };
     h->launches += 6;
-    MOE_TRY(rows(x_perm, m_cap, d, L.xq, L.xs));
-    MOE_TRY(rows(w_gu, 2ll * E * f, d, L.wguq, L.wgus));
+    MOE_TRY(both(x_perm, m_cap, d, m_cap, L.xq, L.xs, L.xq_c, L.xs_c));
+    MOE_TRY(both(w_gu, 2ll * E * f, d, 2ll * f, L.wguq, L.wgus, L.wguq_c, L.wgus_c));
     MOE_TRY(moe::gemm_mx_fwd_gate_up(c, {b + L.xq, b + L.xs}, offsets, {b + L.wguq, b + L.wgus}, au,
                                      hbuf, E, d, f, m_cap, st));
-    MOE_TRY(rows(hbuf, m_cap, f, L.hq, L.hs));
-    MOE_TRY(rows(w_down, static_cast<int64_t>(E) * d, f, L.wdq, L.wds));
+    MOE_TRY(both(hbuf, m_cap, f, m_cap, L.hq, L.hs, L.hq_c, L.hs_c));
+    MOE_TRY(both(w_down, static_cast<int64_t>(E) * d, f, d, L.wdq, L.wds, L.wdq_c, L.wds_c));
     return moe::gemm_mx_fwd_down(c, {b + L.hq, b + L.hs}, offsets, {b + L.wdq, b + L.wds}, o_perm,
                                  E, d, f, m_cap, st);
   }
@@ -468,33 +487,29 @@ moe_status_t moe_grouped_swiglu_bwd(moe_handle_t h, const moe_shape_t* s, const 
     const MxWs L = mx_layout(s);
     auto* b = static_cast<uint8_t*>(ws);
     auto bf = [](const void* p) { return static_cast<const __nv_bfloat16*>(p); };
-    auto rows = [&](const void* in, int64_t r, int64_t cols, size_t q, size_t sc) {
-      return cuda_status(moe::launch_mxfp8_quantize_atoms(bf(in), r, cols, b + q, b + sc, st));
+    auto both = [&](const void* in, int64_t r, int64_t cols, size_t q, size_t sc, size_t qc,
+                    size_t scc) {
+      return cuda_status(moe::launch_mxfp8_quantize_both(bf(in), r, cols, r, b + q, b + sc, b + qc,
+                                                         b + scc, st));
     };
-    auto cols_t = [&](const void* in, int64_t r, int64_t cols, int64_t group, size_t q, size_t sc) {
-      return cuda_status(moe::launch_mxfp8_quantize_cols_t(bf(in), r, cols, group, b + q, b + sc, st));
-    };
-    const int64_t Ed = static_cast<int64_t>(E) * d, E2f = 2ll * E * f;
-    h->launches += 12;
+    // the forward's column-wise copies of W_d, W_gu, H and x_perm
+    const uint8_t* keep = b + scratch_bytes(h, s);
+    h->launches += 6;
     // dgrad of the down projection (+ SwiGLU backward): dO along d, W_d along d
-    MOE_TRY(rows(do_perm, m_cap, d, L.doq, L.dos));
-    MOE_TRY(cols_t(w_down, Ed, f, d, L.wdq_c, L.wds_c));
+    MOE_TRY(both(do_perm, m_cap, d, L.doq, L.dos, L.doq_c, L.dos_c));
     MOE_TRY(moe::gemm_mx_dgrad_down_swiglu(c, {b + L.doq, b + L.dos}, offsets,
-                                           {b + L.wdq_c, b + L.wds_c}, au, dau, E, d, f, m_cap, st));
+                                           {keep + L.wdq_c, keep + L.wds_c}, au, dau, E, d, f,
+                                           m_cap, st));
     // dgrad of gate/up: dAU along 2f, W_gu along 2f
-    MOE_TRY(rows(dau, m_cap, 2ll * f, L.dauq, L.daus));
-    MOE_TRY(cols_t(w_gu, E2f, d, 2ll * f, L.wguq_c, L.wgus_c));
+    MOE_TRY(both(dau, m_cap, 2ll * f, L.dauq, L.daus, L.dauq_c, L.daus_c));
     MOE_TRY(moe::gemm_mx_dgrad_gate_up(c, {b + L.dauq, b + L.daus}, offsets,
-                                       {b + L.wguq_c, b + L.wgus_c}, dx_perm, E, d, f, m_cap, st));
+                                       {keep + L.wguq_c, keep + L.wgus_c}, dx_perm, E, d, f, m_cap,
+                                       st));
     // weight gradients: every operand along tokens
-    MOE_TRY(cols_t(do_perm, m_cap, d, m_cap, L.doq_c, L.dos_c));
-    MOE_TRY(cols_t(hbuf, m_cap, f, m_cap, L.hq_c, L.hs_c));
-    MOE_TRY(moe::gemm_mx_wgrad(c, {b + L.doq_c, b + L.dos_c}, d, {b + L.hq_c, b + L.hs_c}, f,
+    MOE_TRY(moe::gemm_mx_wgrad(c, {b + L.doq_c, b + L.dos_c}, d, {keep + L.hq_c, keep + L.hs_c}, f,
                                offsets, dw_down, E, m_cap, st));
-    MOE_TRY(cols_t(dau, m_cap, 2ll * f, m_cap, L.dauq_c, L.daus_c));
-    MOE_TRY(cols_t(x_perm, m_cap, d, m_cap, L.xq_c, L.xs_c));
-    return moe::gemm_mx_wgrad(c, {b + L.dauq_c, b + L.daus_c}, 2 * f, {b + L.xq_c, b + L.xs_c}, d,
-                              offsets, dw_gu, E, m_cap, st);
+    return moe::gemm_mx_wgrad(c, {b + L.dauq_c, b + L.daus_c}, 2 * f,
+                              {keep + L.xq_c, keep + L.xs_c}, d, offsets, dw_gu, E, m_cap, st);
   }
   h->launches += 4;
   MOE_TRY(moe::gemm_dgrad_down_swiglu(c, do_perm, offsets, w_down, au, dau, E, d, f, m_cap, st));

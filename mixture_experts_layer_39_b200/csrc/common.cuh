@@ -19,6 +19,7 @@ constexpr int kSegAlignMx = 128;
 struct DeviceCtl {
   int status;  // first recorded moe_status_t code, 0 when clean
   int detail;  // kernel-specific detail of the first error (which wait, which index)
+  unsigned ticket;  // routing-count blocks finished in the running launch (0 between launches)
 };
 
 __device__ __forceinline__ void report(DeviceCtl* ctl, int code, int detail) {

@@ -6,11 +6,11 @@
 
 namespace moe {
 
-// Sub-chunk of flat (token, slot) entries handled by one warp in the
-// routing histogram / rank kernels.
-constexpr int kSubChunk = 256;
+// Chunk of tokens (k flat (token, slot) entries each) counted by one warp
+// and ranked and copied by one block of the routing-metadata kernels.
+constexpr int kChunkTokens = 16;
 
-inline int64_t n_subchunks(int T, int k) { return ceil_div64(static_cast<int64_t>(T) * k, kSubChunk); }
+inline int64_t n_subchunks(int T, int /*k*/) { return ceil_div64(T, kChunkTokens); }
 
 // ---- router forward
 cudaError_t launch_router_fused(const __nv_bfloat16* x, const __nv_bfloat16* w_r, const float* bias,
@@ -33,20 +33,21 @@ cudaError_t launch_router_aux_loss(const float* stats, int E, int k, float n_tok
                                    float* loss, float* dprob, cudaStream_t st);
 
 // ---- routing metadata + permute
-cudaError_t launch_route_hist(const int32_t* idx, int T, int k, int E, int32_t* sub_counts,
-                              DeviceCtl* ctl, cudaStream_t st);
-cudaError_t launch_route_scan(int32_t* sub_counts, int64_t n_sub, int E, int align, int32_t* counts,
-                              int32_t* offsets, cudaStream_t st);
-cudaError_t launch_route_rank(const int32_t* idx, int T, int k, int E, const int32_t* sub_base,
-                              const int32_t* offsets, int32_t* row_map, cudaStream_t st);
+// counts, padded offsets and, in sub_counts [E][n_subchunks], the base of
+// every chunk (one launch; its last block scans; `ctl->ticket` must be 0).
+cudaError_t launch_route_count(const int32_t* idx, int T, int k, int E, int align,
+                               int32_t* sub_counts, int32_t* counts, int32_t* offsets,
+                               DeviceCtl* ctl, cudaStream_t st);
+// row_map, and with x_perm non-null the permuted copy (pad rows zeroed).
+cudaError_t launch_route_rank_scatter(const int32_t* idx, const __nv_bfloat16* x, int T, int k,
+                                      int E, const int32_t* sub_base, const int32_t* offsets,
+                                      const int32_t* counts, int d, int32_t* row_map,
+                                      __nv_bfloat16* x_perm, cudaStream_t st);
 // row_src [m_cap]: source token of every routed row, T for pad rows and rows
 // past the last segment.
 cudaError_t launch_route_src(const int32_t* row_map, const int32_t* offsets, const int32_t* counts,
                              int T, int k, int E, int64_t m_cap, int32_t* row_src,
                              cudaStream_t st);
-cudaError_t launch_permute_scatter(const __nv_bfloat16* x, const int32_t* row_map,
-                                   const int32_t* offsets, const int32_t* counts, int T, int d,
-                                   int k, int E, __nv_bfloat16* x_perm, cudaStream_t st);
 
 // ---- combine and backwards
 cudaError_t launch_combine(const __nv_bfloat16* o_perm, const int32_t* row_map, const float* w,
@@ -98,6 +99,12 @@ cudaError_t launch_mxfp8_quantize(const __nv_bfloat16* in, int64_t rows, int64_t
 // rows_per_group multiples of 128.
 cudaError_t launch_mxfp8_quantize_atoms(const __nv_bfloat16* in, int64_t rows, int64_t cols,
                                         uint8_t* q, uint8_t* scales, cudaStream_t st);
+// Both at once from one read: row-wise codes/scales (q_row, s_row) and
+// column-wise ones per group of rows_per_group rows (q_col, s_col); rows a
+// multiple of 32, cols and rows_per_group multiples of 128.
+cudaError_t launch_mxfp8_quantize_both(const __nv_bfloat16* in, int64_t rows, int64_t cols,
+                                       int64_t rows_per_group, uint8_t* q_row, uint8_t* s_row,
+                                       uint8_t* q_col, uint8_t* s_col, cudaStream_t st);
 cudaError_t launch_mxfp8_quantize_cols_t(const __nv_bfloat16* in, int64_t rows, int64_t cols,
                                          int64_t rows_per_group, uint8_t* q, uint8_t* scales,
                                          cudaStream_t st);

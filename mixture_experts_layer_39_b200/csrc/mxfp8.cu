@@ -184,6 +184,95 @@ __global__ void mx_colwise_kernel(const __nv_bfloat16* __restrict__ in, int64_t 
   }
 }
 
+// Both orientations of one operand in one pass (GEMM layouts, atom-ordered
+// scales).  A block of 128 threads takes a tile of 32 rows x 128 columns:
+// thread t loads 16 bytes (8 columns, c8 = t % 16) of rows t/16 + 8i,
+// i = 0..3.
+//   row-wise : blocks of 32 columns span 4 neighbouring lanes, whose maxima
+//              meet by two shuffles; codes to q_row, scales along the row;
+//   column-wise: the tile's 32 rows are one block of every column; each
+//              thread's 4-row maxima meet in shared memory, thread t takes
+//              column t's amax and writes its scale; codes to q_col.
+// The tile's 32 rows never straddle a group (rows_per_group is a multiple of
+// 128), so column blocks follow the per-group atom layout of scale_mode 1.
+__global__ void __launch_bounds__(128)
+    mx_both_kernel(const uint4* __restrict__ in, int64_t rows, int64_t cols, int64_t rows_per_group,
+                   uint2* __restrict__ q_row, uint8_t* __restrict__ s_row, uint2* __restrict__ q_col,
+                   uint8_t* __restrict__ s_col) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float s_part[8][128];
+  __shared__ int s_ecol[128];
+  const int t = threadIdx.x, c8 = t & 15, r0 = t >> 4;
+  const int64_t tiles_c = cols / 128;
+  const int64_t n_tiles = (rows / 32) * tiles_c;
+  const int64_t vec_row = cols / 8;  // 16-byte vectors per row
+  const int64_t n_kb4_row = cols / 128, bpg = rows_per_group / 32;
+  for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+    const int64_t tr = tile / tiles_c, tc = tile - tr * tiles_c;
+    const int64_t row0 = tr * 32, col0 = tc * 128;
+    float v[4][8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 w = __ldg(in + (row0 + r0 + 8 * i) * vec_row + (col0 >> 3) + c8);
+      unpack8(w, v[i]);
+    }
+    // ---- row-wise: block (row, 32 columns) over lanes 4j..4j+3 of this row
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float m = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[i][j]));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      const int e = mx_scale_exp(m);
+      const float inv = pow2_neg(e);
+      uint32_t p[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        p[h] = static_cast<uint32_t>(e4m3x2(v[i][4 * h] * inv, v[i][4 * h + 1] * inv)) |
+               (static_cast<uint32_t>(e4m3x2(v[i][4 * h + 2] * inv, v[i][4 * h + 3] * inv)) << 16);
+      const int64_t r = row0 + r0 + 8 * i;
+      q_row[r * (cols / 8) + (col0 >> 3) + c8] = make_uint2(p[0], p[1]);
+      if ((c8 & 3) == 0)
+        s_row[atom_byte(r, (col0 >> 5) + (c8 >> 2), n_kb4_row)] = static_cast<uint8_t>(e + 127);
+    }
+    // ---- column-wise: the 32 rows of the tile are one block of each column
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float m = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) m = fmaxf(m, fabsf(v[i][j]));
+      s_part[r0][8 * c8 + j] = m;
+    }
+    __syncthreads();
+    {
+      float m = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) m = fmaxf(m, s_part[k][t]);
+      const int e = mx_scale_exp(m);
+      s_ecol[t] = e;
+      const int64_t g = row0 / rows_per_group, rl = (row0 - g * rows_per_group) >> 5;
+      s_col[g * cols * bpg + atom_byte(col0 + t, rl, bpg >> 2)] = static_cast<uint8_t>(e + 127);
+    }
+    __syncthreads();
+    float inv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) inv[j] = pow2_neg(s_ecol[8 * c8 + j]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t p[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        p[h] = static_cast<uint32_t>(e4m3x2(v[i][4 * h] * inv[4 * h], v[i][4 * h + 1] * inv[4 * h + 1])) |
+               (static_cast<uint32_t>(e4m3x2(v[i][4 * h + 2] * inv[4 * h + 2],
+                                             v[i][4 * h + 3] * inv[4 * h + 3])) << 16);
+      q_col[(row0 + r0 + 8 * i) * (cols / 8) + (col0 >> 3) + c8] = make_uint2(p[0], p[1]);
+    }
+    __syncthreads();  // s_part / s_ecol are rewritten by the next tile
+  }
+}
+
 // Picks four columns per thread when every vector access stays aligned.
 cudaError_t launch_colwise(const __nv_bfloat16* in, int64_t rows, int64_t cols, uint8_t* q,
                            uint8_t* scales, int scale_mode, int64_t rows_per_group,
@@ -222,6 +311,17 @@ cudaError_t launch_mxfp8_quantize(const __nv_bfloat16* in, int64_t rows, int64_t
 cudaError_t launch_mxfp8_quantize_atoms(const __nv_bfloat16* in, int64_t rows, int64_t cols,
                                         uint8_t* q, uint8_t* scales, cudaStream_t st) {
   return launch_rowwise(in, rows, cols, q, scales, true, st);
+}
+
+cudaError_t launch_mxfp8_quantize_both(const __nv_bfloat16* in, int64_t rows, int64_t cols,
+                                       int64_t rows_per_group, uint8_t* q_row, uint8_t* s_row,
+                                       uint8_t* q_col, uint8_t* s_col, cudaStream_t st) {
+  const int64_t tiles = (rows / 32) * (cols / 128);
+  const unsigned grid = static_cast<unsigned>(tiles < 148 * 16 ? tiles : 148 * 16);
+  (void)launch_pdl(mx_both_kernel, grid, 128, 0, st, reinterpret_cast<const uint4*>(in), rows, cols,
+                   rows_per_group, reinterpret_cast<uint2*>(q_row), s_row,
+                   reinterpret_cast<uint2*>(q_col), s_col);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_mxfp8_quantize_cols_t(const __nv_bfloat16* in, int64_t rows, int64_t cols,

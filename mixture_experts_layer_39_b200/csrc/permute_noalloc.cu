@@ -2,7 +2,7 @@
 // callers that cannot hand the library any scratch memory.
 //
 // moe_permute needs a small scratch buffer (one expert histogram per
-// 256-entry chunk of the routing ids), which it takes from the caller's
+// 16-token chunk of the routing ids), which it takes from the caller's
 // workspace.  Some callers have no way to provide one: code embedded in a
 // host program that owns all device memory through its own pool and gives
 // plug-ins no allocation hook, or code on a latency-critical path that must
@@ -111,14 +111,13 @@ extern "C" moe_status_t moe_permute_noalloc(moe_handle_t h, const moe_shape_t* s
   if (found != MOE_OK) return found;
 
   auto st = static_cast<cudaStream_t>(stream);
-  h->launches += 4;
-  if (moe::launch_route_hist(topk_idx, T, k, E, sub, h->ctl, st) != cudaSuccess) return MOE_ERR_CUDA;
-  if (moe::launch_route_scan(sub, n_sub, E, moe::seg_align(s), counts, offsets, st) != cudaSuccess)
+  h->launches += 2;
+  if (moe::launch_route_count(topk_idx, T, k, E, moe::seg_align(s), sub, counts, offsets, h->ctl,
+                              st) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (moe::launch_route_rank(topk_idx, T, k, E, sub, offsets, row_map, st) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (moe::launch_permute_scatter(static_cast<const __nv_bfloat16*>(x), row_map, offsets, counts,
-                                  T, d, k, E, static_cast<__nv_bfloat16*>(x_perm), st) != cudaSuccess)
+  if (moe::launch_route_rank_scatter(topk_idx, static_cast<const __nv_bfloat16*>(x), T, k, E, sub,
+                                     offsets, counts, d, row_map,
+                                     static_cast<__nv_bfloat16*>(x_perm), st) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
 }

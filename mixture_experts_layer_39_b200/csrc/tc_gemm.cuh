@@ -519,6 +519,11 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
+// Waits until at most one of this thread's cp.async groups is still pending.
+__device__ __forceinline__ void cp_async_wait_group1() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- the kernel
 template <int BN, int STAGES, int EPI, bool FP8 = false, bool PAIR = false>
 struct SmemPlan {
@@ -536,7 +541,8 @@ struct SmemPlan {
   static constexpr int kMiscOff = kBarOff + kBarBytes;                 // tmem base, abort flag
   static constexpr int kEpiOff = (kMiscOff + 16 + 127) / 128 * 128;    // 4 epilogue warps' buffers
   // per warp: the 4 KB staging buffer, plus (SwiGLU backward) a 4 KB landing
-  // buffer that cp.async fills with the next 32 columns of the saved A and U
+  // buffer; the SwiGLU backward uses both as landing buffers that cp.async
+  // fills with the next two 32-column halves of the saved A and U
   static constexpr int kWarpEpiBytes = kEpiBufBytes + (EPI == EPI_SWIGLU_BWD ? kEpiBufBytes : 0);
   static constexpr int kTileOff = kEpiOff + 4 * kWarpEpiBytes;         // group tile starts
   static constexpr int bytes(int n_groups) { return 1024 + kTileOff + 4 * (n_groups + 1); }
@@ -981,17 +987,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Tile tl = decode_tile<KGROUP, BKE, KMMA, MT>(args, s_tile_start, t);
       const int vrows = quarter_rows(tl);
       const int64_t row_first = quarter_first(tl);  // warp's first row
-      // SwiGLU backward: the saved A and U of the first 32 columns are
-      // requested before waiting for the accumulator, so their latency
-      // overlaps the main loop; each later 32 columns are requested while the
-      // previous ones are computed.
+      // SwiGLU backward: the saved A and U of the first two 32-column halves
+      // are requested before waiting for the accumulator, so their latency
+      // overlaps the main loop; each later half is requested two halves ahead
+      // of its use.
       const __nv_bfloat16* aux = nullptr;
       if constexpr (EPI == EPI_SWIGLU_BWD) {
+        // halves 0 and 1 into the two landing buffers (the staging buffer is
+        // the second: this epilogue stores straight from registers)
         aux = args.aux + row_first * args.ld_aux + static_cast<int64_t>(tl.n_tile) * BN;
-        cp_async_au(lbuf, reinterpret_cast<const uint8_t*>(aux),
-                    reinterpret_cast<const uint8_t*>(aux + args.f), args.ld_aux * 2, vrows, lane,
-                    args.aux);
-        cp_async_commit();
+        const int ncols0 = args.n_cols - tl.n_tile * BN < BN ? args.n_cols - tl.n_tile * BN : BN;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (32 * h < ncols0) {
+            cp_async_au(h ? ebuf : lbuf, reinterpret_cast<const uint8_t*>(aux + 32 * h),
+                        reinterpret_cast<const uint8_t*>(aux + args.f + 32 * h), args.ld_aux * 2,
+                        vrows, lane, args.aux);
+            cp_async_commit();
+          }
+        }
       }
       const bool ok = __all_sync(
           0xffffffffu, mbar_wait(tfull_bar(acc), acc_phase, s_abort, args.wait_ns, true, PAIR));
@@ -1084,54 +1098,54 @@ __global__ void __launch_bounds__(kThreads, 1)
           store_rows(ebuf, lane, vh, reinterpret_cast<uint8_t*>(hh + c), args.ldo2 * 2, vrows);
         }
       } else {  // EPI_SWIGLU_BWD
-        auto* dau = static_cast<__nv_bfloat16*>(args.out) + row_first * args.ldo +
-                    static_cast<int64_t>(tl.n_tile) * BN;
+        // 32 columns at a time; the saved A and U of the next two 32-column
+        // halves are in flight in the two landing buffers while one is
+        // computed (the latency of one L2 round trip under load is about the
+        // time of two halves).  Each lane stores dA and dU of its own row.
+        uint4* drow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) +
+                                               (row_first + lane) * args.ldo +
+                                               static_cast<int64_t>(tl.n_tile) * BN);
+        uint4* urow = drow + args.f / 8;
+        const int nh = ncols / 32;
 #pragma unroll 1
-        for (int c = 0; c < ncols; c += 64) {
-          uint4 ou[8];  // dU in registers; dA goes straight to the staging buffer
+        for (int h = 0; h < nh; ++h) {
+          uint8_t* buf = (h & 1) ? ebuf : lbuf;
+          if (h + 1 < nh) cp_async_wait_group1(); else cp_async_wait_all();
+          __syncwarp();
+          uint4 vau[8];  // this lane's row: A in slots 0-3, U in slots 4-7
+          stage_read_row(buf, lane, vau);
+          __syncwarp();
+          if (h + 2 < nh) {
+            cp_async_au(buf, reinterpret_cast<const uint8_t*>(aux + 32 * (h + 2)),
+                        reinterpret_cast<const uint8_t*>(aux + args.f + 32 * (h + 2)),
+                        args.ld_aux * 2, vrows, lane, args.aux);
+            cp_async_commit();
+          }
+          uint32_t r[32];
+          tmem_ld32(tbase + tcol(32 * h), r);
+          tmem_ld_wait();
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int cc = c + 32 * half;
-            uint4 vau[8];  // this lane's row: A in slots 0-3, U in slots 4-7
-            cp_async_wait_all();
-            __syncwarp();
-            stage_read_row(lbuf, lane, vau);
-            __syncwarp();
-            if (cc + 32 < ncols) {  // the next 32 columns land while these are computed
-              cp_async_au(lbuf, reinterpret_cast<const uint8_t*>(aux + cc + 32),
-                          reinterpret_cast<const uint8_t*>(aux + args.f + cc + 32),
-                          args.ld_aux * 2, vrows, lane, args.aux);
-              cp_async_commit();
+          for (int q = 0; q < 4; ++q) {
+            const uint4 qa = vau[q], qu = vau[4 + q];
+            const float a[8] = {bf16_lo(qa.x), bf16_hi(qa.x), bf16_lo(qa.y), bf16_hi(qa.y),
+                                bf16_lo(qa.z), bf16_hi(qa.z), bf16_lo(qa.w), bf16_hi(qa.w)};
+            const float u[8] = {bf16_lo(qu.x), bf16_hi(qu.x), bf16_lo(qu.y), bf16_hi(qu.y),
+                                bf16_lo(qu.z), bf16_hi(qu.z), bf16_lo(qu.w), bf16_hi(qu.w)};
+            float da[8], du[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float dh = __uint_as_float(r[8 * q + i]);
+              const float sg = sigmoid_fast(a[i]);
+              da[i] = dh * u[i] * sg * (1.0f + a[i] * (1.0f - sg));
+              du[i] = dh * a[i] * sg;
             }
-            uint32_t r[32];
-            tmem_ld32(tbase + tcol(cc), r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 qa = vau[q], qu = vau[4 + q];
-              const float a[8] = {bf16_lo(qa.x), bf16_hi(qa.x), bf16_lo(qa.y), bf16_hi(qa.y),
-                                  bf16_lo(qa.z), bf16_hi(qa.z), bf16_lo(qa.w), bf16_hi(qa.w)};
-              const float u[8] = {bf16_lo(qu.x), bf16_hi(qu.x), bf16_lo(qu.y), bf16_hi(qu.y),
-                                  bf16_lo(qu.z), bf16_hi(qu.z), bf16_lo(qu.w), bf16_hi(qu.w)};
-              float da[8], du[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float dh = __uint_as_float(r[8 * q + i]);
-                const float sg = sigmoid_fast(a[i]);
-                da[i] = dh * u[i] * sg * (1.0f + a[i] * (1.0f - sg));
-                du[i] = dh * a[i] * sg;
-              }
-              *stage_slot(ebuf, lane, 4 * half + q) =
-                  make_uint4(pack_bf16x2(da[0], da[1]), pack_bf16x2(da[2], da[3]),
-                             pack_bf16x2(da[4], da[5]), pack_bf16x2(da[6], da[7]));
-              ou[4 * half + q] = make_uint4(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]),
-                                            pack_bf16x2(du[4], du[5]), pack_bf16x2(du[6], du[7]));
+            if (lane < vrows) {
+              drow[4 * h + q] = make_uint4(pack_bf16x2(da[0], da[1]), pack_bf16x2(da[2], da[3]),
+                                           pack_bf16x2(da[4], da[5]), pack_bf16x2(da[6], da[7]));
+              urow[4 * h + q] = make_uint4(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]),
+                                           pack_bf16x2(du[4], du[5]), pack_bf16x2(du[6], du[7]));
             }
           }
-          __syncwarp();
-          stage_to_global(ebuf, reinterpret_cast<uint8_t*>(dau + c), args.ldo * 2, vrows, lane);
-          __syncwarp();
-          store_rows(ebuf, lane, ou, reinterpret_cast<uint8_t*>(dau + args.f + c), args.ldo * 2, vrows);
         }
       }
       tc_fence_before();
