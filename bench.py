@@ -234,11 +234,17 @@ def measure(L, g, steps, warmup, flush, dev, with_gemm_events=True):
             L.load_stats()
             L.balance_loss()
         if ev: ev[0].record(stream)
-        L.experts_fwd(g["w_gu"], g["w_d"])
-        if L.shared_ff > 0:
-            L.shared_fwd(g["x"], g["w_gu_s"], g["w_d_s"])
+        if L.fuse_combine:  # the shared expert first; the combine runs in the down GEMM
+            if L.shared_ff > 0:
+                L.shared_fwd(g["x"], g["w_gu_s"], g["w_d_s"])
+            L.experts_fwd(g["w_gu"], g["w_d"])
+        else:
+            L.experts_fwd(g["w_gu"], g["w_d"])
+            if L.shared_ff > 0:
+                L.shared_fwd(g["x"], g["w_gu_s"], g["w_d_s"])
         if ev: ev[1].record(stream)
-        L.combine()
+        if not L.fuse_combine:
+            L.combine()
         L.combine_bwd(g["dy"])
         L.router_bwd(g["x"], g["w_r"])
         if ev: ev[2].record(stream)
@@ -421,6 +427,8 @@ def run_ours(args):
         variants["aux_loss"] = bench_cfg(cfg, args.steps, args.warmup, False, aux_alpha=0.01)
         variants["recompute"] = bench_cfg(cfg, args.steps, args.warmup, False, recompute=True)
         variants["gather"] = bench_cfg(cfg, args.steps, args.warmup, False, gather=True)
+        variants["fused_combine"] = bench_cfg(cfg, args.steps, args.warmup, False,
+                                              fuse_combine=True)
         if cfg.name == "e8":
             variants["shared_expert"] = bench_cfg(CONFIGS["e8_shared"], args.steps, args.warmup,
                                                   False, shared_ff=CONFIGS["e8_shared"].shared_ff)
@@ -517,6 +525,11 @@ def run_ours(args):
             line["variants"]["gather"]["what"] = (
                 "no permuted copy of x: the gate/up GEMM and its weight gradient gather the routed "
                 "rows from x with TMA tile::gather4 (moe_route + *_gather entry points)")
+        if "fused_combine" in variants:
+            line["variants"]["fused_combine"]["what"] = (
+                "the weighted unpermute-combine inside the down projection's epilogue "
+                "(moe_permute_src + moe_grouped_swiglu_fwd_combine): the arrival that completes "
+                "a token's rows sums them, same bits as the combine kernel, no separate launch")
         if "shared_expert" in variants:
             sc = CONFIGS["e8_shared"]
             v = variants["shared_expert"]

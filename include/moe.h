@@ -179,7 +179,7 @@ MOE_API moe_status_t moe_permute(moe_handle_t h, const moe_shape_t* s, const voi
  * Same arguments, outputs and device-side checks as moe_permute.  Its scratch
  * is a fixed 1 MiB array inside the library (one per GPU that loads it, held
  * until the process exits), so the shape must satisfy
- *   ceil(T / 16) * E <= MOE_NOALLOC_SCRATCH_INTS,
+ *   (ceil(T / 64) + ceil(T / 512)) * E <= MOE_NOALLOC_SCRATCH_INTS,
  * otherwise MOE_ERR_WORKSPACE is returned before any launch.  The first call
  * on a device looks up the array's device address (a host-side step, done
  * once per device with that device current); make that first call before
@@ -230,6 +230,42 @@ MOE_API moe_status_t moe_grouped_swiglu_recompute(moe_handle_t h, const moe_shap
                                                   const void* x_perm, const int32_t* offsets,
                                                   const void* w_gu, void* au, void* hbuf, void* ws,
                                                   size_t ws_bytes, moe_stream_t stream);
+
+/* moe_permute that also writes row_src [M_cap] int32: the token whose copy
+ * each routed row holds, T on the segments' pad rows (rows past offsets[E]
+ * are not written).  Same passages as moe_permute (Olmo-core 3 introduction
+ * page, section 2; discosf.com article on Olmo-core 3, section 2.1); it
+ * feeds moe_grouped_swiglu_fwd_combine.  Same workspace and checks. */
+MOE_API moe_status_t moe_permute_src(moe_handle_t h, const moe_shape_t* s, const void* x,
+                                     const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                                     int32_t* row_map, int32_t* row_src, void* x_perm, void* ws,
+                                     size_t ws_bytes, moe_stream_t stream);
+
+/* moe_grouped_swiglu_fwd with the weighted unpermute-combine fused into the
+ * down projection's epilogue ("restore" step: discosf.com article on
+ * Olmo-core 3, section 2.1; the grouped GEMM: Olmo-core 3 introduction page,
+ * section 2).  Besides au, h and o_perm it writes
+ *   y[t] = bf16( sum_j topk_w[t,j] * o_perm[row_map[t,j]] + shared_out[t] ),
+ * the same bits as moe_unpermute_combine on the same inputs: every stored
+ * routed row counts one arrival for its token and column tile of 256, and
+ * the epilogue that completes a token's valid rows sums them in slot order
+ * from the stored bf16 rows (no floating-point atomics) and clears the
+ * count.  bf16 only (MOE_ERR_UNSUPPORTED for MXFP8).
+ * In : as moe_grouped_swiglu_fwd, plus row_map [T,k], row_src [M_cap] (from
+ *      moe_permute_src), topk_w [T,k] fp32, shared_out [T,d] bf16 or NULL
+ *      (a shared expert's output, computed before this call).
+ * Out: au (or NULL), h, o_perm as moe_grouped_swiglu_fwd; y [T,d] bf16.
+ * arrivals [T, ceil(d/256)] int32: caller-owned, all zero before the first
+ *      call; every completed call leaves it zero again.  A call stopped by an
+ *      error (MOE_ERR_TIMEOUT, or ids outside [0,E) in the permute) may leave
+ *      counts behind: clear it before the next call. */
+MOE_API moe_status_t moe_grouped_swiglu_fwd_combine(moe_handle_t h, const moe_shape_t* s,
+                                                    const void* x_perm, const int32_t* offsets,
+                                                    const int32_t* row_map, const int32_t* row_src,
+                                                    const float* topk_w, const void* w_gu,
+                                                    const void* w_down, void* au, void* hbuf,
+                                                    void* o_perm, const void* shared_out, void* y,
+                                                    int32_t* arrivals, moe_stream_t stream);
 
 /* ---- Gather forms: the routed copies of x are never written.  Instead of
  * a materialised x_perm, the two expert GEMMs that read routed rows of x

@@ -39,6 +39,8 @@ SIGNATURES = {
     "moe_permute": [P, SP, P, P, P, P, P, P, P, c_size_t, P],
     "moe_permute_noalloc": [P, SP, P, P, P, P, P, P, P],
     "moe_route": [P, SP, P, P, P, P, P, P, c_size_t, P],
+    "moe_permute_src": [P, SP, P, P, P, P, P, P, P, P, c_size_t, P],
+    "moe_grouped_swiglu_fwd_combine": [P, SP, P, P, P, P, P, P, P, P, P, P, P, P, P, P],
     "moe_grouped_swiglu_fwd_gather": [P, SP, P, P, P, P, P, P, P, P, P],
     "moe_grouped_swiglu_recompute_gather": [P, SP, P, P, P, P, P, P, P],
     "moe_grouped_swiglu_bwd_gather": [P, SP, P, P, P, P, P, P, P, P, P, P, P, P, P],

@@ -127,7 +127,7 @@ size_t scratch_bytes(const moe_context* h, const moe_shape_t* s) {
     upd(w.bwd_total);
   }
   upd(align256(static_cast<size_t>(T) * router_ld(static_cast<int>(E)) * 4));       // router logits
-  upd(align256(static_cast<size_t>(moe::n_subchunks(s->T, s->top_k)) * E * 4));    // permute
+  upd(align256(static_cast<size_t>(moe::route_scratch_ints(s->T, s->n_experts)) * 4));  // permute
   upd(router_bwd_layout(h, s).total);                                              // router bwd
   return need;
 }
@@ -271,7 +271,55 @@ moe_status_t moe_permute(moe_handle_t h, const moe_shape_t* s, const void* x,
                                               offsets, h->ctl, st)));
   return cuda_status(moe::launch_route_rank_scatter(
       topk_idx, static_cast<const __nv_bfloat16*>(x), T, k, E, sub, offsets, counts, d, row_map,
-      static_cast<__nv_bfloat16*>(x_perm), st));
+      static_cast<__nv_bfloat16*>(x_perm), nullptr, st));
+}
+
+moe_status_t moe_permute_src(moe_handle_t h, const moe_shape_t* s, const void* x,
+                             const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                             int32_t* row_map, int32_t* row_src, void* x_perm, void* ws,
+                             size_t ws_bytes, moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  if (!all_nonnull(x, topk_idx, counts, offsets, row_map, row_src, x_perm))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(x_perm, 16)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(h, s, ws, ws_bytes));
+  const int T = s->T, d = s->d_model, E = s->n_experts, k = s->top_k;
+  auto st = static_cast<cudaStream_t>(stream);
+  MOE_GUARD(h);
+  auto* sub = static_cast<int32_t*>(ws);
+  h->launches += 2;
+  MOE_TRY(cuda_status(moe::launch_route_count(topk_idx, T, k, E, moe::seg_align(s), sub, counts,
+                                              offsets, h->ctl, st)));
+  return cuda_status(moe::launch_route_rank_scatter(
+      topk_idx, static_cast<const __nv_bfloat16*>(x), T, k, E, sub, offsets, counts, d, row_map,
+      static_cast<__nv_bfloat16*>(x_perm), row_src, st));
+}
+
+moe_status_t moe_grouped_swiglu_fwd_combine(moe_handle_t h, const moe_shape_t* s,
+                                            const void* x_perm, const int32_t* offsets,
+                                            const int32_t* row_map, const int32_t* row_src,
+                                            const float* topk_w, const void* w_gu,
+                                            const void* w_down, void* au, void* hbuf,
+                                            void* o_perm, const void* shared_out, void* y,
+                                            int32_t* arrivals, moe_stream_t stream) {
+  MOE_CHECK_HANDLE(h, s);
+  if (s->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (!all_nonnull(x_perm, offsets, row_map, row_src, topk_w, w_gu, w_down, hbuf, o_perm, y,
+                   arrivals))
+    return MOE_ERR_INVALID_ARG;
+  for (const void* p : {x_perm, w_gu, w_down, static_cast<const void*>(au),
+                        static_cast<const void*>(hbuf), static_cast<const void*>(o_perm),
+                        shared_out, static_cast<const void*>(y)})
+    if (!aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  const int d = s->d_model, f = s->d_ff, E = s->n_experts;
+  const int64_t m_cap = max_rows(s);
+  auto st = static_cast<cudaStream_t>(stream);
+  MOE_GUARD(h);
+  const moe::GemmCtx c = gemm_ctx(h, pair_tiles(s));
+  const moe::CombineArgs cb{row_src, row_map, topk_w, shared_out, y, arrivals, s->T, s->top_k};
+  h->launches += 2;
+  MOE_TRY(moe::gemm_fwd_gate_up(c, x_perm, offsets, w_gu, au, hbuf, E, d, f, m_cap, st));
+  return moe::gemm_fwd_down_combine(c, hbuf, offsets, w_down, o_perm, E, d, f, m_cap, cb, st);
 }
 
 // ---- gather forms (no materialised x_perm; bf16)
@@ -289,7 +337,8 @@ moe_status_t moe_route(moe_handle_t h, const moe_shape_t* s, const int32_t* topk
   MOE_TRY(cuda_status(moe::launch_route_count(topk_idx, T, k, E, moe::seg_align(s), sub, counts,
                                               offsets, h->ctl, st)));
   MOE_TRY(cuda_status(moe::launch_route_rank_scatter(topk_idx, nullptr, T, k, E, sub, offsets,
-                                                     counts, s->d_model, row_map, nullptr, st)));
+                                                     counts, s->d_model, row_map, nullptr, nullptr,
+                                                     st)));
   return cuda_status(
       moe::launch_route_src(row_map, offsets, counts, T, k, E, max_rows(s), row_src, st));
 }

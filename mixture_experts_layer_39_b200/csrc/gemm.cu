@@ -229,6 +229,36 @@ moe_status_t gemm_fwd_down(const GemmCtx& c, const void* h, const int32_t* offse
   return launch<256, false, false, tc::EPI_BF16, false>(ta, tb, a, c.num_sms, st);
 }
 
+moe_status_t gemm_fwd_down_combine(const GemmCtx& c, const void* h, const int32_t* offsets,
+                                   const void* w_d, void* o_perm, int E, int d, int f,
+                                   int64_t m_cap, const CombineArgs& cb, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, h, f, m_cap, 2ull * f, 64, 128)) return MOE_ERR_CUDA;
+  if (!tmap_3d(&tb, w_d, f, d, E, 2ull * f, 2ull * d * f, 64, c.pair_m ? 128 : 256))
+    return MOE_ERR_CUDA;
+  tc::GemmArgs a = base_args(c);
+  set_n(a, d, 256);
+  a.k_blocks = f / tc::BK;
+  a.n_groups = E;
+  a.offsets = offsets;
+  a.total_len = static_cast<int>(m_cap);
+  a.uniform_len = static_cast<int>(m_cap);
+  a.m_cap = m_cap;
+  a.out = o_perm;
+  a.ldo = d;
+  a.row_src = cb.row_src;
+  a.row_map = cb.row_map;
+  a.topk_w = cb.topk_w;
+  a.shared = static_cast<const __nv_bfloat16*>(cb.shared);
+  a.y = static_cast<__nv_bfloat16*>(cb.y);
+  a.arrivals = cb.arrivals;
+  a.n_tok = cb.T;
+  a.top_k = cb.k;
+  if (c.pair_m)
+    return launch<256, false, false, tc::EPI_BF16_COMBINE, false, false, true>(ta, tb, a, c.num_sms, st);
+  return launch<256, false, false, tc::EPI_BF16_COMBINE, false>(ta, tb, a, c.num_sms, st);
+}
+
 moe_status_t gemm_dgrad_down_swiglu(const GemmCtx& c, const void* do_perm, const int32_t* offsets,
                                     const void* w_d, const void* au, void* dau, int E, int d,
                                     int f, int64_t m_cap, cudaStream_t st) {

@@ -28,6 +28,20 @@ moe_status_t gemm_fwd_gate_up(const GemmCtx& c, const void* x_perm, const int32_
 moe_status_t gemm_fwd_down(const GemmCtx& c, const void* h, const int32_t* offsets,
                            const void* w_d, void* o_perm, int E, int d, int f, int64_t m_cap,
                            cudaStream_t st);
+// The down projection with the unpermute-combine fused into its epilogue:
+// also y[t] = bf16(sum_j topk_w[t,j] O[row_map[t,j]] (+ shared[t])).
+struct CombineArgs {
+  const int32_t* row_src;  // [m_cap] token of each routed row, T on pad rows
+  const int32_t* row_map;  // [T, k]
+  const float* topk_w;     // [T, k]
+  const void* shared;      // [T, d] bf16 or nullptr
+  void* y;                 // [T, d] bf16
+  int32_t* arrivals;       // [T, ceil(d / 256)], zero on entry and on return
+  int T, k;
+};
+moe_status_t gemm_fwd_down_combine(const GemmCtx& c, const void* h, const int32_t* offsets,
+                                   const void* w_d, void* o_perm, int E, int d, int f,
+                                   int64_t m_cap, const CombineArgs& cb, cudaStream_t st);
 moe_status_t gemm_dgrad_down_swiglu(const GemmCtx& c, const void* do_perm, const int32_t* offsets,
                                     const void* w_d, const void* au, void* dau, int E, int d,
                                     int f, int64_t m_cap, cudaStream_t st);

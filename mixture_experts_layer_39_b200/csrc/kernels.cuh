@@ -6,11 +6,18 @@
 
 namespace moe {
 
-// Chunk of tokens (k flat (token, slot) entries each) counted by one warp
-// and ranked and copied by one block of the routing-metadata kernels.
+// Routing metadata: a warp counts kCountTokens tokens (k flat (token, slot)
+// entries each), eight such chunks to a block; a block ranks and copies
+// kChunkTokens tokens.
+constexpr int kCountTokens = 64;
 constexpr int kChunkTokens = 16;
 
-inline int64_t n_subchunks(int T, int /*k*/) { return ceil_div64(T, kChunkTokens); }
+inline int64_t count_chunks(int T) { return ceil_div64(T, kCountTokens); }
+inline int64_t count_blocks(int T) { return ceil_div64(count_chunks(T), 8); }
+// int32 scratch of the two routing-metadata launches
+inline int64_t route_scratch_ints(int T, int E) {
+  return static_cast<int64_t>(E) * (count_chunks(T) + count_blocks(T));
+}
 
 // ---- router forward
 cudaError_t launch_router_fused(const __nv_bfloat16* x, const __nv_bfloat16* w_r, const float* bias,
@@ -33,16 +40,18 @@ cudaError_t launch_router_aux_loss(const float* stats, int E, int k, float n_tok
                                    float* loss, float* dprob, cudaStream_t st);
 
 // ---- routing metadata + permute
-// counts, padded offsets and, in sub_counts [E][n_subchunks], the base of
-// every chunk (one launch; its last block scans; `ctl->ticket` must be 0).
+// counts, padded offsets and, in scratch (route_scratch_ints), the chunk and
+// block bases (one launch; its last block scans; `ctl->ticket` must be 0).
 cudaError_t launch_route_count(const int32_t* idx, int T, int k, int E, int align,
-                               int32_t* sub_counts, int32_t* counts, int32_t* offsets,
+                               int32_t* scratch, int32_t* counts, int32_t* offsets,
                                DeviceCtl* ctl, cudaStream_t st);
-// row_map, and with x_perm non-null the permuted copy (pad rows zeroed).
+// row_map, and with x_perm non-null the permuted copy (pad rows zeroed) and,
+// with row_src also non-null, the token of every row in a segment (T on the
+// segments' pad rows; rows past the last segment are not written).
 cudaError_t launch_route_rank_scatter(const int32_t* idx, const __nv_bfloat16* x, int T, int k,
-                                      int E, const int32_t* sub_base, const int32_t* offsets,
+                                      int E, const int32_t* scratch, const int32_t* offsets,
                                       const int32_t* counts, int d, int32_t* row_map,
-                                      __nv_bfloat16* x_perm, cudaStream_t st);
+                                      __nv_bfloat16* x_perm, int32_t* row_src, cudaStream_t st);
 // row_src [m_cap]: source token of every routed row, T for pad rows and rows
 // past the last segment.
 cudaError_t launch_route_src(const int32_t* row_map, const int32_t* offsets, const int32_t* counts,

@@ -9,19 +9,26 @@
 //
 // Metadata is computed in two launches, deterministically, so that the row
 // of every (token, slot) entry is exactly the stable expert-major order.
-// The entries are cut into chunks of kChunkTokens tokens (k entries each).
-//   count        : a warp per chunk counts its experts; the last block to
-//                  finish (a ticket in the handle's control block, no
-//                  waiting) scans, per expert, over the chunks (the base of
-//                  each chunk) and then the padded segment offsets;
-//   rank+scatter : a block of 4 warps per chunk: its first warp walks the
-//                  chunk 32 entries at a time (the rank of an entry among
-//                  equal experts in a batch comes from __match_any_sync, and
-//                  the per-expert running base advances by the batch's
-//                  count), then the 4 warps copy the chunk's tokens to their
-//                  rows; blocks past the chunks zero each segment's pad rows.
-//                  Small blocks keep about 7 resident per SM, so the chunks
-//                  fill the SMs in one balanced wave.
+// The entries are counted in chunks of kCountTokens tokens (k entries each),
+// eight chunks to a block, and ranked and copied in blocks of kChunkTokens
+// tokens.
+//   count        : a warp per chunk counts its experts; each block writes,
+//                  per expert, the prefix of its chunks inside the block and
+//                  the block's total; the last block to finish (a ticket in
+//                  the handle's control block, no waiting) scans the block
+//                  totals per expert and then the padded segment offsets;
+//   rank+scatter : a block of 4 warps per 16 tokens: its first warp adds up
+//                  the bases (segment start + block base + chunk prefix + the
+//                  entries of the chunk before these 16 tokens), walks its
+//                  entries 32 at a time (the rank of an entry among equal
+//                  experts in a batch comes from __match_any_sync, and the
+//                  per-expert running base advances by the batch's count),
+//                  then the 4 warps copy the tokens to their rows; blocks
+//                  past the tokens zero each segment's pad rows.  Small blocks
+//                  keep about 7 resident per SM, so the blocks fill the SMs in
+//                  one balanced wave.
+#include <climits>
+
 #include "kernels.cuh"
 
 namespace moe {
@@ -36,15 +43,17 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
-// Block of kWarps warps; warp w counts chunk blockIdx.x * kWarps + w into
-// sub[e * n_sub + c].  The last block to finish then turns sub into each
-// chunk's base (exclusive scan over chunks, per expert), writes counts and
-// the segments' offsets (starts rounded up to `align` rows) and resets the
-// ticket for the next launch.
+// Block b of kWarps warps; warp w counts chunk c = b * kWarps + w.  Scratch:
+// pre[e * n_sub + c] = the entries of expert e in the block's chunks before c;
+// blk[e * n_blk + b] = the block's total for e, turned by the last block into
+// the exclusive scan over blocks (the block's base).  The last block also
+// writes counts and the segments' offsets (starts rounded up to `align`
+// rows) and resets the ticket for the next launch.
 __global__ void __launch_bounds__(kWarps * 32)
     route_count_kernel(const int32_t* __restrict__ idx, int64_t n_entries, int k, int E,
-                       int64_t n_sub, int align, int32_t* __restrict__ sub,
-                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets, DeviceCtl* ctl) {
+                       int64_t n_sub, int64_t n_blk, int align, int32_t* __restrict__ pre,
+                       int32_t* __restrict__ blk, int32_t* __restrict__ counts,
+                       int32_t* __restrict__ offsets, DeviceCtl* ctl) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ int s_cnt[];  // kWarps x E (reused by the scan)
@@ -56,55 +65,88 @@ __global__ void __launch_bounds__(kWarps * 32)
   __syncwarp();
   const int64_t c = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
   if (c < n_sub) {
-    const int64_t per = static_cast<int64_t>(kChunkTokens) * k;
+    const int64_t per = static_cast<int64_t>(kCountTokens) * k;
     const int64_t beg = c * per;
     const int64_t end = beg + per < n_entries ? beg + per : n_entries;
-    for (int64_t i = beg + lane; i < end; i += 32) {
-      const int e = __ldg(idx + i);
-      if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
-      else report(ctl, MOE_ERR_DEVICE_CHECK, 200);
+    // eight ids per lane in flight at once (a chunk holds at most 64 * 8)
+    for (int64_t i0 = beg; i0 < end; i0 += 32 * 8) {
+      int ids[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t i = i0 + 32 * u + lane;
+        ids[u] = i < end ? __ldg(idx + i) : INT_MIN;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int e = ids[u];
+        if (e == INT_MIN) continue;
+        if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+        else report(ctl, MOE_ERR_DEVICE_CHECK, 200);
+      }
     }
-    __syncwarp();
-    for (int e = lane; e < E; e += 32) sub[static_cast<int64_t>(e) * n_sub + c] = cnt[e];
   }
-  // publish this block's counts, then take a ticket; the last one scans
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kWarps * 32) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const int64_t cw = static_cast<int64_t>(blockIdx.x) * kWarps + w;
+      if (cw < n_sub) pre[static_cast<int64_t>(e) * n_sub + cw] = run;
+      run += s_cnt[w * E + e];
+    }
+    blk[static_cast<int64_t>(e) * n_blk + blockIdx.x] = run;
+  }
+  // publish this block's results, then take a ticket; the last one scans
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) s_ticket = atomicAdd(&ctl->ticket, 1u);
   __syncthreads();
   if (s_ticket != gridDim.x - 1) return;
   __threadfence();
+  // per expert, exclusive scan of the block totals: warp w takes experts
+  // w + kWarps * (4g + q), four at a time, each lane a run of 4 blocks of a
+  // 128-block segment, so that a segment's loads are all in flight at once
   int* s_tot = s_cnt;  // E totals
-  for (int e = warp; e < E; e += kWarps) {
-    int32_t* row = sub + static_cast<int64_t>(e) * n_sub;
-    int carry = 0;
-    for (int64_t base = 0; base < n_sub; base += 32 * 4) {
-      int v[4];
-      int local = 0;
+  for (int e0 = warp; e0 < E; e0 += 4 * kWarps) {
+    int carry[4] = {0, 0, 0, 0};
+    for (int64_t s0 = 0; s0 < n_blk; s0 += 128) {
+      int v[4][4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t i = base + lane * 4 + u;
-        v[u] = i < n_sub ? __ldcg(row + i) : 0;
-        local += v[u];
-      }
-      int incl = local;
+      for (int q = 0; q < 4; ++q) {
+        const int e = e0 + q * kWarps;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
+        for (int u = 0; u < 4; ++u) {
+          const int64_t b = s0 + lane * 4 + u;
+          v[q][u] = (e < E && b < n_blk) ? __ldcg(blk + static_cast<int64_t>(e) * n_blk + b) : 0;
+        }
       }
-      int run = carry + incl - local;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t i = base + lane * 4 + u;
-        if (i < n_sub) row[i] = run;
-        run += v[u];
+      for (int q = 0; q < 4; ++q) {
+        const int e = e0 + q * kWarps;
+        const int local = v[q][0] + v[q][1] + v[q][2] + v[q][3];
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        int run = carry[q] + incl - local;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t b = s0 + lane * 4 + u;
+          if (e < E && b < n_blk) blk[static_cast<int64_t>(e) * n_blk + b] = run;
+          run += v[q][u];
+        }
+        carry[q] += __shfl_sync(0xffffffffu, incl, 31);
       }
-      carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) {
-      counts[e] = carry;
-      s_tot[e] = carry;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = e0 + q * kWarps;
+      if (e < E && lane == 0) {
+        counts[e] = carry[q];
+        s_tot[e] = carry[q];
+      }
     }
   }
   __syncthreads();
@@ -137,39 +179,76 @@ __global__ void __launch_bounds__(kWarps * 32)
   if (threadIdx.x == 0) ctl->ticket = 0u;
 }
 
-// Blocks [0, n_sub): chunk c -- warp 0 ranks its entries into row_map (and
-// shared memory); then, with SCATTER, the block's warps copy each token's
-// row of x to its k rows, two tokens per warp at a time.  Blocks past
-// n_sub (SCATTER only): warp w of block n_sub + b zero-fills the pad rows
-// of expert b * kRsWarps + w.  An entry with an id outside [0, E) gets row -1
-// (the count kernel recorded MOE_ERR_DEVICE_CHECK) and is not copied.
+// Blocks [0, n_rs): tokens [16 b, 16 b + 16) -- warp 0 ranks their entries
+// into row_map (and shared memory; with row_src non-null it also records the
+// token of every row it assigns); then, with SCATTER, the block's warps
+// copy each token's row of x to its k rows, two tokens per warp at a time.
+// Blocks past n_rs (SCATTER only): warp w of block n_rs + b zero-fills the
+// pad rows of expert b * kRsWarps + w (and marks them in row_src with T, when
+// given).  An entry with an id outside [0, E)
+// gets row -1 (the count kernel recorded MOE_ERR_DEVICE_CHECK) and is not
+// copied.
 template <bool SCATTER>
 __global__ void __launch_bounds__(kRsWarps * 32)
     route_rank_scatter_kernel(const int32_t* __restrict__ idx, const uint4* __restrict__ x,
-                              int T, int k, int E, int64_t n_sub,
-                              const int32_t* __restrict__ sub_base,
+                              int T, int k, int E, int64_t n_rs, int64_t n_sub, int64_t n_blk,
+                              const int32_t* __restrict__ pre, const int32_t* __restrict__ blk,
                               const int32_t* __restrict__ offsets,
                               const int32_t* __restrict__ counts, int nvec,
-                              int32_t* __restrict__ row_map, uint4* __restrict__ x_perm) {
+                              int32_t* __restrict__ row_map, uint4* __restrict__ x_perm,
+                              int32_t* __restrict__ row_src) {
   pdl_wait();
   pdl_trigger();
-  extern __shared__ int s_base[];  // E running bases, then the chunk's rows
+  extern __shared__ int s_base[];  // E running bases, then the block's rows
   int* s_rows = s_base + E;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t c = blockIdx.x;
-  if (c < n_sub) {
+  if (c < n_rs) {
+    constexpr int kPerCount = kCountTokens / kChunkTokens;  // rank blocks per count chunk
     const int64_t n_entries = static_cast<int64_t>(T) * k;
     const int64_t per = static_cast<int64_t>(kChunkTokens) * k;
     const int64_t beg = c * per;
     const int64_t end = beg + per < n_entries ? beg + per : n_entries;
     if (warp == 0) {
+      const int64_t cc = c / kPerCount, cb = cc / kWarps;  // count chunk, count block
       for (int e = lane; e < E; e += 32)
-        s_base[e] = __ldg(offsets + e) + sub_base[static_cast<int64_t>(e) * n_sub + c];
+        s_base[e] = __ldg(offsets + e) + blk[static_cast<int64_t>(e) * n_blk + cb] +
+                    pre[static_cast<int64_t>(e) * n_sub + cc];
       __syncwarp();
-      for (int64_t i0 = beg; i0 < end; i0 += 32) {
+      // entries of the count chunk that come before this block's tokens (at
+      // most 48 tokens: 12 ids per lane, all in flight at once)
+      {
+        const int64_t i0 = cc * kCountTokens * static_cast<int64_t>(k);
+        int ids[12];
+#pragma unroll
+        for (int u = 0; u < 12; ++u) {
+          const int64_t i = i0 + 32 * u + lane;
+          ids[u] = i < beg ? __ldg(idx + i) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < 12; ++u)
+          if (ids[u] >= 0 && ids[u] < E) atomicAdd(&s_base[ids[u]], 1);
+        for (int64_t i = i0 + 32 * 12 + lane; i < beg; i += 32) {  // k > 8 only
+          const int e = __ldg(idx + i);
+          if (e >= 0 && e < E) atomicAdd(&s_base[e], 1);
+        }
+      }
+      __syncwarp();
+      // the block's ids (16 tokens x k <= 8: at most 128), all loaded before
+      // the serial walk
+      int ids[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t i = beg + 32 * u + lane;
+        ids[u] = i < end ? __ldg(idx + i) : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t i0 = beg + 32 * u;
+        if (i0 >= end) break;
         const int64_t i = i0 + lane;
         const bool valid = i < end;
-        const int e = valid ? __ldg(idx + i) : -1;
+        const int e = valid ? ids[u] : -1;
         const bool good = valid && e >= 0 && e < E;
         const int key = good ? e : -1 - lane;  // lanes without an expert match only themselves
         const uint32_t peers = __match_any_sync(0xffffffffu, key);
@@ -181,53 +260,70 @@ __global__ void __launch_bounds__(kRsWarps * 32)
         if (valid) {
           row_map[i] = row;
           s_rows[i - beg] = row;
+          if (row_src != nullptr && row >= 0) row_src[row] = static_cast<int32_t>(i / k);
         }
       }
     }
     if constexpr (SCATTER) {
-      __syncthreads();
       const int64_t t0 = c * kChunkTokens;
-      for (int tt = warp; tt < kChunkTokens; tt += 2 * kRsWarps) {
-        // tokens tt and tt + kRsWarps of the chunk (each may be past T)
-        int rows[2][8];
-        bool live[2];
+      // tokens tt and tt + kRsWarps of the chunk (each may be past T), 128
+      // vectors of both at a time: loads first, then the k stores of each
+      auto live_of = [&](int tt) { return tt < kChunkTokens && t0 + tt < T; };
+      auto load_pair = [&](int tt, int v0, uint4 (&val)[2][4]) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (live_of(tt + h * kRsWarps) && v0 + 32 * u < nvec)
+              val[h][u] = __ldg(x + (t0 + tt + h * kRsWarps) * nvec + v0 + 32 * u);
+      };
+      auto store_pair = [&](int tt, int v0, const uint4 (&val)[2][4]) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const int64_t t = t0 + tt + h * kRsWarps;
-          live[h] = tt + h * kRsWarps < kChunkTokens && t < T;
+          if (!live_of(tt + h * kRsWarps)) continue;
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            rows[h][j] = (live[h] && j < k) ? s_rows[(tt + h * kRsWarps) * k + j] : -1;
-        }
-        for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
-          uint4 val[2][4];
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
+          for (int j = 0; j < 8; ++j) {
+            if (j >= k) break;
+            const int row = s_rows[(tt + h * kRsWarps) * k + j];
+            if (row < 0) continue;
+            uint4* dst = x_perm + static_cast<int64_t>(row) * nvec;
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-              if (live[h] && v0 + 32 * u < nvec)
-                val[h][u] = __ldg(x + (t0 + tt + h * kRsWarps) * nvec + v0 + 32 * u);
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              if (rows[h][j] < 0) continue;
-              uint4* dst = x_perm + static_cast<int64_t>(rows[h][j]) * nvec;
-#pragma unroll
-              for (int u = 0; u < 4; ++u)
-                if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = val[h][u];
-            }
+              if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = val[h][u];
+          }
+        }
+      };
+      {
+        // the first pair's first 128 vectors are loaded before waiting for the
+        // ranks, so their latency overlaps warp 0's walk
+        uint4 val[2][4];
+        load_pair(warp, lane, val);
+        __syncthreads();
+        store_pair(warp, lane, val);
+      }
+      for (int v0 = lane + 32 * 4; v0 < nvec; v0 += 32 * 4) {
+        uint4 val[2][4];
+        load_pair(warp, v0, val);
+        store_pair(warp, v0, val);
+      }
+      for (int tt = warp + 2 * kRsWarps; tt < kChunkTokens; tt += 2 * kRsWarps) {
+        for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
+          uint4 val[2][4];
+          load_pair(tt, v0, val);
+          store_pair(tt, v0, val);
         }
       }
     }
   } else if constexpr (SCATTER) {
-    const int e = static_cast<int>((c - n_sub) * kRsWarps + warp);
+    const int e = static_cast<int>((c - n_rs) * kRsWarps + warp);
     if (e >= E) return;
     const int64_t r0 = static_cast<int64_t>(__ldg(offsets + e)) + __ldg(counts + e);
     const int64_t r1 = __ldg(offsets + e + 1);
     const uint4 z = make_uint4(0, 0, 0, 0);
     for (int64_t r = r0; r < r1; ++r)
       for (int v = lane; v < nvec; v += 32) x_perm[r * nvec + v] = z;
+    if (row_src != nullptr)  // pad rows hold no token
+      for (int64_t r = r0 + lane; r < r1; r += 32) row_src[r] = T;
   }
 }
 
@@ -426,30 +522,35 @@ __global__ void __launch_bounds__(kWarps * 32)
 }  // namespace
 
 cudaError_t launch_route_count(const int32_t* idx, int T, int k, int E, int align,
-                               int32_t* sub_counts, int32_t* counts, int32_t* offsets,
+                               int32_t* scratch, int32_t* counts, int32_t* offsets,
                                DeviceCtl* ctl, cudaStream_t st) {
-  const int64_t n_sub = n_subchunks(T, k);
-  const unsigned grid = static_cast<unsigned>(ceil_div64(n_sub, kWarps));
-  (void)launch_pdl(route_count_kernel, grid, kWarps * 32, kWarps * E * sizeof(int), st, idx,
-                   static_cast<int64_t>(T) * k, k, E, n_sub, align, sub_counts, counts, offsets, ctl);
+  const int64_t n_sub = count_chunks(T), n_blk = count_blocks(T);
+  (void)launch_pdl(route_count_kernel, static_cast<unsigned>(n_blk), kWarps * 32,
+                   kWarps * E * sizeof(int), st, idx, static_cast<int64_t>(T) * k, k, E, n_sub,
+                   n_blk, align, scratch, scratch + static_cast<int64_t>(E) * n_sub, counts,
+                   offsets, ctl);
   return cudaGetLastError();
 }
 
 cudaError_t launch_route_rank_scatter(const int32_t* idx, const __nv_bfloat16* x, int T, int k,
-                                      int E, const int32_t* sub_base, const int32_t* offsets,
+                                      int E, const int32_t* scratch, const int32_t* offsets,
                                       const int32_t* counts, int d, int32_t* row_map,
-                                      __nv_bfloat16* x_perm, cudaStream_t st) {
-  const int64_t n_sub = n_subchunks(T, k);
+                                      __nv_bfloat16* x_perm, int32_t* row_src, cudaStream_t st) {
+  const int64_t n_sub = count_chunks(T), n_blk = count_blocks(T);
+  const int64_t n_rs = ceil_div64(T, kChunkTokens);
+  const int32_t* pre = scratch;
+  const int32_t* blk = scratch + static_cast<int64_t>(E) * n_sub;
   const size_t smem = (static_cast<size_t>(E) + static_cast<size_t>(kChunkTokens) * k) * sizeof(int);
   if (x_perm != nullptr) {
-    const unsigned grid = static_cast<unsigned>(n_sub + ceil_div64(E, kRsWarps));
+    const unsigned grid = static_cast<unsigned>(n_rs + ceil_div64(E, kRsWarps));
     (void)launch_pdl(route_rank_scatter_kernel<true>, grid, kRsWarps * 32, smem, st, idx,
-                     reinterpret_cast<const uint4*>(x), T, k, E, n_sub, sub_base, offsets, counts,
-                     d / 8, row_map, reinterpret_cast<uint4*>(x_perm));
+                     reinterpret_cast<const uint4*>(x), T, k, E, n_rs, n_sub, n_blk, pre, blk,
+                     offsets, counts, d / 8, row_map, reinterpret_cast<uint4*>(x_perm), row_src);
   } else {
-    (void)launch_pdl(route_rank_scatter_kernel<false>, static_cast<unsigned>(n_sub), kRsWarps * 32,
-                     smem, st, idx, static_cast<const uint4*>(nullptr), T, k, E, n_sub, sub_base,
-                     offsets, counts, d / 8, row_map, static_cast<uint4*>(nullptr));
+    (void)launch_pdl(route_rank_scatter_kernel<false>, static_cast<unsigned>(n_rs), kRsWarps * 32,
+                     smem, st, idx, static_cast<const uint4*>(nullptr), T, k, E, n_rs, n_sub,
+                     n_blk, pre, blk, offsets, counts, d / 8, row_map,
+                     static_cast<uint4*>(nullptr), static_cast<int32_t*>(nullptr));
   }
   return cudaGetLastError();
 }

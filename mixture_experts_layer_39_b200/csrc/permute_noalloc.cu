@@ -1,8 +1,8 @@
 // moe_permute_noalloc: the routing metadata + permute of moe_permute, for
 // callers that cannot hand the library any scratch memory.
 //
-// moe_permute needs a small scratch buffer (one expert histogram per
-// 16-token chunk of the routing ids), which it takes from the caller's
+// moe_permute needs a small scratch buffer (per expert, a count for every
+// 64 and every 512 tokens of the routing ids), which it takes from the caller's
 // workspace.  Some callers have no way to provide one: code embedded in a
 // host program that owns all device memory through its own pool and gives
 // plug-ins no allocation hook, or code on a latency-critical path that must
@@ -101,8 +101,7 @@ extern "C" moe_status_t moe_permute_noalloc(moe_handle_t h, const moe_shape_t* s
     return MOE_ERR_INVALID_ARG;
   if (!moe::aligned(x, 16) || !moe::aligned(x_perm, 16)) return MOE_ERR_INVALID_ARG;
   const int T = s->T, d = s->d_model, E = s->n_experts, k = s->top_k;
-  const int64_t n_sub = moe::n_subchunks(T, k);
-  if (n_sub * E > kNoallocScratchInts) return MOE_ERR_WORKSPACE;  // shape needs more than 1 MiB
+  if (moe::route_scratch_ints(T, E) > kNoallocScratchInts) return MOE_ERR_WORKSPACE;  // > 1 MiB
 
   moe::DeviceGuard guard(h->device);
   if (!guard.ok) return MOE_ERR_CUDA;
@@ -117,7 +116,7 @@ extern "C" moe_status_t moe_permute_noalloc(moe_handle_t h, const moe_shape_t* s
     return MOE_ERR_CUDA;
   if (moe::launch_route_rank_scatter(topk_idx, static_cast<const __nv_bfloat16*>(x), T, k, E, sub,
                                      offsets, counts, d, row_map,
-                                     static_cast<__nv_bfloat16*>(x_perm), st) != cudaSuccess)
+                                     static_cast<__nv_bfloat16*>(x_perm), nullptr, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
 }

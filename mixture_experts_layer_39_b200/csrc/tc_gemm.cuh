@@ -46,7 +46,10 @@ constexpr int BK = 64;  // bf16 elements per smem row: 128 bytes = one swizzle r
 constexpr int kThreads = 192;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-enum Epi : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_SWIGLU_FWD = 2, EPI_SWIGLU_BWD = 3 };
+// EPI_BF16_COMBINE: the down projection with the unpermute-combine fused into
+// its epilogue (see the epilogue below).
+enum Epi : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_SWIGLU_FWD = 2, EPI_SWIGLU_BWD = 3,
+                 EPI_BF16_COMBINE = 4 };
 
 struct GemmArgs {
   int n_tiles_n;     // tiles along N per (group, m-tile)
@@ -75,6 +78,15 @@ struct GemmArgs {
   // pad rows use src_oob, a row past the matrix that reads as zeros
   const int32_t* row_src;
   int src_oob;
+  // EPI_BF16_COMBINE: row_src[r] = the token of routed row r (T on pad rows);
+  // y [T, n_cols] = bf16(sum_j topk_w[t, j] out[row_map[t, j]] (+ shared[t]));
+  // arrivals [T, n_tiles_n] int32, zero on entry and on return
+  const int32_t* row_map;
+  const float* topk_w;
+  const __nv_bfloat16* shared;
+  __nv_bfloat16* y;
+  int32_t* arrivals;
+  int n_tok, top_k;
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -519,11 +531,6 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
-// Waits until at most one of this thread's cp.async groups is still pending.
-__device__ __forceinline__ void cp_async_wait_group1() {
-  asm volatile("cp.async.wait_group 1;" ::: "memory");
-}
-
 // ---------------------------------------------------------------- the kernel
 template <int BN, int STAGES, int EPI, bool FP8 = false, bool PAIR = false>
 struct SmemPlan {
@@ -541,8 +548,7 @@ struct SmemPlan {
   static constexpr int kMiscOff = kBarOff + kBarBytes;                 // tmem base, abort flag
   static constexpr int kEpiOff = (kMiscOff + 16 + 127) / 128 * 128;    // 4 epilogue warps' buffers
   // per warp: the 4 KB staging buffer, plus (SwiGLU backward) a 4 KB landing
-  // buffer; the SwiGLU backward uses both as landing buffers that cp.async
-  // fills with the next two 32-column halves of the saved A and U
+  // buffer that cp.async fills with the next 32 columns of the saved A and U
   static constexpr int kWarpEpiBytes = kEpiBufBytes + (EPI == EPI_SWIGLU_BWD ? kEpiBufBytes : 0);
   static constexpr int kTileOff = kEpiOff + 4 * kWarpEpiBytes;         // group tile starts
   static constexpr int bytes(int n_groups) { return 1024 + kTileOff + 4 * (n_groups + 1); }
@@ -987,25 +993,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Tile tl = decode_tile<KGROUP, BKE, KMMA, MT>(args, s_tile_start, t);
       const int vrows = quarter_rows(tl);
       const int64_t row_first = quarter_first(tl);  // warp's first row
-      // SwiGLU backward: the saved A and U of the first two 32-column halves
-      // are requested before waiting for the accumulator, so their latency
-      // overlaps the main loop; each later half is requested two halves ahead
-      // of its use.
+      // SwiGLU backward: the saved A and U of the first 32 columns are
+      // requested before waiting for the accumulator, so their latency
+      // overlaps the main loop; each later 32 columns are requested while the
+      // previous ones are computed.
       const __nv_bfloat16* aux = nullptr;
       if constexpr (EPI == EPI_SWIGLU_BWD) {
-        // halves 0 and 1 into the two landing buffers (the staging buffer is
-        // the second: this epilogue stores straight from registers)
         aux = args.aux + row_first * args.ld_aux + static_cast<int64_t>(tl.n_tile) * BN;
-        const int ncols0 = args.n_cols - tl.n_tile * BN < BN ? args.n_cols - tl.n_tile * BN : BN;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (32 * h < ncols0) {
-            cp_async_au(h ? ebuf : lbuf, reinterpret_cast<const uint8_t*>(aux + 32 * h),
-                        reinterpret_cast<const uint8_t*>(aux + args.f + 32 * h), args.ld_aux * 2,
-                        vrows, lane, args.aux);
-            cp_async_commit();
-          }
-        }
+        cp_async_au(lbuf, reinterpret_cast<const uint8_t*>(aux),
+                    reinterpret_cast<const uint8_t*>(aux + args.f), args.ld_aux * 2, vrows, lane,
+                    args.aux);
+        cp_async_commit();
       }
       const bool ok = __all_sync(
           0xffffffffu, mbar_wait(tfull_bar(acc), acc_phase, s_abort, args.wait_ns, true, PAIR));
@@ -1023,7 +1021,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n_left = args.n_cols - tl.n_tile * BN;
       const int ncols = n_left < BN ? n_left : BN;
       const int64_t gofs = KGROUP ? static_cast<int64_t>(tl.group) * args.out_gstride : 0;
-      if constexpr (EPI == EPI_BF16) {
+      if constexpr (EPI == EPI_BF16 || EPI == EPI_BF16_COMBINE) {
         auto* base = static_cast<__nv_bfloat16*>(args.out) + gofs + row_first * args.ldo +
                      static_cast<int64_t>(tl.n_tile) * BN;
 #pragma unroll 1
@@ -1098,54 +1096,54 @@ __global__ void __launch_bounds__(kThreads, 1)
           store_rows(ebuf, lane, vh, reinterpret_cast<uint8_t*>(hh + c), args.ldo2 * 2, vrows);
         }
       } else {  // EPI_SWIGLU_BWD
-        // 32 columns at a time; the saved A and U of the next two 32-column
-        // halves are in flight in the two landing buffers while one is
-        // computed (the latency of one L2 round trip under load is about the
-        // time of two halves).  Each lane stores dA and dU of its own row.
-        uint4* drow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) +
-                                               (row_first + lane) * args.ldo +
-                                               static_cast<int64_t>(tl.n_tile) * BN);
-        uint4* urow = drow + args.f / 8;
-        const int nh = ncols / 32;
+        auto* dau = static_cast<__nv_bfloat16*>(args.out) + row_first * args.ldo +
+                    static_cast<int64_t>(tl.n_tile) * BN;
 #pragma unroll 1
-        for (int h = 0; h < nh; ++h) {
-          uint8_t* buf = (h & 1) ? ebuf : lbuf;
-          if (h + 1 < nh) cp_async_wait_group1(); else cp_async_wait_all();
-          __syncwarp();
-          uint4 vau[8];  // this lane's row: A in slots 0-3, U in slots 4-7
-          stage_read_row(buf, lane, vau);
-          __syncwarp();
-          if (h + 2 < nh) {
-            cp_async_au(buf, reinterpret_cast<const uint8_t*>(aux + 32 * (h + 2)),
-                        reinterpret_cast<const uint8_t*>(aux + args.f + 32 * (h + 2)),
-                        args.ld_aux * 2, vrows, lane, args.aux);
-            cp_async_commit();
-          }
-          uint32_t r[32];
-          tmem_ld32(tbase + tcol(32 * h), r);
-          tmem_ld_wait();
+        for (int c = 0; c < ncols; c += 64) {
+          uint4 ou[8];  // dU in registers; dA goes straight to the staging buffer
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 qa = vau[q], qu = vau[4 + q];
-            const float a[8] = {bf16_lo(qa.x), bf16_hi(qa.x), bf16_lo(qa.y), bf16_hi(qa.y),
-                                bf16_lo(qa.z), bf16_hi(qa.z), bf16_lo(qa.w), bf16_hi(qa.w)};
-            const float u[8] = {bf16_lo(qu.x), bf16_hi(qu.x), bf16_lo(qu.y), bf16_hi(qu.y),
-                                bf16_lo(qu.z), bf16_hi(qu.z), bf16_lo(qu.w), bf16_hi(qu.w)};
-            float da[8], du[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float dh = __uint_as_float(r[8 * q + i]);
-              const float sg = sigmoid_fast(a[i]);
-              da[i] = dh * u[i] * sg * (1.0f + a[i] * (1.0f - sg));
-              du[i] = dh * a[i] * sg;
+          for (int half = 0; half < 2; ++half) {
+            const int cc = c + 32 * half;
+            uint4 vau[8];  // this lane's row: A in slots 0-3, U in slots 4-7
+            cp_async_wait_all();
+            __syncwarp();
+            stage_read_row(lbuf, lane, vau);
+            __syncwarp();
+            if (cc + 32 < ncols) {  // the next 32 columns land while these are computed
+              cp_async_au(lbuf, reinterpret_cast<const uint8_t*>(aux + cc + 32),
+                          reinterpret_cast<const uint8_t*>(aux + args.f + cc + 32),
+                          args.ld_aux * 2, vrows, lane, args.aux);
+              cp_async_commit();
             }
-            if (lane < vrows) {
-              drow[4 * h + q] = make_uint4(pack_bf16x2(da[0], da[1]), pack_bf16x2(da[2], da[3]),
-                                           pack_bf16x2(da[4], da[5]), pack_bf16x2(da[6], da[7]));
-              urow[4 * h + q] = make_uint4(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]),
-                                           pack_bf16x2(du[4], du[5]), pack_bf16x2(du[6], du[7]));
+            uint32_t r[32];
+            tmem_ld32(tbase + tcol(cc), r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 qa = vau[q], qu = vau[4 + q];
+              const float a[8] = {bf16_lo(qa.x), bf16_hi(qa.x), bf16_lo(qa.y), bf16_hi(qa.y),
+                                  bf16_lo(qa.z), bf16_hi(qa.z), bf16_lo(qa.w), bf16_hi(qa.w)};
+              const float u[8] = {bf16_lo(qu.x), bf16_hi(qu.x), bf16_lo(qu.y), bf16_hi(qu.y),
+                                  bf16_lo(qu.z), bf16_hi(qu.z), bf16_lo(qu.w), bf16_hi(qu.w)};
+              float da[8], du[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float dh = __uint_as_float(r[8 * q + i]);
+                const float sg = sigmoid_fast(a[i]);
+                da[i] = dh * u[i] * sg * (1.0f + a[i] * (1.0f - sg));
+                du[i] = dh * a[i] * sg;
+              }
+              *stage_slot(ebuf, lane, 4 * half + q) =
+                  make_uint4(pack_bf16x2(da[0], da[1]), pack_bf16x2(da[2], da[3]),
+                             pack_bf16x2(da[4], da[5]), pack_bf16x2(da[6], da[7]));
+              ou[4 * half + q] = make_uint4(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]),
+                                            pack_bf16x2(du[4], du[5]), pack_bf16x2(du[6], du[7]));
             }
           }
+          __syncwarp();
+          stage_to_global(ebuf, reinterpret_cast<uint8_t*>(dau + c), args.ldo * 2, vrows, lane);
+          __syncwarp();
+          store_rows(ebuf, lane, ou, reinterpret_cast<uint8_t*>(dau + args.f + c), args.ldo * 2, vrows);
         }
       }
       tc_fence_before();
@@ -1155,6 +1153,92 @@ __global__ void __launch_bounds__(kThreads, 1)
         else mbar_arrive(tempty_bar(acc));
       }
       if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
+      if constexpr (EPI == EPI_BF16_COMBINE) {
+        // The warp's rows of this column tile are stored and the accumulator
+        // is released, so what follows overlaps the next tile's main loop.
+        // Publish the rows, then count one arrival per (token, column tile);
+        // the arrival that completes a token's valid rows forms y[t] over the
+        // tile's columns from the stored bf16 rows, in slot order with the
+        // combine kernel's arithmetic (same bits), and clears the count.
+        __threadfence();
+        __syncwarp();
+        int t = -1;
+        int32_t* cnt = nullptr;
+        bool last = false;
+        if (lane < vrows) {
+          const int src = __ldg(args.row_src + row_first + lane);
+          if (src >= 0 && src < args.n_tok) t = src;
+        }
+        if (t >= 0) {
+          int need = 0;
+          for (int j = 0; j < args.top_k; ++j)
+            need += __ldg(args.row_map + static_cast<int64_t>(t) * args.top_k + j) >= 0 ? 1 : 0;
+          cnt = args.arrivals + static_cast<int64_t>(t) * args.n_tiles_n + tl.n_tile;
+          last = atomicAdd(cnt, 1) == need - 1;
+        }
+        uint32_t done = __ballot_sync(0xffffffffu, last);
+        if (done != 0u) __threadfence();
+        const auto* obase = static_cast<const __nv_bfloat16*>(args.out);
+        const int64_t col0 = static_cast<int64_t>(tl.n_tile) * BN;
+        const int n_left = args.n_cols - tl.n_tile * BN;
+        const int ncols = n_left < BN ? n_left : BN;
+        while (done != 0u) {
+          // two completed tokens at a time: all their loads in flight together
+          int64_t tt[2];
+          int srcl[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            srcl[h] = done != 0u ? __ffs(done) - 1 : -1;
+            if (done != 0u) done &= done - 1u;
+            tt[h] = srcl[h] >= 0 ? __shfl_sync(0xffffffffu, t, srcl[h]) : -1;
+          }
+          int rows[2][8];
+          float wt[2][8];
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const bool ok = tt[h] >= 0 && j < args.top_k;
+              rows[h][j] = ok ? __ldg(args.row_map + tt[h] * args.top_k + j) : -1;
+              wt[h][j] = ok ? __ldg(args.topk_w + tt[h] * args.top_k + j) : 0.f;
+            }
+          for (int c = lane * 8; c < ncols; c += 256) {
+            uint4 q[2][8];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                if (rows[h][j] >= 0)
+                  q[h][j] = __ldcg(reinterpret_cast<const uint4*>(obase + rows[h][j] * args.ldo + col0 + c));
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (tt[h] < 0) continue;
+              float acc[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                if (rows[h][j] < 0) continue;
+                float fv[8];
+                unpack8(q[h][j], fv);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(wt[h][j], fv[i], acc[i]);
+              }
+              if (args.shared != nullptr) {  // the shared expert's output, added last
+                float fv[8];
+                unpack8(__ldg(reinterpret_cast<const uint4*>(args.shared + tt[h] * args.ldo + col0 + c)),
+                        fv);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] += fv[i];
+              }
+              *reinterpret_cast<uint4*>(args.y + tt[h] * args.ldo + col0 + c) = pack8(acc);
+            }
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            if (lane == srcl[h]) *cnt = 0;
+        }
+      }
     }
   }
 

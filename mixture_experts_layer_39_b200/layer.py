@@ -16,6 +16,11 @@ With shared_ff > 0 a shared expert runs on every token
 (moe_shared_expert_fwd / _bwd); its output joins the combine and its input
 gradient the permute backward.
 
+With fuse_combine=True (bf16) the weighted unpermute-combine runs inside
+the down projection's epilogue (moe_permute_src ->
+moe_grouped_swiglu_fwd_combine); y has the same bits, and a shared expert's
+forward runs before the routed experts so that its output joins there.
+
 With gather=True (bf16) no permuted copy of x is written: moe_route
 produces the routing metadata and row_src, and the expert GEMMs that read
 routed rows of x gather them from x itself (the *_gather entry points).
@@ -50,7 +55,7 @@ class MoELayer:
                  handle: ops.Handle | None = None, dtype: str = "bf16",
                  fuse_router_dx: bool | None = None, aux_alpha: float = 0.0,
                  aux_reduce: Callable | None = None, shared_ff: int = 0,
-                 recompute: bool = False, gather: bool = False):
+                 recompute: bool = False, gather: bool = False, fuse_combine: bool = False):
         """dtype: "bf16", or "mxfp8" for E4M3/E8M0 expert GEMM operands (the
         library then also aligns expert segments to 128 rows).
         fuse_router_dx: add the router's input gradient inside the permute
@@ -68,8 +73,11 @@ class MoELayer:
         of the backward, and can be shared between layers)."""
         self.recompute = bool(recompute)
         self.gather = bool(gather)
+        self.fuse_combine = bool(fuse_combine)
         if self.gather and dtype != "bf16":
             raise ValueError("the gather forms are bf16 only")
+        if self.fuse_combine and (dtype != "bf16" or self.gather):
+            raise ValueError("the fused combine is bf16 only, with a permuted copy of x")
         self._x = None  # x of the current step (gather forms read it in the GEMMs)
         self.T, self.d, self.f, self.E, self.k = T, d, f, E, k
         dev = torch.device(device)
@@ -89,7 +97,11 @@ class MoELayer:
         self.counts, self.offsets = z(E, dt=I32), z(E + 1, dt=I32)
         self.row_map = z(T, k, dt=I32)
         self.x_perm = None if self.gather else z(M, d)
-        self.row_src = z(M, dt=I32) if self.gather else None
+        self.row_src = z(M, dt=I32) if (self.gather or self.fuse_combine) else None
+        # per (token, 256-column tile) arrival counts of the fused combine:
+        # zero here, left zero by every completed call
+        self.arrivals = (torch.zeros(T, (d + 255) // 256, dtype=I32, device=dev)
+                         if self.fuse_combine else None)
         self.au, self.h = z(M, 2 * f), z(M, f)
         self.o_perm, self.y = z(M, d), z(T, d)
         # backward state
@@ -133,6 +145,10 @@ class MoELayer:
             ops.moe_route(self.handle, self.shape, self.idx, self.counts, self.offsets,
                           self.row_map, self.row_src, self.ws, stream)
             return
+        if self.fuse_combine:
+            ops.moe_permute_src(self.handle, self.shape, x, self.idx, self.counts, self.offsets,
+                                self.row_map, self.row_src, self.x_perm, self.ws, stream)
+            return
         ops.moe_permute(self.handle, self.shape, x, self.idx, self.counts, self.offsets,
                         self.row_map, self.x_perm, self.ws, stream)
 
@@ -142,6 +158,12 @@ class MoELayer:
             ops.moe_grouped_swiglu_fwd_gather(self.handle, self.shape, self._x, self.row_src,
                                               self.offsets, w_gu, w_d, au, self.h, self.o_perm,
                                               stream)
+            return
+        if self.fuse_combine:  # y too (a shared expert's output must be ready)
+            ops.moe_grouped_swiglu_fwd_combine(self.handle, self.shape, self.x_perm, self.offsets,
+                                               self.row_map, self.row_src, self.w, w_gu, w_d, au,
+                                               self.h, self.o_perm, self.o_s, self.y,
+                                               self.arrivals, stream)
             return
         ops.moe_grouped_swiglu_fwd(self.handle, self.shape, self.x_perm, self.offsets, w_gu, w_d,
                                    au, self.h, self.o_perm, self.ws, stream)
@@ -181,6 +203,11 @@ class MoELayer:
             self.load_stats(False, stream)
             n = self.aux_reduce(self.stats) if self.aux_reduce is not None else self.T
             self.balance_loss(None, n, stream)
+        if self.fuse_combine:
+            if self.shared_ff > 0:
+                self.shared_fwd(x, w_gu_s, w_d_s, stream)
+            self.experts_fwd(w_gu, w_d, stream)  # writes y
+            return self.y
         self.experts_fwd(w_gu, w_d, stream)
         if self.shared_ff > 0:
             self.shared_fwd(x, w_gu_s, w_d_s, stream)

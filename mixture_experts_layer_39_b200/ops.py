@@ -161,6 +161,26 @@ def moe_grouped_swiglu_recompute(h, shape, x_perm, offsets, w_gu, au, hbuf, ws, 
           _arg(h, ws, None, "ws"), _nbytes(ws), _stream(h, stream))
 
 
+def moe_permute_src(h, shape, x, topk_idx, counts, offsets, row_map, row_src, x_perm, ws,
+                    stream=None):
+    _call("moe_permute_src", h.ptr, ctypes.byref(shape), _arg(h, x, BF16, "x"),
+          _arg(h, topk_idx, I32, "topk_idx"), _arg(h, counts, I32, "counts"),
+          _arg(h, offsets, I32, "offsets"), _arg(h, row_map, I32, "row_map"),
+          _arg(h, row_src, I32, "row_src"), _arg(h, x_perm, BF16, "x_perm"),
+          _arg(h, ws, None, "ws"), _nbytes(ws), _stream(h, stream))
+
+
+def moe_grouped_swiglu_fwd_combine(h, shape, x_perm, offsets, row_map, row_src, topk_w, w_gu,
+                                   w_down, au, hbuf, o_perm, shared_out, y, arrivals, stream=None):
+    _call("moe_grouped_swiglu_fwd_combine", h.ptr, ctypes.byref(shape),
+          _arg(h, x_perm, BF16, "x_perm"), _arg(h, offsets, I32, "offsets"),
+          _arg(h, row_map, I32, "row_map"), _arg(h, row_src, I32, "row_src"),
+          _arg(h, topk_w, F32, "topk_w"), _arg(h, w_gu, BF16, "w_gu"),
+          _arg(h, w_down, BF16, "w_down"), _arg(h, au, BF16, "au"), _arg(h, hbuf, BF16, "h"),
+          _arg(h, o_perm, BF16, "o_perm"), _arg(h, shared_out, BF16, "shared_out"),
+          _arg(h, y, BF16, "y"), _arg(h, arrivals, I32, "arrivals"), _stream(h, stream))
+
+
 def moe_route(h, shape, topk_idx, counts, offsets, row_map, row_src, ws, stream=None):
     _call("moe_route", h.ptr, ctypes.byref(shape), _arg(h, topk_idx, I32, "topk_idx"),
           _arg(h, counts, I32, "counts"), _arg(h, offsets, I32, "offsets"),

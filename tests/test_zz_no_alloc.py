@@ -50,7 +50,7 @@ def test_noalloc_matches_workspace_permute_twice(cuda_ok, T, d, E, k):
 
 def test_noalloc_rejects_shapes_beyond_its_scratch(cuda_ok):
     h = ops.Handle(0)
-    # ceil(32768/16) * 1024 int32 = 8 MiB > the 1 MiB built-in array
+    # (512 + 64) * 1024 int32 = 2.25 MiB > the 1 MiB built-in array
     shape = ops.make_shape(32768, 256, 256, 1024, 8, MOE_DTYPE_BF16)
     d = torch.empty(16, dtype=torch.bfloat16, device="cuda")
     i = torch.empty(16, dtype=torch.int32, device="cuda")
