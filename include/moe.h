@@ -498,6 +498,31 @@ MOE_API moe_status_t moe_router_aux_loss(moe_handle_t h, const moe_shape_t* s, c
 MOE_API moe_status_t moe_mxfp8_quantize(moe_handle_t h, const void* in, int64_t rows, int64_t cols,
                                 int axis, uint8_t* q, uint8_t* scales, moe_stream_t stream);
 
+/* Both MXFP8 quantisations of a bf16 matrix from one read, written in the
+ * layout the MXFP8 expert GEMMs take: the step the expert calls run on each
+ * operand (Olmo-core 3 introduction page, section 3 "MXFP8"; the same OCP
+ * MX v1.0 per-block rule as moe_mxfp8_quantize):
+ *   row-wise   : blocks of 32 consecutive elements along each row;
+ *   column-wise: blocks of 32 consecutive rows down each column, inside each
+ *                group of rows_per_group rows (the token-axis blocks of one
+ *                expert segment never reach into the next).
+ * Scale codes are in the tensor cores' 512-byte scale-atom order: for a
+ * matrix with MN index r and 32-element contraction block b (n_b4 = number
+ * of contraction blocks / 4), the code sits at byte
+ *   ((r / 128) * n_b4 + b / 4) * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + b % 4.
+ * Row-wise: r = row, b = column / 32, n_b4 = cols / 128.  Column-wise, per
+ * group g (its codes start at byte g * cols * rows_per_group / 32): r =
+ * column, b = (row within the group) / 32, n_b4 = rows_per_group / 128.
+ * In : in [rows, cols] bf16, 16-byte aligned; rows a multiple of
+ *      rows_per_group, rows_per_group and cols multiples of 128.
+ * Out: q_row, q_col [rows, cols] uint8 E4M3 codes (row-major, 16-byte
+ *      aligned); s_row, s_col rows * cols / 32 bytes each (caller-owned).
+ * One launch; MOE_ERR_INVALID_ARG for shapes or alignments outside these. */
+MOE_API moe_status_t moe_mxfp8_quantize_gemm(moe_handle_t h, const void* in, int64_t rows,
+                                             int64_t cols, int64_t rows_per_group, uint8_t* q_row,
+                                             uint8_t* s_row, uint8_t* q_col, uint8_t* s_col,
+                                             moe_stream_t stream);
+
 /* Waits for the device, then returns the status word recorded by kernels
  * (MOE_OK if none) in *device_status and clears it.  The only call that
  * synchronises; not meant for use inside a step.

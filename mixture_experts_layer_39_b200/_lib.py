@@ -57,6 +57,7 @@ SIGNATURES = {
     "moe_router_load_stats": [P, SP, P, P, c_int, P, P, c_size_t, P],
     "moe_router_aux_loss": [P, SP, P, c_int64, ctypes.c_float, P, P, P],
     "moe_mxfp8_quantize": [P, P, c_int64, c_int64, c_int, P, P, P],
+    "moe_mxfp8_quantize_gemm": [P, P, c_int64, c_int64, c_int64, P, P, P, P, P],
     "moe_get_status": [P, ctypes.POINTER(c_int)],
     "moe_get_launch_count": [P, ctypes.POINTER(ctypes.c_uint64)],
     "moe_set_wait_limit": [P, ctypes.c_uint64],

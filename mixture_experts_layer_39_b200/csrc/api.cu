@@ -434,7 +434,7 @@ moe_status_t moe_grouped_swiglu_fwd(moe_handle_t h, const moe_shape_t* s, const 
     auto both = [&](const void* in, int64_t r, int64_t cols, int64_t group, size_t q, size_t sc,
                     size_t qc, size_t scc) {
       return cuda_status(moe::launch_mxfp8_quantize_both(bf(in), r, cols, group, b + q, b + sc,
-                                                         keep + qc, keep + scc, st));
+                                                         keep + qc, keep + scc, h->num_sms, st));
     };
     h->launches += 6;
     MOE_TRY(both(x_perm, m_cap, d, m_cap, L.xq, L.xs, L.xq_c, L.xs_c));
@@ -539,7 +539,7 @@ moe_status_t moe_grouped_swiglu_bwd(moe_handle_t h, const moe_shape_t* s, const 
     auto both = [&](const void* in, int64_t r, int64_t cols, size_t q, size_t sc, size_t qc,
                     size_t scc) {
       return cuda_status(moe::launch_mxfp8_quantize_both(bf(in), r, cols, r, b + q, b + sc, b + qc,
-                                                         b + scc, st));
+                                                         b + scc, h->num_sms, st));
     };
     // the forward's column-wise copies of W_d, W_gu, H and x_perm
     const uint8_t* keep = b + scratch_bytes(h, s);
@@ -745,6 +745,23 @@ moe_status_t moe_mxfp8_quantize(moe_handle_t h, const void* in, int64_t rows, in
   h->launches += 1;
   return cuda_status(moe::launch_mxfp8_quantize(static_cast<const __nv_bfloat16*>(in), rows, cols,
                                                 axis, q, scales, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_mxfp8_quantize_gemm(moe_handle_t h, const void* in, int64_t rows, int64_t cols,
+                                     int64_t rows_per_group, uint8_t* q_row, uint8_t* s_row,
+                                     uint8_t* q_col, uint8_t* s_col, moe_stream_t stream) {
+  if (h == nullptr || !all_nonnull(in, q_row, s_row) || !all_nonnull(q_col, s_col))
+    return MOE_ERR_INVALID_ARG;
+  if (rows < 1 || cols < 1 || rows_per_group < 1 || cols % 128 != 0 || rows_per_group % 128 != 0 ||
+      rows % rows_per_group != 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(in, 16) || !aligned(q_row, 16) || !aligned(q_col, 16)) return MOE_ERR_INVALID_ARG;
+  MOE_GUARD(h);
+  h->launches += 1;
+  return cuda_status(moe::launch_mxfp8_quantize_both(static_cast<const __nv_bfloat16*>(in), rows,
+                                                     cols, rows_per_group, q_row, s_row, q_col,
+                                                     s_col, h->num_sms,
+                                                     static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_get_status(moe_handle_t h, int* device_status) {

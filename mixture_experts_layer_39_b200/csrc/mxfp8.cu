@@ -195,7 +195,10 @@ __global__ void mx_colwise_kernel(const __nv_bfloat16* __restrict__ in, int64_t 
 //              column t's amax and writes its scale; codes to q_col.
 // The tile's 32 rows never straddle a group (rows_per_group is a multiple of
 // 128), so column blocks follow the per-group atom layout of scale_mode 1.
-__global__ void __launch_bounds__(128)
+// Capped at 64 registers a thread, eight blocks (64 KB of loads in flight)
+// fit on an SM, against five at the uncapped 92: 0.79 of the measured copy
+// rate on operand-sized inputs, against 0.67.
+__global__ void __launch_bounds__(128, 8)
     mx_both_kernel(const uint4* __restrict__ in, int64_t rows, int64_t cols, int64_t rows_per_group,
                    uint2* __restrict__ q_row, uint8_t* __restrict__ s_row, uint2* __restrict__ q_col,
                    uint8_t* __restrict__ s_col) {
@@ -315,9 +318,12 @@ cudaError_t launch_mxfp8_quantize_atoms(const __nv_bfloat16* in, int64_t rows, i
 
 cudaError_t launch_mxfp8_quantize_both(const __nv_bfloat16* in, int64_t rows, int64_t cols,
                                        int64_t rows_per_group, uint8_t* q_row, uint8_t* s_row,
-                                       uint8_t* q_col, uint8_t* s_col, cudaStream_t st) {
+                                       uint8_t* q_col, uint8_t* s_col, int num_sms,
+                                       cudaStream_t st) {
+  // two waves of the eight resident blocks per SM, each block walking tiles
   const int64_t tiles = (rows / 32) * (cols / 128);
-  const unsigned grid = static_cast<unsigned>(tiles < 148 * 16 ? tiles : 148 * 16);
+  const int64_t cap = static_cast<int64_t>(num_sms > 0 ? num_sms : 148) * 16;
+  const unsigned grid = static_cast<unsigned>(tiles < cap ? (tiles > 0 ? tiles : 1) : cap);
   (void)launch_pdl(mx_both_kernel, grid, 128, 0, st, reinterpret_cast<const uint4*>(in), rows, cols,
                    rows_per_group, reinterpret_cast<uint2*>(q_row), s_row,
                    reinterpret_cast<uint2*>(q_col), s_col);

@@ -298,3 +298,10 @@ def moe_mxfp8_quantize(h, inp, axis, q, scales, stream=None):
     rows, cols = inp.shape
     _call("moe_mxfp8_quantize", h.ptr, _arg(h, inp, BF16, "in"), rows, cols, axis,
           _arg(h, q, U8, "q"), _arg(h, scales, U8, "scales"), _stream(h, stream))
+
+
+def moe_mxfp8_quantize_gemm(h, inp, rows_per_group, q_row, s_row, q_col, s_col, stream=None):
+    rows, cols = inp.shape
+    _call("moe_mxfp8_quantize_gemm", h.ptr, _arg(h, inp, BF16, "in"), rows, cols, rows_per_group,
+          _arg(h, q_row, U8, "q_row"), _arg(h, s_row, U8, "s_row"), _arg(h, q_col, U8, "q_col"),
+          _arg(h, s_col, U8, "s_col"), _stream(h, stream))

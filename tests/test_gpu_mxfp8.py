@@ -148,3 +148,55 @@ def test_mxfp8_workload_sampled_experts(cuda_ok):
         assert_close(f"dW_d[{e}]", np64(L.dw_d[e]), bwd["dW_d"][0], TOL_MXFP8)
         assert_close(f"dW_gu[{e}]", np64(L.dw_gu[e]), bwd["dW_gu"][0], TOL_MXFP8)
     H.report("full-size mxfp8 (sampled experts)", log0)
+
+
+def _from_atoms(s, n_mn, n_b):
+    """[n_mn, n_b] scale codes read back from the tensor cores' 512-byte atom
+    order: 128 MN indices x 4 contraction blocks per atom, atoms consecutive
+    along the contraction, and inside an atom byte (r % 32) * 16 +
+    ((r / 32) % 4) * 4 + b % 4 (the block-scaled MMA's scale-factor layout
+    for 128 rows and K = 128 per atom)."""
+    r = np.arange(n_mn)[:, None]
+    b = np.arange(n_b)[None, :]
+    idx = ((r // 128) * (n_b // 4) + b // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + b % 4
+    return s[idx]
+
+
+@pytest.mark.parametrize("rows,cols,rpg", [(256, 384, 128), (384, 128, 384), (1024, 256, 256),
+                                           (8192, 1024, 1024)])
+def test_gemm_layout_quantiser_matches_oracle(cuda_ok, rows, cols, rpg):
+    """The quantiser the MXFP8 expert calls run (both orientations from one
+    read, scales in atom order), code for code against the oracle's codec:
+    row-wise blocks along each row, column-wise blocks of 32 rows inside each
+    group of rpg rows.  The largest case has more 32 x 128 tiles than the
+    grid has blocks, so blocks walk several tiles with the next one in flight."""
+    from mixture_experts_layer_39_b200 import ops
+    h = ops.Handle(0)
+    g = torch.Generator().manual_seed(rows + cols)
+    a = torch.randn(rows, cols, generator=g) * torch.exp(torch.randn(rows, 1, generator=g) * 3)
+    a = a * torch.exp(torch.randn(1, cols, generator=g) * 2)
+    a[3] = 0.0                                               # all-zero blocks both ways
+    a[5, :32] = -1e-30
+    a[7, 64:96] = 3e4                                        # saturates nothing: scale follows amax
+    a[9, 96:128] = torch.randn(32, generator=g) * 2e-39      # bf16 subnormals: scale clamp at -127
+    a[:, 1] = torch.randn(rows, generator=g) * 3e-39         # every column block of a column
+    a = a.to(torch.bfloat16)
+    ad = a.cuda()
+    q_row = torch.empty(rows, cols, dtype=torch.uint8, device="cuda")
+    q_col = torch.empty(rows, cols, dtype=torch.uint8, device="cuda")
+    s_row = torch.empty(rows * cols // 32, dtype=torch.uint8, device="cuda")
+    s_col = torch.empty(rows * cols // 32, dtype=torch.uint8, device="cuda")
+    ops.moe_mxfp8_quantize_gemm(h, ad, rpg, q_row, s_row, q_col, s_col)
+    torch.cuda.synchronize()
+    assert h.get_status() == 0
+    a64 = a.double().numpy()
+    qo, so = MX.quantize_blocks(a64, 1)
+    np.testing.assert_array_equal(q_row.cpu().numpy(), qo)
+    np.testing.assert_array_equal(_from_atoms(s_row.cpu().numpy(), rows, cols // 32), so)
+    qc, sc = q_col.cpu().numpy(), s_col.cpu().numpy()
+    per = cols * rpg // 32
+    for gi in range(rows // rpg):
+        qo, so = MX.quantize_blocks(a64[gi * rpg:(gi + 1) * rpg], 0)
+        np.testing.assert_array_equal(qc[gi * rpg:(gi + 1) * rpg], qo)
+        got = _from_atoms(sc[gi * per:(gi + 1) * per], cols, rpg // 32).T
+        np.testing.assert_array_equal(got, so)
