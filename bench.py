@@ -368,7 +368,24 @@ def measure_e2e(L, g, steps, warmup, dev):
     stepper.run(plan(steps), g["w_r"], g["w_gu"], g["w_d"], g["bias"], after=start)
     end = stepper.done_event()
     torch.cuda.synchronize(dev)
-    return start.elapsed_time(end), h2d, d2h
+    e2e_ms = start.elapsed_time(end)
+    # the host link alone: the same per-step copies, both directions at once, no kernels
+    start = torch.cuda.Event(enable_timing=True)
+    start.record(stepper.compute)
+    stepper.copy_in.wait_event(start)
+    stepper.copy_out.wait_event(start)
+    for i in range(steps):
+        with torch.cuda.stream(stepper.copy_in):
+            stepper.x[i & 1].copy_(xs[i & 1], non_blocking=True)
+            stepper.dy[i & 1].copy_(dys[i & 1], non_blocking=True)
+            if routes[0] is not None:
+                stepper.route[i & 1].copy_(routes[i & 1], non_blocking=True)
+        with torch.cuda.stream(stepper.copy_out):
+            ys[i & 1].copy_(stepper.y[i & 1], non_blocking=True)
+            dxs[i & 1].copy_(stepper.dx[i & 1], non_blocking=True)
+    end = stepper.done_event()
+    torch.cuda.synchronize(dev)
+    return e2e_ms, h2d, d2h, start.elapsed_time(end)
 
 
 def run_ours(args):
@@ -409,9 +426,10 @@ def run_ours(args):
         if with_e2e:
             out["memory_bound"] = measure_memory_bound(L, g, flush)
             barrier()
-            e2e_ms, h2d, d2h = measure_e2e(L, g, steps, min(warmup, 3), dev)
+            e2e_ms, h2d, d2h, link_ms = measure_e2e(L, g, steps, min(warmup, 3), dev)
             barrier()
-            out.update({"e2e_total_ms": max_over_ranks(e2e_ms), "h2d": h2d, "d2h": d2h})
+            out.update({"e2e_total_ms": max_over_ranks(e2e_ms), "h2d": h2d, "d2h": d2h,
+                        "link_total_ms": max_over_ranks(link_ms)})
         st = L.handle.get_status()
         if st != 0:
             raise RuntimeError(f"device status {st} after the benchmark")
@@ -473,7 +491,11 @@ def run_ours(args):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": main["h2d"],
                 "d2h_bytes_per_step": main["d2h"],
                 "how": "HostStepper: pinned-host x/dY in, y/dX out every step; copies of "
-                       "neighbouring steps overlap the kernels on two copy streams"},
+                       "neighbouring steps overlap the kernels on two copy streams",
+                "copy_only_ms_per_step": main["link_total_ms"] / K,
+                "of_copy_bound": main["link_total_ms"] / main["e2e_total_ms"],
+                "copy_only_note": "the same copies with no kernels, both directions at once: "
+                                  "the host link's bound on this number"},
         "gpu_launches": main["launches"],
         "grouped_gemm": {"tflops": achieved, "ms_per_step": gemm_ms,
                          "share_of_step": gemm_ms / (main["total_ms"] / K)},
