@@ -1021,7 +1021,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n_left = args.n_cols - tl.n_tile * BN;
       const int ncols = n_left < BN ? n_left : BN;
       const int64_t gofs = KGROUP ? static_cast<int64_t>(tl.group) * args.out_gstride : 0;
-      if constexpr (EPI == EPI_BF16 || EPI == EPI_BF16_COMBINE) {
+      // the warp's part of the accumulator goes back to the MMA issuer
+      auto release_acc = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (PAIR && rank != 0) mbar_arrive_remote(mapa_shared(tempty_bar(acc), 0));
+          else mbar_arrive(tempty_bar(acc));
+        }
+      };
+      // MXFP8 keeps one accumulator (TMEM also holds the scales), so a tile's
+      // epilogue would hold up the next tile's MMAs.  A plain bf16 output
+      // row of 256 columns fits in 128 registers as bf16 pairs: it is read
+      // out of TMEM whole, the accumulator is released, and the stores follow.
+      constexpr bool kEarlyRelease = FP8 && EPI == EPI_BF16 && BN == 256;
+      if constexpr (kEarlyRelease) {
+        auto* base = static_cast<__nv_bfloat16*>(args.out) + gofs + row_first * args.ldo +
+                     static_cast<int64_t>(tl.n_tile) * BN;
+        uint32_t pk[BN / 2];  // bf16 pairs of this lane's row
+#pragma unroll
+        for (int c = 0; c < BN; c += 64) {
+          if (c < ncols) {
+            uint32_t r0[32], r1[32];
+            tmem_ld32(tbase + tcol(c), r0);
+            tmem_ld32(tbase + tcol(c + 32), r1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              pk[c / 2 + i] = zero_acc ? 0u
+                                       : pack_bf16x2(__uint_as_float(r0[2 * i]),
+                                                     __uint_as_float(r0[2 * i + 1]));
+              pk[c / 2 + 16 + i] = zero_acc ? 0u
+                                            : pack_bf16x2(__uint_as_float(r1[2 * i]),
+                                                          __uint_as_float(r1[2 * i + 1]));
+            }
+          }
+        }
+        release_acc();
+#pragma unroll
+        for (int c = 0; c < BN; c += 64) {
+          if (c < ncols) {
+            uint4 v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              v[q] = make_uint4(pk[c / 2 + 4 * q], pk[c / 2 + 4 * q + 1], pk[c / 2 + 4 * q + 2],
+                                pk[c / 2 + 4 * q + 3]);
+            store_rows(ebuf, lane, v, reinterpret_cast<uint8_t*>(base + c), args.ldo * 2, vrows);
+          }
+        }
+      } else if constexpr (EPI == EPI_BF16 || EPI == EPI_BF16_COMBINE) {
         auto* base = static_cast<__nv_bfloat16*>(args.out) + gofs + row_first * args.ldo +
                      static_cast<int64_t>(tl.n_tile) * BN;
 #pragma unroll 1
@@ -1146,12 +1194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           store_rows(ebuf, lane, ou, reinterpret_cast<uint8_t*>(dau + args.f + c), args.ldo * 2, vrows);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (PAIR && rank != 0) mbar_arrive_remote(mapa_shared(tempty_bar(acc), 0));
-        else mbar_arrive(tempty_bar(acc));
-      }
+      if constexpr (!kEarlyRelease) release_acc();
       if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
       if constexpr (EPI == EPI_BF16_COMBINE) {
         // The warp's rows of this column tile are stored and the accumulator
