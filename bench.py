@@ -484,7 +484,8 @@ def run_ours(args):
                    "global_batch": cfg.T * ws, "parallelism": f"replicas{ws}" if ws > 1 else "1 GPU",
                    "l2": "flushed between timed steps outside the step events (512 MiB write, "
                          "then a 512 MiB read of another buffer)"},
-        "roofline": {"bound": "tensor", "kernel": "grouped_gemm_kernel (6 launches per step)",
+        "roofline": {"bound": "tensor", "kernel": "grouped_gemm_kernel: every expert GEMM launch of a step "
+                               "(events around the two expert calls)",
                      "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
                      "peak_source": f"{peak_kind} bf16 burst"},

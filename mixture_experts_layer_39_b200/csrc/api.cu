@@ -32,8 +32,9 @@ bool pair_tiles(const moe_shape_t* s) {
   return static_cast<int64_t>(s->T) * s->top_k >= 1536ll * s->n_experts;
 }
 
-moe::GemmCtx gemm_ctx(const moe_context* h, bool pair_m) {
+moe::GemmCtx gemm_ctx(moe_context* h, bool pair_m) {
   moe::GemmCtx c;
+  c.extra_launches = &h->launches;
   c.num_sms = h->num_sms;
   c.ctl = h->ctl;
   c.pair_m = pair_m;

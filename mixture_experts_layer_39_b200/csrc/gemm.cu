@@ -140,7 +140,8 @@ moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const tc::GemmAr
                          : PAIR ? (BN == 512 ? (BWD ? 3 : 4) : 6)
                                 : (BN == 256 ? 4 : 6);
   if constexpr (BWD || FP8) {
-    if (tc::SmemPlan<BN, STAGES, EPI, FP8, PAIR>::bytes(args.n_groups) > kMaxDynSmem)
+    const size_t need = tc::SmemPlan<BN, STAGES, EPI, FP8, PAIR>::bytes(args.n_groups);
+    if (need > kMaxDynSmem)
       return launch_stages<BN, A_MN, B_MN, EPI, KGROUP, STAGES - 1, FP8, PAIR, GATHER>(
           a, b, sfa, sfb, args, grid, st);
   }
@@ -148,20 +149,33 @@ moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const tc::GemmAr
                                                                               grid, st);
 }
 
+// The last wave of wide weight-gradient tiles keeps every busy pair for a
+// whole wide tile while the others idle.  When that wave holds at most half
+// as many tiles as there are pairs, its tiles run instead as a second launch
+// of 256 x 256 tiles (two per wide tile, one per pair), which ends in about
+// 0.6 of a wide tile's time.  Returns the number of wide tiles moved there.
+int64_t wide_tail(int num_sms, int64_t wide_tiles) {
+  const int64_t units = num_sms / 2 > 0 ? num_sms / 2 : 1;
+  const int64_t rem = wide_tiles % units;
+  return (rem > 0 && 2 * rem <= units) ? rem : 0;
+}
+
 // Weight gradients run 256 x 512 pair tiles ("wide") when the experts'
 // contraction ranges are long (at least 4096 routed rows on average: the
 // single accumulator's epilogue, which no longer overlaps the next tile, is
-// then a few percent of a tile) and 256 x 256 tiles would not fill the SMs'
-// waves enough better.  A wide tile does twice the work of a narrow one in
-// about 0.87 of twice its time (it reads 25% fewer operand bytes per FLOP);
-// tiles = E x M tiles x N tiles, units = CTA pairs.
+// then a few percent of a tile) and the waves come out shorter than with
+// 256 x 256 tiles.  In units of a wide tile's time: a narrow tile takes about
+// 0.575 (half the work at 0.87 of the wide rate: it reads 25% more operand
+// bytes per FLOP) and a tail moved to a narrow launch about 0.6; tiles =
+// E x M tiles x N tiles, units = CTA pairs.
 bool wide_wgrad(int num_sms, int64_t E, int64_t M, int64_t N, int64_t rows) {
   if (rows < 4096 * E) return false;
   const int64_t units = num_sms / 2 > 0 ? num_sms / 2 : 1;
   const int64_t mt = ceil_div64(M, 256);
-  const int64_t waves_n = ceil_div64(E * mt * ceil_div64(N, 256), units);
-  const int64_t waves_w = ceil_div64(E * mt * ceil_div64(N, 512), units);
-  return 174 * waves_w <= 100 * waves_n;
+  const int64_t tiles_n = E * mt * ceil_div64(N, 256);
+  const int64_t tiles_w = E * mt * ceil_div64(N, 512);
+  const int64_t tail = tiles_w % units == 0 ? 0 : (wide_tail(num_sms, tiles_w) > 0 ? 600 : 1000);
+  return 1000 * (tiles_w / units) + tail <= 575 * ceil_div64(tiles_n, units);
 }
 
 tc::GemmArgs base_args(const GemmCtx& c) {
@@ -182,6 +196,40 @@ void set_m(tc::GemmArgs& a, int64_t M, int mt) {
   a.m_rows = static_cast<int>(M);
   a.m_tiles_fixed = static_cast<int>(ceil_div64(M, mt));
 }
+
+// A K-grouped weight gradient on wide tiles, its last wave (wide_tail) as a
+// second launch of 256 x 256 tiles over the same groups and M tiles: wide
+// tile w covers narrow tiles 2w and 2w + 1, so the tail is one contiguous
+// range of the narrow launch's tile list.
+moe_status_t launch_wgrad_wide(const GemmCtx& c, const CUtensorMap& ta, const CUtensorMap& tb,
+                               tc::GemmArgs a, int64_t N, cudaStream_t st) {
+  set_n(a, N, 512);
+  const int64_t tiles = static_cast<int64_t>(a.n_groups) * a.m_tiles_fixed * a.n_tiles_n;
+  const int64_t tail = wide_tail(c.num_sms, tiles);
+  const int64_t head = tiles - tail;
+  if (head > 0) {
+    tc::GemmArgs w = a;
+    if (tail > 0) {
+      w.tile_begin = 0;
+      w.tile_end = static_cast<int>(head);
+    }
+    const int grid = static_cast<int>(2 * head < c.num_sms ? 2 * head : c.num_sms);
+    const moe_status_t r = launch<512, true, true, tc::EPI_BF16, true, false, true>(ta, tb, w, grid, st);
+    if (r != MOE_OK) return r;
+  }
+  if (tail == 0) return MOE_OK;
+  tc::GemmArgs n = a;
+  // two 256-column tiles per wide tile, also where N ends in the first half
+  // of the last wide tile (that tile's second half then writes nothing)
+  n.n_cols = static_cast<int>(N);
+  n.n_tiles_n = 2 * a.n_tiles_n;
+  n.tile_begin = static_cast<int>(2 * head);
+  n.tile_end = static_cast<int>(2 * tiles);
+  if (c.extra_launches != nullptr) ++*c.extra_launches;
+  const int grid = static_cast<int>(4 * tail < c.num_sms ? 4 * tail : c.num_sms);
+  return launch<256, true, true, tc::EPI_BF16, true, false, true>(ta, tb, n, grid, st);
+}
+
 
 }  // namespace
 
@@ -322,9 +370,9 @@ moe_status_t gemm_wgrad_down(const GemmCtx& c, const void* do_perm, const void* 
   a.ldo = f;
   a.out_gstride = static_cast<int64_t>(d) * f;
   set_m(a, d, 2 * tc::BM);  // CTA pairs: 256-row tiles
+  if (wide) return launch_wgrad_wide(c, ta, tb, a, f, st);
   const int64_t tiles = static_cast<int64_t>(E) * a.m_tiles_fixed * a.n_tiles_n;
   const int grid = static_cast<int>(2 * tiles < c.num_sms ? 2 * tiles : c.num_sms);
-  if (wide) return launch<512, true, true, tc::EPI_BF16, true, false, true>(ta, tb, a, grid, st);
   return launch<256, true, true, tc::EPI_BF16, true, false, true>(ta, tb, a, grid, st);
 }
 
@@ -345,9 +393,9 @@ moe_status_t gemm_wgrad_gate_up(const GemmCtx& c, const void* dau, const void* x
   a.ldo = d;
   a.out_gstride = 2ll * f * d;
   set_m(a, 2ll * f, 2 * tc::BM);  // CTA pairs: 256-row tiles
+  if (wide) return launch_wgrad_wide(c, ta, tb, a, d, st);
   const int64_t tiles = static_cast<int64_t>(E) * a.m_tiles_fixed * a.n_tiles_n;
   const int grid = static_cast<int>(2 * tiles < c.num_sms ? 2 * tiles : c.num_sms);
-  if (wide) return launch<512, true, true, tc::EPI_BF16, true, false, true>(ta, tb, a, grid, st);
   return launch<256, true, true, tc::EPI_BF16, true, false, true>(ta, tb, a, grid, st);
 }
 

@@ -14,6 +14,9 @@ struct GemmCtx {
   // time limit of the GEMMs' main-loop waits (the handle's; 0 = give up
   // unless already complete)
   uint64_t wait_ns = 2000000000ull;
+  // launches beyond the fixed count an entry point books (a weight gradient
+  // whose last wave runs as a second launch) are added here
+  uint64_t* extra_launches = nullptr;
 };
 
 // An MXFP8 operand: E4M3 codes and E8M0 scales ([MN index][K/32] bytes).

@@ -115,8 +115,5 @@ cudaError_t launch_mxfp8_quantize_both(const __nv_bfloat16* in, int64_t rows, in
                                        int64_t rows_per_group, uint8_t* q_row, uint8_t* s_row,
                                        uint8_t* q_col, uint8_t* s_col, int num_sms,
                                        cudaStream_t st);
-cudaError_t launch_mxfp8_quantize_cols_t(const __nv_bfloat16* in, int64_t rows, int64_t cols,
-                                         int64_t rows_per_group, uint8_t* q, uint8_t* scales,
-                                         cudaStream_t st);
 
 }  // namespace moe

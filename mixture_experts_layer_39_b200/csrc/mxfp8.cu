@@ -107,14 +107,10 @@ __global__ void mx_rowwise_kernel(const uint4* __restrict__ in, int64_t rows, in
 // of the block is one vector load and one vector store of W codes; the two
 // columns of a bf16 pair are converted by one paired E4M3 conversion (each
 // element rounds on its own, so pairing changes no code).  Scales go to
-// [rows/32, cols] (scale_mode 0) or, for the GEMM operands, per group of
-// rows_per_group rows in atom order with the column as the MN index and the
-// row inside the group as the contraction index (scale_mode 1; cols and
-// rows_per_group multiples of 128).
+// [rows/32, cols].
 template <int W>
 __global__ void mx_colwise_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_t cols,
-                                  uint8_t* __restrict__ q, uint8_t* __restrict__ scales,
-                                  int scale_mode, int64_t rows_per_group) {
+                                  uint8_t* __restrict__ q, uint8_t* __restrict__ scales) {
   static_assert(W == 2 || W == 4, "two or four columns per thread");
   constexpr int NP = W / 2;  // bf16 pairs per row slice
   using In = typename std::conditional<NP == 2, uint2, uint32_t>::type;
@@ -168,19 +164,10 @@ __global__ void mx_colwise_kernel(const __nv_bfloat16* __restrict__ in, int64_t 
              << (16 * j);
       *dst = static_cast<Out>(p);
     }
-    if (scale_mode == 0) {
-      uint32_t s = 0;
+    uint32_t sc = 0;
 #pragma unroll
-      for (int c = 0; c < W; ++c) s |= static_cast<uint32_t>(e[c] + 127) << (8 * c);
-      reinterpret_cast<Out*>(scales)[rb * cgroups + cg] = static_cast<Out>(s);
-    } else {
-      const int64_t bpg = rows_per_group / 32;  // scale blocks per group
-      const int64_t g = rb / bpg, rl = rb - g * bpg;
-      uint8_t* gs = scales + g * cols * bpg;
-#pragma unroll
-      for (int c = 0; c < W; ++c)
-        gs[atom_byte(W * cg + c, rl, bpg >> 2)] = static_cast<uint8_t>(e[c] + 127);
-    }
+    for (int c = 0; c < W; ++c) sc |= static_cast<uint32_t>(e[c] + 127) << (8 * c);
+    reinterpret_cast<Out*>(scales)[rb * cgroups + cg] = static_cast<Out>(sc);
   }
 }
 
@@ -194,7 +181,7 @@ __global__ void mx_colwise_kernel(const __nv_bfloat16* __restrict__ in, int64_t 
 //              thread's 4-row maxima meet in shared memory, thread t takes
 //              column t's amax and writes its scale; codes to q_col.
 // The tile's 32 rows never straddle a group (rows_per_group is a multiple of
-// 128), so column blocks follow the per-group atom layout of scale_mode 1.
+// 128), so the column blocks of each group take their own run of atoms.
 // Capped at 64 registers a thread, eight blocks (64 KB of loads in flight)
 // fit on an SM, against five at the uncapped 92: 0.79 of the measured copy
 // rate on operand-sized inputs, against 0.67.
@@ -278,19 +265,16 @@ __global__ void __launch_bounds__(128, 8)
 
 // Picks four columns per thread when every vector access stays aligned.
 cudaError_t launch_colwise(const __nv_bfloat16* in, int64_t rows, int64_t cols, uint8_t* q,
-                           uint8_t* scales, int scale_mode, int64_t rows_per_group,
-                           cudaStream_t st) {
+                           uint8_t* scales, cudaStream_t st) {
   const bool wide = cols % 4 == 0 && (reinterpret_cast<uintptr_t>(in) & 7) == 0 &&
                     (reinterpret_cast<uintptr_t>(q) & 3) == 0 &&
-                    (scale_mode != 0 || (reinterpret_cast<uintptr_t>(scales) & 3) == 0);
+                    (reinterpret_cast<uintptr_t>(scales) & 3) == 0;
   const int64_t total = (rows / 32) * (cols / (wide ? 4 : 2));
   const unsigned grid = static_cast<unsigned>(ceil_div64(total, 256) < 65535 ? ceil_div64(total, 256) : 65535);
   if (wide)
-    (void)launch_pdl(mx_colwise_kernel<4>, grid, 256, 0, st, in, rows, cols, q, scales, scale_mode,
-                     rows_per_group);
+    (void)launch_pdl(mx_colwise_kernel<4>, grid, 256, 0, st, in, rows, cols, q, scales);
   else
-    (void)launch_pdl(mx_colwise_kernel<2>, grid, 256, 0, st, in, rows, cols, q, scales, scale_mode,
-                     rows_per_group);
+    (void)launch_pdl(mx_colwise_kernel<2>, grid, 256, 0, st, in, rows, cols, q, scales);
   return cudaGetLastError();
 }
 
@@ -308,7 +292,7 @@ cudaError_t launch_rowwise(const __nv_bfloat16* in, int64_t rows, int64_t cols, 
 cudaError_t launch_mxfp8_quantize(const __nv_bfloat16* in, int64_t rows, int64_t cols, int axis,
                                   uint8_t* q, uint8_t* scales, cudaStream_t st) {
   if (axis == 1) return launch_rowwise(in, rows, cols, q, scales, false, st);
-  return launch_colwise(in, rows, cols, q, scales, 0, rows, st);
+  return launch_colwise(in, rows, cols, q, scales, st);
 }
 
 cudaError_t launch_mxfp8_quantize_atoms(const __nv_bfloat16* in, int64_t rows, int64_t cols,
@@ -328,12 +312,6 @@ cudaError_t launch_mxfp8_quantize_both(const __nv_bfloat16* in, int64_t rows, in
                    rows_per_group, reinterpret_cast<uint2*>(q_row), s_row,
                    reinterpret_cast<uint2*>(q_col), s_col);
   return cudaGetLastError();
-}
-
-cudaError_t launch_mxfp8_quantize_cols_t(const __nv_bfloat16* in, int64_t rows, int64_t cols,
-                                         int64_t rows_per_group, uint8_t* q, uint8_t* scales,
-                                         cudaStream_t st) {
-  return launch_colwise(in, rows, cols, q, scales, 1, rows_per_group, st);
 }
 
 }  // namespace moe

@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(kDwThreads)
                      int d, int E, int group_len, float* __restrict__ partial) {
   pdl_wait();
   pdl_trigger();
-  extern __shared__ __align__(16) uint8_t s_raw[];
+  extern __shared__ __align__(128) uint8_t s_raw[];
   uint8_t* s_x = s_raw;                                              // [2][kDwTok][kDwCols] bf16
   float* s_dl = reinterpret_cast<float*>(s_raw + 2 * kDwStageX);      // [2][kDwTok][NE]
   const int64_t col0 = static_cast<int64_t>(blockIdx.x) * kDwCols;

@@ -62,6 +62,9 @@ struct GemmArgs {
   int uniform_len;     // group length when offsets == nullptr
   int total_len;       // clamp of all group boundaries (rows of the grouped operand)
   int m_tiles_fixed;   // K-grouped: M / BM
+  // K-grouped: with tile_end > 0 the launch takes tiles [tile_begin, tile_end)
+  // of the full tile list only (a weight gradient's last wave as its own launch)
+  int tile_begin, tile_end;
   int64_t m_cap;       // M-grouped: rows of the output buffer (store bound)
   void* out;
   int64_t ldo;
@@ -708,6 +711,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     total_tiles = args.n_groups * args.m_tiles_fixed * args.n_tiles_n;
   }
+  int t_begin = 0;
+  if constexpr (KGROUP) {
+    if (args.tile_end > 0) {
+      t_begin = args.tile_begin;
+      total_tiles = args.tile_end < total_tiles ? args.tile_end : total_tiles;
+    }
+  }
 
   if (warp == 0) {
     // ================================================================ producer
@@ -721,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // per-stage: a load is in flight / its phase
       bool ok = true;
-      for (int t = unit; t < total_tiles && ok; t += n_units) {
+      for (int t = t_begin + unit; t < total_tiles && ok; t += n_units) {
         const Tile tl = decode_tile<KGROUP, BKE, KMMA, MT>(args, s_tile_start, t);
         // GATHER: x rows of this lane's 4 rows of the stage (M-grouped: the same
         // rows for the whole tile; K-grouped: loaded one K-block ahead)
@@ -887,7 +897,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_phase = 0;
       uint32_t sf_buf = 0;
       bool ok = true;
-      for (int t = unit; t < total_tiles && ok; t += n_units) {
+      for (int t = t_begin + unit; t < total_tiles && ok; t += n_units) {
         const Tile tl = decode_tile<KGROUP, BKE, KMMA, MT>(args, s_tile_start, t);
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, s_abort, args.wait_ns, true, PAIR)) {
           ok = false;
@@ -989,7 +999,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return n <= 0 ? 0 : (n >= rpw ? rpw : static_cast<int>(n));
       }
     };
-    for (int t = unit; t < total_tiles; t += n_units) {
+    for (int t = t_begin + unit; t < total_tiles; t += n_units) {
       const Tile tl = decode_tile<KGROUP, BKE, KMMA, MT>(args, s_tile_start, t);
       const int vrows = quarter_rows(tl);
       const int64_t row_first = quarter_first(tl);  // warp's first row

@@ -3,7 +3,13 @@ step into one TMEM accumulator), at shapes where those wide tiles are
 chosen: long expert segments and enough tiles to fill the SMs.  Checked
 against the oracle's plain per-expert products (float64 on the GPU's own
 dO_perm, H, dAU and x_perm), with an expert without rows (its tiles write
-zeros), and for determinism (two runs give the same bits)."""
+zeros), and for determinism (two runs give the same bits).
+
+When the last wave of wide tiles would fill at most half of the 74 CTA
+pairs, those tiles run as a second launch of 256 x 256 tiles (two per wide
+tile).  The cases below cover that for both weight gradients, including N
+ending in the first half of the last wide tile (its second half then
+writes nothing)."""
 import numpy as np
 import pytest
 import torch
@@ -17,7 +23,12 @@ pytestmark = pytest.mark.gpu
 
 # T, d, f, E, k: at least 4096 routed rows per expert and enough tiles that
 # 256 x 512 tiles beat 256 x 256 ones on 74 CTA pairs
-CASES = [(8192, 2048, 1024, 4, 2), (6144, 2048, 1024, 3, 2)]
+CASES = [
+    (8192, 2048, 1024, 4, 2),   # wgrad gate/up 128 wide tiles, wgrad down 64: one launch each
+    (6144, 2048, 1024, 3, 2),   # wgrad gate/up 96 wide tiles: the last 22 as a narrow launch
+    (6144, 1792, 1024, 3, 2),   # as above with N = d = 1792: a half-used last wide tile
+    (8192, 3328, 768, 4, 2),    # both weight gradients with a narrow tail, both N ragged
+]
 
 
 def _route(T, E, k, empty, seed):
