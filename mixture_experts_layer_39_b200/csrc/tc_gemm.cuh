@@ -377,6 +377,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+// 32 lanes x 16 consecutive fp32 columns of TMEM.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -1042,10 +1053,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // MXFP8 keeps one accumulator (TMEM also holds the scales), so a tile's
       // epilogue would hold up the next tile's MMAs.  A plain bf16 output
-      // row of 256 columns fits in 128 registers as bf16 pairs: it is read
-      // out of TMEM whole, the accumulator is released, and the stores follow.
-      constexpr bool kEarlyRelease = FP8 && EPI == EPI_BF16 && BN == 256;
-      if constexpr (kEarlyRelease) {
+      // row of 256 columns fits in 128 registers as bf16 pairs, the SwiGLU
+      // forward's A, U and H of 128 columns in 192: they are formed straight
+      // out of TMEM, the accumulator is released, and the stores follow.
+      constexpr bool kEarlyRelease = FP8 && (EPI == EPI_BF16 || EPI == EPI_SWIGLU_FWD) && BN == 256;
+      if constexpr (kEarlyRelease && EPI == EPI_BF16) {
         auto* base = static_cast<__nv_bfloat16*>(args.out) + gofs + row_first * args.ldo +
                      static_cast<int64_t>(tl.n_tile) * BN;
         uint32_t pk[BN / 2];  // bf16 pairs of this lane's row
@@ -1112,6 +1124,49 @@ __global__ void __launch_bounds__(kThreads, 1)
             v[q] = zero_acc ? make_uint4(0, 0, 0, 0)
                             : make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
           store_rows(ebuf, lane, v, reinterpret_cast<uint8_t*>(base + c), args.ldo * 4, vrows);
+        }
+      } else if constexpr (EPI == EPI_SWIGLU_FWD && FP8) {
+        // as above: A, U and H of the warp's rows (3 x 64 registers of bf16
+        // pairs) are formed straight out of TMEM, 16 columns at a time; the
+        // accumulator is released, then the rows are stored
+        constexpr int BNH = BN / 2;
+        const int64_t col0 = static_cast<int64_t>(tl.n_tile) * BNH;
+        auto* au = args.out != nullptr
+                       ? static_cast<__nv_bfloat16*>(args.out) + row_first * args.ldo + col0
+                       : nullptr;
+        auto* hh = static_cast<__nv_bfloat16*>(args.out2) + row_first * args.ldo2 + col0;
+        uint32_t pa[BNH / 2], pu[BNH / 2], ph[BNH / 2];
+#pragma unroll
+        for (int c = 0; c < BNH; c += 16) {
+          uint32_t g[16], u[16];
+          tmem_ld16(tbase + tcol(c), g);
+          tmem_ld16(tbase + tcol(BNH + c), u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float a0 = __uint_as_float(g[2 * i]), a1 = __uint_as_float(g[2 * i + 1]);
+            const float b0 = __uint_as_float(u[2 * i]), b1 = __uint_as_float(u[2 * i + 1]);
+            pa[c / 2 + i] = pack_bf16x2(a0, a1);
+            pu[c / 2 + i] = pack_bf16x2(b0, b1);
+            ph[c / 2 + i] = pack_bf16x2(a0 * sigmoid_fast(a0) * b0, a1 * sigmoid_fast(a1) * b1);
+          }
+        }
+        release_acc();
+        auto put = [&](const uint32_t (&p)[BNH / 2], int c, __nv_bfloat16* dst, int64_t ld) {
+          uint4 v[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            v[q] = make_uint4(p[c / 2 + 4 * q], p[c / 2 + 4 * q + 1], p[c / 2 + 4 * q + 2],
+                              p[c / 2 + 4 * q + 3]);
+          store_rows(ebuf, lane, v, reinterpret_cast<uint8_t*>(dst + c), ld * 2, vrows);
+        };
+#pragma unroll
+        for (int c = 0; c < BNH; c += 64) {
+          if (au != nullptr) {  // [A | U] is not kept when the backward recomputes it
+            put(pa, c, au, args.ldo);
+            put(pu, c, au + args.f, args.ldo);
+          }
+          put(ph, c, hh, args.ldo2);
         }
       } else if constexpr (EPI == EPI_SWIGLU_FWD) {
         constexpr int BNH = BN / 2;
