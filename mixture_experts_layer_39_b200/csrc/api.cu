@@ -26,10 +26,12 @@ int router_ld(int E) { return (E + 127) / 128 * 128; }
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 // 256-row CTA-pair tiles for the M-grouped expert GEMMs when the average
-// expert segment spans at least six of them (tail rows then waste < 1/12 of
-// the tiles); shorter segments keep 128-row tiles.
+// expert segment spans at least four of them; shorter segments (about 512
+// rows at E = 128 and T k = 65536) keep 128-row tiles, whose tail rows waste
+// half as much.  The routing is not known on the host, so a skewed routing
+// with this average (a few long segments) also gets pairs, which suit it.
 bool pair_tiles(const moe_shape_t* s) {
-  return static_cast<int64_t>(s->T) * s->top_k >= 1536ll * s->n_experts;
+  return static_cast<int64_t>(s->T) * s->top_k >= 1024ll * s->n_experts;
 }
 
 moe::GemmCtx gemm_ctx(moe_context* h, bool pair_m) {
