@@ -466,7 +466,7 @@ __global__ void __launch_bounds__(kWarps * 32)
       const int c = __ldg(route_in + t * k + j);
       chosen[j] = c;
       if (c >= 0 && c < E) {
-        const float lc = logits_in[t * E + c] + (bias != nullptr ? __ldg(bias + c) : 0.f);
+        const float lc = logits_in[t * ld_in + c] + (bias != nullptr ? __ldg(bias + c) : 0.f);
         wsel[j] = expf(lc - m) * inv;
       } else if (lane == 0) {
         report(ctl, MOE_ERR_DEVICE_CHECK, 101);

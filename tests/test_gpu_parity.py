@@ -182,6 +182,8 @@ SMALL_CASES = [
     (1600, 256, 256, 6, 2, "skewed"),      # empty experts next to one long segment
     (300, 2304, 256, 8, 2, "learned"),     # d > 2048: router dW over two column slices
     (200, 4096, 128, 16, 4, "bias"),       # d = 4096, E = 16 (router dW: two n-tiles of experts)
+    (700, 256, 256, 200, 6, "random"),     # caller-given ids with the tensor-core router's
+    (500, 384, 128, 96, 3, "random"),      # padded logits rows (stride 256 and 128, not E)
 ]
 
 
