@@ -184,20 +184,23 @@ SMALL_CASES = [
     (200, 4096, 128, 16, 4, "bias"),       # d = 4096, E = 16 (router dW: two n-tiles of experts)
     (700, 256, 256, 200, 6, "random"),     # caller-given ids with the tensor-core router's
     (500, 384, 128, 96, 3, "random"),      # padded logits rows (stride 256 and 128, not E)
+    (300, 256, 256, 48, 3, "random"),      # caller-given ids on the CUDA-core router (16 < E <= 64)
+    (400, 256, 256, 100, 4, "random_renorm"),  # caller-given ids, renormalised gate weights
 ]
 
 
 @pytest.mark.parametrize("case", SMALL_CASES, ids=lambda c: "T%d_d%d_f%d_E%d_k%d_%s" % c)
 def test_small_shapes_every_stage(cuda_ok, case):
     T, d, f, E, k, mode = case
-    cfg = custom_config(T, d, f, E, k, random_routing=(mode == "random"))
+    renorm = mode in ("renorm", "random_renorm")
+    cfg = custom_config(T, d, f, E, k, random_routing=mode in ("random", "random_renorm"))
     inp = make_inputs(cfg, seed=T + E, device="cpu")
     if mode == "skewed":
         inp["bias"] = torch.tensor([4.0, -30.0, 2.0, -30.0, 0.0, -30.0][:E], dtype=torch.float32)
     if mode == "bias":
         inp["bias"] = torch.linspace(-1, 1, E, dtype=torch.float32)
-    L = _run(cfg, _to(inp, "cuda"), renorm=(mode == "renorm"))
-    _check_full(cfg, inp, L, renorm=(mode == "renorm"))
+    L = _run(cfg, _to(inp, "cuda"), renorm=renorm)
+    _check_full(cfg, inp, L, renorm=renorm)
     if mode == "skewed":
         assert (np64(L.counts) == 0).any()
 
