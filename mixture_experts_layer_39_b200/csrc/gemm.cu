@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "gemm.cuh"
+#include "host_ctx.cuh"
 #include "tc_gemm.cuh"
 
 namespace moe {
@@ -89,13 +90,7 @@ moe_status_t launch_stages(const CUtensorMap& a, const CUtensorMap& b, const CUt
                            cudaStream_t st) {
   auto kern = tc::grouped_gemm_kernel<BN, A_MN, B_MN, EPI, KGROUP, STAGES, FP8, PAIR, GATHER>;
   const size_t smem = tc::SmemPlan<BN, STAGES, EPI, FP8, PAIR>::bytes(args.n_groups);
-  static size_t configured = 0;  // largest size this instantiation was opened for
-  if (smem > configured) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    configured = smem;
-  }
+  if (!set_max_dyn_smem(reinterpret_cast<const void*>(kern), smem)) return MOE_ERR_CUDA;
   if (grid <= 0) return MOE_OK;
   if constexpr (PAIR) {
     grid &= ~1;  // whole pairs

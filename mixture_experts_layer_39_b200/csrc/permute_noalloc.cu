@@ -33,6 +33,7 @@
 #include <mutex>
 
 #include "context.cuh"
+#include "host_ctx.cuh"
 #include "kernels.cuh"
 
 namespace {
@@ -47,41 +48,18 @@ std::mutex g_scratch_mu;
 int32_t* g_scratch_addr[kMaxDevices] = {};
 unsigned long long g_scratch_ctx[kMaxDevices] = {};  // context id the address belongs to
 
-// Id of the calling thread's current CUDA context (unique per context
-// created in this process), or 0 when there is none or it cannot be read.
-unsigned long long current_context_id() {
-  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
-  static PFN_cuCtxGetId_v12000 get_id = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
-    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
-  });
-  if (get_current == nullptr || get_id == nullptr) return 0;
-  CUcontext ctx = nullptr;
-  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
-  unsigned long long id = 0;
-  return get_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
-}
-
 // Device address of the array on `device`, which must be the current device.
 moe_status_t scratch_on_device(int device, int32_t** out) {
   if (device < 0 || device >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  const unsigned long long ctx = current_context_id();
+  const unsigned long long ctx = moe::current_context_id();
   if (g_scratch_addr[device] == nullptr || ctx == 0 || ctx != g_scratch_ctx[device]) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_permute_scratch);
     if (e != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
     g_scratch_addr[device] = static_cast<int32_t*>(p);
     // the lookup made the device's primary context current if it was not
-    g_scratch_ctx[device] = ctx != 0 ? ctx : current_context_id();
+    g_scratch_ctx[device] = ctx != 0 ? ctx : moe::current_context_id();
   }
   *out = g_scratch_addr[device];
   return MOE_OK;

@@ -11,6 +11,7 @@
 // file only produces dL (bf16) and the db partial sums.
 #include <type_traits>
 
+#include "host_ctx.cuh"
 #include "kernels.cuh"
 
 namespace moe {
@@ -705,13 +706,8 @@ cudaError_t launch_router_dw(const float* dl, const __nv_bfloat16* x, int T, int
                              cudaStream_t st) {
   if (E <= 16) {
     auto kern = E <= 8 ? router_dw_stream_kernel<8> : router_dw_stream_kernel<16>;
-    static bool opened[2] = {false, false};  // attribute set once per instantiation
-    if (!opened[E <= 8 ? 0 : 1]) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kDsSmem)) != cudaSuccess)
-        return cudaErrorInvalidValue;
-      opened[E <= 8 ? 0 : 1] = true;
-    }
+    if (!set_max_dyn_smem(reinterpret_cast<const void*>(kern), kDsSmem))
+      return cudaErrorInvalidValue;
     const unsigned gx = static_cast<unsigned>(ceil_div64(d, kDsCols));
     (void)launch_pdl(kern, dim3(gx, static_cast<unsigned>(n_chunks)), kDsThreads, kDsSmem, st, dl,
                      x, T, d, E, group_len, partial, ctl);

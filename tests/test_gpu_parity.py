@@ -186,6 +186,8 @@ SMALL_CASES = [
     (500, 384, 128, 96, 3, "random"),      # padded logits rows (stride 256 and 128, not E)
     (300, 256, 256, 48, 3, "random"),      # caller-given ids on the CUDA-core router (16 < E <= 64)
     (400, 256, 256, 100, 4, "random_renorm"),  # caller-given ids, renormalised gate weights
+    (300, 128, 128, 8, 2, "learned"),      # the smallest d and d_ff: one router chunk per warp
+    (300, 128, 256, 100, 3, "bias"),       # d = 128 with the tensor-core router (K = 2 blocks)
 ]
 
 
