@@ -172,6 +172,7 @@ bool all_nonnull(P... p) { return ((p != nullptr) && ...); }
 extern "C" {
 
 moe_status_t moe_create(moe_handle_t* out, int device) {
+  MOE_TRACE();
   if (out == nullptr) return MOE_ERR_INVALID_ARG;
   *out = nullptr;
   int n = 0;
@@ -199,6 +200,7 @@ moe_status_t moe_create(moe_handle_t* out, int device) {
 }
 
 moe_status_t moe_destroy(moe_handle_t h) {
+  MOE_TRACE();
   if (h == nullptr) return MOE_ERR_INVALID_ARG;
   {
     DeviceGuard g(h->device);
@@ -226,6 +228,7 @@ moe_status_t moe_router_topk(moe_handle_t h, const moe_shape_t* s, const void* x
                              const void* w_router, const float* bias, const int32_t* route_in,
                              int32_t* topk_idx, float* topk_w, float* probs, float* logits,
                              void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (!all_nonnull(x, w_router, topk_idx, topk_w, probs)) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(w_router, 16)) return MOE_ERR_INVALID_ARG;
@@ -261,6 +264,7 @@ moe_status_t moe_permute(moe_handle_t h, const moe_shape_t* s, const void* x,
                          const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
                          int32_t* row_map, void* x_perm, void* ws, size_t ws_bytes,
                          moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (!all_nonnull(x, topk_idx, counts, offsets, row_map, x_perm)) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(x_perm, 16)) return MOE_ERR_INVALID_ARG;
@@ -281,6 +285,7 @@ moe_status_t moe_permute_src(moe_handle_t h, const moe_shape_t* s, const void* x
                              const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
                              int32_t* row_map, int32_t* row_src, void* x_perm, void* ws,
                              size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (!all_nonnull(x, topk_idx, counts, offsets, row_map, row_src, x_perm))
     return MOE_ERR_INVALID_ARG;
@@ -305,6 +310,7 @@ moe_status_t moe_grouped_swiglu_fwd_combine(moe_handle_t h, const moe_shape_t* s
                                             const void* w_down, void* au, void* hbuf,
                                             void* o_perm, const void* shared_out, void* y,
                                             int32_t* arrivals, moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (s->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
   if (!all_nonnull(x_perm, offsets, row_map, row_src, topk_w, w_gu, w_down, hbuf, o_perm, y,
@@ -329,6 +335,7 @@ moe_status_t moe_grouped_swiglu_fwd_combine(moe_handle_t h, const moe_shape_t* s
 moe_status_t moe_route(moe_handle_t h, const moe_shape_t* s, const int32_t* topk_idx,
                        int32_t* counts, int32_t* offsets, int32_t* row_map, int32_t* row_src,
                        void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (!all_nonnull(topk_idx, counts, offsets, row_map, row_src)) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_ws(h, s, ws, ws_bytes));
@@ -350,6 +357,7 @@ moe_status_t moe_grouped_swiglu_fwd_gather(moe_handle_t h, const moe_shape_t* s,
                                            const int32_t* row_src, const int32_t* offsets,
                                            const void* w_gu, const void* w_down, void* au,
                                            void* hbuf, void* o_perm, moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (s->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
   if (!all_nonnull(x, row_src, offsets, w_gu, w_down, hbuf, o_perm)) return MOE_ERR_INVALID_ARG;
@@ -371,6 +379,7 @@ moe_status_t moe_grouped_swiglu_recompute_gather(moe_handle_t h, const moe_shape
                                                  const void* x, const int32_t* row_src,
                                                  const int32_t* offsets, const void* w_gu,
                                                  void* au, void* hbuf, moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (s->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
   if (!all_nonnull(x, row_src, offsets, w_gu, au, hbuf)) return MOE_ERR_INVALID_ARG;
@@ -391,6 +400,7 @@ moe_status_t moe_grouped_swiglu_bwd_gather(moe_handle_t h, const moe_shape_t* s,
                                            const void* w_gu, const void* w_down, void* dau,
                                            void* dx_perm, void* dw_gu, void* dw_down,
                                            moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (s->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
   if (!all_nonnull(do_perm, x, row_src, au, hbuf, offsets, w_gu, w_down, dau, dx_perm, dw_gu,
@@ -417,6 +427,7 @@ moe_status_t moe_grouped_swiglu_fwd(moe_handle_t h, const moe_shape_t* s, const 
                                     const int32_t* offsets, const void* w_gu, const void* w_down,
                                     void* au, void* hbuf, void* o_perm, void* ws, size_t ws_bytes,
                                     moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (!all_nonnull(x_perm, offsets, w_gu, w_down, hbuf, o_perm)) return MOE_ERR_INVALID_ARG;
   for (const void* p : {x_perm, w_gu, w_down, static_cast<const void*>(au),
@@ -458,6 +469,7 @@ moe_status_t moe_grouped_swiglu_recompute(moe_handle_t h, const moe_shape_t* s, 
                                           const int32_t* offsets, const void* w_gu, void* au,
                                           void* hbuf, void* ws, size_t ws_bytes,
                                           moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (!all_nonnull(x_perm, offsets, w_gu, au, hbuf)) return MOE_ERR_INVALID_ARG;
   for (const void* p : {x_perm, w_gu, static_cast<const void*>(au), static_cast<const void*>(hbuf)})
@@ -487,6 +499,7 @@ moe_status_t moe_grouped_swiglu_recompute(moe_handle_t h, const moe_shape_t* s, 
 moe_status_t moe_unpermute_combine(moe_handle_t h, const moe_shape_t* s, const void* o_perm,
                                    const int32_t* row_map, const float* topk_w,
                                    const void* shared_out, void* y, moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (!all_nonnull(o_perm, row_map, topk_w, y)) return MOE_ERR_INVALID_ARG;
   if (!aligned(o_perm, 16) || !aligned(y, 16) || !aligned(shared_out, 16))
@@ -505,6 +518,7 @@ moe_status_t moe_unpermute_combine_bwd(moe_handle_t h, const moe_shape_t* s, con
                                        const float* topk_w, const int32_t* offsets,
                                        const int32_t* counts, void* do_perm, float* d_topk_w,
                                        moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (!all_nonnull(dy, o_perm, row_map, topk_w, offsets, counts, do_perm, d_topk_w))
     return MOE_ERR_INVALID_ARG;
@@ -522,6 +536,7 @@ moe_status_t moe_grouped_swiglu_bwd(moe_handle_t h, const moe_shape_t* s, const 
                                     const int32_t* offsets, const void* w_gu, const void* w_down,
                                     void* dau, void* dx_perm, void* dw_gu, void* dw_down, void* ws,
                                     size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (!all_nonnull(do_perm, x_perm, au, hbuf, offsets, w_gu, w_down, dau, dx_perm, dw_gu, dw_down))
     return MOE_ERR_INVALID_ARG;
@@ -576,6 +591,7 @@ moe_status_t moe_grouped_swiglu_bwd(moe_handle_t h, const moe_shape_t* s, const 
 moe_status_t moe_shared_expert_fwd(moe_handle_t h, const moe_shape_t* s, const void* x,
                                    const void* w_gu_s, const void* w_d_s, void* au_s, void* h_s,
                                    void* o_s, moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (s->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
   if (!all_nonnull(x, w_gu_s, w_d_s, au_s, h_s, o_s)) return MOE_ERR_INVALID_ARG;
@@ -595,6 +611,7 @@ moe_status_t moe_shared_expert_bwd(moe_handle_t h, const moe_shape_t* s, const v
                                    const void* x, const void* au_s, const void* h_s,
                                    const void* w_gu_s, const void* w_d_s, void* dau_s, void* dx_s,
                                    void* dw_gu_s, void* dw_d_s, moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (s->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
   if (!all_nonnull(dy, x, au_s, h_s, w_gu_s, w_d_s, dau_s, dx_s, dw_gu_s, dw_d_s))
@@ -618,6 +635,7 @@ moe_status_t moe_shared_expert_bwd(moe_handle_t h, const moe_shape_t* s, const v
 moe_status_t moe_permute_bwd(moe_handle_t h, const moe_shape_t* s, const void* dx_perm,
                              const int32_t* row_map, const float* dx_router, const void* dx_shared,
                              void* dx, moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (!all_nonnull(dx_perm, row_map, dx)) return MOE_ERR_INVALID_ARG;
   if (!aligned(dx_perm, 16) || !aligned(dx, 16) || !aligned(dx_router, 16) ||
@@ -638,6 +656,7 @@ moe_status_t moe_permute_router_bwd(moe_handle_t h, const moe_shape_t* s, const 
                                     const float* probs, const int32_t* topk_idx,
                                     const float* d_probs_aux, const void* w_router,
                                     const void* dx_shared, void* dx, moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (s->n_experts > 64) return MOE_ERR_UNSUPPORTED;
   if (!all_nonnull(dx_perm, row_map, d_topk_w, probs, topk_idx, w_router, dx))
@@ -660,6 +679,7 @@ moe_status_t moe_router_topk_bwd(moe_handle_t h, const moe_shape_t* s, const flo
                                  const float* d_probs_aux, const void* x,
                                  const void* w_router, float* dx_router, void* dw_router,
                                  float* dbias, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (!all_nonnull(d_topk_w, probs, topk_idx, x, w_router, dw_router)) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(dx_router, 16))
@@ -710,6 +730,7 @@ moe_status_t moe_router_topk_bwd(moe_handle_t h, const moe_shape_t* s, const flo
 moe_status_t moe_router_load_stats(moe_handle_t h, const moe_shape_t* s, const float* probs,
                                    const int32_t* counts, int accumulate, float* stats, void* ws,
                                    size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (!all_nonnull(probs, counts, stats)) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_ws(h, s, ws, ws_bytes));
@@ -725,6 +746,7 @@ moe_status_t moe_router_load_stats(moe_handle_t h, const moe_shape_t* s, const f
 moe_status_t moe_router_aux_loss(moe_handle_t h, const moe_shape_t* s, const float* stats,
                                  int64_t n_tokens, float alpha, float* loss, float* d_probs_aux,
                                  moe_stream_t stream) {
+  MOE_TRACE();
   MOE_CHECK_HANDLE(h, s);
   if (stats == nullptr || (loss == nullptr && d_probs_aux == nullptr)) return MOE_ERR_INVALID_ARG;
   if (n_tokens < 1 || !(alpha >= 0.f)) return MOE_ERR_INVALID_ARG;
@@ -737,6 +759,7 @@ moe_status_t moe_router_aux_loss(moe_handle_t h, const moe_shape_t* s, const flo
 
 moe_status_t moe_mxfp8_quantize(moe_handle_t h, const void* in, int64_t rows, int64_t cols,
                                 int axis, uint8_t* q, uint8_t* scales, moe_stream_t stream) {
+  MOE_TRACE();
   if (h == nullptr || !all_nonnull(in, q, scales)) return MOE_ERR_INVALID_ARG;
   if (rows < 1 || cols < 1 || (axis != 0 && axis != 1)) return MOE_ERR_INVALID_ARG;
   if (axis == 1 && (cols % 32 != 0 || !aligned(in, 16) || !aligned(q, 16)))
@@ -753,6 +776,7 @@ moe_status_t moe_mxfp8_quantize(moe_handle_t h, const void* in, int64_t rows, in
 moe_status_t moe_mxfp8_quantize_gemm(moe_handle_t h, const void* in, int64_t rows, int64_t cols,
                                      int64_t rows_per_group, uint8_t* q_row, uint8_t* s_row,
                                      uint8_t* q_col, uint8_t* s_col, moe_stream_t stream) {
+  MOE_TRACE();
   if (h == nullptr || !all_nonnull(in, q_row, s_row) || !all_nonnull(q_col, s_col))
     return MOE_ERR_INVALID_ARG;
   if (rows < 1 || cols < 1 || rows_per_group < 1 || cols % 128 != 0 || rows_per_group % 128 != 0 ||
@@ -768,6 +792,7 @@ moe_status_t moe_mxfp8_quantize_gemm(moe_handle_t h, const void* in, int64_t row
 }
 
 moe_status_t moe_get_status(moe_handle_t h, int* device_status) {
+  MOE_TRACE();
   if (h == nullptr || device_status == nullptr) return MOE_ERR_INVALID_ARG;
   MOE_GUARD(h);
   if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;

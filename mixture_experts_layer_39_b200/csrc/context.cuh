@@ -1,6 +1,8 @@
 // The library handle behind moe_handle_t (private to libmoe.so).
 #pragma once
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 
 struct moe_context {
@@ -12,6 +14,20 @@ struct moe_context {
 };
 
 namespace moe {
+
+// One NVTX range per entry point that touches the device, named for the
+// entry point, pushed on entry and popped on every return: a timeline tool
+// (Nsight Systems, or any NVTX client) then shows each call's host span
+// around the kernels it launched.  With no tool attached the header-only
+// NVTX 3 calls go to empty functions.
+struct TraceRange {
+  explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+  ~TraceRange() { nvtxRangePop(); }
+  TraceRange(const TraceRange&) = delete;
+  TraceRange& operator=(const TraceRange&) = delete;
+};
+
+#define MOE_TRACE() const ::moe::TraceRange _moe_trace(__func__)
 
 // Makes the handle's device current for the duration of a call.
 struct DeviceGuard {

@@ -71,6 +71,7 @@ extern "C" moe_status_t moe_permute_noalloc(moe_handle_t h, const moe_shape_t* s
                                             const int32_t* topk_idx, int32_t* counts,
                                             int32_t* offsets, int32_t* row_map, void* x_perm,
                                             moe_stream_t stream) {
+  MOE_TRACE();
   if (h == nullptr) return MOE_ERR_INVALID_ARG;
   const moe_status_t shape_ok = moe::check_shape(s);
   if (shape_ok != MOE_OK) return shape_ok;
