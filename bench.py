@@ -162,15 +162,31 @@ def blas_threads():
     return os.cpu_count() or 1
 
 
-def size_oracle_sample(cfg, seconds):
-    """Tokens per oracle step so that one step costs about `seconds`."""
-    T_s = min(128, cfg.T)
+def _oracle_seconds(cfg, T_s):
     args = _oracle_inputs(cfg, T_s)
     t0 = time.perf_counter()
     _oracle_step(*args[:4], args[4], cfg.k, args[5], args[6])
-    dt = max(time.perf_counter() - t0, 1e-3)
-    T_fit = int(T_s * seconds / dt)
-    return max(min(128, cfg.T), min(cfg.T, T_fit // 64 * 64 if T_fit >= 64 else T_fit))
+    return max(time.perf_counter() - t0, 1e-3)
+
+
+def size_oracle_sample(cfg, seconds):
+    """Tokens per oracle step so that one step costs about `seconds`.  A step
+    has a fixed part (every expert's full weights are rounded and their
+    gradients formed whatever the token count) and a part linear in the
+    tokens, so two probe sizes fit t = a + b T and the sample solves it."""
+    T1 = min(128, cfg.T)
+    T2 = min(4 * T1, cfg.T)
+    _oracle_seconds(cfg, T1)  # first touch of the weights and BLAS threads, not timed
+    t1 = _oracle_seconds(cfg, T1)
+    if T2 == T1:
+        return T1
+    t2 = _oracle_seconds(cfg, T2)
+    b = (t2 - t1) / (T2 - T1)
+    if b <= 0:
+        b = t2 / T2
+    a = max(t1 - b * T1, 0.0)
+    T_fit = int(max(seconds - a, 0.0) / b)
+    return max(T1, min(cfg.T, T_fit // 64 * 64 if T_fit >= 64 else T_fit))
 
 
 def cpu_baseline(cfg, seconds):
