@@ -29,6 +29,8 @@ import sys
 import tempfile
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
@@ -203,6 +205,28 @@ def cpu_baseline(cfg, seconds):
 
 
 # ------------------------------------------------------------------ our arm
+def gini(counts):
+    """Gini coefficient of the per-expert routed-row counts: 0 when every
+    expert gets the same load, (E - 1) / E when one expert gets all of it.
+    With the counts sorted ascending, c_1 <= ... <= c_E,
+    G = 2 * sum_i i * c_i / (E * sum_i c_i) - (E + 1) / E."""
+    c = np.sort(np.asarray(counts, dtype=np.float64).ravel())
+    E, total = c.size, c.sum()
+    if E == 0 or total <= 0:
+        return 0.0
+    i = np.arange(1, E + 1, dtype=np.float64)
+    return float(2.0 * np.dot(i, c) / (E * total) - (E + 1.0) / E)
+
+
+def load_report(counts):
+    """Per-expert load of one step's routing, read from the device counts
+    after the timed region: the real load, not a balance score."""
+    c = np.asarray(counts, dtype=np.int64).ravel()
+    return {"max_over_mean_load": float(c.max() / c.mean()), "max_count": int(c.max()),
+            "min_count": int(c.min()), "mean_count": float(c.mean()),
+            "zero_experts": int((c == 0).sum()), "gini": gini(c)}
+
+
 def gemm_traffic(cfg_name):
     """DRAM bytes per step of the grouped-GEMM launches from the committed ncu
     summary, only while the kernel sources are the ones it was taken on."""
@@ -523,8 +547,7 @@ def run_ours(args):
         "gpu_launches": main["launches"],
         "grouped_gemm": {"tflops": achieved, "ms_per_step": gemm_ms,
                          "share_of_step": gemm_ms / (main["total_ms"] / K)},
-        "routing": {"max_over_mean_load": float(counts.max() / counts.mean()),
-                    "zero_experts": int((counts == 0).sum())},
+        "routing": load_report(counts),
         "memory_bound": {
             "peak_gb_s": peaks["hbm_gbs"], "peak_source": f"{peak_kind} copy",
             "timing": "each call alone, CUDA events, L2 flushed before it, median of 10 (rank 0)",
@@ -546,9 +569,7 @@ def run_ours(args):
             "ms_per_step": skew["total_ms"] / K,
             "grouped_gemm_tflops": sc.gemm_flops_fwd_bwd()
             / (statistics.mean(skew["gemm_ms"]) / 1e3) / 1e12,
-            "routing": {"max_over_mean_load": float(sk_counts.max() / sk_counts.mean()),
-                        "max_count": int(sk_counts.max()), "mean_count": float(sk_counts.mean()),
-                        "zero_experts": int((sk_counts == 0).sum())}}
+            "routing": load_report(sk_counts)}
     if variants:
         base_ms = main["total_ms"] / K
         line["variants"] = {}

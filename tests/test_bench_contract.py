@@ -29,3 +29,27 @@ def test_reference_arm_json_line():
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_load_report_gini():
+    """The Gini coefficient of the per-expert loads (the sorted-sum form the
+    bench uses) against its closed forms, 0 for equal loads and (E - 1) / E
+    when one expert takes every row, and against the mean-absolute-difference
+    definition, sum_ij |c_i - c_j| / (2 n sum_i c_i), on random counts."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import bench
+    E = 16
+    assert bench.gini(np.full(E, 37)) == 0.0
+    one = np.zeros(E, dtype=np.int64)
+    one[5] = 1000
+    assert abs(bench.gini(one) - (E - 1) / E) < 1e-12
+    rng = np.random.default_rng(0)
+    for _ in range(5):
+        c = rng.integers(0, 500, size=int(rng.integers(2, 200)))
+        mad = np.abs(c[:, None] - c[None, :]).sum()   # sum over all ordered pairs
+        ref = mad / (2 * c.size * c.sum())
+        assert abs(bench.gini(c) - ref) < 1e-12
+    r = bench.load_report(np.array([0, 4, 4, 8]))
+    assert r["zero_experts"] == 1 and r["max_count"] == 8 and r["min_count"] == 0
+    assert r["max_over_mean_load"] == 2.0 and abs(r["gini"] - 0.375) < 1e-12
