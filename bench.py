@@ -726,7 +726,7 @@ def run_reference(args):
     from mixture_experts_layer_39_b200.inputs import CONFIGS
     cfg = CONFIGS[args.workload]
     per_step = max(0.5, 150.0 / max(1, args.steps + args.warmup))
-    T_s = size_oracle_sample(cfg, min(per_step, 5.0))
+    T_s = size_oracle_sample(cfg, min(per_step, 4.0))
     inp = _oracle_inputs(cfg, T_s)
     for _ in range(args.warmup):
         _oracle_step(*inp[:4], inp[4], cfg.k, inp[5], inp[6])
