@@ -37,6 +37,9 @@
  *     caller-written topk_idx, a bounded wait that ran out) never trap: the
  *     kernel records a code in the handle's status word, skips the bad
  *     entry, and moe_get_status reports it later.
+ *   - Every call that takes a stream, and moe_create, moe_destroy and
+ *     moe_get_status, opens one NVTX range named for itself and closes it
+ *     before returning (NVTX 3, header-only; a no-op without a tool).
  *   - Layouts are row-major.  bf16 = bfloat16 (round to nearest even).
  *   - Supported shapes: 1 <= k <= min(E, 8), 1 <= E <= 1024, T >= 1,
  *     d_model and d_ff multiples of 128.
