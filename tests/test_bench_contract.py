@@ -53,3 +53,24 @@ def test_load_report_gini():
     r = bench.load_report(np.array([0, 4, 4, 8]))
     assert r["zero_experts"] == 1 and r["max_count"] == 8 and r["min_count"] == 0
     assert r["max_over_mean_load"] == 2.0 and abs(r["gini"] - 0.375) < 1e-12
+
+
+def test_reference_arm_under_torchrun_two_ranks():
+    """Launched the way an N-GPU run is (torchrun, one process per rank), the
+    reference arm runs on rank 0 only: exactly one JSON line, n_gpus = 2,
+    every rank exits 0.  No GPU and no process group are needed for it."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                        "--nproc-per-node", "2", "--master-addr", "127.0.0.1",
+                        "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+                        "--impl", "reference", "--workload", "tiny", "--steps", "1",
+                        "--warmup", "0", "--gpus", "2"],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
